@@ -1,0 +1,382 @@
+#!/usr/bin/env python
+"""Benchmark of the Prism dynamic block-sparse video self-attention layer.
+
+One step = one pass of the whole path over one synthetic layer:
+prism_plan -> prism_select -> prism_attn_fwd -> prism_attn_bwd, on the
+native-2K training grid (T=56, H=96, W=160: 860,160 tokens, 24 heads,
+head_dim 128, bf16, Top-k 4%, Top-p 0.9) unless --workload says otherwise.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl prism|reference]
+
+Prints one JSON line (rank 0).  `value` is the effective TFLOP/s of the whole
+step over all ranks, counting only the computed blocks: (4 + 10) * P * D per
+layer, P = number of computed (query, key) token pairs.  Multi-GPU runs are
+weak scaling: every rank runs its own independent layer (seeded by rank);
+ranks exchange nothing but the timing barrier.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from dynamic_block_sparse_stats_b200 import _lib, api  # noqa: E402
+from dynamic_block_sparse_stats_b200.synth import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "Prism sparse-attn fwd+bwd ms/layer & effective TFLOP/s at ~860K tokens"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for name, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- flops
+def computed_pairs(p, pl, sel):
+    """P = sum over heads and query blocks i of B_i * sum_{j in S_i} B_j."""
+    NB = p.T * p.H * p.W // 64
+    row_ptr = sel.row_ptr.long()
+    counts = row_ptr[1:] - row_ptr[:-1]
+    Bsz = pl.blocks[:, :, 1].reshape(-1).long()            # [heads*NB] (garbage past n_blocks)
+    rows = torch.arange(p.heads * NB, device=row_ptr.device)
+    valid = (rows % NB) < pl.n_blocks.long().repeat_interleave(NB)
+    Bq = torch.where(valid, Bsz, torch.zeros_like(Bsz))
+    row_of = torch.repeat_interleave(rows, counts)
+    head_of = row_of // NB
+    col = sel.col[:sel.nnz].long()
+    Bk = Bsz[head_of * NB + col]
+    return int((Bq[row_of] * Bk).sum().item())
+
+
+# ----------------------------------------------------------------------------- oracle sample
+def oracle_sample(w, inp, p, pl, sel, head=0, n_rows=2, seed=0):
+    """Time the CPU oracle on a bounded sample of the same layer: the plan and
+    the selection of one head over the full grid, and forward+backward
+    attention of `n_rows` random query blocks of that head.  Returns the
+    extrapolated layer time and the sample description."""
+    from threadpoolctl import threadpool_info
+
+    from oracle import prism_oracle as O
+    T, H, W = w.T, w.H, w.W
+    Vh = inp["V"][:, head:head + 1].float().cpu().numpy()
+    Qh = inp["Q"][:, head:head + 1].float().cpu().numpy()
+    Kh = inp["K"][:, head:head + 1].float().cpu().numpy()
+    a = inp["a"].cpu().numpy()
+    dOh = inp["dO"][:, head:head + 1].float().cpu().numpy() if "dO" in inp else None
+    t0 = time.perf_counter()
+    opl = O.plan(Vh, a, T, H, W)
+    t1 = time.perf_counter()
+    osel = O.select(Qh, Kh, opl, w.topk_frac, w.topk_abs, w.top_p)
+    t2 = time.perf_counter()
+    hp = opl.heads[0]
+    nb = hp.blocks.shape[0]
+    rng = np.random.default_rng(seed)
+    rows = sorted(rng.choice(nb, size=min(n_rows, nb), replace=False).tolist())
+    sub = [[osel[0][i] for i in rows]]
+    scale = float(np.float32(1.0 / math.sqrt(w.head_dim)))
+    t3 = time.perf_counter()
+    O.attention_fwd(Qh, Kh, Vh, opl, sub, scale)
+    if dOh is not None:
+        O.attention_bwd(Qh, Kh, Vh, dOh, opl, sub, scale)
+    t4 = time.perf_counter()
+    pairs_sample = sum(int(hp.blocks[i, 4]) * int(sum(hp.blocks[j, 4] for j in ids)) for (i, ids, _) in sub[0])
+    P_total = computed_pairs(p, pl, sel)
+    attn_time = (t4 - t3) * (P_total / max(pairs_sample, 1))
+    layer_time = w.heads * ((t1 - t0) + (t2 - t1)) + attn_time
+    threads = max([t.get("num_threads", 1) for t in threadpool_info()] + [1])
+    desc = (f"oracle plan+select of head {head} over the full {T}x{H}x{W} grid "
+            f"({(t1 - t0):.2f}s + {(t2 - t1):.2f}s, x{w.heads} heads) and fwd"
+            f"{'+bwd' if dOh is not None else ''} of {len(rows)} query blocks ({t4 - t3:.2f}s, "
+            f"x{P_total / max(pairs_sample, 1):.0f} by computed pairs); extrapolated layer time {layer_time:.1f}s")
+    return layer_time, desc, threads, (t4 - t0)
+
+
+# ----------------------------------------------------------------------------- main arms
+def run_prism(args, w, rank, world, device):
+    lib = _lib.load()
+    p = api.params_for(w)
+    inp = make_inputs(w, device, seed=rank)
+    N, h, D = w.N, w.heads, w.head_dim
+    Q, K, V, a = inp["Q"], inp["K"], inp["V"], inp["a"]
+    dO = inp.get("dO")
+    backward = dO is not None
+    # buffers reused by every step
+    pl = api.plan(p, V, a)
+    sel = api.select(p, pl, Q, K)
+    sel = api.select(p, pl, Q, K, cap=int(sel.nnz * 1.1) + 1024)
+    fw = api.attn_fwd(p, pl, sel, Q, K, V)
+    O_, lse = fw.O, fw.lse
+    grads = None
+    bws = None
+    if backward:
+        grads = api.attn_bwd(p, pl, sel, Q, K, V, O_, dO, lse)
+        bws = torch.empty(lib.prism_attn_workspace_size(api.C.byref(p), 1), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    stages = ["plan", "select", "fwd", "bwd"] if backward else ["plan", "select", "fwd"]
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        api.plan(p, V, a, out=pl)
+        if ev is not None:
+            ev[1].record(stream)
+        api.select(p, pl, Q, K, out=sel)
+        if ev is not None:
+            ev[2].record(stream)
+        api.attn_fwd(p, pl, sel, Q, K, V, O=O_, lse=lse, ws=fw.ws)
+        if ev is not None:
+            ev[3].record(stream)
+        if backward:
+            api.attn_bwd(p, pl, sel, Q, K, V, O_, dO, lse, out=grads, ws=bws)
+            if ev is not None:
+                ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    P = computed_pairs(p, pl, sel)
+    flops_fwd, flops_bwd = 4.0 * P * D, (10.0 * P * D if backward else 0.0)
+    flops = flops_fwd + flops_bwd
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(args.steps)]
+    clk = ClockSampler(torch.cuda.current_device())
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clk.start()
+    l0 = lib.prism_kernel_launches()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    launches = lib.prism_kernel_launches() - l0
+    clocks = clk.stop()
+    ms = t_start.elapsed_time(t_end) / args.steps
+    stage_ms = {s: statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps))
+                for i, s in enumerate(stages)}
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+
+    # end to end through host buffers
+    e2e = None
+    if not args.no_e2e:
+        hin = {k: inp[k].cpu().pin_memory() for k in (["Q", "K", "V", "a"] + (["dO"] if backward else []))}
+        outs = [O_] + (list(grads) if backward else [])
+        hout = [torch.empty_like(t, device="cpu").pin_memory() for t in outs]
+        dev = {"Q": Q, "K": K, "V": V, "a": a, "dO": dO}
+        h2d = sum(t.numel() * t.element_size() for t in hin.values())
+        d2h = sum(t.numel() * t.element_size() for t in hout)
+
+        def step_e2e():
+            for k_, t in hin.items():
+                dev[k_].copy_(t, non_blocking=True)
+            step()
+            for src, dst in zip(outs, hout):
+                dst.copy_(src, non_blocking=True)
+
+        step_e2e()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        ksteps = max(1, min(args.steps, 3))
+        for _ in range(ksteps):
+            step_e2e()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = torch.tensor([e0.elapsed_time(e1) / ksteps], dtype=torch.float64, device=device)
+        if world > 1:
+            torch.distributed.all_reduce(ems, op=torch.distributed.ReduceOp.MAX)
+        e2e = {"value": world * flops / (float(ems.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": float(ems.item()), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "steps": ksteps}
+        del hin, hout
+
+    peaks, peak_src = load_peaks()
+    dominant = "bwd" if backward else "fwd"
+    dom_flops = flops_bwd if backward else flops_fwd
+    achieved = dom_flops / (stage_ms[dominant] * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    roofline = {"kernel": f"prism_attn_{dominant} call ({'attn_bwd' if backward else 'attn_fwd'} kernels)",
+                "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_source": f"{peak_src} bf16 sustained", "traffic": None,
+                "algorithmic": f"{'10' if backward else '4'}*P*D = {dom_flops:.4e} FLOP per launch"}
+    plan_bytes = N * h * D * 2 + N * 4
+    stage_roofline = {
+        "plan_GBps": plan_bytes / (stage_ms["plan"] * 1e-3) / 1e9,
+        "plan_frac_hbm": plan_bytes / (stage_ms["plan"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "fwd_TFLOPs": flops_fwd / (stage_ms["fwd"] * 1e-3) / 1e12,
+        "fwd_frac_bf16": flops_fwd / (stage_ms["fwd"] * 1e-3) / 1e12 / peak,
+    }
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        layer_time, desc, threads, wall = oracle_sample(w, inp, p, pl, sel)
+        cpu = {"value": flops / layer_time / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": desc, "host_cpus": os.cpu_count(), "sample_wall_s": wall}
+
+    density = P / (float(N) * N * h)
+    line = {
+        "metric": METRIC, "value": world * flops / (ms_max * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded generator; stands in for the pages' 2K-Bench latents)",
+        "config": {"workload": w.name, "T": w.T, "H": w.H, "W": w.W, "tokens": N, "heads": h, "head_dim": D,
+                   "topk_frac": w.topk_frac, "top_p": w.top_p, "backward": backward,
+                   "parallelism": f"weak x{world} (independent layers, no collectives)",
+                   "l2": "inputs larger than L2 (each bf16 tensor %.2f GB)" % (N * h * D * 2 / 1e9),
+                   "pairs": P, "pair_density": density, "nnz_blocks": sel.nnz},
+        "stage_ms": stage_ms, "stage_roofline": stage_roofline,
+        "clocks": clocks, "e2e": e2e, "gpu_launches": launches, "roofline": roofline, "cpu_baseline": cpu,
+    }
+    return line
+
+
+def run_reference(args, w, rank, world):
+    """The CPU oracle as the reference arm: each step is a bounded sample of the
+    same layer (plan + selection of one head, fwd+bwd of two query blocks),
+    extrapolated to the layer by computed pairs."""
+    if rank != 0:
+        return None
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_inputs(w, dev, seed=0)
+    p = api.params_for(w)
+    if dev == "cuda":
+        pl = api.plan(p, inp["V"], inp["a"])
+        sel = api.select(p, pl, inp["Q"], inp["K"])
+    else:
+        raise RuntimeError("the reference arm needs the selection size of the layer (CUDA) for extrapolation")
+    times, desc, threads = [], "", 1
+    for k in range(args.warmup + args.steps):
+        lt, desc, threads, _wall = oracle_sample(w, inp, p, pl, sel, head=k % w.heads, seed=k)
+        if k >= args.warmup:
+            times.append(lt)
+    P = computed_pairs(p, pl, sel)
+    flops = (4.0 + (10.0 if w.backward else 0.0)) * P * w.head_dim
+    layer = statistics.mean(times)
+    v = flops / layer / 1e12
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": layer * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded generator; stands in for the pages' 2K-Bench latents)",
+            "config": {"workload": w.name, "T": w.T, "H": w.H, "W": w.W, "tokens": w.N, "heads": w.heads,
+                       "head_dim": w.head_dim, "topk_frac": w.topk_frac, "top_p": w.top_p},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["prism", "reference"], default="prism")
+    ap.add_argument("--workload", default="2k_train", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+
+    if args.impl == "reference":
+        line = run_reference(args, w, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the prism arm has no CPU path)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    try:
+        line = run_prism(args, w, rank, world, device)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

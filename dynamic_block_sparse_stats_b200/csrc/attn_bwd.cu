@@ -1,0 +1,704 @@
+// prism_attn_bwd: gradients of the block-sparse attention through the
+// selected blocks only, on tcgen05 tensor cores.
+//
+// Method: Prism digest ("Prism：为原生 2K 视频音频联合生成设计的动态稀疏注意力"),
+// training section: shape assignment and block selection are constants; the
+// gradient flows only through the sparse attention of the selected blocks.
+// The arithmetic is the softmax-attention backward with the softmax recomputed
+// from the forward's log-sum-exp:
+//   P = exp(s*scale - lse), dP = dO V^T, Delta_q = sum_c dO_qc O_qc,
+//   dS = P (dP - Delta), dQ = scale dS K, dK = scale dS^T Q, dV = P^T dO.
+//
+// Two kernels, no atomics (deterministic):
+//   dq_kernel    one CTA per 128-query tile; walks the CSR like the forward:
+//                S = Q K^T, dP = dO V^T (TMEM), dS -> TMEM (bf16),
+//                dQ += dS K (TS MMA).
+//   dkdv_kernel  one CTA per 128-key tile; walks the transpose (CSC):
+//                S^T = K Q^T, dP^T = V dO^T (TMEM), P^T and dS^T -> TMEM
+//                (bf16), dV += P^T dO, dK += dS^T Q (TS MMAs).
+// Roles as in the forward: warp 0 TMA producer, warp 1 TMEM owner and MMA
+// issuer, warps 2-5 one thread per TMEM lane (row).
+#include "attn_walk.cuh"
+
+namespace prism {
+namespace bwd {
+using namespace attn;
+
+constexpr int NSTAGE = 2;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------------------
+// prep: dOp[h][p] = dO[perm][h], delta[h][p] = sum_c dO*O, lse2[h][p] = lse*log2e
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const int32_t *__restrict__ perm, int N, int heads,
+                                                       const uint16_t *__restrict__ dO,
+                                                       const uint16_t *__restrict__ O,
+                                                       const float *__restrict__ lse, uint16_t *__restrict__ dOp,
+                                                       float *__restrict__ lse2p, float *__restrict__ deltap) {
+  constexpr int G = D / 8;  // lanes per row
+  const size_t g = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t r = g / G;
+  const int v = (int)(g % G);
+  const size_t rows = (size_t)heads * N;
+  const bool live = r < rows;
+  float acc = 0.f;
+  if (live) {
+    const int h = (int)(r / N);
+    const int n = perm[r];
+    const size_t src = ((size_t)n * heads + h) * D + v * 8;
+    const uint4 a = __ldg(reinterpret_cast<const uint4 *>(dO + src));
+    const uint4 b = __ldg(reinterpret_cast<const uint4 *>(O + src));
+    *reinterpret_cast<uint4 *>(dOp + r * D + v * 8) = a;
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      acc = fmaf(bf16lo(aw[q]), bf16lo(bw[q]), acc);
+      acc = fmaf(bf16hi(aw[q]), bf16hi(bw[q]), acc);
+    }
+    if (v == 0) lse2p[r] = lse[(size_t)h * N + n] * kLog2e;
+  }
+#pragma unroll
+  for (int o = 1; o < G; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (live && v == 0) deltap[r] = acc;
+}
+
+// ---------------------------------------------------------------------------
+// dQ kernel
+// ---------------------------------------------------------------------------
+template <int D>
+struct DqSmem {
+  static constexpr int CHUNKS = D / 64;
+  static constexpr int TILE = 128 * D * 2;  // 128 rows of bf16
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_DO = OFF_Q + TILE;
+  static constexpr int OFF_K = OFF_DO + TILE;
+  static constexpr int OFF_V = OFF_K + NSTAGE * TILE;
+  static constexpr int OFF_BAR = OFF_V + NSTAGE * TILE;
+  static constexpr int BYTES = OFF_BAR + 256;
+};
+
+struct DqBars {
+  uint64_t qdo_full;
+  uint64_t k_full[NSTAGE];
+  uint64_t v_full[NSTAGE];
+  uint64_t kv_empty[NSTAGE];
+  uint64_t s_full, dp_full, ds_ready, dq_done;
+  int meta[NSTAGE];
+  uint32_t tmem_base;
+  int ntiles, nunits, abort;
+};
+
+template <int D>
+__device__ __forceinline__ void store_row(void *out, bool fp32, size_t off, const uint32_t (&o)[32], float mul) {
+  if (fp32) {
+    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(out) + off);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      dst[i] = make_float4(__uint_as_float(o[4 * i]) * mul, __uint_as_float(o[4 * i + 1]) * mul,
+                           __uint_as_float(o[4 * i + 2]) * mul, __uint_as_float(o[4 * i + 3]) * mul);
+  } else {
+    uint4 v[4];
+    uint32_t *pv = reinterpret_cast<uint32_t *>(v);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) pv[i] = pack_bf16(__uint_as_float(o[2 * i]) * mul, __uint_as_float(o[2 * i + 1]) * mul);
+    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(out) + off);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dst[i] = v[i];
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    dq_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapDO,
+              const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
+              const int32_t *__restrict__ row_ptr, const int32_t *__restrict__ col, const int32_t *__restrict__ blocks,
+              const int32_t *__restrict__ unit_block, const int32_t *__restrict__ tile_units,
+              const int32_t *__restrict__ perm, const float *__restrict__ lse2p, const float *__restrict__ deltap,
+              void *__restrict__ dQ, int grad_fp32, int N, int heads, float scale_log2, float sm_scale,
+              int *status) {
+  using L = DqSmem<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  DqBars &bar = *reinterpret_cast<DqBars *>(smem + L::OFF_BAR);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, h = blockIdx.y;
+  const int NB = N / 64;
+  const int32_t *blocks_h = blocks + (size_t)h * NB * 4;
+
+  if (threadIdx.x == 0) bar.abort = *reinterpret_cast<volatile int *>(status);
+  __syncthreads();
+  if (bar.abort) return;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar.qdo_full, 1);
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(&bar.k_full[s], 1);
+      mbar_init(&bar.v_full[s], 1);
+      mbar_init(&bar.kv_empty[s], 1);
+    }
+    mbar_init(&bar.s_full, 1);
+    mbar_init(&bar.dp_full, 1);
+    mbar_init(&bar.ds_ready, 128);
+    mbar_init(&bar.dq_done, 1);
+    bar.nunits = tile_units[(size_t)h * (N / 128) + tile];
+    bar.ntiles = (bar.nunits + 1) >> 1;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bar.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar.tmem_base;
+  const int ntiles = bar.ntiles, nunits = bar.nunits;
+  const uint32_t tS = tmem, tP = tmem + 128, tQ = tmem + 256;
+
+  if (warp == 0) {
+    const int b0 = unit_block[(size_t)h * NB + 2 * tile], b1 = unit_block[(size_t)h * NB + 2 * tile + 1];
+    UnitWalk w;
+    cursor_init(w.a, row_ptr[h * NB + b0], row_ptr[h * NB + b0 + 1]);
+    if (b1 != b0) {
+      cursor_init(w.b, row_ptr[h * NB + b1], row_ptr[h * NB + b1 + 1]);
+      w.mask_a = 1;
+      w.mask_b = 2;
+    } else {
+      cursor_init(w.b, 0, 0);
+      w.mask_a = 3;
+      w.mask_b = 0;
+    }
+    w.cur_cnt = w.cur_k = 0;
+    w.cur_ub = 0;
+    w.cur_mask = 0;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bar.qdo_full, 2 * L::TILE);
+#pragma unroll
+      for (int c = 0; c < L::CHUNKS; ++c) {
+        tma_load_2d(smem + L::OFF_Q + c * (128 * 128), &mapQ, &bar.qdo_full, c * 64, h * N + tile * 128);
+        tma_load_2d(smem + L::OFF_DO + c * (128 * 128), &mapDO, &bar.qdo_full, c * 64, h * N + tile * 128);
+      }
+    }
+    for (int j = 0; j < ntiles; ++j) {
+      const int s = j % NSTAGE;
+      uint32_t ua, ub = 0;
+      int ma, mb = 0, nu = 1;
+      walk_next(w, col, blocks_h, ua, ma);
+      if (2 * j + 2 <= nunits) {
+        walk_next(w, col, blocks_h, ub, mb);
+        nu = 2;
+      }
+      ua = min(ua, (uint32_t)(NB - 1));
+      ub = min(ub, (uint32_t)(NB - 1));
+      if (lane == 0) {
+        bool ok = true;
+        if (j >= NSTAGE) ok = mbar_wait(&bar.kv_empty[s], ((j / NSTAGE) - 1) & 1, status, 21);
+        if (!ok) bar.abort = 1;
+        if (ok) {
+          bar.meta[s] = nu | (ma << 4) | (mb << 8);
+          uint8_t *ks = smem + L::OFF_K + s * L::TILE;
+          uint8_t *vs = smem + L::OFF_V + s * L::TILE;
+          const int bytes = nu * 64 * D * 2;
+          mbar_arrive_expect_tx(&bar.k_full[s], bytes);
+#pragma unroll
+          for (int c = 0; c < L::CHUNKS; ++c) {
+            tma_load_2d(ks + c * (128 * 128), &mapK, &bar.k_full[s], c * 64, h * N + (int)ua * 64);
+            if (nu == 2) tma_load_2d(ks + c * (128 * 128) + 64 * 128, &mapK, &bar.k_full[s], c * 64, h * N + (int)ub * 64);
+          }
+          mbar_arrive_expect_tx(&bar.v_full[s], bytes);
+#pragma unroll
+          for (int c = 0; c < L::CHUNKS; ++c) {
+            tma_load_2d(vs + c * (128 * 128), &mapV, &bar.v_full[s], c * 64, h * N + (int)ua * 64);
+            if (nu == 2) tma_load_2d(vs + c * (128 * 128) + 64 * 128, &mapV, &bar.v_full[s], c * 64, h * N + (int)ub * 64);
+          }
+        }
+      }
+      __syncwarp();
+      if (*reinterpret_cast<volatile int *>(&bar.abort)) break;
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_full = idesc_bf16(128, 128, 0), id_half = idesc_bf16(128, 64, 0);
+      const uint32_t id_dq = idesc_bf16(128, D, 1);
+      const uint32_t sQ = smem_u32(smem + L::OFF_Q), sDO = smem_u32(smem + L::OFF_DO);
+      bool ok = mbar_wait(&bar.qdo_full, 0, status, 22);
+      tc_fence_after();
+      for (int j = 0; ok && j <= ntiles; ++j) {
+        if (j >= 1) {  // dQ += dS_{j-1} K_{j-1}
+          const int jj = j - 1, s = jj % NSTAGE;
+          ok = mbar_wait(&bar.ds_ready, jj & 1, status, 23);
+          if (!ok) break;
+          tc_fence_after();
+          const int nu = bar.meta[s] & 15;
+          const uint32_t sK = smem_u32(smem + L::OFF_K + s * L::TILE);
+          for (int ks = 0; ks < nu * 4; ++ks)
+            mma_ts(tQ, tP + ks * 8, sdesc_sw128(sK + ks * 2048, 128 * 128, 1024), id_dq,
+                   (jj > 0 || ks > 0) ? 1u : 0u);
+          mma_commit(&bar.dq_done);
+          mma_commit(&bar.kv_empty[s]);
+        }
+        if (j < ntiles) {
+          const int s = j % NSTAGE;
+          ok = mbar_wait(&bar.k_full[s], (j / NSTAGE) & 1, status, 24);
+          if (!ok) break;
+          tc_fence_after();
+          const int nu = bar.meta[s] & 15;
+          const uint32_t id = nu == 2 ? id_full : id_half;
+          const uint32_t sK = smem_u32(smem + L::OFF_K + s * L::TILE);
+          const uint32_t sV = smem_u32(smem + L::OFF_V + s * L::TILE);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+            mma_ss(tS, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), id, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&bar.s_full);
+          ok = mbar_wait(&bar.v_full[s], (j / NSTAGE) & 1, status, 25);
+          if (ok && j >= 1) ok = mbar_wait(&bar.dq_done, (j - 1) & 1, status, 26);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+            mma_ss(tP, sdesc_sw128(sDO + off, 16, 1024), sdesc_sw128(sV + off, 16, 1024), id, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&bar.dp_full);
+        }
+      }
+      if (!ok) bar.abort = 1;
+    }
+    __syncwarp();
+  } else {
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    const int half = row >> 6;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const size_t prow = (size_t)h * N + (size_t)tile * 128 + row;
+    const float lse2 = lse2p[prow], dl = deltap[prow];
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      const int s = j % NSTAGE;
+      ok = mbar_wait(&bar.s_full, j & 1, status, 27);
+      if (ok) ok = mbar_wait(&bar.dp_full, j & 1, status, 28);
+      if (!ok) break;
+      tc_fence_after();
+      const int meta = bar.meta[s];
+      const int nu = meta & 15;
+      for (int c = 0; c < 2 * nu; ++c) {
+        const int m = (c < 2) ? (meta >> 4) : (meta >> 8);
+        const bool valid = (m >> half) & 1;
+        uint32_t sv[32], dv[32], pk[16];
+        tmem_ld32(tS + lane_off + c * 32, sv);
+        tmem_ld32(tP + lane_off + c * 32, dv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float d0 = 0.f, d1 = 0.f;
+          if (valid) {
+            const float p0 = exp2f(fmaf(__uint_as_float(sv[i]), scale_log2, -lse2));
+            const float p1 = exp2f(fmaf(__uint_as_float(sv[i + 1]), scale_log2, -lse2));
+            d0 = p0 * (__uint_as_float(dv[i]) - dl);
+            d1 = p1 * (__uint_as_float(dv[i + 1]) - dl);
+          }
+          pk[i / 2] = pack_bf16(d0, d1);
+        }
+        tmem_st16(tP + lane_off + c * 16, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar.ds_ready);
+    }
+    if (ok && ntiles > 0) ok = mbar_wait(&bar.dq_done, (ntiles - 1) & 1, status, 29);
+    if (ok) {
+      tc_fence_after();
+      const int n = perm[prow];
+      const size_t off = ((size_t)n * heads + h) * D;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t o[32];
+        if (ntiles > 0) {
+          tmem_ld32(tQ + lane_off + c, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
+        store_row<D>(dQ, grad_fp32 != 0, off + c, o, sm_scale);
+      }
+    } else {
+      bar.abort = 1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dK/dV kernel
+// ---------------------------------------------------------------------------
+template <int D>
+struct KvSmem {
+  static constexpr int CHUNKS = D / 64;
+  static constexpr int TILE = 128 * D * 2;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + TILE;
+  static constexpr int OFF_Q = OFF_V + TILE;                 // ring of query tiles
+  static constexpr int OFF_DO = OFF_Q + NSTAGE * TILE;       // ring of dO tiles
+  static constexpr int OFF_STAT = OFF_DO + NSTAGE * TILE;    // [NSTAGE][2][128] floats: lse2, delta
+  static constexpr int OFF_BAR = OFF_STAT + NSTAGE * 2 * 128 * 4;
+  static constexpr int BYTES = OFF_BAR + 256;
+};
+
+struct KvBars {
+  uint64_t kv_full;
+  uint64_t q_full[NSTAGE];
+  uint64_t q_empty[NSTAGE];
+  uint64_t s_full, dp_full, ds_ready, mm_done;
+  int meta[NSTAGE];
+  uint32_t tmem_base;
+  int ntiles, nunits, abort;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    dkdv_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapDO,
+                const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
+                const int32_t *__restrict__ col_ptr, const int32_t *__restrict__ rowidx,
+                const int32_t *__restrict__ blocks, const int32_t *__restrict__ unit_block,
+                const int32_t *__restrict__ tile_units, const int32_t *__restrict__ perm,
+                const float *__restrict__ lse2p, const float *__restrict__ deltap, void *__restrict__ dK,
+                void *__restrict__ dV, int grad_fp32, int N, int heads, float scale_log2, float sm_scale,
+                int *status) {
+  using L = KvSmem<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  KvBars &bar = *reinterpret_cast<KvBars *>(smem + L::OFF_BAR);
+  float *stat = reinterpret_cast<float *>(smem + L::OFF_STAT);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, h = blockIdx.y;
+  const int NB = N / 64;
+  const int32_t *blocks_h = blocks + (size_t)h * NB * 4;
+
+  if (threadIdx.x == 0) bar.abort = *reinterpret_cast<volatile int *>(status);
+  __syncthreads();
+  if (bar.abort) return;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar.kv_full, 1);
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(&bar.q_full[s], 1);
+      mbar_init(&bar.q_empty[s], 1);
+    }
+    mbar_init(&bar.s_full, 1);
+    mbar_init(&bar.dp_full, 1);
+    mbar_init(&bar.ds_ready, 128);
+    mbar_init(&bar.mm_done, 1);
+    bar.nunits = tile_units[(size_t)h * (N / 128) + tile];
+    bar.ntiles = (bar.nunits + 1) >> 1;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bar.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar.tmem_base;
+  const int ntiles = bar.ntiles, nunits = bar.nunits;
+  const uint32_t tS = tmem, tP = tmem + 128, tV = tmem + 256, tK = tmem + 256 + D;
+
+  if (warp == 0) {
+    const int b0 = unit_block[(size_t)h * NB + 2 * tile], b1 = unit_block[(size_t)h * NB + 2 * tile + 1];
+    UnitWalk w;
+    cursor_init(w.a, col_ptr[h * NB + b0], col_ptr[h * NB + b0 + 1]);
+    if (b1 != b0) {
+      cursor_init(w.b, col_ptr[h * NB + b1], col_ptr[h * NB + b1 + 1]);
+      w.mask_a = 1;
+      w.mask_b = 2;
+    } else {
+      cursor_init(w.b, 0, 0);
+      w.mask_a = 3;
+      w.mask_b = 0;
+    }
+    w.cur_cnt = w.cur_k = 0;
+    w.cur_ub = 0;
+    w.cur_mask = 0;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bar.kv_full, 2 * L::TILE);
+#pragma unroll
+      for (int c = 0; c < L::CHUNKS; ++c) {
+        tma_load_2d(smem + L::OFF_K + c * (128 * 128), &mapK, &bar.kv_full, c * 64, h * N + tile * 128);
+        tma_load_2d(smem + L::OFF_V + c * (128 * 128), &mapV, &bar.kv_full, c * 64, h * N + tile * 128);
+      }
+    }
+    for (int j = 0; j < ntiles; ++j) {
+      const int s = j % NSTAGE;
+      uint32_t ua, ub = 0;
+      int ma, mb = 0, nu = 1;
+      walk_next(w, rowidx, blocks_h, ua, ma);
+      if (2 * j + 2 <= nunits) {
+        walk_next(w, rowidx, blocks_h, ub, mb);
+        nu = 2;
+      }
+      ua = min(ua, (uint32_t)(NB - 1));
+      ub = min(ub, (uint32_t)(NB - 1));
+      if (lane == 0) {
+        bool ok = true;
+        if (j >= NSTAGE) ok = mbar_wait(&bar.q_empty[s], ((j / NSTAGE) - 1) & 1, status, 41);
+        if (!ok) bar.abort = 1;
+        if (ok) {
+          bar.meta[s] = nu | (ma << 4) | (mb << 8);
+          uint8_t *qs = smem + L::OFF_Q + s * L::TILE;
+          uint8_t *ds = smem + L::OFF_DO + s * L::TILE;
+          float *st = stat + s * 256;
+          mbar_arrive_expect_tx(&bar.q_full[s], nu * (2 * 64 * D * 2 + 2 * 64 * 4));
+          for (int u = 0; u < nu; ++u) {
+            const int un = u == 0 ? (int)ua : (int)ub;
+#pragma unroll
+            for (int c = 0; c < L::CHUNKS; ++c) {
+              tma_load_2d(qs + c * (128 * 128) + u * 64 * 128, &mapQ, &bar.q_full[s], c * 64, h * N + un * 64);
+              tma_load_2d(ds + c * (128 * 128) + u * 64 * 128, &mapDO, &bar.q_full[s], c * 64, h * N + un * 64);
+            }
+            bulk_load(st + u * 64, lse2p + (size_t)h * N + (size_t)un * 64, 256, &bar.q_full[s]);
+            bulk_load(st + 128 + u * 64, deltap + (size_t)h * N + (size_t)un * 64, 256, &bar.q_full[s]);
+          }
+        }
+      }
+      __syncwarp();
+      if (*reinterpret_cast<volatile int *>(&bar.abort)) break;
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_full = idesc_bf16(128, 128, 0), id_half = idesc_bf16(128, 64, 0);
+      const uint32_t id_acc = idesc_bf16(128, D, 1);
+      const uint32_t sK = smem_u32(smem + L::OFF_K), sV = smem_u32(smem + L::OFF_V);
+      bool ok = mbar_wait(&bar.kv_full, 0, status, 42);
+      tc_fence_after();
+      for (int j = 0; ok && j <= ntiles; ++j) {
+        if (j >= 1) {  // dV += P^T dO, dK += dS^T Q  (tile j-1)
+          const int jj = j - 1, s = jj % NSTAGE;
+          ok = mbar_wait(&bar.ds_ready, jj & 1, status, 43);
+          if (!ok) break;
+          tc_fence_after();
+          const int nu = bar.meta[s] & 15;
+          const uint32_t sQ = smem_u32(smem + L::OFF_Q + s * L::TILE);
+          const uint32_t sDO = smem_u32(smem + L::OFF_DO + s * L::TILE);
+          for (int ks = 0; ks < nu * 4; ++ks) {
+            const uint32_t acc = (jj > 0 || ks > 0) ? 1u : 0u;
+            mma_ts(tV, tS + ks * 8, sdesc_sw128(sDO + ks * 2048, 128 * 128, 1024), id_acc, acc);
+            mma_ts(tK, tP + ks * 8, sdesc_sw128(sQ + ks * 2048, 128 * 128, 1024), id_acc, acc);
+          }
+          mma_commit(&bar.mm_done);
+          mma_commit(&bar.q_empty[s]);
+        }
+        if (j < ntiles) {
+          const int s = j % NSTAGE;
+          ok = mbar_wait(&bar.q_full[s], (j / NSTAGE) & 1, status, 44);
+          if (ok && j >= 1) ok = mbar_wait(&bar.mm_done, (j - 1) & 1, status, 45);
+          if (!ok) break;
+          tc_fence_after();
+          const int nu = bar.meta[s] & 15;
+          const uint32_t id = nu == 2 ? id_full : id_half;
+          const uint32_t sQ = smem_u32(smem + L::OFF_Q + s * L::TILE);
+          const uint32_t sDO = smem_u32(smem + L::OFF_DO + s * L::TILE);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+            mma_ss(tS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), id, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&bar.s_full);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+            mma_ss(tP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sDO + off, 16, 1024), id, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&bar.dp_full);
+        }
+      }
+      if (!ok) bar.abort = 1;
+    }
+    __syncwarp();
+  } else {
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;  // key row of the tile
+    const int half = row >> 6;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      const int s = j % NSTAGE;
+      ok = mbar_wait(&bar.s_full, j & 1, status, 47);
+      if (ok) ok = mbar_wait(&bar.dp_full, j & 1, status, 48);
+      if (!ok) break;
+      tc_fence_after();
+      const int meta = bar.meta[s];
+      const int nu = meta & 15;
+      const float *l2 = stat + s * 256, *dl = stat + s * 256 + 128;
+      for (int c = 0; c < 2 * nu; ++c) {
+        const int m = (c < 2) ? (meta >> 4) : (meta >> 8);
+        const bool valid = (m >> half) & 1;
+        uint32_t sv[32], dv[32], pp[16], pd[16];
+        tmem_ld32(tS + lane_off + c * 32, sv);
+        tmem_ld32(tP + lane_off + c * 32, dv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
+          if (valid) {
+            const int q = c * 32 + i;
+            p0 = exp2f(fmaf(__uint_as_float(sv[i]), scale_log2, -l2[q]));
+            p1 = exp2f(fmaf(__uint_as_float(sv[i + 1]), scale_log2, -l2[q + 1]));
+            d0 = p0 * (__uint_as_float(dv[i]) - dl[q]);
+            d1 = p1 * (__uint_as_float(dv[i + 1]) - dl[q + 1]);
+          }
+          pp[i / 2] = pack_bf16(p0, p1);
+          pd[i / 2] = pack_bf16(d0, d1);
+        }
+        tmem_st16(tS + lane_off + c * 16, pp);
+        tmem_st16(tP + lane_off + c * 16, pd);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar.ds_ready);
+    }
+    if (ok && ntiles > 0) ok = mbar_wait(&bar.mm_done, (ntiles - 1) & 1, status, 49);
+    if (ok) {
+      tc_fence_after();
+      const size_t prow = (size_t)h * N + (size_t)tile * 128 + row;
+      const int n = perm[prow];
+      const size_t off = ((size_t)n * heads + h) * D;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t o[32];
+        if (ntiles > 0) {
+          tmem_ld32(tV + lane_off + c, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
+        store_row<D>(dV, grad_fp32 != 0, off + c, o, 1.0f);
+        if (ntiles > 0) {
+          tmem_ld32(tK + lane_off + c, o);
+          tmem_wait_ld();
+        }
+        store_row<D>(dK, grad_fp32 != 0, off + c, o, sm_scale);
+      }
+    } else {
+      bar.abort = 1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace bwd
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+struct BwdWs {
+  WsHeader *hdr;
+  uint16_t *Qp, *Kp, *Vp, *dOp;
+  float *lse2p, *deltap;
+  int32_t *unit_block, *tu_q, *tu_k;
+};
+static BwdWs carve_bwd(const prism_params &p, void *ws) {
+  const size_t N = (size_t)p.T * p.H * p.W, h = p.heads, D = p.head_dim;
+  const size_t tens = align_up(sizeof(uint16_t) * h * N * D, 256);
+  char *w = static_cast<char *>(ws);
+  BwdWs b;
+  b.hdr = reinterpret_cast<WsHeader *>(w);
+  w += kWsHeader;
+  b.Qp = reinterpret_cast<uint16_t *>(w);
+  w += tens;
+  b.Kp = reinterpret_cast<uint16_t *>(w);
+  w += tens;
+  b.Vp = reinterpret_cast<uint16_t *>(w);
+  w += tens;
+  b.dOp = reinterpret_cast<uint16_t *>(w);
+  w += tens;
+  b.lse2p = reinterpret_cast<float *>(w);
+  w += align_up(sizeof(float) * h * N, 256);
+  b.deltap = reinterpret_cast<float *>(w);
+  w += align_up(sizeof(float) * h * N, 256);
+  b.unit_block = reinterpret_cast<int32_t *>(w);
+  w += align_up(sizeof(int32_t) * h * (N / 64), 256);
+  b.tu_q = reinterpret_cast<int32_t *>(w);
+  w += align_up(sizeof(int32_t) * h * (N / 128), 256);
+  b.tu_k = reinterpret_cast<int32_t *>(w);
+  return b;
+}
+
+size_t attn_bwd_ws_bytes(const prism_params &p) {
+  const size_t N = (size_t)p.T * p.H * p.W, h = p.heads, D = p.head_dim;
+  return kWsHeader + 4 * align_up(sizeof(uint16_t) * h * N * D, 256) + 2 * align_up(sizeof(float) * h * N, 256) +
+         align_up(sizeof(int32_t) * h * (N / 64), 256) + 2 * align_up(sizeof(int32_t) * h * (N / 128), 256);
+}
+
+template <int D>
+static cudaError_t run_bwd(const prism_params &p, const prism_plan_t &plan, const prism_select_t &sel,
+                           const BwdWs &w, void *dQ, void *dK, void *dV, int grad_fp32, cudaStream_t st) {
+  const int N = p.T * p.H * p.W;
+  const long long rows = (long long)p.heads * N;
+  CUtensorMap mQ128, mDO128, mK64, mV64, mQ64, mDO64, mK128, mV128;
+  cudaError_t e;
+  if ((e = make_rows_map(&mQ128, w.Qp, rows, D, 128)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&mDO128, w.dOp, rows, D, 128)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&mK64, w.Kp, rows, D, 64)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&mV64, w.Vp, rows, D, 64)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&mQ64, w.Qp, rows, D, 64)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&mDO64, w.dOp, rows, D, 64)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&mK128, w.Kp, rows, D, 128)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&mV128, w.Vp, rows, D, 128)) != cudaSuccess) return e;
+  const float scale = effective_scale(p);
+  const float scale_log2 = scale * bwd::kLog2e;
+  dim3 grid(N / 128, p.heads);
+  const int s1 = bwd::KvSmem<D>::BYTES + 1024;
+  cudaFuncSetAttribute(bwd::dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, s1);
+  bwd::dkdv_kernel<D><<<grid, bwd::kThreads, s1, st>>>(mQ64, mDO64, mK128, mV128, sel.col_ptr, sel.row, plan.blocks,
+                                                       w.unit_block, w.tu_k, plan.perm, w.lse2p, w.deltap, dK, dV,
+                                                       grad_fp32, N, p.heads, scale_log2, scale, &w.hdr->status);
+  const int s2 = bwd::DqSmem<D>::BYTES + 1024;
+  cudaFuncSetAttribute(bwd::dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, s2);
+  bwd::dq_kernel<D><<<grid, bwd::kThreads, s2, st>>>(mQ128, mDO128, mK64, mV64, sel.row_ptr, sel.col, plan.blocks,
+                                                     w.unit_block, w.tu_q, plan.perm, w.lse2p, w.deltap, dQ,
+                                                     grad_fp32, N, p.heads, scale_log2, scale, &w.hdr->status);
+  count_launches(2);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_bwd(const prism_params &p, const prism_plan_t &plan, const prism_select_t &sel,
+                            const uint16_t *Q, const uint16_t *K, const uint16_t *V, const uint16_t *O,
+                            const uint16_t *dO, const float *lse, void *dQ, void *dK, void *dV, int grad_fp32,
+                            void *ws, cudaStream_t st) {
+  const int N = p.T * p.H * p.W, NB = N / 64, D = p.head_dim;
+  BwdWs w = carve_bwd(p, ws);
+  cudaError_t e;
+  if ((e = launch_permute3(plan.perm, N, p.heads, D, Q, K, V, w.Qp, w.Kp, w.Vp, st)) != cudaSuccess) return e;
+  const size_t total = (size_t)p.heads * N * (D / 8);
+  if (D == 128)
+    bwd::bwd_prep_kernel<128><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(plan.perm, N, p.heads, dO, O, lse,
+                                                                              w.dOp, w.lse2p, w.deltap);
+  else
+    bwd::bwd_prep_kernel<64><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(plan.perm, N, p.heads, dO, O, lse,
+                                                                             w.dOp, w.lse2p, w.deltap);
+  count_launches(1);
+  if ((e = launch_unit_block(plan.blocks, plan.n_blocks, NB, p.heads, w.unit_block, st)) != cudaSuccess) return e;
+  if ((e = launch_tile_units(sel.row_ptr, sel.col, plan.blocks, w.unit_block, N, p.heads, w.tu_q, st)) != cudaSuccess)
+    return e;
+  if ((e = launch_tile_units(sel.col_ptr, sel.row, plan.blocks, w.unit_block, N, p.heads, w.tu_k, st)) != cudaSuccess)
+    return e;
+  return D == 128 ? run_bwd<128>(p, plan, sel, w, dQ, dK, dV, grad_fp32, st)
+                  : run_bwd<64>(p, plan, sel, w, dQ, dK, dV, grad_fp32, st);
+}
+
+}  // namespace prism

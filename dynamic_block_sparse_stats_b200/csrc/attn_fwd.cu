@@ -1,0 +1,548 @@
+// prism_attn_fwd: exact attention of each query over the tokens of its
+// selected key blocks, on tcgen05 tensor cores with TMEM accumulators.
+//
+// Method: Prism digest ("Prism：为原生 2K 视频音频联合生成设计的动态稀疏注意力"),
+// section on hybrid block selection (exact attention with the full query
+// tokens and the selected key/value blocks, online softmax, no full attention
+// matrix; the output goes back to the original order) and the training
+// section (the kernel walks blocks of any volume in 64-token units).
+//
+// Work unit: one CTA per 128-query tile of one head, in permuted order.  A
+// tile is two 64-token units; both belong to one block (B >= 128), or to two
+// 64-token blocks of the same zone, in which case the tile walks the union of
+// their selections and masks each key unit per row half.  Keys are streamed
+// as tiles of two 64-token units (any two units of the walk).
+//
+// Roles (192 threads):
+//   warp 0      TMA producer: Q once, then K and V units into a 2-stage ring.
+//   warp 1      allocates TMEM; lane 0 issues tcgen05.mma:
+//                 S[b] = Q K^T  (SS, fp32 in TMEM, double buffered)
+//                 O   += P V    (TS: P is read from TMEM where S[b] was)
+//   warps 2-5   softmax, one thread per query row: reads S[b], online max
+//               with lazy rescaling of O (only when the max grows by more
+//               than 2^8), writes P as bf16 into TMEM, and finally
+//               normalises O and scatters it to natural token order.
+#include "attn_walk.cuh"
+
+namespace prism {
+
+namespace fwd {
+using namespace attn;
+
+constexpr int BM = 128;          // query rows per CTA
+constexpr int NSTAGE = 2;        // K/V ring depth
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (factor 256)
+
+template <int D>
+struct Smem {
+  static constexpr int CHUNKS = D / 64;                     // 128-byte swizzle chunks per row
+  static constexpr int Q_BYTES = BM * D * 2;                // 128 rows
+  static constexpr int KV_BYTES = 128 * D * 2;              // one key tile (two units)
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NSTAGE * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NSTAGE * KV_BYTES;
+  static constexpr int BYTES = OFF_BAR + 256;
+};
+
+struct Bars {
+  uint64_t q_full;
+  uint64_t k_full[NSTAGE];
+  uint64_t v_full[NSTAGE];
+  uint64_t kv_empty[NSTAGE];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t pv_done[2];
+  int meta[NSTAGE];  // nunits | mask0 << 4 | mask1 << 8
+  uint32_t tmem_base;
+  int ntiles;
+  int nunits;
+  int abort;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+                    const __grid_constant__ CUtensorMap mapV, const int32_t *__restrict__ row_ptr,
+                    const int32_t *__restrict__ col, const int32_t *__restrict__ blocks,
+                    const int32_t *__restrict__ unit_block, const int32_t *__restrict__ tile_units,
+                    const int32_t *__restrict__ perm, uint16_t *__restrict__ O, float *__restrict__ lse, int N,
+                    int heads, float scale_log2, int *status) {
+  using L = Smem<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars &bar = *reinterpret_cast<Bars *>(smem + L::OFF_BAR);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, h = blockIdx.y;
+  const int NB = N / 64;
+  const int32_t *blocks_h = blocks + (size_t)h * NB * 4;
+
+  // a CTA that starts after another one gave up does no work
+  if (threadIdx.x == 0) bar.abort = *reinterpret_cast<volatile int *>(status);
+  __syncthreads();
+  if (bar.abort) return;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar.q_full, 1);
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(&bar.k_full[s], 1);
+      mbar_init(&bar.v_full[s], 1);
+      mbar_init(&bar.kv_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bar.s_full[b], 1);
+      mbar_init(&bar.p_full[b], 128);
+      mbar_init(&bar.pv_done[b], 1);
+    }
+    bar.nunits = tile_units[(size_t)h * (N / BM) + tile];
+    bar.ntiles = (bar.nunits + 1) >> 1;
+    bar.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bar.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar.tmem_base;
+  const int ntiles = bar.ntiles;
+  const int nunits = bar.nunits;
+  const uint32_t tS[2] = {tmem, tmem + 128};
+  const uint32_t tO = tmem + 256;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    const int u0 = 2 * tile, u1 = 2 * tile + 1;
+    const int b0 = unit_block[(size_t)h * NB + u0], b1 = unit_block[(size_t)h * NB + u1];
+    UnitWalk w;
+    const int r0 = h * NB + b0, r1 = h * NB + b1;
+    cursor_init(w.a, row_ptr[r0], row_ptr[r0 + 1]);
+    if (b1 != b0) {
+      cursor_init(w.b, row_ptr[r1], row_ptr[r1 + 1]);
+      w.mask_a = 1;
+      w.mask_b = 2;
+    } else {
+      cursor_init(w.b, 0, 0);
+      w.mask_a = 3;
+      w.mask_b = 0;
+    }
+    w.cur_cnt = 0;
+    w.cur_k = 0;
+    w.cur_ub = 0;
+    w.cur_mask = 0;
+    if (lane == 0) {
+      prefetch_tensormap(&mapQ);
+      prefetch_tensormap(&mapK);
+      prefetch_tensormap(&mapV);
+      mbar_arrive_expect_tx(&bar.q_full, L::Q_BYTES);
+#pragma unroll
+      for (int c = 0; c < L::CHUNKS; ++c)
+        tma_load_2d(smem + L::OFF_Q + c * (BM * 128), &mapQ, &bar.q_full, c * 64, h * N + tile * BM);
+    }
+    for (int j = 0; j < ntiles; ++j) {
+      const int s = j % NSTAGE;
+      uint32_t ua, ub = 0;
+      int ma, mb = 0, nu = 1;
+      walk_next(w, col, blocks_h, ua, ma);
+      if (2 * j + 2 <= nunits) {
+        walk_next(w, col, blocks_h, ub, mb);
+        nu = 2;
+      }
+      ua = min(ua, (uint32_t)(NB - 1));  // a well-formed walk never clamps
+      ub = min(ub, (uint32_t)(NB - 1));
+      if (lane == 0) {
+        bool ok = true;
+        if (j >= NSTAGE) ok = mbar_wait(&bar.kv_empty[s], ((j / NSTAGE) - 1) & 1, status, 1);
+        if (!ok) bar.abort = 1;
+        if (ok) {
+          bar.meta[s] = nu | (ma << 4) | (mb << 8);
+          uint8_t *ks = smem + L::OFF_K + s * L::KV_BYTES;
+          uint8_t *vs = smem + L::OFF_V + s * L::KV_BYTES;
+          const int bytes = nu * 64 * D * 2;
+          mbar_arrive_expect_tx(&bar.k_full[s], bytes);
+#pragma unroll
+          for (int c = 0; c < L::CHUNKS; ++c) {
+            tma_load_2d(ks + c * (128 * 128), &mapK, &bar.k_full[s], c * 64, h * N + (int)ua * 64);
+            if (nu == 2) tma_load_2d(ks + c * (128 * 128) + 64 * 128, &mapK, &bar.k_full[s], c * 64, h * N + (int)ub * 64);
+          }
+          mbar_arrive_expect_tx(&bar.v_full[s], bytes);
+#pragma unroll
+          for (int c = 0; c < L::CHUNKS; ++c) {
+            tma_load_2d(vs + c * (128 * 128), &mapV, &bar.v_full[s], c * 64, h * N + (int)ua * 64);
+            if (nu == 2) tma_load_2d(vs + c * (128 * 128) + 64 * 128, &mapV, &bar.v_full[s], c * 64, h * N + (int)ub * 64);
+          }
+        }
+      }
+      __syncwarp();
+      if (*reinterpret_cast<volatile int *>(&bar.abort)) break;
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s_full = idesc_bf16(128, 128, 0);
+      const uint32_t idesc_s_half = idesc_bf16(128, 64, 0);
+      const uint32_t idesc_o = idesc_bf16(128, D, 1);
+      const uint32_t sQ = smem_u32(smem + L::OFF_Q);
+      bool ok = mbar_wait(&bar.q_full, 0, status, 2);
+      tc_fence_after();
+      for (int j = 0; ok && j <= ntiles; ++j) {
+        if (j < ntiles) {
+          const int s = j % NSTAGE, b = j & 1;
+          ok = mbar_wait(&bar.k_full[s], (j / NSTAGE) & 1, status, 3);
+          if (ok && j >= 2) ok = mbar_wait(&bar.pv_done[b], ((j - 2) >> 1) & 1, status, 4);
+          if (!ok) break;
+          tc_fence_after();
+          const int nu = bar.meta[s] & 15;
+          const uint32_t sK = smem_u32(smem + L::OFF_K + s * L::KV_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+            const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sK + off, 16, 1024);
+            mma_ss(tS[b], ad, bd, nu == 2 ? idesc_s_full : idesc_s_half, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&bar.s_full[b]);
+        }
+        if (j >= 1) {
+          const int jj = j - 1, s = jj % NSTAGE, b = jj & 1;
+          ok = mbar_wait(&bar.p_full[b], (jj >> 1) & 1, status, 5);
+          if (ok) ok = mbar_wait(&bar.v_full[s], (jj / NSTAGE) & 1, status, 6);
+          if (!ok) break;
+          tc_fence_after();
+          const int nu = bar.meta[s] & 15;
+          const uint32_t sV = smem_u32(smem + L::OFF_V + s * L::KV_BYTES);
+          for (int ks = 0; ks < nu * 4; ++ks) {
+            const uint64_t bd = sdesc_sw128(sV + ks * 2048, 128 * 128, 1024);
+            mma_ts(tO, tS[b] + ks * 8, bd, idesc_o, (jj > 0 || ks > 0) ? 1u : 0u);
+          }
+          mma_commit(&bar.pv_done[b]);
+          mma_commit(&bar.kv_empty[s]);
+        }
+      }
+      if (!ok) bar.abort = 1;
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    const int half = row >> 6;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      const int s = j % NSTAGE, b = j & 1;
+      ok = mbar_wait(&bar.s_full[b], (j >> 1) & 1, status, 7);
+      if (!ok) break;
+      tc_fence_after();
+      const int meta = bar.meta[s];
+      const int nu = meta & 15;
+      const bool ok0 = ((meta >> 4) >> half) & 1;
+      const bool ok1 = nu == 2 && (((meta >> 8) >> half) & 1);
+      uint32_t r[4][32];
+      tmem_ld32(tS[b] + lane_off + 0, r[0]);
+      tmem_ld32(tS[b] + lane_off + 32, r[1]);
+      if (nu == 2) {
+        tmem_ld32(tS[b] + lane_off + 64, r[2]);
+        tmem_ld32(tS[b] + lane_off + 96, r[3]);
+      }
+      tmem_wait_ld();
+      float mt = -INFINITY;
+      if (ok0) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mt = fmaxf(mt, __uint_as_float(r[q][i]));
+      }
+      if (ok1) {
+#pragma unroll
+        for (int q = 2; q < 4; ++q)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mt = fmaxf(mt, __uint_as_float(r[q][i]));
+      }
+      mt *= scale_log2;
+      if (mt > m + kRescaleLog2 || (m == -INFINITY && mt > -INFINITY)) {
+        // new reference maximum: rescale the running sum and, once O holds
+        // earlier tiles, the accumulator rows of this thread
+        const float alpha = (m == -INFINITY) ? 0.f : exp2f(m - mt);
+        if (j > 0 && m != -INFINITY) {
+          ok = mbar_wait(&bar.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, status, 8);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < D; c += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + lane_off + c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tO + lane_off + c, o);
+          }
+          tmem_wait_st();
+        }
+        l *= alpha;
+        m = mt;
+      }
+      // P = exp2(s * scale_log2 - m), bf16, packed two keys per column
+      uint32_t pk[64];
+      float ls = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const bool valid = (q < 2) ? ok0 : ok1;
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float p0 = 0.f, p1 = 0.f;
+          if (valid) {
+            p0 = exp2f(fmaf(__uint_as_float(r[q][i]), scale_log2, -m));
+            p1 = exp2f(fmaf(__uint_as_float(r[q][i + 1]), scale_log2, -m));
+          }
+          ls += p0 + p1;
+          pk[q * 16 + i / 2] = pack_bf16(p0, p1);
+        }
+      }
+      l += ls;
+      tmem_st32(tS[b] + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      if (nu == 2) tmem_st32(tS[b] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar.p_full[b]);
+    }
+    // epilogue
+    if (ok && ntiles > 0) ok = mbar_wait(&bar.pv_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, status, 9);
+    if (ok) {
+      tc_fence_after();
+      const int p = tile * BM + row;
+      const int n = perm[(size_t)h * N + p];
+      const float inv = (l > 0.f) ? 1.0f / l : 0.f;
+      uint16_t *dst = O + ((size_t)n * heads + h) * D;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t o[32];
+        if (ntiles > 0) {
+          tmem_ld32(tO + lane_off + c, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
+        uint4 v[4];
+        uint32_t *pv = reinterpret_cast<uint32_t *>(v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pv[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) reinterpret_cast<uint4 *>(dst + c)[i] = v[i];
+      }
+      // natural-log LSE: ln 2 * (m + log2 l)
+      lse[(size_t)h * N + n] = (l > 0.f) ? 0.69314718055994531f * (m + log2f(l)) : -INFINITY;
+    } else {
+      bar.abort = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// pre-passes
+// ---------------------------------------------------------------------------
+// unit_block[h][u] = block of 64-token unit u.
+__global__ void unit_block_kernel(const int32_t *__restrict__ blocks, const int32_t *__restrict__ n_blocks, int NB,
+                                  int32_t *__restrict__ unit_block) {
+  const int h = blockIdx.y;
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= n_blocks[h]) return;
+  const int32_t *e = blocks + ((size_t)h * NB + b) * 4;
+  const int u0 = e[0] >> 6, nu = e[1] >> 6;
+  for (int k = 0; k < nu; ++k) unit_block[(size_t)h * NB + u0 + k] = b;
+}
+
+// tile_units[h][t] = key units walked by query tile t (union of the two row
+// lists when the tile holds two 64-token blocks).  One warp per tile.
+__global__ void tile_units_kernel(const int32_t *__restrict__ row_ptr, const int32_t *__restrict__ col,
+                                  const int32_t *__restrict__ blocks, const int32_t *__restrict__ unit_block, int N,
+                                  int heads, int32_t *__restrict__ tile_units) {
+  const int NB = N / 64, NT = N / BM;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (gw >= NT * heads) return;
+  const int h = gw / NT, t = gw % NT;
+  const int32_t *blocks_h = blocks + (size_t)h * NB * 4;
+  const int b0 = unit_block[(size_t)h * NB + 2 * t], b1 = unit_block[(size_t)h * NB + 2 * t + 1];
+  const int s0 = row_ptr[h * NB + b0], e0 = row_ptr[h * NB + b0 + 1];
+  long long cnt = 0;
+  for (int q = s0 + lane; q < e0; q += 32) cnt += blocks_h[(size_t)col[q] * 4 + 1] >> 6;
+  if (b1 != b0) {
+    const int s1 = row_ptr[h * NB + b1], e1 = row_ptr[h * NB + b1 + 1];
+    for (int q = s1 + lane; q < e1; q += 32) {
+      const int j = col[q];
+      int lo = s0, hi = e0;  // binary search j in the first list
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (col[mid] < j)
+          lo = mid + 1;
+        else
+          hi = mid;
+      }
+      if (!(lo < e0 && col[lo] == j)) cnt += blocks_h[(size_t)j * 4 + 1] >> 6;
+    }
+  }
+  cnt = warp_sum(cnt);
+  if (lane == 0) tile_units[(size_t)h * NT + t] = (int32_t)cnt;
+}
+
+// dst[h][p][:] = src[perm[h][p]][h][:]
+__global__ void permute3_kernel(const int32_t *__restrict__ perm, int N, int heads, int D,
+                                const uint16_t *__restrict__ s0, const uint16_t *__restrict__ s1,
+                                const uint16_t *__restrict__ s2, uint16_t *__restrict__ d0, uint16_t *__restrict__ d1,
+                                uint16_t *__restrict__ d2) {
+  const int vpr = D / 8;  // 16-byte vectors per row
+  const size_t g = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t rows = (size_t)heads * N;
+  if (g >= rows * vpr) return;
+  const size_t r = g / vpr;
+  const int v = (int)(g % vpr);
+  const int h = (int)(r / N);
+  const int n = perm[r];
+  const size_t src = ((size_t)n * heads + h) * D + v * 8, dst = r * D + v * 8;
+  *reinterpret_cast<uint4 *>(d0 + dst) = __ldg(reinterpret_cast<const uint4 *>(s0 + src));
+  if (s1) *reinterpret_cast<uint4 *>(d1 + dst) = __ldg(reinterpret_cast<const uint4 *>(s1 + src));
+  if (s2) *reinterpret_cast<uint4 *>(d2 + dst) = __ldg(reinterpret_cast<const uint4 *>(s2 + src));
+}
+
+}  // namespace fwd
+
+cudaError_t launch_permute3(const int32_t *perm, int N, int heads, int D, const uint16_t *s0, const uint16_t *s1,
+                            const uint16_t *s2, uint16_t *d0, uint16_t *d1, uint16_t *d2, cudaStream_t st) {
+  const size_t total = (size_t)heads * N * (D / 8);
+  fwd::permute3_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(perm, N, heads, D, s0, s1, s2, d0, d1, d2);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unit_block(const int32_t *blocks, const int32_t *n_blocks, int NB, int heads,
+                              int32_t *unit_block, cudaStream_t st) {
+  fwd::unit_block_kernel<<<dim3((NB + 255) / 256, heads), 256, 0, st>>>(blocks, n_blocks, NB, unit_block);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tile_units(const int32_t *ptr, const int32_t *idx, const int32_t *blocks,
+                              const int32_t *unit_block, int N, int heads, int32_t *tile_units, cudaStream_t st) {
+  const int warps = (N / 128) * heads;
+  fwd::tile_units_kernel<<<(warps * 32 + 255) / 256, 256, 0, st>>>(ptr, idx, blocks, unit_block, N, heads,
+                                                                   tile_units);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// tensor maps
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 map over rows of D elements: box = 64 elements x box_rows, 128B swizzle.
+cudaError_t make_rows_map(CUtensorMap *map, const void *base, long long rows, int D, int box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+struct FwdWs {
+  WsHeader *hdr;
+  uint16_t *Qp, *Kp, *Vp;
+  int32_t *unit_block, *tile_units;
+};
+static FwdWs carve_fwd(const prism_params &p, void *ws) {
+  const size_t N = (size_t)p.T * p.H * p.W, h = p.heads, D = p.head_dim;
+  const size_t tens = align_up(sizeof(uint16_t) * h * N * D, 256);
+  char *w = static_cast<char *>(ws);
+  FwdWs f;
+  f.hdr = reinterpret_cast<WsHeader *>(w);
+  w += kWsHeader;
+  f.Qp = reinterpret_cast<uint16_t *>(w);
+  w += tens;
+  f.Kp = reinterpret_cast<uint16_t *>(w);
+  w += tens;
+  f.Vp = reinterpret_cast<uint16_t *>(w);
+  w += tens;
+  f.unit_block = reinterpret_cast<int32_t *>(w);
+  w += align_up(sizeof(int32_t) * h * (N / 64), 256);
+  f.tile_units = reinterpret_cast<int32_t *>(w);
+  return f;
+}
+
+size_t attn_fwd_ws_bytes(const prism_params &p) {
+  const size_t N = (size_t)p.T * p.H * p.W, h = p.heads, D = p.head_dim;
+  return kWsHeader + 3 * align_up(sizeof(uint16_t) * h * N * D, 256) + align_up(sizeof(int32_t) * h * (N / 64), 256) +
+         align_up(sizeof(int32_t) * h * (N / 128), 256);
+}
+
+template <int D>
+static cudaError_t run_fwd(const prism_params &p, const prism_plan_t &plan, const prism_select_t &sel,
+                           const FwdWs &w, uint16_t *O, float *lse, cudaStream_t st) {
+  const int N = p.T * p.H * p.W;
+  CUtensorMap mQ, mK, mV;
+  cudaError_t e;
+  if ((e = make_rows_map(&mQ, w.Qp, (long long)p.heads * N, D, 128)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&mK, w.Kp, (long long)p.heads * N, D, 64)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&mV, w.Vp, (long long)p.heads * N, D, 64)) != cudaSuccess) return e;
+  const int smem = fwd::Smem<D>::BYTES + 1024;
+  cudaFuncSetAttribute(fwd::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const float scale_log2 = effective_scale(p) * 1.4426950408889634f;
+  dim3 grid(N / fwd::BM, p.heads);
+  fwd::attn_fwd_kernel<D><<<grid, fwd::kThreads, smem, st>>>(mQ, mK, mV, sel.row_ptr, sel.col, plan.blocks,
+                                                             w.unit_block, w.tile_units, plan.perm, O, lse, N,
+                                                             p.heads, scale_log2, &w.hdr->status);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_fwd(const prism_params &p, const prism_plan_t &plan, const prism_select_t &sel,
+                            const uint16_t *Q, const uint16_t *K, const uint16_t *V, uint16_t *O, float *lse,
+                            void *ws, cudaStream_t st) {
+  const int N = p.T * p.H * p.W, NB = N / 64, D = p.head_dim;
+  FwdWs w = carve_fwd(p, ws);
+  cudaError_t e;
+  if ((e = launch_permute3(plan.perm, N, p.heads, D, Q, K, V, w.Qp, w.Kp, w.Vp, st)) != cudaSuccess) return e;
+  if ((e = launch_unit_block(plan.blocks, plan.n_blocks, NB, p.heads, w.unit_block, st)) != cudaSuccess) return e;
+  if ((e = launch_tile_units(sel.row_ptr, sel.col, plan.blocks, w.unit_block, N, p.heads, w.tile_units, st)) !=
+      cudaSuccess)
+    return e;
+  return D == 128 ? run_fwd<128>(p, plan, sel, w, O, lse, st) : run_fwd<64>(p, plan, sel, w, O, lse, st);
+}
+
+}  // namespace prism

@@ -1,0 +1,56 @@
+// Internal declarations shared by the translation units of libprism.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace prism {
+
+// plan.cu
+size_t plan_ws_bytes(const prism_params &p);
+cudaError_t launch_plan(const prism_params &p, const uint16_t *V, const float *a, const prism_plan_t &out, void *ws,
+                        cudaStream_t st);
+
+// select.cu
+size_t select_ws_bytes(const prism_params &p);
+size_t select_max_nb(const prism_params &p);
+cudaError_t launch_select(const prism_params &p, const prism_plan_t &plan, const uint16_t *Q, const uint16_t *K,
+                          prism_select_t &out, void *ws, cudaStream_t st, long long *nnz_out);
+
+// attn_fwd.cu
+size_t attn_fwd_ws_bytes(const prism_params &p);
+cudaError_t launch_attn_fwd(const prism_params &p, const prism_plan_t &plan, const prism_select_t &sel,
+                            const uint16_t *Q, const uint16_t *K, const uint16_t *V, uint16_t *O, float *lse,
+                            void *ws, cudaStream_t st);
+
+// attn_bwd.cu
+size_t attn_bwd_ws_bytes(const prism_params &p);
+cudaError_t launch_attn_bwd(const prism_params &p, const prism_plan_t &plan, const prism_select_t &sel,
+                            const uint16_t *Q, const uint16_t *K, const uint16_t *V, const uint16_t *O,
+                            const uint16_t *dO, const float *lse, void *dQ, void *dK, void *dV, int grad_fp32,
+                            void *ws, cudaStream_t st);
+
+// shared launch helper: token gather into permuted head-major order
+// dst[h][p][:] = src[perm[h][p]][h][:] for up to three tensors at once.
+cudaError_t launch_permute3(const int32_t *perm, int N, int heads, int D, const uint16_t *s0, const uint16_t *s1,
+                            const uint16_t *s2, uint16_t *d0, uint16_t *d1, uint16_t *d2, cudaStream_t st);
+
+float effective_scale(const prism_params &p);
+
+// attention pre-passes (attn_fwd.cu), shared by the backward
+cudaError_t launch_unit_block(const int32_t *blocks, const int32_t *n_blocks, int NB, int heads,
+                              int32_t *unit_block, cudaStream_t st);
+// tile_units[h][t]: 64-token units walked by 128-token tile t over the rows
+// (ptr, idx) of its one or two blocks (CSR for query tiles, CSC for key tiles).
+cudaError_t launch_tile_units(const int32_t *ptr, const int32_t *idx, const int32_t *blocks,
+                              const int32_t *unit_block, int N, int heads, int32_t *tile_units, cudaStream_t st);
+// 2-D bf16 tensor map over rows of D elements, box 64 x box_rows, 128B swizzle.
+cudaError_t make_rows_map(CUtensorMap *map, const void *base, long long rows, int D, int box_rows);
+
+// host-side count of kernel launches (prism_kernel_launches)
+void count_launches(int n);
+
+}  // namespace prism

@@ -1,0 +1,246 @@
+/*
+ * prism.h -- C ABI of the Prism dynamic block-sparse video self-attention
+ * path for NVIDIA B200 (sm_100a).
+ *
+ * The path, per attention layer and head (Prism digest, "Prism：为原生 2K
+ * 视频音频联合生成设计的动态稀疏注意力", overview and Fig. 2 description):
+ *   prism_plan      8x8x8 macro-zones -> variation indicator g_d(m) and
+ *                   density rho(m) -> block volume B(m) in {64,128,256}
+ *                   -> block shape (nearest log2 candidate to l*) ->
+ *                   block-contiguous permutation.
+ *   prism_select    block means of Q and K -> block scores -> hybrid
+ *                   Top-k U Top-p key-block sets (CSR, and its transpose).
+ *   prism_attn_fwd  exact attention of every query over the tokens of its
+ *                   selected key blocks; output in natural token order.
+ *   prism_attn_bwd  gradients through the same selected blocks only.
+ *
+ * Conventions shared by every call
+ *   Layout.  Batch 1.  Natural raster token order n = (t*H + y)*W + x over
+ *     a T x H x W latent grid, N = T*H*W.  Q, K, V, O, dO, dQ, dK, dV are
+ *     bf16 (passed as uint16_t bit patterns) laid out [N][heads][head_dim],
+ *     contiguous.  The A2V norm map a2v_norm is fp32 [N].
+ *   Sizes.  Z = (T/8)(H/8)(W/8) zones; NB = N/64 is the most blocks a head
+ *     can have (every zone at B = 64).
+ *   Memory.  Every pointer argument is DEVICE memory unless stated
+ *     otherwise.  The caller allocates and owns every buffer, including the
+ *     workspaces sized by the *_workspace_size() queries; the library never
+ *     allocates device memory.  Workspaces must be 256-byte aligned and may
+ *     not be shared by calls that run concurrently.
+ *   Execution.  Calls enqueue kernels on `stream` and return without waiting,
+ *     except prism_select, which waits once on `stream` to read the number
+ *     of selected entries (nnz).
+ *   Errors.  Every call returns a prism_status.  Nothing is thrown across the
+ *     ABI.  prism_last_error() returns a message for the calling thread's
+ *     last failing call.  Kernels that time out on an internal wait record
+ *     PRISM_ERR_TIMEOUT in the workspace; prism_workspace_status() reads it.
+ */
+#ifndef PRISM_H
+#define PRISM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *prism_stream_t; /* the same type as cudaStream_t */
+
+typedef enum prism_status {
+  PRISM_OK = 0,
+  PRISM_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad param   */
+  PRISM_ERR_UNSUPPORTED = 2,  /* T/H/W not multiples of 8, head_dim not 64/128 */
+  PRISM_ERR_CAPACITY = 3,     /* an output or workspace is too small          */
+  PRISM_ERR_CUDA = 4,         /* a CUDA runtime call failed                   */
+  PRISM_ERR_TIMEOUT = 5       /* a kernel gave up on an internal wait         */
+} prism_status;
+
+/*
+ * Parameters of one layer.
+ *   T, H, W        latent grid; each a positive multiple of 8 (macro-zone
+ *                  edge Z_T = Z_H = Z_W = 8, Prism digest, Fig. 2 text).
+ *   heads          number of attention heads (>= 1).
+ *   head_dim       D, 64 or 128.
+ *   tau128, tau256 density thresholds (0.5 and 0.25 on the pages, digest
+ *                  section on information density).  rho >= tau128 gives
+ *                  B = 64, tau256 <= rho < tau128 gives 128, else 256.
+ *   eps            the small constant of g_d(m) (1e-6 here; "a tiny
+ *                  constant" on the pages).
+ *   topk_frac      Top-k as a kept fraction of key blocks, rounded up
+ *                  (ignored when topk_abs > 0).
+ *   topk_abs       Top-k as an absolute block count when > 0.
+ *   top_p          Top-p threshold (0.2 on the pages' default, 0.9 in the
+ *                  benchmark grids).
+ *   sm_scale       attention scale; 0 selects 1/sqrt(head_dim).  The same
+ *                  scale multiplies the block scores.
+ */
+typedef struct prism_params {
+  int32_t T, H, W;
+  int32_t heads, head_dim;
+  float tau128, tau256, eps;
+  float topk_frac;
+  int32_t topk_abs;
+  float top_p;
+  float sm_scale;
+} prism_params;
+
+/*
+ * Output of prism_plan.  All arrays are device memory owned by the caller.
+ *   zone_shape [heads][Z]     candidate id 0..15 of each zone (id order:
+ *                             volume ascending, then (b_T,b_H,b_W)
+ *                             lexicographic: 0 (2,4,8) ... 15 (8,8,4)).
+ *   zone_g     [heads][Z][3]  g_T, g_H, g_W (float64).  May be NULL.
+ *   zone_rho   [heads][Z]     normalised density rho(m) (float64). May be NULL.
+ *   n_blocks   [heads]        number of blocks of each head.
+ *   blocks     [heads][NB][4] per block: {p0, B, n0, shape id}: first
+ *                             permuted position, volume, natural index of
+ *                             the block's first (origin) token, candidate id.
+ *                             Entries at index >= n_blocks[h] are unspecified.
+ *   perm       [heads][N]     natural token index at permuted position p.
+ *   inv_perm   [heads][N]     permuted position of natural token n.  May be
+ *                             NULL.
+ * Permuted order: zones in raster order (zW fastest), zone m occupying
+ * positions [512m, 512m+512); blocks in raster order of the zone's block
+ * grid; tokens in raster (t,y,x) order inside a block.
+ */
+typedef struct prism_plan_t {
+  uint8_t *zone_shape;
+  double *zone_g;
+  double *zone_rho;
+  int32_t *n_blocks;
+  int32_t *blocks;
+  int32_t *perm;
+  int32_t *inv_perm;
+} prism_plan_t;
+
+/* Bytes of workspace prism_plan needs (0 on invalid params). */
+size_t prism_plan_workspace_size(const prism_params *p);
+
+/*
+ * prism_plan -- zone statistics, variation indicator, density, volume,
+ * shape and permutation, per head.
+ *   Zone statistics: the channel variance of mean-pooled V along each axis
+ *   (r_{v,d}), the A2V-norm coupling abar(m) and direction shares
+ *   vhat_{a,d}(m), and rho_raw(m) = intra-zone spatial variance + temporal
+ *   frame-difference variance (digest, section on zone guidance and the
+ *   rho_raw equation; xyznot.com review "Prism: динамическое разреженное
+ *   внимание ...", Method sections 1-2).  g_d = r_{v,d} + abar*vhat_{a,d}
+ *   + eps; l*_d closed form; nearest candidate in log2 space.
+ *   V         bf16 [N][heads][head_dim].
+ *   a2v_norm  fp32 [N] norm of the previous layer's audio-to-video
+ *             attention output per video token, or NULL for the first
+ *             layer (video guidance only).
+ *   out       arrays to fill (see prism_plan_t).
+ *   workspace, ws_bytes  at least prism_plan_workspace_size(p) bytes.
+ * Returns PRISM_OK, PRISM_ERR_INVALID_ARG, PRISM_ERR_UNSUPPORTED,
+ * PRISM_ERR_CAPACITY (ws_bytes too small) or PRISM_ERR_CUDA.
+ */
+int prism_plan(const prism_params *p, const uint16_t *V, const float *a2v_norm,
+               const prism_plan_t *out, void *workspace, size_t ws_bytes,
+               prism_stream_t stream);
+
+/*
+ * Output of prism_select.  Rows are indexed r = h*NB + i (head h, query
+ * block i); rows i >= n_blocks[h] are empty.
+ *   row_ptr [heads*NB + 1]  CSR offsets into col.
+ *   col     [cap]           selected key-block ids, ascending in each row.
+ *   cap     capacity of col (and of row) in entries (host value, in).
+ *   nnz     entries written (host value, out).  When nnz > cap the call
+ *           returns PRISM_ERR_CAPACITY and nnz is the capacity needed.
+ *   col_ptr [heads*NB + 1]  CSC offsets (transpose), or NULL to skip it.
+ *   row     [cap]           query-block ids of each key block, ascending.
+ */
+typedef struct prism_select_t {
+  int32_t *row_ptr;
+  int32_t *col;
+  int64_t cap;
+  int64_t nnz;
+  int32_t *col_ptr;
+  int32_t *row;
+} prism_select_t;
+
+/* Bytes of workspace prism_select needs (0 on invalid params). */
+size_t prism_select_workspace_size(const prism_params *p);
+
+/*
+ * prism_select -- hybrid block selection (digest, section on hybrid block
+ * selection; review, Method section 3): per head, block means Qbar_i and
+ * Kbar_j over each block's tokens, scores s_ij = (Qbar_i . Kbar_j) * scale,
+ * P_i = softmax_j(s_i), S_i = Top-k(P_i, k) U Top-p(P_i, top_p).
+ * Precision: block means are fp32 running sums over the block's tokens in
+ * raster order times 1/B; scores are fp32 running sums over channels of
+ * separately rounded products, times the scale; the Top-p cumulative sum
+ * is accumulated in float64.  Order: score descending, then key id
+ * ascending; "passes p" is read as ">= p" with the crossing block kept.
+ *   plan   output of prism_plan for the same params.
+ *   Q, K   bf16 [N][heads][head_dim].
+ *   out    see prism_select_t; out->nnz is written.
+ * Waits once on `stream`.  Returns PRISM_OK, PRISM_ERR_INVALID_ARG,
+ * PRISM_ERR_UNSUPPORTED, PRISM_ERR_CAPACITY or PRISM_ERR_CUDA.
+ */
+int prism_select(const prism_params *p, const prism_plan_t *plan,
+                 const uint16_t *Q, const uint16_t *K, prism_select_t *out,
+                 void *workspace, size_t ws_bytes, prism_stream_t stream);
+
+/* Bytes of workspace prism_attn_fwd (backward = 0) or prism_attn_bwd
+ * (backward = 1) needs (0 on invalid params). */
+size_t prism_attn_workspace_size(const prism_params *p, int backward);
+
+/*
+ * prism_attn_fwd -- exact attention over the selected blocks (digest,
+ * section on hybrid selection: full query tokens against the keys and
+ * values of the selected key blocks, online softmax, no full attention
+ * matrix; 64-token units, training section).  For every query token q of
+ * block i:  O_q = sum_k softmax_k(q.k * scale) v_k  over the tokens k of
+ * the blocks in S_i;  lse_q = log sum_k exp(q.k * scale).
+ *   Q, K, V   bf16 [N][heads][head_dim].
+ *   O         bf16 [N][heads][head_dim], natural order (inverse permutation
+ *             applied).
+ *   lse       fp32 [heads][N], natural order (natural log).
+ * Runs on tcgen05 tensor cores (bf16 operands, fp32 accumulation).
+ * Returns PRISM_OK, PRISM_ERR_INVALID_ARG, PRISM_ERR_UNSUPPORTED,
+ * PRISM_ERR_CAPACITY or PRISM_ERR_CUDA.
+ */
+int prism_attn_fwd(const prism_params *p, const prism_plan_t *plan,
+                   const prism_select_t *sel, const uint16_t *Q,
+                   const uint16_t *K, const uint16_t *V, uint16_t *O,
+                   float *lse, void *workspace, size_t ws_bytes,
+                   prism_stream_t stream);
+
+/*
+ * prism_attn_bwd -- gradients of prism_attn_fwd through the selected blocks
+ * only; the plan and the selection are constants (digest, training section).
+ *   O, lse    outputs of prism_attn_fwd for the same inputs.
+ *   dO        bf16 [N][heads][head_dim] upstream gradient.
+ *   dQ,dK,dV  [N][heads][head_dim]; bf16 when grad_fp32 == 0, fp32 else.
+ * sel must carry the transpose (col_ptr/row non-NULL).
+ * Returns PRISM_OK, PRISM_ERR_INVALID_ARG, PRISM_ERR_UNSUPPORTED,
+ * PRISM_ERR_CAPACITY or PRISM_ERR_CUDA.
+ */
+int prism_attn_bwd(const prism_params *p, const prism_plan_t *plan,
+                   const prism_select_t *sel, const uint16_t *Q,
+                   const uint16_t *K, const uint16_t *V, const uint16_t *O,
+                   const uint16_t *dO, const float *lse, void *dQ, void *dK,
+                   void *dV, int grad_fp32, void *workspace, size_t ws_bytes,
+                   prism_stream_t stream);
+
+/* Waits on `stream` and returns the status a kernel recorded in
+ * `workspace` (PRISM_OK or PRISM_ERR_TIMEOUT), or PRISM_ERR_CUDA. */
+int prism_workspace_status(const void *workspace, prism_stream_t stream);
+
+/* Message of the calling thread's last failing call ("" if none).  The
+ * string is owned by the library and valid until the thread's next call. */
+const char *prism_last_error(void);
+
+/* Number of kernels this process has launched through the library so far
+ * (host-side counter, incremented at every launch; never reset). */
+uint64_t prism_kernel_launches(void);
+
+/* Library version, "major.minor.patch". */
+const char *prism_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PRISM_H */

@@ -1,0 +1,82 @@
+"""The C-ABI library loads, exports every function include/prism.h declares,
+and validates arguments on the host (no GPU needed: every check below
+returns before any CUDA call)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from dynamic_block_sparse_stats_b200 import _lib, api
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "prism.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(prism_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_what_the_binding_exports():
+    assert declared_functions() == sorted(_lib.EXPORTS)
+
+
+def test_library_loads_and_exports_every_symbol():
+    lib = _lib.load()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.prism_version().decode().count(".") == 2
+
+
+def test_struct_layouts_match_header():
+    assert C.sizeof(_lib.PrismParams) == 12 * 4
+    assert C.sizeof(_lib.PrismPlan) == 7 * 8
+    assert C.sizeof(_lib.PrismSelect) == 6 * 8
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(T=12), _lib.PRISM_ERR_UNSUPPORTED),
+    (dict(head_dim=96), _lib.PRISM_ERR_UNSUPPORTED),
+    (dict(heads=0), _lib.PRISM_ERR_INVALID_ARG),
+    (dict(top_p=-0.5), _lib.PRISM_ERR_INVALID_ARG),
+    (dict(tau128=0.1, tau256=0.2), _lib.PRISM_ERR_INVALID_ARG),
+])
+def test_invalid_params_are_rejected_before_any_cuda_call(bad, code):
+    lib = _lib.load()
+    kw = dict(T=8, H=16, W=16, heads=1, head_dim=64, topk_abs=2, top_p=0.9)
+    kw.update(bad)
+    p = api.params(**kw)
+    assert lib.prism_plan_workspace_size(C.byref(p)) == 0
+    plan = _lib.PrismPlan(8, 8, 8, 8, 8, 8, 8)  # non-null dummies, never dereferenced
+    rc = lib.prism_plan(C.byref(p), C.c_void_p(8), None, C.byref(plan), C.c_void_p(256), 1 << 20, None)
+    assert rc == code
+    assert lib.prism_last_error().decode()
+
+
+def test_null_pointers_and_short_workspace_are_rejected():
+    lib = _lib.load()
+    p = api.params(8, 16, 16, 1, 64, topk_abs=2)
+    plan = _lib.PrismPlan(8, 8, 8, 8, 8, 8, 8)
+    assert lib.prism_plan(C.byref(p), None, None, C.byref(plan), C.c_void_p(256), 1 << 20, None) == \
+        _lib.PRISM_ERR_INVALID_ARG
+    need = lib.prism_plan_workspace_size(C.byref(p))
+    assert need > 256
+    rc = lib.prism_plan(C.byref(p), C.c_void_p(8), None, C.byref(plan), C.c_void_p(256), need - 1, None)
+    assert rc == _lib.PRISM_ERR_CAPACITY and "need" in lib.prism_last_error().decode()
+    rc = lib.prism_plan(C.byref(p), C.c_void_p(8), None, C.byref(plan), C.c_void_p(264), need, None)
+    assert rc == _lib.PRISM_ERR_INVALID_ARG  # misaligned workspace
+    sel = _lib.PrismSelect(8, 8, 10, 0, 8, None)  # col_ptr without row
+    assert lib.prism_select(C.byref(p), C.byref(plan), C.c_void_p(8), C.c_void_p(8), C.byref(sel),
+                            C.c_void_p(256), 1 << 30, None) == _lib.PRISM_ERR_INVALID_ARG
+    assert lib.prism_attn_bwd(C.byref(p), C.byref(plan), C.byref(_lib.PrismSelect(8, 8, 10, 0, None, None)),
+                              *([C.c_void_p(8)] * 9), 0, C.c_void_p(256), 1 << 30, None) == _lib.PRISM_ERR_INVALID_ARG
+
+
+def test_workspace_sizes_grow_with_the_grid():
+    lib = _lib.load()
+    small = api.params(8, 16, 16, 1, 64)
+    big = api.params(56, 96, 160, 24, 128)
+    for f in (lib.prism_plan_workspace_size, lib.prism_select_workspace_size):
+        assert 0 < f(C.byref(small)) < f(C.byref(big))
+    assert lib.prism_attn_workspace_size(C.byref(big), 0) >= 3 * 860160 * 24 * 128 * 2

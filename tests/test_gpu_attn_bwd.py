@@ -1,0 +1,128 @@
+"""GPU parity of prism_attn_bwd (tcgen05 dQ and dK/dV kernels) against the
+float64 oracle on the library's plan and selection: dQ, dK, dV within
+max-abs 2e-2 and mean-abs 2e-3 (fp32 gradient outputs), and equality with
+PyTorch autograd of dense attention when every block is selected."""
+import numpy as np
+import pytest
+import torch
+
+from dynamic_block_sparse_stats_b200 import api
+from dynamic_block_sparse_stats_b200.synth import WORKLOADS, make_inputs
+from oracle import prism_oracle as O
+from tests.helpers import oracle_plan_from_shapes, scale_of, to_np
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS, MEAN_ABS = 2e-2, 2e-3
+
+
+def _lists(sel, NB, heads, nb):
+    row_ptr = to_np(sel.row_ptr).astype(np.int64)
+    col = to_np(sel.col)[:sel.nnz]
+    col_ptr = to_np(sel.col_ptr).astype(np.int64)
+    rows = to_np(sel.row)[:sel.nnz]
+    csr = [[col[row_ptr[h * NB + i]:row_ptr[h * NB + i + 1]] for i in range(nb[h])] for h in range(heads)]
+    csc = [[rows[col_ptr[h * NB + j]:col_ptr[h * NB + j + 1]] for j in range(nb[h])] for h in range(heads)]
+    return csr, csc
+
+
+def _run(name, grad_fp32=True, **over):
+    w = WORKLOADS[name]
+    inp = make_inputs(w, "cuda", with_grad=True)
+    p = api.params_for(w, **over)
+    pl = api.plan(p, inp["V"], inp["a"])
+    sel = api.select(p, pl, inp["Q"], inp["K"])
+    fw = api.attn_fwd(p, pl, sel, inp["Q"], inp["K"], inp["V"])
+    bws = torch.empty(api._lib.load().prism_attn_workspace_size(api.C.byref(p), 1), dtype=torch.uint8,
+                      device="cuda")
+    g = api.attn_bwd(p, pl, sel, inp["Q"], inp["K"], inp["V"], fw.O, inp["dO"], fw.lse, grad_fp32=grad_fp32, ws=bws)
+    torch.cuda.synchronize()
+    assert api.workspace_status(bws) == 0 and api.workspace_status(fw.ws) == 0
+    return w, inp, p, pl, sel, fw, g
+
+
+def _check(name, heads=None, n_sample=None, seed=0):
+    w, inp, p, pl, sel, fw, (dQ, dK, dV) = _run(name)
+    NB = w.N // 64
+    nb = to_np(pl.n_blocks)
+    shapes = to_np(pl.zone_shape)
+    ref_plan = oracle_plan_from_shapes(w.T, w.H, w.W, [shapes[h] for h in range(w.heads)])
+    csr, csc = _lists(sel, NB, w.heads, nb)
+    Q, K, V, dO = (inp[x].float().cpu().numpy() for x in ("Q", "K", "V", "dO"))
+    gQ, gK, gV = to_np(dQ), to_np(dK), to_np(dV)
+    scale = scale_of(w.head_dim)
+    rng = np.random.default_rng(seed)
+    errs = {"dQ": [], "dK": [], "dV": []}
+    for h in (range(w.heads) if heads is None else heads):
+        hp = ref_plan.heads[h]
+        sub = O.Plan(w.T, w.H, w.W, [hp])
+        if n_sample is None:
+            sel_h = [[(i, csr[h][i], {}) for i in range(nb[h])]]
+            rQ, rK, rV = O.attention_bwd(Q[:, h:h + 1], K[:, h:h + 1], V[:, h:h + 1], dO[:, h:h + 1], sub, sel_h, scale)
+            for nm, got, ref in (("dQ", gQ, rQ), ("dK", gK, rK), ("dV", gV, rV)):
+                errs[nm].append(np.abs(got[:, h] - ref[:, 0]).reshape(-1))
+            continue
+        for i in rng.choice(nb[h], size=min(n_sample, nb[h]), replace=False):
+            rQ, _, _ = O.attention_bwd(Q[:, h:h + 1], K[:, h:h + 1], V[:, h:h + 1], dO[:, h:h + 1], sub,
+                                       [[(int(i), csr[h][i], {})]], scale)
+            toks = hp.perm[hp.blocks[i, 5]:hp.blocks[i, 5] + hp.blocks[i, 4]]
+            errs["dQ"].append(np.abs(gQ[toks, h] - rQ[toks, 0]).reshape(-1))
+        for j in rng.choice(nb[h], size=min(n_sample, nb[h]), replace=False):
+            users = [(int(i), csr[h][int(i)], {}) for i in csc[h][j]]
+            _, rK, rV = O.attention_bwd(Q[:, h:h + 1], K[:, h:h + 1], V[:, h:h + 1], dO[:, h:h + 1], sub, [users],
+                                        scale)
+            toks = hp.perm[hp.blocks[j, 5]:hp.blocks[j, 5] + hp.blocks[j, 4]]
+            errs["dK"].append(np.abs(gK[toks, h] - rK[toks, 0]).reshape(-1))
+            errs["dV"].append(np.abs(gV[toks, h] - rV[toks, 0]).reshape(-1))
+    for nm, e in errs.items():
+        e = np.concatenate(e)
+        print(f"{name} {nm}: max-abs {e.max():.3e} mean-abs {e.mean():.3e} over {e.size}")
+        assert e.max() <= MAX_ABS and e.mean() <= MEAN_ABS, nm
+    for t in (dQ, dK, dV):
+        assert torch.isfinite(t).all()
+
+
+def test_bwd_tiny():
+    _check("tiny")
+
+
+def test_bwd_small_d128():
+    _check("small")
+
+
+def test_bwd_small_d64_multihead():
+    _check("small_d64")
+
+
+def test_bwd_720p_sampled_blocks():
+    _check("720p", heads=[3, 17], n_sample=12)
+
+
+def test_bwd_select_all_equals_dense_autograd():
+    w = WORKLOADS["small_d64"]
+    NB = w.N // 64
+    _, inp, p, pl, sel, fw, (dQ, dK, dV) = _run("small_d64", topk_abs=NB, top_p=0.5)
+    q, k, v = (inp[x].float().permute(1, 0, 2).requires_grad_(True) for x in ("Q", "K", "V"))
+    s = torch.einsum("hqd,hkd->hqk", q, k) * scale_of(w.head_dim)
+    o = torch.softmax(s, dim=-1) @ v
+    o.backward(inp["dO"].float().permute(1, 0, 2))
+    for nm, got, ref in (("dQ", dQ, q.grad), ("dK", dK, k.grad), ("dV", dV, v.grad)):
+        d = (got - ref.permute(1, 0, 2)).abs()
+        print(f"select-all {nm}: max {d.max().item():.3e} mean {d.mean().item():.3e}")
+        assert d.max().item() <= MAX_ABS and d.mean().item() <= MEAN_ABS
+
+
+def test_bwd_bf16_outputs_track_fp32_outputs():
+    _, _, _, _, _, _, g32 = _run("small", grad_fp32=True)
+    _, _, _, _, _, _, g16 = _run("small", grad_fp32=False)
+    for a, b in zip(g32, g16):
+        assert b.dtype == torch.bfloat16
+        rel = ((b.float() - a).abs() / (a.abs() + 1e-3)).max().item()
+        assert rel < 1e-2
+
+
+def test_bwd_is_deterministic():
+    _, _, _, _, _, _, g1 = _run("small")
+    _, _, _, _, _, _, g2 = _run("small")
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b)

@@ -93,6 +93,26 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ----------------------------------------------------------------------------- ranks
+def rank_seed(rank: int) -> int:
+    """Each rank runs its own independent layer (weak scaling)."""
+    return rank
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a per-rank time over all ranks (identity on one rank)."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Units processed by all ranks per second, timed by the slowest rank."""
+    return world * units_per_rank / (ms_max * 1e-3)
+
+
 # ----------------------------------------------------------------------------- flops
 def computed_pairs(p, pl, sel):
     """P = sum over heads and query blocks i of B_i * sum_{j in S_i} B_j."""
@@ -157,7 +177,7 @@ def oracle_sample(w, inp, p, pl, sel, head=0, n_rows=2, seed=0):
 def run_prism(args, w, rank, world, device):
     lib = _lib.load()
     p = api.params_for(w)
-    inp = make_inputs(w, device, seed=rank)
+    inp = make_inputs(w, device, seed=rank_seed(rank))
     N, h, D = w.N, w.heads, w.head_dim
     Q, K, V, a = inp["Q"], inp["K"], inp["V"], inp["a"]
     dO = inp.get("dO")
@@ -167,11 +187,11 @@ def run_prism(args, w, rank, world, device):
     sel = api.select(p, pl, Q, K)
     sel = api.select(p, pl, Q, K, cap=int(sel.nnz * 1.1) + 1024)
     fw = api.attn_fwd(p, pl, sel, Q, K, V)
-    O_, lse = fw.O, fw.lse
+    O_, lse, O_res = fw.O, fw.lse, fw.O_res
     grads = None
     bws = None
     if backward:
-        grads = api.attn_bwd(p, pl, sel, Q, K, V, O_, dO, lse)
+        grads = api.attn_bwd(p, pl, sel, Q, K, V, O_, dO, lse, O_res=O_res)
         bws = torch.empty(lib.prism_attn_workspace_size(api.C.byref(p), 1), dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
     stages = ["plan", "select", "fwd", "bwd"] if backward else ["plan", "select", "fwd"]
@@ -185,11 +205,11 @@ def run_prism(args, w, rank, world, device):
         api.select(p, pl, Q, K, out=sel)
         if ev is not None:
             ev[2].record(stream)
-        api.attn_fwd(p, pl, sel, Q, K, V, O=O_, lse=lse, ws=fw.ws)
+        api.attn_fwd(p, pl, sel, Q, K, V, O=O_, lse=lse, ws=fw.ws, O_res=O_res)
         if ev is not None:
             ev[3].record(stream)
         if backward:
-            api.attn_bwd(p, pl, sel, Q, K, V, O_, dO, lse, out=grads, ws=bws)
+            api.attn_bwd(p, pl, sel, Q, K, V, O_, dO, lse, out=grads, ws=bws, O_res=O_res)
             if ev is not None:
                 ev[4].record(stream)
 
@@ -221,10 +241,7 @@ def run_prism(args, w, rank, world, device):
     ms = t_start.elapsed_time(t_end) / args.steps
     stage_ms = {s: statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps))
                 for i, s in enumerate(stages)}
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(ms, world, device)
 
     # end to end through host buffers
     e2e = None
@@ -255,11 +272,9 @@ def run_prism(args, w, rank, world, device):
             step_e2e()
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = torch.tensor([e0.elapsed_time(e1) / ksteps], dtype=torch.float64, device=device)
-        if world > 1:
-            torch.distributed.all_reduce(ems, op=torch.distributed.ReduceOp.MAX)
-        e2e = {"value": world * flops / (float(ems.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "ms_per_step": float(ems.item()), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+        ems = max_over_ranks(e0.elapsed_time(e1) / ksteps, world, device)
+        e2e = {"value": whole_job_rate(flops, world, ems) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": ems, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": ksteps}
         del hin, hout
 
@@ -288,7 +303,7 @@ def run_prism(args, w, rank, world, device):
 
     density = P / (float(N) * N * h)
     line = {
-        "metric": METRIC, "value": world * flops / (ms_max * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "metric": METRIC, "value": whole_job_rate(flops, world, ms_max) / 1e12, "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded generator; stands in for the pages' 2K-Bench latents)",

@@ -18,8 +18,9 @@ PRISM_ERR_UNSUPPORTED = 2
 PRISM_ERR_CAPACITY = 3
 PRISM_ERR_CUDA = 4
 PRISM_ERR_TIMEOUT = 5
+PRISM_ERR_RANGE = 6
 STATUS_NAMES = {0: "PRISM_OK", 1: "PRISM_ERR_INVALID_ARG", 2: "PRISM_ERR_UNSUPPORTED", 3: "PRISM_ERR_CAPACITY",
-                4: "PRISM_ERR_CUDA", 5: "PRISM_ERR_TIMEOUT"}
+                4: "PRISM_ERR_CUDA", 5: "PRISM_ERR_TIMEOUT", 6: "PRISM_ERR_RANGE"}
 
 # Every function the header declares, with its ctypes signature.
 EXPORTS = (
@@ -71,9 +72,10 @@ def load() -> C.CDLL:
         "prism_select_workspace_size": (sz, [P(PrismParams)]),
         "prism_select": (C.c_int, [P(PrismParams), P(PrismPlan), vp, vp, P(PrismSelect), vp, sz, st]),
         "prism_attn_workspace_size": (sz, [P(PrismParams), C.c_int]),
-        "prism_attn_fwd": (C.c_int, [P(PrismParams), P(PrismPlan), P(PrismSelect), vp, vp, vp, vp, vp, vp, sz, st]),
+        "prism_attn_fwd": (C.c_int, [P(PrismParams), P(PrismPlan), P(PrismSelect), vp, vp, vp, vp, vp, vp, vp, sz,
+                                     st]),
         "prism_attn_bwd": (C.c_int, [P(PrismParams), P(PrismPlan), P(PrismSelect), vp, vp, vp, vp, vp, vp, vp, vp,
-                                     vp, C.c_int, vp, sz, st]),
+                                     vp, vp, C.c_int, vp, sz, st]),
         "prism_workspace_status": (C.c_int, [vp, st]),
         "prism_last_error": (C.c_char_p, []),
         "prism_version": (C.c_char_p, []),

@@ -167,27 +167,33 @@ class FwdResult:
     O: torch.Tensor
     lse: torch.Tensor
     ws: torch.Tensor
+    O_res: torch.Tensor | None = None
 
 
-def attn_fwd(p: PrismParams, pl: Plan, sel: Selection, Q, K, V, O=None, lse=None, ws=None,
-             stream=None) -> FwdResult:
-    """prism_attn_fwd: attention over the selected blocks; O natural order, lse [heads, N]."""
+def attn_fwd(p: PrismParams, pl: Plan, sel: Selection, Q, K, V, O=None, lse=None, ws=None, O_res=None,
+             residual: bool = True, stream=None) -> FwdResult:
+    """prism_attn_fwd: attention over the selected blocks; O natural order,
+    lse [heads, N]; with `residual`, also O's bf16 rounding residual for the
+    backward's Delta."""
     N = p.T * p.H * p.W
     for name, t in (("Q", Q), ("K", K), ("V", V)):
         _check_tensor(t, name, torch.bfloat16, (N, p.heads, p.head_dim))
     lib = _lib.load()
     O = O if O is not None else torch.empty_like(Q)
+    if residual and O_res is None:
+        O_res = torch.empty_like(Q)
     lse = lse if lse is not None else torch.empty((p.heads, N), dtype=torch.float32, device=Q.device)
     ws = ws if ws is not None else _workspace(lib.prism_attn_workspace_size(C.byref(p), 0), Q.device)
     cpl, cs = pl.c_struct(), sel.c_struct()
-    check(lib.prism_attn_fwd(C.byref(p), C.byref(cpl), C.byref(cs), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse),
-                             _ptr(ws), ws.numel(), _stream(stream)))
-    return FwdResult(O, lse, ws)
+    check(lib.prism_attn_fwd(C.byref(p), C.byref(cpl), C.byref(cs), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
+                             _ptr(O_res) if residual else None, _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return FwdResult(O, lse, ws, O_res if residual else None)
 
 
 def attn_bwd(p: PrismParams, pl: Plan, sel: Selection, Q, K, V, O, dO, lse, grad_fp32=False, out=None, ws=None,
-             stream=None):
-    """prism_attn_bwd: dQ, dK, dV through the selected blocks (natural order)."""
+             O_res=None, stream=None):
+    """prism_attn_bwd: dQ, dK, dV through the selected blocks (natural order).
+    Pass the forward's O_res for an fp32-accurate Delta."""
     N = p.T * p.H * p.W
     lib = _lib.load()
     dt = torch.float32 if grad_fp32 else torch.bfloat16
@@ -196,9 +202,9 @@ def attn_bwd(p: PrismParams, pl: Plan, sel: Selection, Q, K, V, O, dO, lse, grad
     ws = ws if ws is not None else _workspace(lib.prism_attn_workspace_size(C.byref(p), 1), Q.device)
     cpl, cs = pl.c_struct(), sel.c_struct()
     dQ, dK, dV = out
-    check(lib.prism_attn_bwd(C.byref(p), C.byref(cpl), C.byref(cs), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO),
-                             _ptr(lse), _ptr(dQ), _ptr(dK), _ptr(dV), int(bool(grad_fp32)), _ptr(ws), ws.numel(),
-                             _stream(stream)))
+    check(lib.prism_attn_bwd(C.byref(p), C.byref(cpl), C.byref(cs), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
+                             _ptr(O_res), _ptr(dO), _ptr(lse), _ptr(dQ), _ptr(dK), _ptr(dV), int(bool(grad_fp32)),
+                             _ptr(ws), ws.numel(), _stream(stream)))
     return dQ, dK, dV
 
 

@@ -143,8 +143,8 @@ size_t prism_attn_workspace_size(const prism_params *p, int backward) {
 }
 
 int prism_attn_fwd(const prism_params *p, const prism_plan_t *plan, const prism_select_t *sel, const uint16_t *Q,
-                   const uint16_t *K, const uint16_t *V, uint16_t *O, float *lse, void *workspace, size_t ws_bytes,
-                   prism_stream_t stream) {
+                   const uint16_t *K, const uint16_t *V, uint16_t *O, uint16_t *O_res, float *lse, void *workspace,
+                   size_t ws_bytes, prism_stream_t stream) {
   int rc;
   if ((rc = check_params(p)) != PRISM_OK) return rc;
   if (!Q || !K || !V || !O || !lse) return fail(PRISM_ERR_INVALID_ARG, "Q, K, V, O or lse is NULL");
@@ -153,15 +153,15 @@ int prism_attn_fwd(const prism_params *p, const prism_plan_t *plan, const prism_
   if ((rc = check_ws(workspace, ws_bytes, attn_fwd_ws_bytes(*p))) != PRISM_OK) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(workspace, 0, kWsHeader, st);
-  if (e == cudaSuccess) e = launch_attn_fwd(*p, *plan, *sel, Q, K, V, O, lse, workspace, st);
+  if (e == cudaSuccess) e = launch_attn_fwd(*p, *plan, *sel, Q, K, V, O, O_res, lse, workspace, st);
   if (e != cudaSuccess) return cuda_fail(e, "prism_attn_fwd");
   g_last_error.clear();
   return PRISM_OK;
 }
 
 int prism_attn_bwd(const prism_params *p, const prism_plan_t *plan, const prism_select_t *sel, const uint16_t *Q,
-                   const uint16_t *K, const uint16_t *V, const uint16_t *O, const uint16_t *dO, const float *lse,
-                   void *dQ, void *dK, void *dV, int grad_fp32, void *workspace, size_t ws_bytes,
+                   const uint16_t *K, const uint16_t *V, const uint16_t *O, const uint16_t *O_res, const uint16_t *dO,
+                   const float *lse, void *dQ, void *dK, void *dV, int grad_fp32, void *workspace, size_t ws_bytes,
                    prism_stream_t stream) {
   int rc;
   if ((rc = check_params(p)) != PRISM_OK) return rc;
@@ -173,7 +173,8 @@ int prism_attn_bwd(const prism_params *p, const prism_plan_t *plan, const prism_
   if ((rc = check_ws(workspace, ws_bytes, attn_bwd_ws_bytes(*p))) != PRISM_OK) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(workspace, 0, kWsHeader, st);
-  if (e == cudaSuccess) e = launch_attn_bwd(*p, *plan, *sel, Q, K, V, O, dO, lse, dQ, dK, dV, grad_fp32, workspace, st);
+  if (e == cudaSuccess)
+    e = launch_attn_bwd(*p, *plan, *sel, Q, K, V, O, O_res, dO, lse, dQ, dK, dV, grad_fp32, workspace, st);
   if (e != cudaSuccess) return cuda_fail(e, "prism_attn_bwd");
   g_last_error.clear();
   return PRISM_OK;

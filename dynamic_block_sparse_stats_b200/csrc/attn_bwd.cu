@@ -11,11 +11,12 @@
 //
 // Two kernels, no atomics (deterministic):
 //   dq_kernel    one CTA per 128-query tile; walks the CSR like the forward:
-//                S = Q K^T, dP = dO V^T (TMEM), dS -> TMEM (bf16),
+//                S = Q K^T, dP = dO V^T (TMEM), dS -> TMEM (fp16),
 //                dQ += dS K (TS MMA).
 //   dkdv_kernel  one CTA per 128-key tile; walks the transpose (CSC):
 //                S^T = K Q^T, dP^T = V dO^T (TMEM), P^T and dS^T -> TMEM
-//                (bf16), dV += P^T dO, dK += dS^T Q (TS MMAs).
+//                (fp16), dV += P^T dO, dK += dS^T Q (TS MMAs).
+// Operands are fp16 (exact conversions of the bf16 inputs, see the forward).
 // Roles as in the forward: warp 0 TMA producer, warp 1 TMEM owner and MMA
 // issuer, warps 2-5 one thread per TMEM lane (row).
 #include "attn_walk.cuh"
@@ -30,14 +31,17 @@ constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ---------------------------------------------------------------------------
-// prep: dOp[h][p] = dO[perm][h], delta[h][p] = sum_c dO*O, lse2[h][p] = lse*log2e
+// prep: dOp[h][p] = fp16(dO[perm][h]), delta[h][p] = sum_c dO*(O + O_res)
+// (O_res, the forward's bf16 rounding residual, may be NULL), lse2 = lse*log2e
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const int32_t *__restrict__ perm, int N, int heads,
                                                        const uint16_t *__restrict__ dO,
                                                        const uint16_t *__restrict__ O,
+                                                       const uint16_t *__restrict__ O_res,
                                                        const float *__restrict__ lse, uint16_t *__restrict__ dOp,
-                                                       float *__restrict__ lse2p, float *__restrict__ deltap) {
+                                                       float *__restrict__ lse2p, float *__restrict__ deltap,
+                                                       int *status) {
   constexpr int G = D / 8;  // lanes per row
   const size_t g = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const size_t r = g / G;
@@ -51,12 +55,17 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const int32_t *__restrict
     const size_t src = ((size_t)n * heads + h) * D + v * 8;
     const uint4 a = __ldg(reinterpret_cast<const uint4 *>(dO + src));
     const uint4 b = __ldg(reinterpret_cast<const uint4 *>(O + src));
-    *reinterpret_cast<uint4 *>(dOp + r * D + v * 8) = a;
-    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+    bool bad = false;
+    *reinterpret_cast<uint4 *>(dOp + r * D + v * 8) =
+        make_uint4(bf16x2_to_f16x2(a.x, bad), bf16x2_to_f16x2(a.y, bad), bf16x2_to_f16x2(a.z, bad),
+                   bf16x2_to_f16x2(a.w, bad));
+    if (bad) record_status(status, PRISM_ERR_RANGE, 101);
+    const uint4 c = O_res ? __ldg(reinterpret_cast<const uint4 *>(O_res + src)) : make_uint4(0, 0, 0, 0);
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w}, cw[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      acc = fmaf(bf16lo(aw[q]), bf16lo(bw[q]), acc);
-      acc = fmaf(bf16hi(aw[q]), bf16hi(bw[q]), acc);
+      acc = fmaf(bf16lo(aw[q]), bf16lo(bw[q]) + bf16lo(cw[q]), acc);
+      acc = fmaf(bf16hi(aw[q]), bf16hi(bw[q]) + bf16hi(cw[q]), acc);
     }
     if (v == 0) lse2p[r] = lse[(size_t)h * N + n] * kLog2e;
   }
@@ -220,8 +229,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t id_full = idesc_bf16(128, 128, 0), id_half = idesc_bf16(128, 64, 0);
-      const uint32_t id_dq = idesc_bf16(128, D, 1);
+      const uint32_t id_full = idesc_f16(128, 128, 0), id_half = idesc_f16(128, 64, 0);
+      const uint32_t id_dq = idesc_f16(128, D, 1);
       const uint32_t sQ = smem_u32(smem + L::OFF_Q), sDO = smem_u32(smem + L::OFF_DO);
       bool ok = mbar_wait(&bar.qdo_full, 0, status, 22);
       tc_fence_after();
@@ -279,8 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
       const int s = j % NSTAGE;
-      ok = mbar_wait(&bar.s_full, j & 1, status, 27);
-      if (ok) ok = mbar_wait(&bar.dp_full, j & 1, status, 28);
+      ok = mbar_wait_warp(&bar.s_full, j & 1, status, 27);
+      if (ok) ok = mbar_wait_warp(&bar.dp_full, j & 1, status, 28);
       if (!ok) break;
       tc_fence_after();
       const int meta = bar.meta[s];
@@ -301,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             d0 = p0 * (__uint_as_float(dv[i]) - dl);
             d1 = p1 * (__uint_as_float(dv[i + 1]) - dl);
           }
-          pk[i / 2] = pack_bf16(d0, d1);
+          pk[i / 2] = pack_f16(d0, d1);
         }
         tmem_st16(tP + lane_off + c * 16, pk);
       }
@@ -309,7 +318,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&bar.ds_ready);
     }
-    if (ok && ntiles > 0) ok = mbar_wait(&bar.dq_done, (ntiles - 1) & 1, status, 29);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok && ntiles > 0) ok = mbar_wait_warp(&bar.dq_done, (ntiles - 1) & 1, status, 29);
     if (ok) {
       tc_fence_after();
       const int n = perm[prow];
@@ -474,8 +484,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t id_full = idesc_bf16(128, 128, 0), id_half = idesc_bf16(128, 64, 0);
-      const uint32_t id_acc = idesc_bf16(128, D, 1);
+      const uint32_t id_full = idesc_f16(128, 128, 0), id_half = idesc_f16(128, 64, 0);
+      const uint32_t id_acc = idesc_f16(128, D, 1);
       const uint32_t sK = smem_u32(smem + L::OFF_K), sV = smem_u32(smem + L::OFF_V);
       bool ok = mbar_wait(&bar.kv_full, 0, status, 42);
       tc_fence_after();
@@ -531,8 +541,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
       const int s = j % NSTAGE;
-      ok = mbar_wait(&bar.s_full, j & 1, status, 47);
-      if (ok) ok = mbar_wait(&bar.dp_full, j & 1, status, 48);
+      ok = mbar_wait_warp(&bar.s_full, j & 1, status, 47);
+      if (ok) ok = mbar_wait_warp(&bar.dp_full, j & 1, status, 48);
       if (!ok) break;
       tc_fence_after();
       const int meta = bar.meta[s];
@@ -555,8 +565,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             d0 = p0 * (__uint_as_float(dv[i]) - dl[q]);
             d1 = p1 * (__uint_as_float(dv[i + 1]) - dl[q + 1]);
           }
-          pp[i / 2] = pack_bf16(p0, p1);
-          pd[i / 2] = pack_bf16(d0, d1);
+          pp[i / 2] = pack_f16(p0, p1);
+          pd[i / 2] = pack_f16(d0, d1);
         }
         tmem_st16(tS + lane_off + c * 16, pp);
         tmem_st16(tP + lane_off + c * 16, pd);
@@ -565,7 +575,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&bar.ds_ready);
     }
-    if (ok && ntiles > 0) ok = mbar_wait(&bar.mm_done, (ntiles - 1) & 1, status, 49);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok && ntiles > 0) ok = mbar_wait_warp(&bar.mm_done, (ntiles - 1) & 1, status, 49);
     if (ok) {
       tc_fence_after();
       const size_t prow = (size_t)h * N + (size_t)tile * 128 + row;
@@ -678,19 +689,23 @@ static cudaError_t run_bwd(const prism_params &p, const prism_plan_t &plan, cons
 
 cudaError_t launch_attn_bwd(const prism_params &p, const prism_plan_t &plan, const prism_select_t &sel,
                             const uint16_t *Q, const uint16_t *K, const uint16_t *V, const uint16_t *O,
-                            const uint16_t *dO, const float *lse, void *dQ, void *dK, void *dV, int grad_fp32,
-                            void *ws, cudaStream_t st) {
+                            const uint16_t *O_res, const uint16_t *dO, const float *lse, void *dQ, void *dK,
+                            void *dV, int grad_fp32, void *ws, cudaStream_t st) {
   const int N = p.T * p.H * p.W, NB = N / 64, D = p.head_dim;
   BwdWs w = carve_bwd(p, ws);
   cudaError_t e;
-  if ((e = launch_permute3(plan.perm, N, p.heads, D, Q, K, V, w.Qp, w.Kp, w.Vp, st)) != cudaSuccess) return e;
+  if ((e = launch_permute3(plan.perm, N, p.heads, D, Q, K, V, w.Qp, w.Kp, w.Vp, &w.hdr->status, st)) !=
+      cudaSuccess)
+    return e;
   const size_t total = (size_t)p.heads * N * (D / 8);
   if (D == 128)
-    bwd::bwd_prep_kernel<128><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(plan.perm, N, p.heads, dO, O, lse,
-                                                                              w.dOp, w.lse2p, w.deltap);
+    bwd::bwd_prep_kernel<128><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(plan.perm, N, p.heads, dO, O, O_res, lse,
+                                                                              w.dOp, w.lse2p, w.deltap,
+                                                                              &w.hdr->status);
   else
-    bwd::bwd_prep_kernel<64><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(plan.perm, N, p.heads, dO, O, lse,
-                                                                             w.dOp, w.lse2p, w.deltap);
+    bwd::bwd_prep_kernel<64><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(plan.perm, N, p.heads, dO, O, O_res, lse,
+                                                                             w.dOp, w.lse2p, w.deltap,
+                                                                             &w.hdr->status);
   count_launches(1);
   if ((e = launch_unit_block(plan.blocks, plan.n_blocks, NB, p.heads, w.unit_block, st)) != cudaSuccess) return e;
   if ((e = launch_tile_units(sel.row_ptr, sel.col, plan.blocks, w.unit_block, N, p.heads, w.tu_q, st)) != cudaSuccess)

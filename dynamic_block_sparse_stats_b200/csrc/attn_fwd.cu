@@ -20,7 +20,7 @@
 //                 O   += P V    (TS: P is read from TMEM where S[b] was)
 //   warps 2-5   softmax, one thread per query row: reads S[b], online max
 //               with lazy rescaling of O (only when the max grows by more
-//               than 2^8), writes P as bf16 into TMEM, and finally
+//               than 2^8), writes P as fp16 into TMEM, and finally
 //               normalises O and scatters it to natural token order.
 #include "attn_walk.cuh"
 
@@ -68,8 +68,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap mapV, const int32_t *__restrict__ row_ptr,
                     const int32_t *__restrict__ col, const int32_t *__restrict__ blocks,
                     const int32_t *__restrict__ unit_block, const int32_t *__restrict__ tile_units,
-                    const int32_t *__restrict__ perm, uint16_t *__restrict__ O, float *__restrict__ lse, int N,
-                    int heads, float scale_log2, int *status) {
+                    const int32_t *__restrict__ perm, uint16_t *__restrict__ O, uint16_t *__restrict__ O_res,
+                    float *__restrict__ lse, int N, int heads, float scale_log2, int *status) {
   using L = Smem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -183,9 +183,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc_s_full = idesc_bf16(128, 128, 0);
-      const uint32_t idesc_s_half = idesc_bf16(128, 64, 0);
-      const uint32_t idesc_o = idesc_bf16(128, D, 1);
+      const uint32_t idesc_s_full = idesc_f16(128, 128, 0);
+      const uint32_t idesc_s_half = idesc_f16(128, 64, 0);
+      const uint32_t idesc_o = idesc_f16(128, D, 1);
       const uint32_t sQ = smem_u32(smem + L::OFF_Q);
       bool ok = mbar_wait(&bar.q_full, 0, status, 2);
       tc_fence_after();
@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
       const int s = j % NSTAGE, b = j & 1;
-      ok = mbar_wait(&bar.s_full[b], (j >> 1) & 1, status, 7);
+      ok = mbar_wait_warp(&bar.s_full[b], (j >> 1) & 1, status, 7);
       if (!ok) break;
       tc_fence_after();
       const int meta = bar.meta[s];
@@ -265,12 +265,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; ++i) mt = fmaxf(mt, __uint_as_float(r[q][i]));
       }
       mt *= scale_log2;
-      if (mt > m + kRescaleLog2 || (m == -INFINITY && mt > -INFINITY)) {
-        // new reference maximum: rescale the running sum and, once O holds
-        // earlier tiles, the accumulator rows of this thread
-        const float alpha = (m == -INFINITY) ? 0.f : exp2f(m - mt);
-        if (j > 0 && m != -INFINITY) {
-          ok = mbar_wait(&bar.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, status, 8);
+      // A row takes a new reference maximum only when it grows by more than
+      // 2^8 (or on its first valid key).  The decision to touch O is made per
+      // warp, because tcgen05.ld/st are warp-collective; rows that keep their
+      // maximum use alpha = 1.
+      const bool want = mt > m + kRescaleLog2 || (m == -INFINITY && mt > -INFINITY);
+      if (__any_sync(0xffffffffu, want)) {
+        const float m_new = want ? mt : m;
+        const float alpha = (m == -INFINITY) ? 0.f : exp2f(m - m_new);
+        if (j > 0 && __any_sync(0xffffffffu, want && m != -INFINITY)) {
+          ok = mbar_wait_warp(&bar.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, status, 8);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll 1
@@ -285,9 +289,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_st();
         }
         l *= alpha;
-        m = mt;
+        m = m_new;
       }
-      // P = exp2(s * scale_log2 - m), bf16, packed two keys per column
+      // P = exp2(s * scale_log2 - m), fp16, packed two keys per column
       uint32_t pk[64];
       float ls = 0.f;
 #pragma unroll
@@ -301,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             p1 = exp2f(fmaf(__uint_as_float(r[q][i + 1]), scale_log2, -m));
           }
           ls += p0 + p1;
-          pk[q * 16 + i / 2] = pack_bf16(p0, p1);
+          pk[q * 16 + i / 2] = pack_f16(p0, p1);
         }
       }
       l += ls;
@@ -312,7 +316,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bar.p_full[b]);
     }
     // epilogue
-    if (ok && ntiles > 0) ok = mbar_wait(&bar.pv_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, status, 9);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok && ntiles > 0) ok = mbar_wait_warp(&bar.pv_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, status, 9);
     if (ok) {
       tc_fence_after();
       const int p = tile * BM + row;
@@ -329,13 +334,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = 0u;
         }
-        uint4 v[4];
-        uint32_t *pv = reinterpret_cast<uint32_t *>(v);
+        uint4 v[4], rv[4];
+        uint32_t *pv = reinterpret_cast<uint32_t *>(v), *pr = reinterpret_cast<uint32_t *>(rv);
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pv[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+        for (int i = 0; i < 16; ++i) {
+          const float x0 = __uint_as_float(o[2 * i]) * inv, x1 = __uint_as_float(o[2 * i + 1]) * inv;
+          pv[i] = pack_bf16(x0, x1);
+          pr[i] = pack_bf16(x0 - bf16lo(pv[i]), x1 - bf16hi(pv[i]));  // rounding residual
+        }
 #pragma unroll
         for (int i = 0; i < 4; ++i) reinterpret_cast<uint4 *>(dst + c)[i] = v[i];
+        if (O_res) {
+          uint16_t *rdst = O_res + ((size_t)n * heads + h) * D;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) reinterpret_cast<uint4 *>(rdst + c)[i] = rv[i];
+        }
       }
       // natural-log LSE: ln 2 * (m + log2 l)
       lse[(size_t)h * N + n] = (l > 0.f) ? 0.69314718055994531f * (m + log2f(l)) : -INFINITY;
@@ -400,11 +413,17 @@ __global__ void tile_units_kernel(const int32_t *__restrict__ row_ptr, const int
   if (lane == 0) tile_units[(size_t)h * NT + t] = (int32_t)cnt;
 }
 
-// dst[h][p][:] = src[perm[h][p]][h][:]
+__device__ __forceinline__ uint4 to_f16x8(uint4 v, bool &bad) {
+  return make_uint4(bf16x2_to_f16x2(v.x, bad), bf16x2_to_f16x2(v.y, bad), bf16x2_to_f16x2(v.z, bad),
+                    bf16x2_to_f16x2(v.w, bad));
+}
+
+// dst[h][p][:] = fp16(src[perm[h][p]][h][:]); a value outside the fp16 range
+// records PRISM_ERR_RANGE in *status.
 __global__ void permute3_kernel(const int32_t *__restrict__ perm, int N, int heads, int D,
                                 const uint16_t *__restrict__ s0, const uint16_t *__restrict__ s1,
                                 const uint16_t *__restrict__ s2, uint16_t *__restrict__ d0, uint16_t *__restrict__ d1,
-                                uint16_t *__restrict__ d2) {
+                                uint16_t *__restrict__ d2, int *status) {
   const int vpr = D / 8;  // 16-byte vectors per row
   const size_t g = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const size_t rows = (size_t)heads * N;
@@ -414,17 +433,21 @@ __global__ void permute3_kernel(const int32_t *__restrict__ perm, int N, int hea
   const int h = (int)(r / N);
   const int n = perm[r];
   const size_t src = ((size_t)n * heads + h) * D + v * 8, dst = r * D + v * 8;
-  *reinterpret_cast<uint4 *>(d0 + dst) = __ldg(reinterpret_cast<const uint4 *>(s0 + src));
-  if (s1) *reinterpret_cast<uint4 *>(d1 + dst) = __ldg(reinterpret_cast<const uint4 *>(s1 + src));
-  if (s2) *reinterpret_cast<uint4 *>(d2 + dst) = __ldg(reinterpret_cast<const uint4 *>(s2 + src));
+  bool bad = false;
+  *reinterpret_cast<uint4 *>(d0 + dst) = to_f16x8(__ldg(reinterpret_cast<const uint4 *>(s0 + src)), bad);
+  if (s1) *reinterpret_cast<uint4 *>(d1 + dst) = to_f16x8(__ldg(reinterpret_cast<const uint4 *>(s1 + src)), bad);
+  if (s2) *reinterpret_cast<uint4 *>(d2 + dst) = to_f16x8(__ldg(reinterpret_cast<const uint4 *>(s2 + src)), bad);
+  if (bad) record_status(status, PRISM_ERR_RANGE, 100);
 }
 
 }  // namespace fwd
 
 cudaError_t launch_permute3(const int32_t *perm, int N, int heads, int D, const uint16_t *s0, const uint16_t *s1,
-                            const uint16_t *s2, uint16_t *d0, uint16_t *d1, uint16_t *d2, cudaStream_t st) {
+                            const uint16_t *s2, uint16_t *d0, uint16_t *d1, uint16_t *d2, int *status,
+                            cudaStream_t st) {
   const size_t total = (size_t)heads * N * (D / 8);
-  fwd::permute3_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(perm, N, heads, D, s0, s1, s2, d0, d1, d2);
+  fwd::permute3_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(perm, N, heads, D, s0, s1, s2, d0, d1, d2,
+                                                                       status);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -464,7 +487,7 @@ static EncodeTiledFn get_encode() {
   return fn;
 }
 
-// 2-D bf16 map over rows of D elements: box = 64 elements x box_rows, 128B swizzle.
+// 2-D fp16 map over rows of D elements: box = 64 elements x box_rows, 128B swizzle.
 cudaError_t make_rows_map(CUtensorMap *map, const void *base, long long rows, int D, int box_rows) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return cudaErrorNotSupported;
@@ -472,7 +495,7 @@ cudaError_t make_rows_map(CUtensorMap *map, const void *base, long long rows, in
   const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
   const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box,
                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
@@ -513,7 +536,7 @@ size_t attn_fwd_ws_bytes(const prism_params &p) {
 
 template <int D>
 static cudaError_t run_fwd(const prism_params &p, const prism_plan_t &plan, const prism_select_t &sel,
-                           const FwdWs &w, uint16_t *O, float *lse, cudaStream_t st) {
+                           const FwdWs &w, uint16_t *O, uint16_t *O_res, float *lse, cudaStream_t st) {
   const int N = p.T * p.H * p.W;
   CUtensorMap mQ, mK, mV;
   cudaError_t e;
@@ -525,24 +548,26 @@ static cudaError_t run_fwd(const prism_params &p, const prism_plan_t &plan, cons
   const float scale_log2 = effective_scale(p) * 1.4426950408889634f;
   dim3 grid(N / fwd::BM, p.heads);
   fwd::attn_fwd_kernel<D><<<grid, fwd::kThreads, smem, st>>>(mQ, mK, mV, sel.row_ptr, sel.col, plan.blocks,
-                                                             w.unit_block, w.tile_units, plan.perm, O, lse, N,
-                                                             p.heads, scale_log2, &w.hdr->status);
+                                                             w.unit_block, w.tile_units, plan.perm, O, O_res, lse,
+                                                             N, p.heads, scale_log2, &w.hdr->status);
   count_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_attn_fwd(const prism_params &p, const prism_plan_t &plan, const prism_select_t &sel,
-                            const uint16_t *Q, const uint16_t *K, const uint16_t *V, uint16_t *O, float *lse,
-                            void *ws, cudaStream_t st) {
+                            const uint16_t *Q, const uint16_t *K, const uint16_t *V, uint16_t *O, uint16_t *O_res,
+                            float *lse, void *ws, cudaStream_t st) {
   const int N = p.T * p.H * p.W, NB = N / 64, D = p.head_dim;
   FwdWs w = carve_fwd(p, ws);
   cudaError_t e;
-  if ((e = launch_permute3(plan.perm, N, p.heads, D, Q, K, V, w.Qp, w.Kp, w.Vp, st)) != cudaSuccess) return e;
+  if ((e = launch_permute3(plan.perm, N, p.heads, D, Q, K, V, w.Qp, w.Kp, w.Vp, &w.hdr->status, st)) !=
+      cudaSuccess)
+    return e;
   if ((e = launch_unit_block(plan.blocks, plan.n_blocks, NB, p.heads, w.unit_block, st)) != cudaSuccess) return e;
   if ((e = launch_tile_units(sel.row_ptr, sel.col, plan.blocks, w.unit_block, N, p.heads, w.tile_units, st)) !=
       cudaSuccess)
     return e;
-  return D == 128 ? run_fwd<128>(p, plan, sel, w, O, lse, st) : run_fwd<64>(p, plan, sel, w, O, lse, st);
+  return D == 128 ? run_fwd<128>(p, plan, sel, w, O, O_res, lse, st) : run_fwd<64>(p, plan, sel, w, O, O_res, lse, st);
 }
 
 }  // namespace prism

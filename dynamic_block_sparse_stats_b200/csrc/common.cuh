@@ -29,6 +29,12 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // (cycles of the SM clock; about 2 s at 1.9 GHz).
 constexpr long long kWaitLimitCycles = 4000000000LL;
 
+__device__ __forceinline__ void record_status(int *status, int code, int where) {
+  if (status) {
+    atomicCAS(status, 0, code);
+    atomicExch(status + 1, where);
+  }
+}
 __device__ __forceinline__ void record_timeout(int *status, int where) {
   if (status) {
     atomicExch(status, (int)PRISM_ERR_TIMEOUT);
@@ -52,6 +58,18 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// bf16 pair -> fp16 pair (exact for |x| <= 65504 and |x| >= 2^-14); sets
+// *bad when a value lies outside the fp16 range.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v, bool &bad) {
+  const float lo = bf16lo(v), hi = bf16hi(v);
+  bad |= !(fabsf(lo) <= 65504.f) || !(fabsf(hi) <= 65504.f);
+  return pack_f16(lo, hi);
 }
 
 // ---------------------------------------------------------------------------
@@ -101,6 +119,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *s
     }
   }
   return true;
+}
+
+// Bounded wait whose outcome is the same for every lane of the warp, so that
+// the .sync.aligned tcgen05 instructions that follow stay convergent.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, int *status, int where) {
+  const bool ok = mbar_wait(bar, parity, status, where);
+  return __all_sync(0xffffffffu, ok);
 }
 
 // ---------------------------------------------------------------------------
@@ -218,12 +243,15 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   d |= (uint64_t)2 << 61;
   return d;
 }
-// Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulation.
-//   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format
-//   (1 = bf16), 15 A major (0 = K), 16 B major (0 = K, 1 = MN),
-//   17-22 N >> 3, 24-28 M >> 4.
+// Instruction descriptor for kind::f16 with fp32 accumulation.
+//   bits 4-5 D format (1 = f32), 7-9 A format, 10-12 B format (0 = f16,
+//   1 = bf16; A and B always the same type), 15 A major (0 = K), 16 B major
+//   (0 = K, 1 = MN), 17-22 N >> 3, 24-28 M >> 4.
 __host__ __device__ constexpr uint32_t idesc_bf16(uint32_t M, uint32_t N, uint32_t b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn_major << 16) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_f16(uint32_t M, uint32_t N, uint32_t b_mn_major) {
+  return (1u << 4) | (b_mn_major << 16) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
 // ---------------------------------------------------------------------------

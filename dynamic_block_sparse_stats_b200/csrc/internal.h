@@ -23,20 +23,23 @@ cudaError_t launch_select(const prism_params &p, const prism_plan_t &plan, const
 // attn_fwd.cu
 size_t attn_fwd_ws_bytes(const prism_params &p);
 cudaError_t launch_attn_fwd(const prism_params &p, const prism_plan_t &plan, const prism_select_t &sel,
-                            const uint16_t *Q, const uint16_t *K, const uint16_t *V, uint16_t *O, float *lse,
-                            void *ws, cudaStream_t st);
+                            const uint16_t *Q, const uint16_t *K, const uint16_t *V, uint16_t *O, uint16_t *O_res,
+                            float *lse, void *ws, cudaStream_t st);
 
 // attn_bwd.cu
 size_t attn_bwd_ws_bytes(const prism_params &p);
 cudaError_t launch_attn_bwd(const prism_params &p, const prism_plan_t &plan, const prism_select_t &sel,
                             const uint16_t *Q, const uint16_t *K, const uint16_t *V, const uint16_t *O,
-                            const uint16_t *dO, const float *lse, void *dQ, void *dK, void *dV, int grad_fp32,
-                            void *ws, cudaStream_t st);
+                            const uint16_t *O_res, const uint16_t *dO, const float *lse, void *dQ, void *dK,
+                            void *dV, int grad_fp32, void *ws, cudaStream_t st);
 
-// shared launch helper: token gather into permuted head-major order
-// dst[h][p][:] = src[perm[h][p]][h][:] for up to three tensors at once.
+// shared launch helper: token gather into permuted head-major order with the
+// bf16 -> fp16 conversion of the attention operands:
+// dst[h][p][:] = fp16(src[perm[h][p]][h][:]) for up to three tensors at once;
+// out-of-range values record PRISM_ERR_RANGE in *status.
 cudaError_t launch_permute3(const int32_t *perm, int N, int heads, int D, const uint16_t *s0, const uint16_t *s1,
-                            const uint16_t *s2, uint16_t *d0, uint16_t *d1, uint16_t *d2, cudaStream_t st);
+                            const uint16_t *s2, uint16_t *d0, uint16_t *d1, uint16_t *d2, int *status,
+                            cudaStream_t st);
 
 float effective_scale(const prism_params &p);
 
@@ -47,7 +50,7 @@ cudaError_t launch_unit_block(const int32_t *blocks, const int32_t *n_blocks, in
 // (ptr, idx) of its one or two blocks (CSR for query tiles, CSC for key tiles).
 cudaError_t launch_tile_units(const int32_t *ptr, const int32_t *idx, const int32_t *blocks,
                               const int32_t *unit_block, int N, int heads, int32_t *tile_units, cudaStream_t st);
-// 2-D bf16 tensor map over rows of D elements, box 64 x box_rows, 128B swizzle.
+// 2-D fp16 tensor map over rows of D elements, box 64 x box_rows, 128B swizzle.
 cudaError_t make_rows_map(CUtensorMap *map, const void *base, long long rows, int D, int box_rows);
 
 // host-side count of kernel launches (prism_kernel_launches)

@@ -52,7 +52,8 @@ typedef enum prism_status {
   PRISM_ERR_UNSUPPORTED = 2,  /* T/H/W not multiples of 8, head_dim not 64/128 */
   PRISM_ERR_CAPACITY = 3,     /* an output or workspace is too small          */
   PRISM_ERR_CUDA = 4,         /* a CUDA runtime call failed                   */
-  PRISM_ERR_TIMEOUT = 5       /* a kernel gave up on an internal wait         */
+  PRISM_ERR_TIMEOUT = 5,      /* a kernel gave up on an internal wait         */
+  PRISM_ERR_RANGE = 6         /* an attention input is outside the fp16 range */
 } prism_status;
 
 /*
@@ -196,21 +197,31 @@ size_t prism_attn_workspace_size(const prism_params *p, int backward);
  *   Q, K, V   bf16 [N][heads][head_dim].
  *   O         bf16 [N][heads][head_dim], natural order (inverse permutation
  *             applied).
+ *   O_res     bf16 [N][heads][head_dim] or NULL: the rounding residual
+ *             O_fp32 - O (rounded to bf16), so that O + O_res carries the
+ *             fp32 accumulator to ~2^-17 relative.  prism_attn_bwd uses it
+ *             for Delta = rowsum(dO * O); without it Delta is formed from the
+ *             bf16 O, whose rounding dominates the gradient error of rows
+ *             with sharp attention.
  *   lse       fp32 [heads][N], natural order (natural log).
- * Runs on tcgen05 tensor cores (bf16 operands, fp32 accumulation).
+ * Runs on tcgen05 tensor cores with fp32 accumulation.  The operands are
+ * fp16: Q, K, V convert exactly from bf16 for |x| <= 65504 (a larger value
+ * records PRISM_ERR_RANGE in the workspace); the probabilities P (in [0, 256]
+ * under the lazy rescaling) are rounded to fp16, 8x finer than bf16.
  * Returns PRISM_OK, PRISM_ERR_INVALID_ARG, PRISM_ERR_UNSUPPORTED,
  * PRISM_ERR_CAPACITY or PRISM_ERR_CUDA.
  */
 int prism_attn_fwd(const prism_params *p, const prism_plan_t *plan,
                    const prism_select_t *sel, const uint16_t *Q,
                    const uint16_t *K, const uint16_t *V, uint16_t *O,
-                   float *lse, void *workspace, size_t ws_bytes,
-                   prism_stream_t stream);
+                   uint16_t *O_res, float *lse, void *workspace,
+                   size_t ws_bytes, prism_stream_t stream);
 
 /*
  * prism_attn_bwd -- gradients of prism_attn_fwd through the selected blocks
  * only; the plan and the selection are constants (digest, training section).
  *   O, lse    outputs of prism_attn_fwd for the same inputs.
+ *   O_res     the forward's O_res, or NULL (Delta from the bf16 O alone).
  *   dO        bf16 [N][heads][head_dim] upstream gradient.
  *   dQ,dK,dV  [N][heads][head_dim]; bf16 when grad_fp32 == 0, fp32 else.
  * sel must carry the transpose (col_ptr/row non-NULL).
@@ -220,12 +231,16 @@ int prism_attn_fwd(const prism_params *p, const prism_plan_t *plan,
 int prism_attn_bwd(const prism_params *p, const prism_plan_t *plan,
                    const prism_select_t *sel, const uint16_t *Q,
                    const uint16_t *K, const uint16_t *V, const uint16_t *O,
-                   const uint16_t *dO, const float *lse, void *dQ, void *dK,
-                   void *dV, int grad_fp32, void *workspace, size_t ws_bytes,
+                   const uint16_t *O_res, const uint16_t *dO,
+                   const float *lse, void *dQ, void *dK, void *dV,
+                   int grad_fp32, void *workspace, size_t ws_bytes,
                    prism_stream_t stream);
 
 /* Waits on `stream` and returns the status a kernel recorded in
- * `workspace` (PRISM_OK or PRISM_ERR_TIMEOUT), or PRISM_ERR_CUDA. */
+ * `workspace`: PRISM_OK, PRISM_ERR_TIMEOUT, or PRISM_ERR_RANGE (an attention
+ * call met a Q/K/V/dO value with |x| > 65504, the largest fp16 value; the
+ * attention tensor-core operands are fp16, to which bf16 converts exactly in
+ * that range), or PRISM_ERR_CUDA. */
 int prism_workspace_status(const void *workspace, prism_stream_t stream);
 
 /* Message of the calling thread's last failing call ("" if none).  The

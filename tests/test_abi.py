@@ -70,7 +70,7 @@ def test_null_pointers_and_short_workspace_are_rejected():
     assert lib.prism_select(C.byref(p), C.byref(plan), C.c_void_p(8), C.c_void_p(8), C.byref(sel),
                             C.c_void_p(256), 1 << 30, None) == _lib.PRISM_ERR_INVALID_ARG
     assert lib.prism_attn_bwd(C.byref(p), C.byref(plan), C.byref(_lib.PrismSelect(8, 8, 10, 0, None, None)),
-                              *([C.c_void_p(8)] * 9), 0, C.c_void_p(256), 1 << 30, None) == _lib.PRISM_ERR_INVALID_ARG
+                              *([C.c_void_p(8)] * 10), 0, C.c_void_p(256), 1 << 30, None) == _lib.PRISM_ERR_INVALID_ARG
 
 
 def test_workspace_sizes_grow_with_the_grid():

@@ -48,8 +48,10 @@ def test_plan_matches_oracle(name):
     excluded = 0
     for k, h in enumerate(heads):
         hp = ref.heads[k]
-        np.testing.assert_allclose(rho[h], hp.rho, rtol=1e-9, atol=1e-12)
-        np.testing.assert_allclose(g[h], hp.g, rtol=1e-9, atol=1e-12)
+        # statistic values: fp32 partial sums of <= 8 terms combined in float64
+        # (<= 8 fp32 ulps relative); the decisions below are compared exactly
+        np.testing.assert_allclose(rho[h], hp.rho, rtol=1e-6, atol=1e-12)
+        np.testing.assert_allclose(g[h], hp.g, rtol=1e-6, atol=1e-12)
         diff = shapes[h] != hp.shape
         tie = (hp.vol_margin <= TIE) | (hp.shape_margin <= TIE)
         assert not (diff & ~tie).any(), f"head {h}: shape differs outside ties at zones {np.nonzero(diff & ~tie)}"
@@ -134,7 +136,7 @@ def test_layer_one_without_a2v_norms():
     pl = api.plan(p, inp["V"], None)
     ref = O.plan(inp["V"].float().cpu().numpy(), None, w.T, w.H, w.W)
     for h, hp in enumerate(ref.heads):
-        np.testing.assert_allclose(to_np(pl.zone_g)[h], hp.g, rtol=1e-9)
+        np.testing.assert_allclose(to_np(pl.zone_g)[h], hp.g, rtol=1e-6)
         tie = (hp.vol_margin <= TIE) | (hp.shape_margin <= TIE)
         assert ((to_np(pl.zone_shape)[h] == hp.shape) | tie).all()
 

@@ -26,7 +26,7 @@ STATUS_NAMES = {0: "PRISM_OK", 1: "PRISM_ERR_INVALID_ARG", 2: "PRISM_ERR_UNSUPPO
 EXPORTS = (
     "prism_plan_workspace_size", "prism_plan", "prism_select_workspace_size", "prism_select",
     "prism_attn_workspace_size", "prism_attn_fwd", "prism_attn_bwd", "prism_workspace_status",
-    "prism_last_error", "prism_version", "prism_kernel_launches",
+    "prism_last_error", "prism_version", "prism_kernel_launches", "prism_plan_noalloc",
 )
 
 
@@ -80,6 +80,7 @@ def load() -> C.CDLL:
         "prism_last_error": (C.c_char_p, []),
         "prism_version": (C.c_char_p, []),
         "prism_kernel_launches": (C.c_uint64, []),
+        "prism_plan_noalloc": (C.c_int, [P(PrismParams), vp, vp, P(PrismPlan), st]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)

@@ -73,6 +73,18 @@ static int check_ws(void *ws, size_t bytes, size_t need) {
   return PRISM_OK;
 }
 
+// Argument checks of prism_plan, for other entry points that plan the same way.
+int check_plan_call(const prism_params *p, const uint16_t *V, const prism_plan_t *out) {
+  int rc;
+  if ((rc = check_params(p)) != PRISM_OK) return rc;
+  if (!V) return fail(PRISM_ERR_INVALID_ARG, "V is NULL");
+  return check_plan(out);
+}
+
+int report_error(int code, const char *msg) { return fail(code, "%s", msg); }
+
+void clear_error() { g_last_error.clear(); }
+
 }  // namespace prism
 
 using namespace prism;

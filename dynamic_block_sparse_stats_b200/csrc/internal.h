@@ -56,4 +56,9 @@ cudaError_t make_rows_map(CUtensorMap *map, const void *base, long long rows, in
 // host-side count of kernel launches (prism_kernel_launches)
 void count_launches(int n);
 
+// api.cu: prism_plan's argument checks; error reporting for prism_last_error
+int check_plan_call(const prism_params *p, const uint16_t *V, const prism_plan_t *out);
+int report_error(int code, const char *msg);
+void clear_error();
+
 }  // namespace prism

@@ -358,12 +358,16 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["prism", "reference"], default="prism")
     ap.add_argument("--workload", default="2k_train", choices=sorted(WORKLOADS))
+    ap.add_argument("--backward", action="store_true", help="time the backward on any workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[args.workload]
+    if args.backward and not w.backward:
+        import dataclasses
+        w = dataclasses.replace(w, backward=True)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

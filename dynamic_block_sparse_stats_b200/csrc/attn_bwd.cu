@@ -167,21 +167,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tS = tmem, tP = tmem + 128, tQ = tmem + 256;
 
   if (warp == 0) {
-    const int b0 = unit_block[(size_t)h * NB + 2 * tile], b1 = unit_block[(size_t)h * NB + 2 * tile + 1];
-    UnitWalk w;
-    cursor_init(w.a, row_ptr[h * NB + b0], row_ptr[h * NB + b0 + 1]);
-    if (b1 != b0) {
-      cursor_init(w.b, row_ptr[h * NB + b1], row_ptr[h * NB + b1 + 1]);
-      w.mask_a = 1;
-      w.mask_b = 2;
-    } else {
-      cursor_init(w.b, 0, 0);
-      w.mask_a = 3;
-      w.mask_b = 0;
-    }
-    w.cur_cnt = w.cur_k = 0;
-    w.cur_ub = 0;
-    w.cur_mask = 0;
+    const int blk[2] = {unit_block[(size_t)h * NB + 2 * tile], unit_block[(size_t)h * NB + 2 * tile + 1]};
+    UnitWalk<2> w;
+    walk_init<2>(w, blk, 2, row_ptr, h * NB);
     if (lane == 0) {
       mbar_arrive_expect_tx(&bar.qdo_full, 2 * L::TILE);
 #pragma unroll
@@ -194,9 +182,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int s = j % NSTAGE;
       uint32_t ua, ub = 0;
       int ma, mb = 0, nu = 1;
-      walk_next(w, col, blocks_h, ua, ma);
+      walk_next<2>(w, col, blocks_h, ua, ma);
       if (2 * j + 2 <= nunits) {
-        walk_next(w, col, blocks_h, ub, mb);
+        walk_next<2>(w, col, blocks_h, ub, mb);
         nu = 2;
       }
       ua = min(ua, (uint32_t)(NB - 1));
@@ -423,21 +411,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tS = tmem, tP = tmem + 128, tV = tmem + 256, tK = tmem + 256 + D;
 
   if (warp == 0) {
-    const int b0 = unit_block[(size_t)h * NB + 2 * tile], b1 = unit_block[(size_t)h * NB + 2 * tile + 1];
-    UnitWalk w;
-    cursor_init(w.a, col_ptr[h * NB + b0], col_ptr[h * NB + b0 + 1]);
-    if (b1 != b0) {
-      cursor_init(w.b, col_ptr[h * NB + b1], col_ptr[h * NB + b1 + 1]);
-      w.mask_a = 1;
-      w.mask_b = 2;
-    } else {
-      cursor_init(w.b, 0, 0);
-      w.mask_a = 3;
-      w.mask_b = 0;
-    }
-    w.cur_cnt = w.cur_k = 0;
-    w.cur_ub = 0;
-    w.cur_mask = 0;
+    const int blk[2] = {unit_block[(size_t)h * NB + 2 * tile], unit_block[(size_t)h * NB + 2 * tile + 1]};
+    UnitWalk<2> w;
+    walk_init<2>(w, blk, 2, col_ptr, h * NB);
     if (lane == 0) {
       mbar_arrive_expect_tx(&bar.kv_full, 2 * L::TILE);
 #pragma unroll
@@ -450,9 +426,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int s = j % NSTAGE;
       uint32_t ua, ub = 0;
       int ma, mb = 0, nu = 1;
-      walk_next(w, rowidx, blocks_h, ua, ma);
+      walk_next<2>(w, rowidx, blocks_h, ua, ma);
       if (2 * j + 2 <= nunits) {
-        walk_next(w, rowidx, blocks_h, ub, mb);
+        walk_next<2>(w, rowidx, blocks_h, ub, mb);
         nu = 2;
       }
       ua = min(ua, (uint32_t)(NB - 1));
@@ -708,9 +684,11 @@ cudaError_t launch_attn_bwd(const prism_params &p, const prism_plan_t &plan, con
                                                                              &w.hdr->status);
   count_launches(1);
   if ((e = launch_unit_block(plan.blocks, plan.n_blocks, NB, p.heads, w.unit_block, st)) != cudaSuccess) return e;
-  if ((e = launch_tile_units(sel.row_ptr, sel.col, plan.blocks, w.unit_block, N, p.heads, w.tu_q, st)) != cudaSuccess)
+  if ((e = launch_tile_units(sel.row_ptr, sel.col, plan.blocks, w.unit_block, N, p.heads, 2, w.tu_q, st)) !=
+      cudaSuccess)
     return e;
-  if ((e = launch_tile_units(sel.col_ptr, sel.row, plan.blocks, w.unit_block, N, p.heads, w.tu_k, st)) != cudaSuccess)
+  if ((e = launch_tile_units(sel.col_ptr, sel.row, plan.blocks, w.unit_block, N, p.heads, 2, w.tu_k, st)) !=
+      cudaSuccess)
     return e;
   return D == 128 ? run_bwd<128>(p, plan, sel, w, dQ, dK, dV, grad_fp32, st)
                   : run_bwd<64>(p, plan, sel, w, dQ, dK, dV, grad_fp32, st);

@@ -29,21 +29,20 @@ namespace prism {
 namespace fwd {
 using namespace attn;
 
-constexpr int BM = 128;          // query rows per CTA
+constexpr int BQ = 256;          // query rows per CTA: two 128-row tiles
 constexpr int NSTAGE = 2;        // K/V ring depth
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;    // 12 warps
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (factor 256)
 
 template <int D>
 struct Smem {
   static constexpr int CHUNKS = D / 64;                     // 128-byte swizzle chunks per row
-  static constexpr int Q_BYTES = BM * D * 2;                // 128 rows
-  static constexpr int KV_BYTES = 128 * D * 2;              // one key tile (two units)
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NSTAGE * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + NSTAGE * KV_BYTES;
+  static constexpr int TILE = 128 * D * 2;                  // 128 rows of fp16
+  static constexpr int OFF_Q = 0;                           // two query tiles
+  static constexpr int OFF_K = OFF_Q + 2 * TILE;
+  static constexpr int OFF_V = OFF_K + NSTAGE * TILE;
+  static constexpr int OFF_BAR = OFF_V + NSTAGE * TILE;
   static constexpr int BYTES = OFF_BAR + 256;
 };
 
@@ -52,15 +51,36 @@ struct Bars {
   uint64_t k_full[NSTAGE];
   uint64_t v_full[NSTAGE];
   uint64_t kv_empty[NSTAGE];
-  uint64_t s_full[2];
+  uint64_t s_full[2];   // per query tile
   uint64_t p_full[2];
   uint64_t pv_done[2];
-  int meta[NSTAGE];  // nunits | mask0 << 4 | mask1 << 8
+  int meta[NSTAGE];     // units | maskA << 4 | maskB << 8  (masks: bit = 64-row quarter)
   uint32_t tmem_base;
   int ntiles;
   int nunits;
   int abort;
 };
+
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// (a0, a1) * (b, b) + (c, c) and (a0, a1) + (b0, b1) on paired fp32 lanes
+__device__ __forceinline__ float2 ffma2(float2 a, float b, float c) {
+  uint64_t d;
+  const uint64_t av = *reinterpret_cast<uint64_t *>(&a);
+  float2 bb = make_float2(b, b), cc = make_float2(c, c);
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(av), "l"(*reinterpret_cast<uint64_t *>(&bb)),
+      "l"(*reinterpret_cast<uint64_t *>(&cc)));
+  return *reinterpret_cast<float2 *>(&d);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(*reinterpret_cast<uint64_t *>(&a)),
+      "l"(*reinterpret_cast<uint64_t *>(&b)));
+  return *reinterpret_cast<float2 *>(&d);
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -75,7 +95,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars &bar = *reinterpret_cast<Bars *>(smem + L::OFF_BAR);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.x, h = blockIdx.y;
+  const int quad = blockIdx.x, h = blockIdx.y;
   const int NB = N / 64;
   const int32_t *blocks_h = blocks + (size_t)h * NB * 4;
 
@@ -91,12 +111,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar.v_full[s], 1);
       mbar_init(&bar.kv_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bar.s_full[b], 1);
-      mbar_init(&bar.p_full[b], 128);
-      mbar_init(&bar.pv_done[b], 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bar.s_full[t], 1);
+      mbar_init(&bar.p_full[t], 128);
+      mbar_init(&bar.pv_done[t], 1);
     }
-    bar.nunits = tile_units[(size_t)h * (N / BM) + tile];
+    bar.nunits = tile_units[(size_t)h * (N / BQ) + quad];
     bar.ntiles = (bar.nunits + 1) >> 1;
     bar.abort = 0;
     fence_barrier_init();
@@ -111,45 +131,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bar.tmem_base;
   const int ntiles = bar.ntiles;
   const int nunits = bar.nunits;
-  const uint32_t tS[2] = {tmem, tmem + 128};
-  const uint32_t tO = tmem + 256;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    const int u0 = 2 * tile, u1 = 2 * tile + 1;
-    const int b0 = unit_block[(size_t)h * NB + u0], b1 = unit_block[(size_t)h * NB + u1];
-    UnitWalk w;
-    const int r0 = h * NB + b0, r1 = h * NB + b1;
-    cursor_init(w.a, row_ptr[r0], row_ptr[r0 + 1]);
-    if (b1 != b0) {
-      cursor_init(w.b, row_ptr[r1], row_ptr[r1 + 1]);
-      w.mask_a = 1;
-      w.mask_b = 2;
-    } else {
-      cursor_init(w.b, 0, 0);
-      w.mask_a = 3;
-      w.mask_b = 0;
-    }
-    w.cur_cnt = 0;
-    w.cur_k = 0;
-    w.cur_ub = 0;
-    w.cur_mask = 0;
+    int blk[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) blk[q] = unit_block[(size_t)h * NB + 4 * quad + q];
+    UnitWalk<4> w;
+    walk_init<4>(w, blk, 4, row_ptr, h * NB);
     if (lane == 0) {
       prefetch_tensormap(&mapQ);
       prefetch_tensormap(&mapK);
       prefetch_tensormap(&mapV);
-      mbar_arrive_expect_tx(&bar.q_full, L::Q_BYTES);
+      mbar_arrive_expect_tx(&bar.q_full, 2 * L::TILE);
 #pragma unroll
-      for (int c = 0; c < L::CHUNKS; ++c)
-        tma_load_2d(smem + L::OFF_Q + c * (BM * 128), &mapQ, &bar.q_full, c * 64, h * N + tile * BM);
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int c = 0; c < L::CHUNKS; ++c)
+          tma_load_2d(smem + L::OFF_Q + t * L::TILE + c * (128 * 128), &mapQ, &bar.q_full, c * 64,
+                      h * N + quad * BQ + t * 128);
     }
     for (int j = 0; j < ntiles; ++j) {
       const int s = j % NSTAGE;
       uint32_t ua, ub = 0;
       int ma, mb = 0, nu = 1;
-      walk_next(w, col, blocks_h, ua, ma);
+      walk_next<4>(w, col, blocks_h, ua, ma);
       if (2 * j + 2 <= nunits) {
-        walk_next(w, col, blocks_h, ub, mb);
+        walk_next<4>(w, col, blocks_h, ub, mb);
         nu = 2;
       }
       ua = min(ua, (uint32_t)(NB - 1));  // a well-formed walk never clamps
@@ -160,8 +168,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) bar.abort = 1;
         if (ok) {
           bar.meta[s] = nu | (ma << 4) | (mb << 8);
-          uint8_t *ks = smem + L::OFF_K + s * L::KV_BYTES;
-          uint8_t *vs = smem + L::OFF_V + s * L::KV_BYTES;
+          uint8_t *ks = smem + L::OFF_K + s * L::TILE;
+          uint8_t *vs = smem + L::OFF_V + s * L::TILE;
           const int bytes = nu * 64 * D * 2;
           mbar_arrive_expect_tx(&bar.k_full[s], bytes);
 #pragma unroll
@@ -186,83 +194,74 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_s_full = idesc_f16(128, 128, 0);
       const uint32_t idesc_s_half = idesc_f16(128, 64, 0);
       const uint32_t idesc_o = idesc_f16(128, D, 1);
-      const uint32_t sQ = smem_u32(smem + L::OFF_Q);
       bool ok = mbar_wait(&bar.q_full, 0, status, 2);
       tc_fence_after();
-      for (int j = 0; ok && j <= ntiles; ++j) {
-        if (j < ntiles) {
-          const int s = j % NSTAGE, b = j & 1;
-          ok = mbar_wait(&bar.k_full[s], (j / NSTAGE) & 1, status, 3);
-          if (ok && j >= 2) ok = mbar_wait(&bar.pv_done[b], ((j - 2) >> 1) & 1, status, 4);
+      for (int j = 0; ok && j < ntiles; ++j) {
+        const int s = j % NSTAGE;
+        ok = mbar_wait(&bar.k_full[s], (j / NSTAGE) & 1, status, 3);
+        if (!ok) break;
+        tc_fence_after();
+        const int nu = bar.meta[s] & 15;
+        const uint32_t sK = smem_u32(smem + L::OFF_K + s * L::TILE);
+        for (int t = 0; t < 2; ++t) {
+          // S_t is free once the PV of the previous key tile read its P
+          if (j >= 1) ok = mbar_wait(&bar.pv_done[t], (j - 1) & 1, status, 4);
           if (!ok) break;
           tc_fence_after();
-          const int nu = bar.meta[s] & 15;
-          const uint32_t sK = smem_u32(smem + L::OFF_K + s * L::KV_BYTES);
+          const uint32_t sQ = smem_u32(smem + L::OFF_Q + t * L::TILE);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-            const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(sK + off, 16, 1024);
-            mma_ss(tS[b], ad, bd, nu == 2 ? idesc_s_full : idesc_s_half, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + 128 * t, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024),
+                   nu == 2 ? idesc_s_full : idesc_s_half, kk > 0 ? 1u : 0u);
           }
-          mma_commit(&bar.s_full[b]);
+          mma_commit(&bar.s_full[t]);
         }
-        if (j >= 1) {
-          const int jj = j - 1, s = jj % NSTAGE, b = jj & 1;
-          ok = mbar_wait(&bar.p_full[b], (jj >> 1) & 1, status, 5);
-          if (ok) ok = mbar_wait(&bar.v_full[s], (jj / NSTAGE) & 1, status, 6);
+        if (!ok) break;
+        ok = mbar_wait(&bar.v_full[s], (j / NSTAGE) & 1, status, 6);
+        const uint32_t sV = smem_u32(smem + L::OFF_V + s * L::TILE);
+        for (int t = 0; ok && t < 2; ++t) {
+          ok = mbar_wait(&bar.p_full[t], j & 1, status, 5);
           if (!ok) break;
           tc_fence_after();
-          const int nu = bar.meta[s] & 15;
-          const uint32_t sV = smem_u32(smem + L::OFF_V + s * L::KV_BYTES);
-          for (int ks = 0; ks < nu * 4; ++ks) {
-            const uint64_t bd = sdesc_sw128(sV + ks * 2048, 128 * 128, 1024);
-            mma_ts(tO, tS[b] + ks * 8, bd, idesc_o, (jj > 0 || ks > 0) ? 1u : 0u);
-          }
-          mma_commit(&bar.pv_done[b]);
-          mma_commit(&bar.kv_empty[s]);
+          for (int ks = 0; ks < nu * 4; ++ks)
+            mma_ts(tmem + 256 + t * D, tmem + 128 * t + ks * 8, sdesc_sw128(sV + ks * 2048, 128 * 128, 1024),
+                   idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
+          mma_commit(&bar.pv_done[t]);
         }
+        mma_commit(&bar.kv_empty[s]);
       }
       if (!ok) bar.abort = 1;
     }
     __syncwarp();
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
+    const int t = (warp - 4) >> 2;  // query tile of this warpgroup
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
-    const int half = row >> 6;
+    const int qbit = 2 * t + (row >> 6);  // 64-row quarter of the CTA (warp-uniform)
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const uint32_t tS = tmem + 128 * t, tO = tmem + 256 + t * D;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
-      const int s = j % NSTAGE, b = j & 1;
-      ok = mbar_wait_warp(&bar.s_full[b], (j >> 1) & 1, status, 7);
+      const int s = j % NSTAGE;
+      ok = mbar_wait_warp(&bar.s_full[t], j & 1, status, 7);
       if (!ok) break;
       tc_fence_after();
       const int meta = bar.meta[s];
       const int nu = meta & 15;
-      const bool ok0 = ((meta >> 4) >> half) & 1;
-      const bool ok1 = nu == 2 && (((meta >> 8) >> half) & 1);
-      uint32_t r[4][32];
-      tmem_ld32(tS[b] + lane_off + 0, r[0]);
-      tmem_ld32(tS[b] + lane_off + 32, r[1]);
-      if (nu == 2) {
-        tmem_ld32(tS[b] + lane_off + 64, r[2]);
-        tmem_ld32(tS[b] + lane_off + 96, r[3]);
-      }
-      tmem_wait_ld();
+      const bool v0 = ((meta >> 4) >> qbit) & 1;
+      const bool v1 = nu == 2 && (((meta >> 8) >> qbit) & 1);
+      // pass 1: maximum over the valid columns of this row
       float mt = -INFINITY;
-      if (ok0) {
+      for (int c = 0; c < 2 * nu; ++c) {
+        if (!((c < 2) ? v0 : v1)) continue;  // warp-uniform
+        uint32_t r[32];
+        tmem_ld32(tS + lane_off + c * 32, r);
+        tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 2; ++q)
-#pragma unroll
-          for (int i = 0; i < 32; ++i) mt = fmaxf(mt, __uint_as_float(r[q][i]));
-      }
-      if (ok1) {
-#pragma unroll
-        for (int q = 2; q < 4; ++q)
-#pragma unroll
-          for (int i = 0; i < 32; ++i) mt = fmaxf(mt, __uint_as_float(r[q][i]));
+        for (int i = 0; i < 32; i += 2) mt = fmaxf(mt, fmaxf(__uint_as_float(r[i]), __uint_as_float(r[i + 1])));
       }
       mt *= scale_log2;
       // A row takes a new reference maximum only when it grows by more than
@@ -272,9 +271,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool want = mt > m + kRescaleLog2 || (m == -INFINITY && mt > -INFINITY);
       if (__any_sync(0xffffffffu, want)) {
         const float m_new = want ? mt : m;
-        const float alpha = (m == -INFINITY) ? 0.f : exp2f(m - m_new);
+        const float alpha = (m == -INFINITY) ? 0.f : ex2f(m - m_new);
         if (j > 0 && __any_sync(0xffffffffu, want && m != -INFINITY)) {
-          ok = mbar_wait_warp(&bar.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, status, 8);
+          ok = mbar_wait_warp(&bar.pv_done[t], (j - 1) & 1, status, 8);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll 1
@@ -291,36 +290,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         l *= alpha;
         m = m_new;
       }
-      // P = exp2(s * scale_log2 - m), fp16, packed two keys per column
-      uint32_t pk[64];
-      float ls = 0.f;
+      // pass 2: P = exp2(s * scale_log2 - m) in fp16, two keys per column
+      float2 ls = make_float2(0.f, 0.f);
+      for (int c = 0; c < 2 * nu; ++c) {
+        uint32_t pk[16];
+        if ((c < 2) ? v0 : v1) {
+          uint32_t r[32];
+          tmem_ld32(tS + lane_off + c * 32, r);
+          tmem_wait_ld();
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const bool valid = (q < 2) ? ok0 : ok1;
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float p0 = 0.f, p1 = 0.f;
-          if (valid) {
-            p0 = exp2f(fmaf(__uint_as_float(r[q][i]), scale_log2, -m));
-            p1 = exp2f(fmaf(__uint_as_float(r[q][i + 1]), scale_log2, -m));
+          for (int i = 0; i < 32; i += 2) {
+            float2 x = ffma2(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), scale_log2, -m);
+            float2 p = make_float2(ex2f(x.x), ex2f(x.y));
+            ls = fadd2(ls, p);
+            pk[i / 2] = pack_f16(p.x, p.y);
           }
-          ls += p0 + p1;
-          pk[q * 16 + i / 2] = pack_f16(p0, p1);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = 0u;
         }
+        tmem_st16(tS + lane_off + c * 16, pk);
       }
-      l += ls;
-      tmem_st32(tS[b] + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      if (nu == 2) tmem_st32(tS[b] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      l += ls.x + ls.y;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar.p_full[b]);
+      mbar_arrive(&bar.p_full[t]);
     }
     // epilogue
     ok = __all_sync(0xffffffffu, ok);
-    if (ok && ntiles > 0) ok = mbar_wait_warp(&bar.pv_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, status, 9);
+    if (ok && ntiles > 0) ok = mbar_wait_warp(&bar.pv_done[t], (ntiles - 1) & 1, status, 9);
     if (ok) {
       tc_fence_after();
-      const int p = tile * BM + row;
+      const int p = quad * BQ + t * 128 + row;
       const int n = perm[(size_t)h * N + p];
       const float inv = (l > 0.f) ? 1.0f / l : 0.f;
       uint16_t *dst = O + ((size_t)n * heads + h) * D;
@@ -379,34 +380,50 @@ __global__ void unit_block_kernel(const int32_t *__restrict__ blocks, const int3
   for (int k = 0; k < nu; ++k) unit_block[(size_t)h * NB + u0 + k] = b;
 }
 
-// tile_units[h][t] = key units walked by query tile t (union of the two row
-// lists when the tile holds two 64-token blocks).  One warp per tile.
-__global__ void tile_units_kernel(const int32_t *__restrict__ row_ptr, const int32_t *__restrict__ col,
+// tile_units[h][t] = 64-token units walked by tile t (UPT units) over the
+// union of the rows of its distinct blocks (CSR rows for query tiles, CSC
+// rows for key tiles).  One warp per tile.
+template <int UPT>
+__global__ void tile_units_kernel(const int32_t *__restrict__ ptr, const int32_t *__restrict__ idx,
                                   const int32_t *__restrict__ blocks, const int32_t *__restrict__ unit_block, int N,
                                   int heads, int32_t *__restrict__ tile_units) {
-  const int NB = N / 64, NT = N / BM;
+  const int NB = N / 64, NT = N / (64 * UPT);
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (gw >= NT * heads) return;
   const int h = gw / NT, t = gw % NT;
   const int32_t *blocks_h = blocks + (size_t)h * NB * 4;
-  const int b0 = unit_block[(size_t)h * NB + 2 * t], b1 = unit_block[(size_t)h * NB + 2 * t + 1];
-  const int s0 = row_ptr[h * NB + b0], e0 = row_ptr[h * NB + b0 + 1];
+  int b[UPT];
+#pragma unroll
+  for (int q = 0; q < UPT; ++q) b[q] = unit_block[(size_t)h * NB + UPT * t + q];
   long long cnt = 0;
-  for (int q = s0 + lane; q < e0; q += 32) cnt += blocks_h[(size_t)col[q] * 4 + 1] >> 6;
-  if (b1 != b0) {
-    const int s1 = row_ptr[h * NB + b1], e1 = row_ptr[h * NB + b1 + 1];
-    for (int q = s1 + lane; q < e1; q += 32) {
-      const int j = col[q];
-      int lo = s0, hi = e0;  // binary search j in the first list
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (col[mid] < j)
-          lo = mid + 1;
-        else
-          hi = mid;
+#pragma unroll
+  for (int q = 0; q < UPT; ++q) {
+    bool dup = false;
+#pragma unroll
+    for (int r = 0; r < q; ++r) dup |= (b[r] == b[q]);
+    if (dup) continue;
+    const int s = ptr[h * NB + b[q]], e = ptr[h * NB + b[q] + 1];
+    for (int k = s + lane; k < e; k += 32) {
+      const int j = idx[k];
+      bool seen = false;  // already counted through an earlier distinct block's row
+#pragma unroll
+      for (int r = 0; r < q; ++r) {
+        bool first = true;
+#pragma unroll
+        for (int u = 0; u < r; ++u) first &= (b[u] != b[r]);
+        if (!first || seen) continue;
+        int lo = ptr[h * NB + b[r]], hi = ptr[h * NB + b[r] + 1];
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (idx[mid] < j)
+            lo = mid + 1;
+          else
+            hi = mid;
+        }
+        seen = lo < ptr[h * NB + b[r] + 1] && idx[lo] == j;
       }
-      if (!(lo < e0 && col[lo] == j)) cnt += blocks_h[(size_t)j * 4 + 1] >> 6;
+      if (!seen) cnt += blocks_h[(size_t)j * 4 + 1] >> 6;
     }
   }
   cnt = warp_sum(cnt);
@@ -460,10 +477,15 @@ cudaError_t launch_unit_block(const int32_t *blocks, const int32_t *n_blocks, in
 }
 
 cudaError_t launch_tile_units(const int32_t *ptr, const int32_t *idx, const int32_t *blocks,
-                              const int32_t *unit_block, int N, int heads, int32_t *tile_units, cudaStream_t st) {
-  const int warps = (N / 128) * heads;
-  fwd::tile_units_kernel<<<(warps * 32 + 255) / 256, 256, 0, st>>>(ptr, idx, blocks, unit_block, N, heads,
-                                                                   tile_units);
+                              const int32_t *unit_block, int N, int heads, int units_per_tile, int32_t *tile_units,
+                              cudaStream_t st) {
+  const int warps = (N / (64 * units_per_tile)) * heads;
+  if (units_per_tile == 4)
+    fwd::tile_units_kernel<4><<<(warps * 32 + 255) / 256, 256, 0, st>>>(ptr, idx, blocks, unit_block, N, heads,
+                                                                        tile_units);
+  else
+    fwd::tile_units_kernel<2><<<(warps * 32 + 255) / 256, 256, 0, st>>>(ptr, idx, blocks, unit_block, N, heads,
+                                                                        tile_units);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -531,7 +553,7 @@ static FwdWs carve_fwd(const prism_params &p, void *ws) {
 size_t attn_fwd_ws_bytes(const prism_params &p) {
   const size_t N = (size_t)p.T * p.H * p.W, h = p.heads, D = p.head_dim;
   return kWsHeader + 3 * align_up(sizeof(uint16_t) * h * N * D, 256) + align_up(sizeof(int32_t) * h * (N / 64), 256) +
-         align_up(sizeof(int32_t) * h * (N / 128), 256);
+         align_up(sizeof(int32_t) * h * (N / 256), 256);
 }
 
 template <int D>
@@ -546,7 +568,7 @@ static cudaError_t run_fwd(const prism_params &p, const prism_plan_t &plan, cons
   const int smem = fwd::Smem<D>::BYTES + 1024;
   cudaFuncSetAttribute(fwd::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   const float scale_log2 = effective_scale(p) * 1.4426950408889634f;
-  dim3 grid(N / fwd::BM, p.heads);
+  dim3 grid(N / fwd::BQ, p.heads);
   fwd::attn_fwd_kernel<D><<<grid, fwd::kThreads, smem, st>>>(mQ, mK, mV, sel.row_ptr, sel.col, plan.blocks,
                                                              w.unit_block, w.tile_units, plan.perm, O, O_res, lse,
                                                              N, p.heads, scale_log2, &w.hdr->status);
@@ -564,7 +586,7 @@ cudaError_t launch_attn_fwd(const prism_params &p, const prism_plan_t &plan, con
       cudaSuccess)
     return e;
   if ((e = launch_unit_block(plan.blocks, plan.n_blocks, NB, p.heads, w.unit_block, st)) != cudaSuccess) return e;
-  if ((e = launch_tile_units(sel.row_ptr, sel.col, plan.blocks, w.unit_block, N, p.heads, w.tile_units, st)) !=
+  if ((e = launch_tile_units(sel.row_ptr, sel.col, plan.blocks, w.unit_block, N, p.heads, 4, w.tile_units, st)) !=
       cudaSuccess)
     return e;
   return D == 128 ? run_fwd<128>(p, plan, sel, w, O, O_res, lse, st) : run_fwd<64>(p, plan, sel, w, O, O_res, lse, st);

@@ -37,37 +37,71 @@ __device__ __forceinline__ uint32_t cursor_peek(Cursor &c, const int32_t *__rest
   return __shfl_sync(0xffffffffu, c.reg, c.pos - c.base);
 }
 
+// Merge of up to NL sorted rows (the distinct blocks of a query or key tile)
+// into one ascending stream of 64-token units.  Each unit carries a mask:
+// bit q is set when the block of the tile's q-th 64-row quarter selected it.
+template <int NL>
 struct UnitWalk {
-  Cursor a, b;
-  int mask_a, mask_b;
+  Cursor c[NL];
+  int mask[NL];
   uint32_t cur_ub;
   int cur_cnt, cur_k, cur_mask;
 };
-__device__ __forceinline__ void walk_next(UnitWalk &w, const int32_t *__restrict__ col,
+
+// Set up the walk for a tile made of `nq` units whose blocks are blk[0..nq):
+// slot q holds the row of quarter q's block unless an earlier quarter has
+// the same block (then the slot stays empty and that quarter's bit is added
+// to the earlier slot's mask).  All indices are compile-time after unrolling.
+template <int NL>
+__device__ __forceinline__ void walk_init(UnitWalk<NL> &w, const int (&blk)[NL], int nq,
+                                          const int32_t *__restrict__ ptr, int row0) {
+#pragma unroll
+  for (int q = 0; q < NL; ++q) {
+    bool dup = false;
+#pragma unroll
+    for (int r = 0; r < q; ++r) dup |= (blk[r] == blk[q]);
+    const bool live = q < nq && !dup;
+    if (live)
+      cursor_init(w.c[q], ptr[row0 + blk[q]], ptr[row0 + blk[q] + 1]);
+    else
+      cursor_init(w.c[q], 0, 0);
+    int m = 0;
+#pragma unroll
+    for (int r = q; r < NL; ++r)
+      if (r < nq && blk[r] == blk[q]) m |= 1 << r;
+    w.mask[q] = live ? m : 0;
+  }
+  w.cur_cnt = 0;
+  w.cur_k = 0;
+  w.cur_ub = 0;
+  w.cur_mask = 0;
+}
+
+template <int NL>
+__device__ __forceinline__ void walk_next(UnitWalk<NL> &w, const int32_t *__restrict__ col,
                                           const int32_t *__restrict__ blocks_h, uint32_t &unit, int &mask) {
   if (w.cur_k >= w.cur_cnt) {
-    const uint32_t ea = cursor_peek(w.a, col, blocks_h);
-    const uint32_t eb = cursor_peek(w.b, col, blocks_h);
-    const uint32_t ka = ea == kEnd ? kEnd : (ea & 0x0fffffffu);
-    const uint32_t kb = eb == kEnd ? kEnd : (eb & 0x0fffffffu);
-    uint32_t e;
-    if (ka < kb) {
-      e = ea;
-      w.cur_mask = w.mask_a;
-      ++w.a.pos;
-    } else if (kb < ka) {
-      e = eb;
-      w.cur_mask = w.mask_b;
-      ++w.b.pos;
-    } else {
-      e = ea;
-      w.cur_mask = w.mask_a | w.mask_b;
-      ++w.a.pos;
-      ++w.b.pos;
+    uint32_t e[NL], key[NL];
+    uint32_t kmin = kEnd;
+#pragma unroll
+    for (int r = 0; r < NL; ++r) {
+      e[r] = cursor_peek(w.c[r], col, blocks_h);
+      key[r] = e[r] == kEnd ? kEnd : (e[r] & 0x0fffffffu);
+      kmin = min(kmin, key[r]);
     }
-    w.cur_ub = e & 0x0fffffffu;
-    w.cur_cnt = (int)(e >> 28) + 1;
+    uint32_t ent = kEnd;
+    int m = 0;
+#pragma unroll
+    for (int r = 0; r < NL; ++r)
+      if (key[r] == kmin && kmin != kEnd) {
+        ent = e[r];
+        m |= w.mask[r];
+        ++w.c[r].pos;
+      }
+    w.cur_ub = ent & 0x0fffffffu;
+    w.cur_cnt = (int)(ent >> 28) + 1;
     w.cur_k = 0;
+    w.cur_mask = m;
   }
   unit = w.cur_ub + (uint32_t)w.cur_k;
   mask = w.cur_mask;

@@ -46,10 +46,12 @@ float effective_scale(const prism_params &p);
 // attention pre-passes (attn_fwd.cu), shared by the backward
 cudaError_t launch_unit_block(const int32_t *blocks, const int32_t *n_blocks, int NB, int heads,
                               int32_t *unit_block, cudaStream_t st);
-// tile_units[h][t]: 64-token units walked by 128-token tile t over the rows
-// (ptr, idx) of its one or two blocks (CSR for query tiles, CSC for key tiles).
+// tile_units[h][t]: 64-token units walked by tile t (units_per_tile = 2 or 4
+// units) over the union of the rows (ptr, idx) of its distinct blocks (CSR
+// for query tiles, CSC for key tiles).
 cudaError_t launch_tile_units(const int32_t *ptr, const int32_t *idx, const int32_t *blocks,
-                              const int32_t *unit_block, int N, int heads, int32_t *tile_units, cudaStream_t st);
+                              const int32_t *unit_block, int N, int heads, int units_per_tile, int32_t *tile_units,
+                              cudaStream_t st);
 // 2-D fp16 tensor map over rows of D elements, box 64 x box_rows, 128B swizzle.
 cudaError_t make_rows_map(CUtensorMap *map, const void *base, long long rows, int D, int box_rows);
 

@@ -74,6 +74,10 @@ WORKLOADS = {
                           regions=2, radius=4, a_regions=1),
     "720p": Workload("720p", 24, 48, 80, 24, 128, topk_frac=0.08, top_p=0.9,
                      regions=3, radius=6, a_regions=2),
+    # 720p grid with 8 heads: every tensor (189 MB) exceeds L2, a few GB in
+    # total -- sized for kernel profiling
+    "720p_h8": Workload("720p_h8", 24, 48, 80, 8, 128, topk_frac=0.08, top_p=0.9,
+                        regions=3, radius=6, a_regions=2),
     "1080p": Workload("1080p", 32, 72, 120, 24, 128, topk_frac=0.06, top_p=0.9,
                       regions=6, radius=8, a_regions=3, static_frac=0.3),
     "2k": Workload("2k", 56, 96, 160, 24, 128, topk_frac=0.04, top_p=0.9,

@@ -17,16 +17,17 @@
 //                S^T = K Q^T, dP^T = V dO^T (TMEM), P^T and dS^T -> TMEM
 //                (fp16), dV += P^T dO, dK += dS^T Q (TS MMAs).
 // Operands are fp16 (exact conversions of the bf16 inputs, see the forward).
-// Roles as in the forward: warp 0 TMA producer, warp 1 TMEM owner and MMA
-// issuer, warps 2-5 one thread per TMEM lane (row).
+// Roles: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer, warps 4-11
+// two compute warpgroups (one thread per TMEM lane) taking alternate steps of
+// one 64-token unit; each step has its own TMEM buffers, so the compute of a
+// step overlaps the MMAs of the next.
 #include "attn_walk.cuh"
 
 namespace prism {
 namespace bwd {
 using namespace attn;
 
-constexpr int NSTAGE = 2;
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 4-11 two compute warpgroups
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -75,30 +76,12 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const int32_t *__restrict
 }
 
 // ---------------------------------------------------------------------------
-// dQ kernel
+// Shared pieces of the two kernels.  Both walk 64-token units of the
+// streamed side, one unit per step; two compute warpgroups take alternate
+// steps, each with its own TMEM buffer pair, so the compute of step i
+// overlaps the MMAs of step i+1.
 // ---------------------------------------------------------------------------
-template <int D>
-struct DqSmem {
-  static constexpr int CHUNKS = D / 64;
-  static constexpr int TILE = 128 * D * 2;  // 128 rows of bf16
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_DO = OFF_Q + TILE;
-  static constexpr int OFF_K = OFF_DO + TILE;
-  static constexpr int OFF_V = OFF_K + NSTAGE * TILE;
-  static constexpr int OFF_BAR = OFF_V + NSTAGE * TILE;
-  static constexpr int BYTES = OFF_BAR + 256;
-};
-
-struct DqBars {
-  uint64_t qdo_full;
-  uint64_t k_full[NSTAGE];
-  uint64_t v_full[NSTAGE];
-  uint64_t kv_empty[NSTAGE];
-  uint64_t s_full, dp_full, ds_ready, dq_done;
-  int meta[NSTAGE];
-  uint32_t tmem_base;
-  int ntiles, nunits, abort;
-};
+constexpr int NS = 4;  // ring depth (steps of one 64-token unit)
 
 template <int D>
 __device__ __forceinline__ void store_row(void *out, bool fp32, size_t off, const uint32_t (&o)[32], float mul) {
@@ -118,6 +101,34 @@ __device__ __forceinline__ void store_row(void *out, bool fp32, size_t off, cons
     for (int i = 0; i < 4; ++i) dst[i] = v[i];
   }
 }
+
+// ---------------------------------------------------------------------------
+// dQ kernel: one CTA per 128-query tile; steps over the key units of the
+// union of its rows' selections.
+//   TMEM: dQ [0, D); step buffer b: S at 128+128b, dP (then dS) at 192+128b.
+// ---------------------------------------------------------------------------
+template <int D>
+struct DqSmem {
+  static constexpr int CHUNKS = D / 64;
+  static constexpr int TILE = 128 * D * 2;  // 128 rows of fp16
+  static constexpr int UNIT = 64 * D * 2;   // 64 rows
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_DO = OFF_Q + TILE;
+  static constexpr int OFF_K = OFF_DO + TILE;
+  static constexpr int OFF_V = OFF_K + NS * UNIT;
+  static constexpr int OFF_BAR = OFF_V + NS * UNIT;
+  static constexpr int BYTES = OFF_BAR + 256;
+};
+
+struct DqBars {
+  uint64_t qdo_full;
+  uint64_t k_full[NS], v_full[NS], kv_empty[NS];
+  uint64_t s_full[2], dp_full[2], ds_ready[2], dq_done[2];
+  uint64_t fin;  // single use: every MMA of the tile has completed
+  int mask[NS];
+  uint32_t tmem_base;
+  int nsteps, abort;
+};
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -142,17 +153,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (bar.abort) return;
   if (threadIdx.x == 0) {
     mbar_init(&bar.qdo_full, 1);
-    for (int s = 0; s < NSTAGE; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&bar.k_full[s], 1);
       mbar_init(&bar.v_full[s], 1);
       mbar_init(&bar.kv_empty[s], 1);
     }
-    mbar_init(&bar.s_full, 1);
-    mbar_init(&bar.dp_full, 1);
-    mbar_init(&bar.ds_ready, 128);
-    mbar_init(&bar.dq_done, 1);
-    bar.nunits = tile_units[(size_t)h * (N / 128) + tile];
-    bar.ntiles = (bar.nunits + 1) >> 1;
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bar.s_full[b], 1);
+      mbar_init(&bar.dp_full[b], 1);
+      mbar_init(&bar.ds_ready[b], 128);
+      mbar_init(&bar.dq_done[b], 1);
+    }
+    mbar_init(&bar.fin, 1);
+    bar.nsteps = tile_units[(size_t)h * (N / 128) + tile];
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -163,8 +176,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bar.tmem_base;
-  const int ntiles = bar.ntiles, nunits = bar.nunits;
-  const uint32_t tS = tmem, tP = tmem + 128, tQ = tmem + 256;
+  const int nsteps = bar.nsteps;
+  const uint32_t tQ = tmem;
 
   if (warp == 0) {
     const int blk[2] = {unit_block[(size_t)h * NB + 2 * tile], unit_block[(size_t)h * NB + 2 * tile + 1]};
@@ -178,38 +191,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(smem + L::OFF_DO + c * (128 * 128), &mapDO, &bar.qdo_full, c * 64, h * N + tile * 128);
       }
     }
-    for (int j = 0; j < ntiles; ++j) {
-      const int s = j % NSTAGE;
-      uint32_t ua, ub = 0;
-      int ma, mb = 0, nu = 1;
-      walk_next<2>(w, col, blocks_h, ua, ma);
-      if (2 * j + 2 <= nunits) {
-        walk_next<2>(w, col, blocks_h, ub, mb);
-        nu = 2;
-      }
-      ua = min(ua, (uint32_t)(NB - 1));
-      ub = min(ub, (uint32_t)(NB - 1));
+    for (int j = 0; j < nsteps; ++j) {
+      const int s = j % NS;
+      uint32_t u;
+      int m;
+      walk_next<2>(w, col, blocks_h, u, m);
+      u = min(u, (uint32_t)(NB - 1));  // a well-formed walk never clamps
       if (lane == 0) {
         bool ok = true;
-        if (j >= NSTAGE) ok = mbar_wait(&bar.kv_empty[s], ((j / NSTAGE) - 1) & 1, status, 21);
+        if (j >= NS) ok = mbar_wait(&bar.kv_empty[s], ((j / NS) - 1) & 1, status, 21);
         if (!ok) bar.abort = 1;
         if (ok) {
-          bar.meta[s] = nu | (ma << 4) | (mb << 8);
-          uint8_t *ks = smem + L::OFF_K + s * L::TILE;
-          uint8_t *vs = smem + L::OFF_V + s * L::TILE;
-          const int bytes = nu * 64 * D * 2;
-          mbar_arrive_expect_tx(&bar.k_full[s], bytes);
+          bar.mask[s] = m;
+          mbar_arrive_expect_tx(&bar.k_full[s], L::UNIT);
 #pragma unroll
-          for (int c = 0; c < L::CHUNKS; ++c) {
-            tma_load_2d(ks + c * (128 * 128), &mapK, &bar.k_full[s], c * 64, h * N + (int)ua * 64);
-            if (nu == 2) tma_load_2d(ks + c * (128 * 128) + 64 * 128, &mapK, &bar.k_full[s], c * 64, h * N + (int)ub * 64);
-          }
-          mbar_arrive_expect_tx(&bar.v_full[s], bytes);
+          for (int c = 0; c < L::CHUNKS; ++c)
+            tma_load_2d(smem + L::OFF_K + s * L::UNIT + c * (64 * 128), &mapK, &bar.k_full[s], c * 64,
+                        h * N + (int)u * 64);
+          mbar_arrive_expect_tx(&bar.v_full[s], L::UNIT);
 #pragma unroll
-          for (int c = 0; c < L::CHUNKS; ++c) {
-            tma_load_2d(vs + c * (128 * 128), &mapV, &bar.v_full[s], c * 64, h * N + (int)ua * 64);
-            if (nu == 2) tma_load_2d(vs + c * (128 * 128) + 64 * 128, &mapV, &bar.v_full[s], c * 64, h * N + (int)ub * 64);
-          }
+          for (int c = 0; c < L::CHUNKS; ++c)
+            tma_load_2d(smem + L::OFF_V + s * L::UNIT + c * (64 * 128), &mapV, &bar.v_full[s], c * 64,
+                        h * N + (int)u * 64);
         }
       }
       __syncwarp();
@@ -217,110 +220,113 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t id_full = idesc_f16(128, 128, 0), id_half = idesc_f16(128, 64, 0);
-      const uint32_t id_dq = idesc_f16(128, D, 1);
+      const uint32_t id64 = idesc_f16(128, 64, 0), id_dq = idesc_f16(128, D, 1);
       const uint32_t sQ = smem_u32(smem + L::OFF_Q), sDO = smem_u32(smem + L::OFF_DO);
       bool ok = mbar_wait(&bar.qdo_full, 0, status, 22);
       tc_fence_after();
-      for (int j = 0; ok && j <= ntiles; ++j) {
-        if (j >= 1) {  // dQ += dS_{j-1} K_{j-1}
-          const int jj = j - 1, s = jj % NSTAGE;
-          ok = mbar_wait(&bar.ds_ready, jj & 1, status, 23);
+      for (int i = 0; ok && i <= nsteps; ++i) {
+        if (i < nsteps) {  // S_i = Q K_i^T, dP_i = dO V_i^T into buffer i&1
+          const int s = i % NS, b = i & 1;
+          const uint32_t tS = tmem + 128 + 128 * b, tP = tS + 64;
+          ok = mbar_wait(&bar.k_full[s], (i / NS) & 1, status, 24);
           if (!ok) break;
           tc_fence_after();
-          const int nu = bar.meta[s] & 15;
-          const uint32_t sK = smem_u32(smem + L::OFF_K + s * L::TILE);
-          for (int ks = 0; ks < nu * 4; ++ks)
-            mma_ts(tQ, tP + ks * 8, sdesc_sw128(sK + ks * 2048, 128 * 128, 1024), id_dq,
-                   (jj > 0 || ks > 0) ? 1u : 0u);
-          mma_commit(&bar.dq_done);
+          const uint32_t sK = smem_u32(smem + L::OFF_K + s * L::UNIT);
+          const uint32_t sV = smem_u32(smem + L::OFF_V + s * L::UNIT);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tS, sdesc_sw128(sQ + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024),
+                   sdesc_sw128(sK + (kk >> 2) * (64 * 128) + (kk & 3) * 32, 16, 1024), id64, kk > 0 ? 1u : 0u);
+          mma_commit(&bar.s_full[b]);
+          ok = mbar_wait(&bar.v_full[s], (i / NS) & 1, status, 25);
+          if (ok && i >= 2) ok = mbar_wait(&bar.dq_done[b], ((i - 2) >> 1) & 1, status, 26);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tP, sdesc_sw128(sDO + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024),
+                   sdesc_sw128(sV + (kk >> 2) * (64 * 128) + (kk & 3) * 32, 16, 1024), id64, kk > 0 ? 1u : 0u);
+          mma_commit(&bar.dp_full[b]);
+        }
+        if (i >= 1) {  // dQ += dS_{i-1} K_{i-1}
+          const int jj = i - 1, s = jj % NS, b = jj & 1;
+          const uint32_t tP = tmem + 192 + 128 * b;
+          ok = mbar_wait(&bar.ds_ready[b], (jj >> 1) & 1, status, 23);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t sK = smem_u32(smem + L::OFF_K + s * L::UNIT);
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_ts(tQ, tP + ks * 8, sdesc_sw128(sK + ks * 2048, 64 * 128, 1024), id_dq, (jj > 0 || ks > 0) ? 1u : 0u);
+          mma_commit(&bar.dq_done[b]);
           mma_commit(&bar.kv_empty[s]);
         }
-        if (j < ntiles) {
-          const int s = j % NSTAGE;
-          ok = mbar_wait(&bar.k_full[s], (j / NSTAGE) & 1, status, 24);
-          if (!ok) break;
-          tc_fence_after();
-          const int nu = bar.meta[s] & 15;
-          const uint32_t id = nu == 2 ? id_full : id_half;
-          const uint32_t sK = smem_u32(smem + L::OFF_K + s * L::TILE);
-          const uint32_t sV = smem_u32(smem + L::OFF_V + s * L::TILE);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-            mma_ss(tS, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), id, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&bar.s_full);
-          ok = mbar_wait(&bar.v_full[s], (j / NSTAGE) & 1, status, 25);
-          if (ok && j >= 1) ok = mbar_wait(&bar.dq_done, (j - 1) & 1, status, 26);
-          if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-            mma_ss(tP, sdesc_sw128(sDO + off, 16, 1024), sdesc_sw128(sV + off, 16, 1024), id, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&bar.dp_full);
-        }
       }
+      if (ok && nsteps > 0) mma_commit(&bar.fin);
       if (!ok) bar.abort = 1;
     }
     __syncwarp();
-  } else {
+  } else if (warp >= 4) {
+    const int g = (warp - 4) >> 2;  // warpgroup: steps with i % 2 == g
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
-    const int half = row >> 6;
+    const int half = row >> 6;  // warp-uniform
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const size_t prow = (size_t)h * N + (size_t)tile * 128 + row;
     const float lse2 = lse2p[prow], dl = deltap[prow];
+    const uint32_t tS = tmem + 128 + 128 * g, tP = tS + 64;
     bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
-      const int s = j % NSTAGE;
-      ok = mbar_wait_warp(&bar.s_full, j & 1, status, 27);
-      if (ok) ok = mbar_wait_warp(&bar.dp_full, j & 1, status, 28);
+    for (int i = g; i < nsteps; i += 2) {
+      const int ph = (i >> 1) & 1;
+      ok = mbar_wait_warp(&bar.s_full[g], ph, status, 27);
+      if (ok) ok = mbar_wait_warp(&bar.dp_full[g], ph, status, 28);
       if (!ok) break;
       tc_fence_after();
-      const int meta = bar.meta[s];
-      const int nu = meta & 15;
-      for (int c = 0; c < 2 * nu; ++c) {
-        const int m = (c < 2) ? (meta >> 4) : (meta >> 8);
-        const bool valid = (m >> half) & 1;
-        uint32_t sv[32], dv[32], pk[16];
-        tmem_ld32(tS + lane_off + c * 32, sv);
-        tmem_ld32(tP + lane_off + c * 32, dv);
-        tmem_wait_ld();
+      const bool valid = (bar.mask[i % NS] >> half) & 1;
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float d0 = 0.f, d1 = 0.f;
-          if (valid) {
-            const float p0 = exp2f(fmaf(__uint_as_float(sv[i]), scale_log2, -lse2));
-            const float p1 = exp2f(fmaf(__uint_as_float(sv[i + 1]), scale_log2, -lse2));
-            d0 = p0 * (__uint_as_float(dv[i]) - dl);
-            d1 = p1 * (__uint_as_float(dv[i + 1]) - dl);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[16];
+        if (valid) {
+          uint32_t sv[32], dv[32];
+          tmem_ld32(tS + lane_off + c * 32, sv);
+          tmem_ld32(tP + lane_off + c * 32, dv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; k += 2) {
+            const float2 x = ffma2(make_float2(__uint_as_float(sv[k]), __uint_as_float(sv[k + 1])), scale_log2, -lse2);
+            const float2 p = make_float2(ex2f(x.x), ex2f(x.y));
+            const float2 d = fmul2(p, fsub2(make_float2(__uint_as_float(dv[k]), __uint_as_float(dv[k + 1])),
+                                            make_float2(dl, dl)));
+            pk[k / 2] = pack_f16(d.x, d.y);
           }
-          pk[i / 2] = pack_f16(d0, d1);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) pk[k] = 0u;
         }
         tmem_st16(tP + lane_off + c * 16, pk);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar.ds_ready);
+      mbar_arrive(&bar.ds_ready[g]);
     }
+    // A parity wait on dq_done could match an older phase for the warpgroup
+    // that did not run the step before the last; the single-use barrier
+    // cannot.
     ok = __all_sync(0xffffffffu, ok);
-    if (ok && ntiles > 0) ok = mbar_wait_warp(&bar.dq_done, (ntiles - 1) & 1, status, 29);
+    if (ok && nsteps > 0) ok = mbar_wait_warp(&bar.fin, 0, status, 29);
     if (ok) {
       tc_fence_after();
       const int n = perm[prow];
       const size_t off = ((size_t)n * heads + h) * D;
 #pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
+      for (int c = g * (D / 2); c < (g + 1) * (D / 2); c += 32) {
         uint32_t o[32];
-        if (ntiles > 0) {
+        if (nsteps > 0) {
           tmem_ld32(tQ + lane_off + c, o);
           tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0u;
+          for (int k = 0; k < 32; ++k) o[k] = 0u;
         }
         store_row<D>(dQ, grad_fp32 != 0, off + c, o, sm_scale);
       }
@@ -337,29 +343,33 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// dK/dV kernel
+// dK/dV kernel: one CTA per 128-key tile; steps over the query units of the
+// union of its blocks' columns (the transpose of the selection).
+//   TMEM: dV [0, D), dK [128, 128+D); step buffer b: S^T (then P^T) at
+//   256+128b, dP^T (then dS^T) at 320+128b.
 // ---------------------------------------------------------------------------
 template <int D>
 struct KvSmem {
   static constexpr int CHUNKS = D / 64;
   static constexpr int TILE = 128 * D * 2;
+  static constexpr int UNIT = 64 * D * 2;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + TILE;
-  static constexpr int OFF_Q = OFF_V + TILE;                 // ring of query tiles
-  static constexpr int OFF_DO = OFF_Q + NSTAGE * TILE;       // ring of dO tiles
-  static constexpr int OFF_STAT = OFF_DO + NSTAGE * TILE;    // [NSTAGE][2][128] floats: lse2, delta
-  static constexpr int OFF_BAR = OFF_STAT + NSTAGE * 2 * 128 * 4;
+  static constexpr int OFF_Q = OFF_V + TILE;                // ring of query units
+  static constexpr int OFF_DO = OFF_Q + NS * UNIT;          // ring of dO units
+  static constexpr int OFF_STAT = OFF_DO + NS * UNIT;       // [NS][2][64] floats: lse2, delta
+  static constexpr int OFF_BAR = OFF_STAT + NS * 2 * 64 * 4;
   static constexpr int BYTES = OFF_BAR + 256;
 };
 
 struct KvBars {
   uint64_t kv_full;
-  uint64_t q_full[NSTAGE];
-  uint64_t q_empty[NSTAGE];
-  uint64_t s_full, dp_full, ds_ready, mm_done;
-  int meta[NSTAGE];
+  uint64_t q_full[NS], q_empty[NS];
+  uint64_t s_full[2], dp_full[2], ds_ready[2], dv_done[2], dk_done[2];
+  uint64_t fin;  // single use: every MMA of the tile has completed
+  int mask[NS];
   uint32_t tmem_base;
-  int ntiles, nunits, abort;
+  int nsteps, abort;
 };
 
 template <int D>
@@ -387,16 +397,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (bar.abort) return;
   if (threadIdx.x == 0) {
     mbar_init(&bar.kv_full, 1);
-    for (int s = 0; s < NSTAGE; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&bar.q_full[s], 1);
       mbar_init(&bar.q_empty[s], 1);
     }
-    mbar_init(&bar.s_full, 1);
-    mbar_init(&bar.dp_full, 1);
-    mbar_init(&bar.ds_ready, 128);
-    mbar_init(&bar.mm_done, 1);
-    bar.nunits = tile_units[(size_t)h * (N / 128) + tile];
-    bar.ntiles = (bar.nunits + 1) >> 1;
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bar.s_full[b], 1);
+      mbar_init(&bar.dp_full[b], 1);
+      mbar_init(&bar.ds_ready[b], 128);
+      mbar_init(&bar.dv_done[b], 1);
+      mbar_init(&bar.dk_done[b], 1);
+    }
+    mbar_init(&bar.fin, 1);
+    bar.nsteps = tile_units[(size_t)h * (N / 128) + tile];
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -407,8 +420,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bar.tmem_base;
-  const int ntiles = bar.ntiles, nunits = bar.nunits;
-  const uint32_t tS = tmem, tP = tmem + 128, tV = tmem + 256, tK = tmem + 256 + D;
+  const int nsteps = bar.nsteps;
+  const uint32_t tV = tmem, tK = tmem + 128;
 
   if (warp == 0) {
     const int blk[2] = {unit_block[(size_t)h * NB + 2 * tile], unit_block[(size_t)h * NB + 2 * tile + 1]};
@@ -422,37 +435,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(smem + L::OFF_V + c * (128 * 128), &mapV, &bar.kv_full, c * 64, h * N + tile * 128);
       }
     }
-    for (int j = 0; j < ntiles; ++j) {
-      const int s = j % NSTAGE;
-      uint32_t ua, ub = 0;
-      int ma, mb = 0, nu = 1;
-      walk_next<2>(w, rowidx, blocks_h, ua, ma);
-      if (2 * j + 2 <= nunits) {
-        walk_next<2>(w, rowidx, blocks_h, ub, mb);
-        nu = 2;
-      }
-      ua = min(ua, (uint32_t)(NB - 1));
-      ub = min(ub, (uint32_t)(NB - 1));
+    for (int j = 0; j < nsteps; ++j) {
+      const int s = j % NS;
+      uint32_t u;
+      int m;
+      walk_next<2>(w, rowidx, blocks_h, u, m);
+      u = min(u, (uint32_t)(NB - 1));
       if (lane == 0) {
         bool ok = true;
-        if (j >= NSTAGE) ok = mbar_wait(&bar.q_empty[s], ((j / NSTAGE) - 1) & 1, status, 41);
+        if (j >= NS) ok = mbar_wait(&bar.q_empty[s], ((j / NS) - 1) & 1, status, 41);
         if (!ok) bar.abort = 1;
         if (ok) {
-          bar.meta[s] = nu | (ma << 4) | (mb << 8);
-          uint8_t *qs = smem + L::OFF_Q + s * L::TILE;
-          uint8_t *ds = smem + L::OFF_DO + s * L::TILE;
-          float *st = stat + s * 256;
-          mbar_arrive_expect_tx(&bar.q_full[s], nu * (2 * 64 * D * 2 + 2 * 64 * 4));
-          for (int u = 0; u < nu; ++u) {
-            const int un = u == 0 ? (int)ua : (int)ub;
+          bar.mask[s] = m;
+          mbar_arrive_expect_tx(&bar.q_full[s], 2 * L::UNIT + 2 * 64 * 4);
 #pragma unroll
-            for (int c = 0; c < L::CHUNKS; ++c) {
-              tma_load_2d(qs + c * (128 * 128) + u * 64 * 128, &mapQ, &bar.q_full[s], c * 64, h * N + un * 64);
-              tma_load_2d(ds + c * (128 * 128) + u * 64 * 128, &mapDO, &bar.q_full[s], c * 64, h * N + un * 64);
-            }
-            bulk_load(st + u * 64, lse2p + (size_t)h * N + (size_t)un * 64, 256, &bar.q_full[s]);
-            bulk_load(st + 128 + u * 64, deltap + (size_t)h * N + (size_t)un * 64, 256, &bar.q_full[s]);
+          for (int c = 0; c < L::CHUNKS; ++c) {
+            tma_load_2d(smem + L::OFF_Q + s * L::UNIT + c * (64 * 128), &mapQ, &bar.q_full[s], c * 64,
+                        h * N + (int)u * 64);
+            tma_load_2d(smem + L::OFF_DO + s * L::UNIT + c * (64 * 128), &mapDO, &bar.q_full[s], c * 64,
+                        h * N + (int)u * 64);
           }
+          bulk_load(stat + s * 128, lse2p + (size_t)h * N + (size_t)u * 64, 256, &bar.q_full[s]);
+          bulk_load(stat + s * 128 + 64, deltap + (size_t)h * N + (size_t)u * 64, 256, &bar.q_full[s]);
         }
       }
       __syncwarp();
@@ -460,120 +464,127 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t id_full = idesc_f16(128, 128, 0), id_half = idesc_f16(128, 64, 0);
-      const uint32_t id_acc = idesc_f16(128, D, 1);
+      const uint32_t id64 = idesc_f16(128, 64, 0), id_acc = idesc_f16(128, D, 1);
       const uint32_t sK = smem_u32(smem + L::OFF_K), sV = smem_u32(smem + L::OFF_V);
       bool ok = mbar_wait(&bar.kv_full, 0, status, 42);
       tc_fence_after();
-      for (int j = 0; ok && j <= ntiles; ++j) {
-        if (j >= 1) {  // dV += P^T dO, dK += dS^T Q  (tile j-1)
-          const int jj = j - 1, s = jj % NSTAGE;
-          ok = mbar_wait(&bar.ds_ready, jj & 1, status, 43);
+      for (int i = 0; ok && i <= nsteps; ++i) {
+        if (i < nsteps) {  // S^T_i = K Q_i^T, dP^T_i = V dO_i^T into buffer i&1
+          const int s = i % NS, b = i & 1;
+          const uint32_t tS = tmem + 256 + 128 * b, tP = tS + 64;
+          ok = mbar_wait(&bar.q_full[s], (i / NS) & 1, status, 44);
+          if (ok && i >= 2) ok = mbar_wait(&bar.dv_done[b], ((i - 2) >> 1) & 1, status, 45);
           if (!ok) break;
           tc_fence_after();
-          const int nu = bar.meta[s] & 15;
-          const uint32_t sQ = smem_u32(smem + L::OFF_Q + s * L::TILE);
-          const uint32_t sDO = smem_u32(smem + L::OFF_DO + s * L::TILE);
-          for (int ks = 0; ks < nu * 4; ++ks) {
-            const uint32_t acc = (jj > 0 || ks > 0) ? 1u : 0u;
-            mma_ts(tV, tS + ks * 8, sdesc_sw128(sDO + ks * 2048, 128 * 128, 1024), id_acc, acc);
-            mma_ts(tK, tP + ks * 8, sdesc_sw128(sQ + ks * 2048, 128 * 128, 1024), id_acc, acc);
-          }
-          mma_commit(&bar.mm_done);
+          const uint32_t sQ = smem_u32(smem + L::OFF_Q + s * L::UNIT);
+          const uint32_t sDO = smem_u32(smem + L::OFF_DO + s * L::UNIT);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tS, sdesc_sw128(sK + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024),
+                   sdesc_sw128(sQ + (kk >> 2) * (64 * 128) + (kk & 3) * 32, 16, 1024), id64, kk > 0 ? 1u : 0u);
+          mma_commit(&bar.s_full[b]);
+          if (i >= 2) ok = mbar_wait(&bar.dk_done[b], ((i - 2) >> 1) & 1, status, 46);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tP, sdesc_sw128(sV + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024),
+                   sdesc_sw128(sDO + (kk >> 2) * (64 * 128) + (kk & 3) * 32, 16, 1024), id64, kk > 0 ? 1u : 0u);
+          mma_commit(&bar.dp_full[b]);
+        }
+        if (i >= 1) {  // dV += P^T dO, dK += dS^T Q  (step i-1)
+          const int jj = i - 1, s = jj % NS, b = jj & 1;
+          const uint32_t tS = tmem + 256 + 128 * b, tP = tS + 64;
+          ok = mbar_wait(&bar.ds_ready[b], (jj >> 1) & 1, status, 43);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t sQ = smem_u32(smem + L::OFF_Q + s * L::UNIT);
+          const uint32_t sDO = smem_u32(smem + L::OFF_DO + s * L::UNIT);
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_ts(tV, tS + ks * 8, sdesc_sw128(sDO + ks * 2048, 64 * 128, 1024), id_acc, (jj > 0 || ks > 0) ? 1u : 0u);
+          mma_commit(&bar.dv_done[b]);
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_ts(tK, tP + ks * 8, sdesc_sw128(sQ + ks * 2048, 64 * 128, 1024), id_acc, (jj > 0 || ks > 0) ? 1u : 0u);
+          mma_commit(&bar.dk_done[b]);
           mma_commit(&bar.q_empty[s]);
         }
-        if (j < ntiles) {
-          const int s = j % NSTAGE;
-          ok = mbar_wait(&bar.q_full[s], (j / NSTAGE) & 1, status, 44);
-          if (ok && j >= 1) ok = mbar_wait(&bar.mm_done, (j - 1) & 1, status, 45);
-          if (!ok) break;
-          tc_fence_after();
-          const int nu = bar.meta[s] & 15;
-          const uint32_t id = nu == 2 ? id_full : id_half;
-          const uint32_t sQ = smem_u32(smem + L::OFF_Q + s * L::TILE);
-          const uint32_t sDO = smem_u32(smem + L::OFF_DO + s * L::TILE);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-            mma_ss(tS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), id, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&bar.s_full);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-            mma_ss(tP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sDO + off, 16, 1024), id, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&bar.dp_full);
-        }
       }
+      if (ok && nsteps > 0) mma_commit(&bar.fin);
       if (!ok) bar.abort = 1;
     }
     __syncwarp();
-  } else {
+  } else if (warp >= 4) {
+    const int g = (warp - 4) >> 2;
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;  // key row of the tile
-    const int half = row >> 6;
+    const int half = row >> 6;       // warp-uniform
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const uint32_t tS = tmem + 256 + 128 * g, tP = tS + 64;
     bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
-      const int s = j % NSTAGE;
-      ok = mbar_wait_warp(&bar.s_full, j & 1, status, 47);
-      if (ok) ok = mbar_wait_warp(&bar.dp_full, j & 1, status, 48);
+    for (int i = g; i < nsteps; i += 2) {
+      const int ph = (i >> 1) & 1, s = i % NS;
+      ok = mbar_wait_warp(&bar.s_full[g], ph, status, 47);
+      if (ok) ok = mbar_wait_warp(&bar.dp_full[g], ph, status, 48);
+      // the stage's statistics were written by the async proxy: observe the
+      // stage's own barrier (already complete; the stage cannot be refilled
+      // before this step releases it) so those writes are visible here
+      if (ok) ok = mbar_wait_warp(&bar.q_full[s], (i / NS) & 1, status, 50);
       if (!ok) break;
       tc_fence_after();
-      const int meta = bar.meta[s];
-      const int nu = meta & 15;
-      const float *l2 = stat + s * 256, *dl = stat + s * 256 + 128;
-      for (int c = 0; c < 2 * nu; ++c) {
-        const int m = (c < 2) ? (meta >> 4) : (meta >> 8);
-        const bool valid = (m >> half) & 1;
-        uint32_t sv[32], dv[32], pp[16], pd[16];
-        tmem_ld32(tS + lane_off + c * 32, sv);
-        tmem_ld32(tP + lane_off + c * 32, dv);
-        tmem_wait_ld();
+      const bool valid = (bar.mask[s] >> half) & 1;
+      const float *l2 = stat + s * 128, *dl = stat + s * 128 + 64;
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
-          if (valid) {
-            const int q = c * 32 + i;
-            p0 = exp2f(fmaf(__uint_as_float(sv[i]), scale_log2, -l2[q]));
-            p1 = exp2f(fmaf(__uint_as_float(sv[i + 1]), scale_log2, -l2[q + 1]));
-            d0 = p0 * (__uint_as_float(dv[i]) - dl[q]);
-            d1 = p1 * (__uint_as_float(dv[i + 1]) - dl[q + 1]);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pp[16], pd[16];
+        if (valid) {
+          uint32_t sv[32], dv[32];
+          tmem_ld32(tS + lane_off + c * 32, sv);
+          tmem_ld32(tP + lane_off + c * 32, dv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; k += 2) {
+            const int q = c * 32 + k;
+            const float2 x = ffma2(make_float2(__uint_as_float(sv[k]), __uint_as_float(sv[k + 1])),
+                                   make_float2(scale_log2, scale_log2), make_float2(-l2[q], -l2[q + 1]));
+            const float2 p = make_float2(ex2f(x.x), ex2f(x.y));
+            const float2 d = fmul2(p, fsub2(make_float2(__uint_as_float(dv[k]), __uint_as_float(dv[k + 1])),
+                                            make_float2(dl[q], dl[q + 1])));
+            pp[k / 2] = pack_f16(p.x, p.y);
+            pd[k / 2] = pack_f16(d.x, d.y);
           }
-          pp[i / 2] = pack_f16(p0, p1);
-          pd[i / 2] = pack_f16(d0, d1);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) pp[k] = pd[k] = 0u;
         }
         tmem_st16(tS + lane_off + c * 16, pp);
         tmem_st16(tP + lane_off + c * 16, pd);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar.ds_ready);
+      mbar_arrive(&bar.ds_ready[g]);
     }
     ok = __all_sync(0xffffffffu, ok);
-    if (ok && ntiles > 0) ok = mbar_wait_warp(&bar.mm_done, (ntiles - 1) & 1, status, 49);
+    if (ok && nsteps > 0) ok = mbar_wait_warp(&bar.fin, 0, status, 49);
     if (ok) {
       tc_fence_after();
       const size_t prow = (size_t)h * N + (size_t)tile * 128 + row;
       const int n = perm[prow];
       const size_t off = ((size_t)n * heads + h) * D;
+      // warpgroup 0 writes dV, warpgroup 1 writes dK
+      const uint32_t src = g == 0 ? tV : tK;
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
         uint32_t o[32];
-        if (ntiles > 0) {
-          tmem_ld32(tV + lane_off + c, o);
+        if (nsteps > 0) {
+          tmem_ld32(src + lane_off + c, o);
           tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0u;
+          for (int k = 0; k < 32; ++k) o[k] = 0u;
         }
-        store_row<D>(dV, grad_fp32 != 0, off + c, o, 1.0f);
-        if (ntiles > 0) {
-          tmem_ld32(tK + lane_off + c, o);
-          tmem_wait_ld();
-        }
-        store_row<D>(dK, grad_fp32 != 0, off + c, o, sm_scale);
+        store_row<D>(g == 0 ? dV : dK, grad_fp32 != 0, off + c, o, g == 0 ? 1.0f : sm_scale);
       }
     } else {
       bar.abort = 1;
@@ -636,7 +647,7 @@ static cudaError_t run_bwd(const prism_params &p, const prism_plan_t &plan, cons
                            const BwdWs &w, void *dQ, void *dK, void *dV, int grad_fp32, cudaStream_t st) {
   const int N = p.T * p.H * p.W;
   const long long rows = (long long)p.heads * N;
-  CUtensorMap mQ128, mDO128, mK64, mV64, mQ64, mDO64, mK128, mV128;
+  CUtensorMap mQ128, mDO128, mK64, mV64, mQ64, mDO64, mK128, mV128;  // box rows 128 or 64
   cudaError_t e;
   if ((e = make_rows_map(&mQ128, w.Qp, rows, D, 128)) != cudaSuccess) return e;
   if ((e = make_rows_map(&mDO128, w.dOp, rows, D, 128)) != cudaSuccess) return e;

@@ -61,27 +61,6 @@ struct Bars {
   int abort;
 };
 
-__device__ __forceinline__ float ex2f(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-// (a0, a1) * (b, b) + (c, c) and (a0, a1) + (b0, b1) on paired fp32 lanes
-__device__ __forceinline__ float2 ffma2(float2 a, float b, float c) {
-  uint64_t d;
-  const uint64_t av = *reinterpret_cast<uint64_t *>(&a);
-  float2 bb = make_float2(b, b), cc = make_float2(c, c);
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(av), "l"(*reinterpret_cast<uint64_t *>(&bb)),
-      "l"(*reinterpret_cast<uint64_t *>(&cc)));
-  return *reinterpret_cast<float2 *>(&d);
-}
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(*reinterpret_cast<uint64_t *>(&a)),
-      "l"(*reinterpret_cast<uint64_t *>(&b)));
-  return *reinterpret_cast<float2 *>(&d);
-}
-
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,

@@ -255,6 +255,43 @@ __host__ __device__ constexpr uint32_t idesc_f16(uint32_t M, uint32_t N, uint32_
 }
 
 // ---------------------------------------------------------------------------
+// fast arithmetic for the attention softmax
+// ---------------------------------------------------------------------------
+// 2^x by the MUFU instruction (flush-to-zero; relative error ~2^-22, far below
+// the fp16 rounding the result goes through).
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint64_t f2u(float2 a) { return *reinterpret_cast<uint64_t *>(&a); }
+__device__ __forceinline__ float2 u2f(uint64_t a) { return *reinterpret_cast<float2 *>(&a); }
+// paired fp32 lanes (one instruction for two values)
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)), "l"(f2u(c)));
+  return u2f(d);
+}
+__device__ __forceinline__ float2 ffma2(float2 a, float b, float c) {
+  return ffma2(a, make_float2(b, b), make_float2(c, c));
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
+  return u2f(d);
+}
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
+  return u2f(d);
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
+  return u2f(d);
+}
+
+// ---------------------------------------------------------------------------
 // block-wide helpers
 // ---------------------------------------------------------------------------
 template <typename T>

@@ -130,6 +130,79 @@ def computed_pairs(p, pl, sel):
     return int((Bq[row_of] * Bk).sum().item())
 
 
+# ----------------------------------------------------------------------------- kernel rooflines
+def read_kernel_times(lib):
+    out = {}
+    for i in range(_lib.KERNEL_TIMING_IDS):
+        n, ms, name = _lib.C.c_int(0), _lib.C.c_double(0.0), _lib.C.c_char_p()
+        _lib.check(lib.prism_kernel_timing_read(i, _lib.C.byref(n), _lib.C.byref(ms), _lib.C.byref(name)))
+        out[name.value.decode()] = (n.value, ms.value)
+    return out
+
+
+def kernel_rooflines(ktimes, P, D, N, h, nb, peaks, peak_src, steps):
+    """Per kernel: launches, ms per launch (CUDA events on the launching
+    stream, timed region), algorithmic work per launch and its fraction of the
+    measured peak (sustained bf16 for tensor kernels inside this long step;
+    the STREAM copy bandwidth for HBM-bound kernels)."""
+    tensor_peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    hbm = peaks["hbm_gbs"]
+    sum_nb2 = float((nb.double() ** 2).sum().item())
+    spec = {
+        # name: (bound, work per step, unit, description)
+        "attn_fwd": ("tensor", 4.0 * P * D, "TFLOP/s", "4*P*D FLOP (QK^T and PV on the computed pairs)"),
+        "attn_bwd_dkdv": ("tensor", 8.0 * P * D, "TFLOP/s", "8*P*D FLOP (S^T, dP^T, dV, dK on the computed pairs)"),
+        "attn_bwd_dq": ("tensor", 6.0 * P * D, "TFLOP/s", "6*P*D FLOP (S, dP, dQ on the computed pairs)"),
+        "zone_video_stats": ("hbm", 2.0 * N * h * D, "GB/s", "one read of V: 2*N*h*D bytes"),
+        "block_mean": ("hbm", 4.0 * N * h * D, "GB/s", "one read of Q and K: 4*N*h*D bytes"),
+        "block_score": ("alu", 2.0 * D * sum_nb2, "TFLOP/s", "2*D*sum_h Nb^2 fp32 FLOP (mul + add)"),
+        "select_row": ("alu", None, None, "per-row radix selection over N_b scores"),
+    }
+    out = {}
+    for name, (n, ms) in ktimes.items():
+        bound, work, unit, desc = spec[name]
+        rec = {"launches": n, "total_ms": ms, "ms_per_launch": ms / n if n else None, "bound": bound,
+               "algorithmic": desc, "unit": unit, "achieved": None, "peak": None, "frac": None, "peak_source": None}
+        if n and work is not None:
+            # `work` is per step; kernels launched once per head per step share
+            # it evenly
+            per_launch = work * steps / n
+            sec = (ms / n) * 1e-3
+            if bound == "tensor":
+                rec["achieved"] = per_launch / sec / 1e12
+                rec["peak"] = tensor_peak
+                rec["peak_source"] = f"{peak_src} bf16 sustained"
+            elif bound == "hbm":
+                rec["achieved"] = per_launch / sec / 1e9
+                rec["peak"] = hbm
+                rec["peak_source"] = f"{peak_src} HBM copy"
+            else:
+                rec["achieved"] = per_launch / sec / 1e12
+                # FP32 SIMT: 148 SMs x 128 lanes x (1 op per lane per cycle) at the max SM clock
+                rec["peak"] = 148 * 128 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+                rec["peak_source"] = "derived: 148 SMs x 128 fp32 lanes x max SM clock (one FMUL or FADD each)"
+            rec["frac"] = rec["achieved"] / rec["peak"]
+        out[name] = rec
+    return out
+
+
+def stored_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None
+    when the summary is missing or the kernel's source changed since."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f).get(kernel)
+    if not d:
+        return None
+    src = os.path.join(ROOT, "dynamic_block_sparse_stats_b200", "csrc", d["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != d["source_sha256"]:
+        return None
+    return d["bytes_per_launch"]
+
+
 # ----------------------------------------------------------------------------- oracle sample
 def oracle_sample(w, inp, p, pl, sel, head=0, n_rows=2, seed=0):
     """Time the CPU oracle on a bounded sample of the same layer: the plan and
@@ -221,6 +294,7 @@ def run_prism(args, w, rank, world, device):
     flops = flops_fwd + flops_bwd
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(args.steps)]
+    lib.prism_kernel_timing(1)
     clk = ClockSampler(torch.cuda.current_device())
     if world > 1:
         torch.distributed.barrier()
@@ -238,6 +312,8 @@ def run_prism(args, w, rank, world, device):
         torch.distributed.barrier()
     launches = lib.prism_kernel_launches() - l0
     clocks = clk.stop()
+    ktimes = read_kernel_times(lib)
+    lib.prism_kernel_timing(0)
     ms = t_start.elapsed_time(t_end) / args.steps
     stage_ms = {s: statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps))
                 for i, s in enumerate(stages)}
@@ -279,20 +355,21 @@ def run_prism(args, w, rank, world, device):
         del hin, hout
 
     peaks, peak_src = load_peaks()
-    dominant = "bwd" if backward else "fwd"
-    dom_flops = flops_bwd if backward else flops_fwd
-    achieved = dom_flops / (stage_ms[dominant] * 1e-3) / 1e12
+    nb = pl.n_blocks.long()
+    kernels = kernel_rooflines(ktimes, P, D, N, h, nb, peaks, peak_src, args.steps)
+    dom = max((k for k in kernels if kernels[k]["launches"]), key=lambda k: kernels[k]["total_ms"])
+    kd = kernels[dom]
+    roofline = {"kernel": dom, "bound": kd["bound"], "achieved": kd["achieved"], "peak": kd["peak"],
+                "unit": kd["unit"], "frac": kd["frac"], "peak_source": kd["peak_source"],
+                "traffic": stored_traffic(dom), "algorithmic": kd["algorithmic"],
+                "ms_per_launch": kd["ms_per_launch"]}
     peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
-    roofline = {"kernel": f"prism_attn_{dominant} call ({'attn_bwd' if backward else 'attn_fwd'} kernels)",
-                "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "peak_source": f"{peak_src} bf16 sustained", "traffic": None,
-                "algorithmic": f"{'10' if backward else '4'}*P*D = {dom_flops:.4e} FLOP per launch"}
     plan_bytes = N * h * D * 2 + N * 4
     stage_roofline = {
         "plan_GBps": plan_bytes / (stage_ms["plan"] * 1e-3) / 1e9,
         "plan_frac_hbm": plan_bytes / (stage_ms["plan"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
-        "fwd_TFLOPs": flops_fwd / (stage_ms["fwd"] * 1e-3) / 1e12,
-        "fwd_frac_bf16": flops_fwd / (stage_ms["fwd"] * 1e-3) / 1e12 / peak,
+        "fwd_call_TFLOPs": flops_fwd / (stage_ms["fwd"] * 1e-3) / 1e12,
+        "fwd_call_frac_bf16": flops_fwd / (stage_ms["fwd"] * 1e-3) / 1e12 / peak,
     }
 
     cpu = None
@@ -312,7 +389,7 @@ def run_prism(args, w, rank, world, device):
                    "parallelism": f"weak x{world} (independent layers, no collectives)",
                    "l2": "inputs larger than L2 (each bf16 tensor %.2f GB)" % (N * h * D * 2 / 1e9),
                    "pairs": P, "pair_density": density, "nnz_blocks": sel.nnz},
-        "stage_ms": stage_ms, "stage_roofline": stage_roofline,
+        "stage_ms": stage_ms, "stage_roofline": stage_roofline, "kernels": kernels,
         "clocks": clocks, "e2e": e2e, "gpu_launches": launches, "roofline": roofline, "cpu_baseline": cpu,
     }
     return line

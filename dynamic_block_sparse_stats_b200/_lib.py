@@ -27,7 +27,9 @@ EXPORTS = (
     "prism_plan_workspace_size", "prism_plan", "prism_select_workspace_size", "prism_select",
     "prism_attn_workspace_size", "prism_attn_fwd", "prism_attn_bwd", "prism_workspace_status",
     "prism_last_error", "prism_version", "prism_kernel_launches", "prism_plan_noalloc",
+    "prism_kernel_timing", "prism_kernel_timing_read",
 )
+KERNEL_TIMING_IDS = 7
 
 
 class PrismParams(C.Structure):
@@ -81,6 +83,8 @@ def load() -> C.CDLL:
         "prism_version": (C.c_char_p, []),
         "prism_kernel_launches": (C.c_uint64, []),
         "prism_plan_noalloc": (C.c_int, [P(PrismParams), vp, vp, P(PrismPlan), st]),
+        "prism_kernel_timing": (C.c_int, [C.c_int]),
+        "prism_kernel_timing_read": (C.c_int, [C.c_int, P(C.c_int), P(C.c_double), P(C.c_char_p)]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)

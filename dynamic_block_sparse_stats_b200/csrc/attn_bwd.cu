@@ -18,9 +18,9 @@
 //                (fp16), dV += P^T dO, dK += dS^T Q (TS MMAs).
 // Operands are fp16 (exact conversions of the bf16 inputs, see the forward).
 // Roles: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer, warps 4-11
-// two compute warpgroups (one thread per TMEM lane) taking alternate steps of
-// one 64-token unit; each step has its own TMEM buffers, so the compute of a
-// step overlaps the MMAs of the next.
+// two compute warpgroups (one thread per TMEM lane), each taking one 32-token
+// half of every 64-token step.  Steps alternate between two TMEM buffer
+// pairs, so the compute of a step overlaps the MMAs of the next.
 #include "attn_walk.cuh"
 
 namespace prism {
@@ -77,9 +77,9 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const int32_t *__restrict
 
 // ---------------------------------------------------------------------------
 // Shared pieces of the two kernels.  Both walk 64-token units of the
-// streamed side, one unit per step; two compute warpgroups take alternate
-// steps, each with its own TMEM buffer pair, so the compute of step i
-// overlaps the MMAs of step i+1.
+// streamed side, one unit per step, alternating between two TMEM buffer
+// pairs so the compute of step i overlaps the MMAs of step i+1; the two
+// compute warpgroups split each step's 64 columns.
 // ---------------------------------------------------------------------------
 constexpr int NS = 4;  // ring depth (steps of one 64-token unit)
 
@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bar.s_full[b], 1);
       mbar_init(&bar.dp_full[b], 1);
-      mbar_init(&bar.ds_ready[b], 128);
+      mbar_init(&bar.ds_ready[b], 256);
       mbar_init(&bar.dq_done[b], 1);
     }
     mbar_init(&bar.fin, 1);
@@ -267,47 +267,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    const int g = (warp - 4) >> 2;  // warpgroup: steps with i % 2 == g
+    const int g = (warp - 4) >> 2;  // warpgroup: 32-key chunk g of every step
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const int half = row >> 6;  // warp-uniform
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const size_t prow = (size_t)h * N + (size_t)tile * 128 + row;
     const float lse2 = lse2p[prow], dl = deltap[prow];
-    const uint32_t tS = tmem + 128 + 128 * g, tP = tS + 64;
     bool ok = true;
-    for (int i = g; i < nsteps; i += 2) {
-      const int ph = (i >> 1) & 1;
-      ok = mbar_wait_warp(&bar.s_full[g], ph, status, 27);
-      if (ok) ok = mbar_wait_warp(&bar.dp_full[g], ph, status, 28);
+    for (int i = 0; i < nsteps; ++i) {
+      const int b = i & 1, ph = (i >> 1) & 1;
+      const uint32_t tS = tmem + 128 + 128 * b, tP = tS + 64;
+      ok = mbar_wait_warp(&bar.s_full[b], ph, status, 27);
+      if (ok) ok = mbar_wait_warp(&bar.dp_full[b], ph, status, 28);
       if (!ok) break;
       tc_fence_after();
       const bool valid = (bar.mask[i % NS] >> half) & 1;
+      uint32_t pk[16];
+      if (valid) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32(tS + lane_off + g * 32, sv);
+        tmem_ld32(tP + lane_off + g * 32, dv);
+        tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t pk[16];
-        if (valid) {
-          uint32_t sv[32], dv[32];
-          tmem_ld32(tS + lane_off + c * 32, sv);
-          tmem_ld32(tP + lane_off + c * 32, dv);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; k += 2) {
-            const float2 x = ffma2(make_float2(__uint_as_float(sv[k]), __uint_as_float(sv[k + 1])), scale_log2, -lse2);
-            const float2 p = make_float2(ex2f(x.x), ex2f(x.y));
-            const float2 d = fmul2(p, fsub2(make_float2(__uint_as_float(dv[k]), __uint_as_float(dv[k + 1])),
-                                            make_float2(dl, dl)));
-            pk[k / 2] = pack_f16(d.x, d.y);
-          }
-        } else {
-#pragma unroll
-          for (int k = 0; k < 16; ++k) pk[k] = 0u;
+        for (int k = 0; k < 32; k += 2) {
+          const float2 x = ffma2(make_float2(__uint_as_float(sv[k]), __uint_as_float(sv[k + 1])), scale_log2, -lse2);
+          const float2 p = make_float2(ex2f(x.x), ex2f(x.y));
+          const float2 d = fmul2(p, fsub2(make_float2(__uint_as_float(dv[k]), __uint_as_float(dv[k + 1])),
+                                          make_float2(dl, dl)));
+          pk[k / 2] = pack_f16(d.x, d.y);
         }
-        tmem_st16(tP + lane_off + c * 16, pk);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) pk[k] = 0u;
       }
+      tmem_st16(tP + lane_off + g * 16, pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar.ds_ready[g]);
+      mbar_arrive(&bar.ds_ready[b]);
     }
     // A parity wait on dq_done could match an older phase for the warpgroup
     // that did not run the step before the last; the single-use barrier
@@ -404,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bar.s_full[b], 1);
       mbar_init(&bar.dp_full[b], 1);
-      mbar_init(&bar.ds_ready[b], 128);
+      mbar_init(&bar.ds_ready[b], 256);
       mbar_init(&bar.dv_done[b], 1);
       mbar_init(&bar.dk_done[b], 1);
     }
@@ -516,17 +513,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    const int g = (warp - 4) >> 2;
+    const int g = (warp - 4) >> 2;   // warpgroup: 32-query chunk g of every step
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;  // key row of the tile
     const int half = row >> 6;       // warp-uniform
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    const uint32_t tS = tmem + 256 + 128 * g, tP = tS + 64;
     bool ok = true;
-    for (int i = g; i < nsteps; i += 2) {
-      const int ph = (i >> 1) & 1, s = i % NS;
-      ok = mbar_wait_warp(&bar.s_full[g], ph, status, 47);
-      if (ok) ok = mbar_wait_warp(&bar.dp_full[g], ph, status, 48);
+    for (int i = 0; i < nsteps; ++i) {
+      const int b = i & 1, ph = (i >> 1) & 1, s = i % NS;
+      const uint32_t tS = tmem + 256 + 128 * b, tP = tS + 64;
+      ok = mbar_wait_warp(&bar.s_full[b], ph, status, 47);
+      if (ok) ok = mbar_wait_warp(&bar.dp_full[b], ph, status, 48);
       // the stage's statistics were written by the async proxy: observe the
       // stage's own barrier (already complete; the stage cannot be refilled
       // before this step releases it) so those writes are visible here
@@ -534,36 +531,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const bool valid = (bar.mask[s] >> half) & 1;
-      const float *l2 = stat + s * 128, *dl = stat + s * 128 + 64;
+      const float4 *l2 = reinterpret_cast<const float4 *>(stat + s * 128 + g * 32);
+      const float4 *dl = reinterpret_cast<const float4 *>(stat + s * 128 + 64 + g * 32);
+      uint32_t pp[16], pd[16];
+      if (valid) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32(tS + lane_off + g * 32, sv);
+        tmem_ld32(tP + lane_off + g * 32, dv);
+        tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t pp[16], pd[16];
-        if (valid) {
-          uint32_t sv[32], dv[32];
-          tmem_ld32(tS + lane_off + c * 32, sv);
-          tmem_ld32(tP + lane_off + c * 32, dv);
-          tmem_wait_ld();
+        for (int k4 = 0; k4 < 8; ++k4) {
+          const float4 lq = l2[k4], dq = dl[k4];
 #pragma unroll
-          for (int k = 0; k < 32; k += 2) {
-            const int q = c * 32 + k;
+          for (int u = 0; u < 2; ++u) {
+            const int k = 4 * k4 + 2 * u;
+            const float2 lm = u ? make_float2(-lq.z, -lq.w) : make_float2(-lq.x, -lq.y);
+            const float2 dd = u ? make_float2(dq.z, dq.w) : make_float2(dq.x, dq.y);
             const float2 x = ffma2(make_float2(__uint_as_float(sv[k]), __uint_as_float(sv[k + 1])),
-                                   make_float2(scale_log2, scale_log2), make_float2(-l2[q], -l2[q + 1]));
+                                   make_float2(scale_log2, scale_log2), lm);
             const float2 p = make_float2(ex2f(x.x), ex2f(x.y));
-            const float2 d = fmul2(p, fsub2(make_float2(__uint_as_float(dv[k]), __uint_as_float(dv[k + 1])),
-                                            make_float2(dl[q], dl[q + 1])));
+            const float2 d = fmul2(p, fsub2(make_float2(__uint_as_float(dv[k]), __uint_as_float(dv[k + 1])), dd));
             pp[k / 2] = pack_f16(p.x, p.y);
             pd[k / 2] = pack_f16(d.x, d.y);
           }
-        } else {
-#pragma unroll
-          for (int k = 0; k < 16; ++k) pp[k] = pd[k] = 0u;
         }
-        tmem_st16(tS + lane_off + c * 16, pp);
-        tmem_st16(tP + lane_off + c * 16, pd);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) pp[k] = pd[k] = 0u;
       }
+      tmem_st16(tS + lane_off + g * 16, pp);
+      tmem_st16(tP + lane_off + g * 16, pd);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar.ds_ready[g]);
+      mbar_arrive(&bar.ds_ready[b]);
     }
     ok = __all_sync(0xffffffffu, ok);
     if (ok && nsteps > 0) ok = mbar_wait_warp(&bar.fin, 0, status, 49);
@@ -662,14 +662,20 @@ static cudaError_t run_bwd(const prism_params &p, const prism_plan_t &plan, cons
   dim3 grid(N / 128, p.heads);
   const int s1 = bwd::KvSmem<D>::BYTES + 1024;
   cudaFuncSetAttribute(bwd::dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, s1);
+  {
+  KernelTimer kt_(KT_ATTN_DKDV, st);
   bwd::dkdv_kernel<D><<<grid, bwd::kThreads, s1, st>>>(mQ64, mDO64, mK128, mV128, sel.col_ptr, sel.row, plan.blocks,
                                                        w.unit_block, w.tu_k, plan.perm, w.lse2p, w.deltap, dK, dV,
                                                        grad_fp32, N, p.heads, scale_log2, scale, &w.hdr->status);
+  }
   const int s2 = bwd::DqSmem<D>::BYTES + 1024;
   cudaFuncSetAttribute(bwd::dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, s2);
+  {
+  KernelTimer kt_(KT_ATTN_DQ, st);
   bwd::dq_kernel<D><<<grid, bwd::kThreads, s2, st>>>(mQ128, mDO128, mK64, mV64, sel.row_ptr, sel.col, plan.blocks,
                                                      w.unit_block, w.tu_q, plan.perm, w.lse2p, w.deltap, dQ,
                                                      grad_fp32, N, p.heads, scale_log2, scale, &w.hdr->status);
+  }
   count_launches(2);
   return cudaGetLastError();
 }

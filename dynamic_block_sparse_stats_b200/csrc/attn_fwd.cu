@@ -548,6 +548,7 @@ static cudaError_t run_fwd(const prism_params &p, const prism_plan_t &plan, cons
   cudaFuncSetAttribute(fwd::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   const float scale_log2 = effective_scale(p) * 1.4426950408889634f;
   dim3 grid(N / fwd::BQ, p.heads);
+  KernelTimer kt_(KT_ATTN_FWD, st);
   fwd::attn_fwd_kernel<D><<<grid, fwd::kThreads, smem, st>>>(mQ, mK, mV, sel.row_ptr, sel.col, plan.blocks,
                                                              w.unit_block, w.tile_units, plan.perm, O, O_res, lse,
                                                              N, p.heads, scale_log2, &w.hdr->status);

@@ -58,6 +58,29 @@ cudaError_t make_rows_map(CUtensorMap *map, const void *base, long long rows, in
 // host-side count of kernel launches (prism_kernel_launches)
 void count_launches(int n);
 
+// timing.cu: optional event timing of the main kernels (prism_kernel_timing)
+enum KernelTimingId {
+  KT_ZONE_STATS = 0,
+  KT_BLOCK_MEAN,
+  KT_BLOCK_SCORE,
+  KT_SELECT_ROW,
+  KT_ATTN_FWD,
+  KT_ATTN_DKDV,
+  KT_ATTN_DQ,
+  KT_COUNT
+};
+// Records an event on `st` at construction and at destruction when timing is
+// enabled; wrap exactly one kernel launch.
+class KernelTimer {
+ public:
+  KernelTimer(int id, cudaStream_t st);
+  ~KernelTimer();
+
+ private:
+  cudaStream_t st_;
+  int idx_;
+};
+
 // api.cu: prism_plan's argument checks; error reporting for prism_last_error
 int check_plan_call(const prism_params *p, const uint16_t *V, const prism_plan_t *out);
 int report_error(int code, const char *msg);

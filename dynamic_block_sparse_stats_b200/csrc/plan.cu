@@ -406,6 +406,8 @@ cudaError_t launch_plan(const prism_params &p, const uint16_t *V, const float *a
   int32_t *zone_first = reinterpret_cast<int32_t *>(w);
 
   dim3 g1(Z, p.heads);
+  {
+  KernelTimer kt_(KT_ZONE_STATS, st);
   if (p.head_dim == 128) {
     const int sm = 2 * 8 * 8 * 128 * sizeof(float);
     cudaFuncSetAttribute(zone_video_stats_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
@@ -413,6 +415,7 @@ cudaError_t launch_plan(const prism_params &p, const uint16_t *V, const float *a
   } else {
     const int sm = 2 * 8 * 8 * 64 * sizeof(float);
     zone_video_stats_kernel<64><<<g1, 256, sm, st>>>(V, p.T, p.H, p.W, p.heads, vstats);
+  }
   }
   if (a) zone_a2v_stats_kernel<<<Z, 64, 0, st>>>(a, p.T, p.H, p.W, astats);
   plan_finalize_kernel<<<p.heads, 1024, 0, st>>>(vstats, a ? astats : nullptr, Z, p.T, p.H, p.W, p.heads, NB,

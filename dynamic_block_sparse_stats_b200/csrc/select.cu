@@ -599,12 +599,15 @@ cudaError_t launch_select(const prism_params &p, const prism_plan_t &plan, const
   if ((err = cudaMemsetAsync(w.counts, 0, sizeof(int32_t) * p.heads * NB, st)) != cudaSuccess) return err;
 
   dim3 gm(NB, p.heads);
+  {
+  KernelTimer kt_(KT_BLOCK_MEAN, st);
   if (D == 128)
     block_mean_kernel<128><<<gm, 128, 0, st>>>(Q, K, plan.blocks, plan.n_blocks, p.H, p.W, p.heads, NB, w.qbar,
                                                w.kbar);
   else
     block_mean_kernel<64><<<gm, 64, 0, st>>>(Q, K, plan.blocks, plan.n_blocks, p.H, p.W, p.heads, NB, w.qbar,
                                              w.kbar);
+  }
   const float scale = effective_scale(p);
   const int tiles = (NB + 127) / 128;
   const size_t sel_smem = (size_t)8 * ((NB + 3) & ~3);
@@ -612,12 +615,18 @@ cudaError_t launch_select(const prism_params &p, const prism_plan_t &plan, const
   for (int h = 0; h < p.heads; ++h) {
     const float *qb = w.qbar + (size_t)h * NB * D;
     const float *kb = w.kbar + (size_t)h * NB * D;
-    if (D == 128)
-      block_score_kernel<128><<<dim3(tiles, tiles), 256, 0, st>>>(qb, kb, plan.n_blocks + h, NB, scale, w.S);
-    else
-      block_score_kernel<64><<<dim3(tiles, tiles), 256, 0, st>>>(qb, kb, plan.n_blocks + h, NB, scale, w.S);
-    select_row_kernel<<<NB, kSelThreads, sel_smem, st>>>(w.S, NB, plan.n_blocks + h, p.topk_frac, p.topk_abs,
-                                                         p.top_p, w.counts + (size_t)h * NB);
+    {
+      KernelTimer kt_(KT_BLOCK_SCORE, st);
+      if (D == 128)
+        block_score_kernel<128><<<dim3(tiles, tiles), 256, 0, st>>>(qb, kb, plan.n_blocks + h, NB, scale, w.S);
+      else
+        block_score_kernel<64><<<dim3(tiles, tiles), 256, 0, st>>>(qb, kb, plan.n_blocks + h, NB, scale, w.S);
+    }
+    {
+      KernelTimer kt_(KT_SELECT_ROW, st);
+      select_row_kernel<<<NB, kSelThreads, sel_smem, st>>>(w.S, NB, plan.n_blocks + h, p.topk_frac, p.topk_abs,
+                                                           p.top_p, w.counts + (size_t)h * NB);
+    }
     scan_kernel<<<1, 1024, 0, st>>>(w.counts + (size_t)h * NB, NB, out.row_ptr + (size_t)h * NB, &w.hdr->nnz,
                                     h == p.heads - 1);
     csr_fill_kernel<<<NB, 128, 0, st>>>(w.S, NB, plan.n_blocks + h, w.counts + (size_t)h * NB,

@@ -278,6 +278,21 @@ const char *prism_last_error(void);
  * (host-side counter, incremented at every launch; never reset). */
 uint64_t prism_kernel_launches(void);
 
+/* Optional timing of the library's main kernels, for measurement.  When
+ * enabled, every launch of the zone-statistics, block-mean, block-score,
+ * row-selection, forward-attention and the two backward-attention kernels is
+ * bracketed by a CUDA event pair recorded on its launching stream.
+ * prism_kernel_timing(1) clears the records and enables; (0) clears and
+ * disables.  Returns PRISM_OK. */
+int prism_kernel_timing(int enable);
+
+/* Reads the records of kernel `id` (0 .. 6, in the order listed above): waits
+ * for its events, and returns the number of timed launches, their total
+ * milliseconds and the kernel's name (library-owned string).  Returns
+ * PRISM_OK, PRISM_ERR_INVALID_ARG (id out of range) or PRISM_ERR_CUDA. */
+int prism_kernel_timing_read(int id, int *launches, double *total_ms,
+                             const char **name);
+
 /* Library version, "major.minor.patch". */
 const char *prism_version(void);
 

@@ -204,11 +204,14 @@ def stored_traffic(kernel):
 
 
 # ----------------------------------------------------------------------------- oracle sample
-def oracle_sample(w, inp, p, pl, sel, head=0, n_rows=2, seed=0):
+def oracle_sample(w, inp, head=0, n_rows=2, seed=0):
     """Time the CPU oracle on a bounded sample of the same layer: the plan and
     the selection of one head over the full grid, and forward+backward
-    attention of `n_rows` random query blocks of that head.  Returns the
-    extrapolated layer time and the sample description."""
+    attention of `n_rows` random query blocks of that head.  The layer time
+    is extrapolated from the oracle's own numbers only: plan and selection
+    times x heads, attention time x (computed pairs of the head's full
+    selection x heads) / (pairs of the sampled blocks).  Returns (layer time,
+    layer computed pairs, description, threads, wall seconds)."""
     from threadpoolctl import threadpool_info
 
     from oracle import prism_oracle as O
@@ -235,15 +238,17 @@ def oracle_sample(w, inp, p, pl, sel, head=0, n_rows=2, seed=0):
         O.attention_bwd(Qh, Kh, Vh, dOh, opl, sub, scale)
     t4 = time.perf_counter()
     pairs_sample = sum(int(hp.blocks[i, 4]) * int(sum(hp.blocks[j, 4] for j in ids)) for (i, ids, _) in sub[0])
-    P_total = computed_pairs(p, pl, sel)
+    pairs_head = sum(int(hp.blocks[i, 4]) * int(hp.blocks[ids, 4].sum()) for (i, ids, _) in osel[0])
+    P_total = pairs_head * w.heads
     attn_time = (t4 - t3) * (P_total / max(pairs_sample, 1))
     layer_time = w.heads * ((t1 - t0) + (t2 - t1)) + attn_time
     threads = max([t.get("num_threads", 1) for t in threadpool_info()] + [1])
     desc = (f"oracle plan+select of head {head} over the full {T}x{H}x{W} grid "
             f"({(t1 - t0):.2f}s + {(t2 - t1):.2f}s, x{w.heads} heads) and fwd"
             f"{'+bwd' if dOh is not None else ''} of {len(rows)} query blocks ({t4 - t3:.2f}s, "
-            f"x{P_total / max(pairs_sample, 1):.0f} by computed pairs); extrapolated layer time {layer_time:.1f}s")
-    return layer_time, desc, threads, (t4 - t0)
+            f"x{P_total / max(pairs_sample, 1):.0f} by computed pairs, the head's pairs x{w.heads} heads); "
+            f"extrapolated layer time {layer_time:.1f}s")
+    return layer_time, P_total, desc, threads, (t4 - t0)
 
 
 # ----------------------------------------------------------------------------- main arms
@@ -374,8 +379,9 @@ def run_prism(args, w, rank, world, device):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        layer_time, desc, threads, wall = oracle_sample(w, inp, p, pl, sel)
-        cpu = {"value": flops / layer_time / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+        layer_time, P_or, desc, threads, wall = oracle_sample(w, inp)
+        flops_or = (4.0 + (10.0 if backward else 0.0)) * P_or * D
+        cpu = {"value": flops_or / layer_time / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": desc, "host_cpus": os.cpu_count(), "sample_wall_s": wall}
 
     density = P / (float(N) * N * h)
@@ -401,29 +407,25 @@ def run_reference(args, w, rank, world):
     extrapolated to the layer by computed pairs."""
     if rank != 0:
         return None
+    # inputs are drawn by the seeded generator (on the GPU when there is one,
+    # only for speed); every computation below is the CPU oracle's
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    inp = make_inputs(w, dev, seed=0)
-    p = api.params_for(w)
-    if dev == "cuda":
-        pl = api.plan(p, inp["V"], inp["a"])
-        sel = api.select(p, pl, inp["Q"], inp["K"])
-    else:
-        raise RuntimeError("the reference arm needs the selection size of the layer (CUDA) for extrapolation")
-    times, desc, threads = [], "", 1
+    inp = make_inputs(w, dev, seed=0)  # oracle_sample moves one head at a time to the host
+    times, rates, desc, threads = [], [], "", 1
     for k in range(args.warmup + args.steps):
-        lt, desc, threads, _wall = oracle_sample(w, inp, p, pl, sel, head=k % w.heads, seed=k)
+        lt, P, desc, threads, _wall = oracle_sample(w, inp, head=k % w.heads, seed=k)
         if k >= args.warmup:
             times.append(lt)
-    P = computed_pairs(p, pl, sel)
-    flops = (4.0 + (10.0 if w.backward else 0.0)) * P * w.head_dim
+            rates.append((4.0 + (10.0 if w.backward else 0.0)) * P * w.head_dim / lt)
     layer = statistics.mean(times)
-    v = flops / layer / 1e12
+    v = statistics.mean(rates) / 1e12
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": layer * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded generator; stands in for the pages' 2K-Bench latents)",
             "config": {"workload": w.name, "T": w.T, "H": w.H, "W": w.W, "tokens": w.N, "heads": w.heads,
-                       "head_dim": w.head_dim, "topk_frac": w.topk_frac, "top_p": w.top_p},
+                       "head_dim": w.head_dim, "topk_frac": w.topk_frac, "top_p": w.top_p, "backward": w.backward,
+                       "parallelism": "rank 0 only (CPU oracle)"},
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 

@@ -221,7 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t id64 = idesc_f16(128, 64, 0), id_dq = idesc_f16(128, D, 1);
-      const uint32_t sQ = smem_u32(smem + L::OFF_Q), sDO = smem_u32(smem + L::OFF_DO);
+      const uint64_t dQd = sdesc_sw128(smem_u32(smem + L::OFF_Q), 16, 1024);
+      const uint64_t dDOd = sdesc_sw128(smem_u32(smem + L::OFF_DO), 16, 1024);
       bool ok = mbar_wait(&bar.qdo_full, 0, status, 22);
       tc_fence_after();
       for (int i = 0; ok && i <= nsteps; ++i) {
@@ -231,12 +232,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait(&bar.k_full[s], (i / NS) & 1, status, 24);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t sK = smem_u32(smem + L::OFF_K + s * L::UNIT);
-          const uint32_t sV = smem_u32(smem + L::OFF_V + s * L::UNIT);
+          const uint64_t dK = sdesc_sw128(smem_u32(smem + L::OFF_K + s * L::UNIT), 16, 1024);
+          const uint64_t dV = sdesc_sw128(smem_u32(smem + L::OFF_V + s * L::UNIT), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tS, sdesc_sw128(sQ + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024),
-                   sdesc_sw128(sK + (kk >> 2) * (64 * 128) + (kk & 3) * 32, 16, 1024), id64, kk > 0 ? 1u : 0u);
+            mma_ss(tS, dQd + kslice16(kk, 128 * 128), dK + kslice16(kk, 64 * 128), id64, kk > 0 ? 1u : 0u);
           mma_commit(&bar.s_full[b]);
           ok = mbar_wait(&bar.v_full[s], (i / NS) & 1, status, 25);
           if (ok && i >= 2) ok = mbar_wait(&bar.dq_done[b], ((i - 2) >> 1) & 1, status, 26);
@@ -244,8 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tP, sdesc_sw128(sDO + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024),
-                   sdesc_sw128(sV + (kk >> 2) * (64 * 128) + (kk & 3) * 32, 16, 1024), id64, kk > 0 ? 1u : 0u);
+            mma_ss(tP, dDOd + kslice16(kk, 128 * 128), dV + kslice16(kk, 64 * 128), id64, kk > 0 ? 1u : 0u);
           mma_commit(&bar.dp_full[b]);
         }
         if (i >= 1) {  // dQ += dS_{i-1} K_{i-1}
@@ -254,10 +253,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait(&bar.ds_ready[b], (jj >> 1) & 1, status, 23);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t sK = smem_u32(smem + L::OFF_K + s * L::UNIT);
+          const uint64_t dKmn = sdesc_sw128(smem_u32(smem + L::OFF_K + s * L::UNIT), 64 * 128, 1024);
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
-            mma_ts(tQ, tP + ks * 8, sdesc_sw128(sK + ks * 2048, 64 * 128, 1024), id_dq, (jj > 0 || ks > 0) ? 1u : 0u);
+            mma_ts(tQ, tP + ks * 8, dKmn + (uint64_t)ks * 128, id_dq, (jj > 0 || ks > 0) ? 1u : 0u);
           mma_commit(&bar.dq_done[b]);
           mma_commit(&bar.kv_empty[s]);
         }
@@ -462,7 +461,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t id64 = idesc_f16(128, 64, 0), id_acc = idesc_f16(128, D, 1);
-      const uint32_t sK = smem_u32(smem + L::OFF_K), sV = smem_u32(smem + L::OFF_V);
+      const uint64_t dKd = sdesc_sw128(smem_u32(smem + L::OFF_K), 16, 1024);
+      const uint64_t dVd = sdesc_sw128(smem_u32(smem + L::OFF_V), 16, 1024);
       bool ok = mbar_wait(&bar.kv_full, 0, status, 42);
       tc_fence_after();
       for (int i = 0; ok && i <= nsteps; ++i) {
@@ -473,20 +473,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok && i >= 2) ok = mbar_wait(&bar.dv_done[b], ((i - 2) >> 1) & 1, status, 45);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t sQ = smem_u32(smem + L::OFF_Q + s * L::UNIT);
-          const uint32_t sDO = smem_u32(smem + L::OFF_DO + s * L::UNIT);
+          const uint64_t dQs = sdesc_sw128(smem_u32(smem + L::OFF_Q + s * L::UNIT), 16, 1024);
+          const uint64_t dDOs = sdesc_sw128(smem_u32(smem + L::OFF_DO + s * L::UNIT), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tS, sdesc_sw128(sK + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024),
-                   sdesc_sw128(sQ + (kk >> 2) * (64 * 128) + (kk & 3) * 32, 16, 1024), id64, kk > 0 ? 1u : 0u);
+            mma_ss(tS, dKd + kslice16(kk, 128 * 128), dQs + kslice16(kk, 64 * 128), id64, kk > 0 ? 1u : 0u);
           mma_commit(&bar.s_full[b]);
           if (i >= 2) ok = mbar_wait(&bar.dk_done[b], ((i - 2) >> 1) & 1, status, 46);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tP, sdesc_sw128(sV + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024),
-                   sdesc_sw128(sDO + (kk >> 2) * (64 * 128) + (kk & 3) * 32, 16, 1024), id64, kk > 0 ? 1u : 0u);
+            mma_ss(tP, dVd + kslice16(kk, 128 * 128), dDOs + kslice16(kk, 64 * 128), id64, kk > 0 ? 1u : 0u);
           mma_commit(&bar.dp_full[b]);
         }
         if (i >= 1) {  // dV += P^T dO, dK += dS^T Q  (step i-1)
@@ -495,15 +493,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait(&bar.ds_ready[b], (jj >> 1) & 1, status, 43);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t sQ = smem_u32(smem + L::OFF_Q + s * L::UNIT);
-          const uint32_t sDO = smem_u32(smem + L::OFF_DO + s * L::UNIT);
+          const uint64_t dQmn = sdesc_sw128(smem_u32(smem + L::OFF_Q + s * L::UNIT), 64 * 128, 1024);
+          const uint64_t dDOmn = sdesc_sw128(smem_u32(smem + L::OFF_DO + s * L::UNIT), 64 * 128, 1024);
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
-            mma_ts(tV, tS + ks * 8, sdesc_sw128(sDO + ks * 2048, 64 * 128, 1024), id_acc, (jj > 0 || ks > 0) ? 1u : 0u);
+            mma_ts(tV, tS + ks * 8, dDOmn + (uint64_t)ks * 128, id_acc, (jj > 0 || ks > 0) ? 1u : 0u);
           mma_commit(&bar.dv_done[b]);
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
-            mma_ts(tK, tP + ks * 8, sdesc_sw128(sQ + ks * 2048, 64 * 128, 1024), id_acc, (jj > 0 || ks > 0) ? 1u : 0u);
+            mma_ts(tK, tP + ks * 8, dQmn + (uint64_t)ks * 128, id_acc, (jj > 0 || ks > 0) ? 1u : 0u);
           mma_commit(&bar.dk_done[b]);
           mma_commit(&bar.q_empty[s]);
         }

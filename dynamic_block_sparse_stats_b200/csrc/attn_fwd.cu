@@ -173,6 +173,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_s_full = idesc_f16(128, 128, 0);
       const uint32_t idesc_s_half = idesc_f16(128, 64, 0);
       const uint32_t idesc_o = idesc_f16(128, D, 1);
+      const uint64_t dQ0 = sdesc_sw128(smem_u32(smem + L::OFF_Q), 16, 1024);
+      const uint64_t dQ1 = sdesc_sw128(smem_u32(smem + L::OFF_Q + L::TILE), 16, 1024);
       bool ok = mbar_wait(&bar.q_full, 0, status, 2);
       tc_fence_after();
       for (int j = 0; ok && j < ntiles; ++j) {
@@ -181,31 +183,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const int nu = bar.meta[s] & 15;
-        const uint32_t sK = smem_u32(smem + L::OFF_K + s * L::TILE);
+        const uint32_t idesc_s = nu == 2 ? idesc_s_full : idesc_s_half;
+        const uint64_t dK = sdesc_sw128(smem_u32(smem + L::OFF_K + s * L::TILE), 16, 1024);
+        const uint64_t dV = sdesc_sw128(smem_u32(smem + L::OFF_V + s * L::TILE), 128 * 128, 1024);
         for (int t = 0; t < 2; ++t) {
           // S_t is free once the PV of the previous key tile read its P
           if (j >= 1) ok = mbar_wait(&bar.pv_done[t], (j - 1) & 1, status, 4);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t sQ = smem_u32(smem + L::OFF_Q + t * L::TILE);
+          const uint64_t dQt = t ? dQ1 : dQ0;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-            mma_ss(tmem + 128 * t, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024),
-                   nu == 2 ? idesc_s_full : idesc_s_half, kk > 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tmem + 128 * t, dQt + kslice16(kk, 128 * 128), dK + kslice16(kk, 128 * 128), idesc_s,
+                   kk > 0 ? 1u : 0u);
           mma_commit(&bar.s_full[t]);
         }
         if (!ok) break;
         ok = mbar_wait(&bar.v_full[s], (j / NSTAGE) & 1, status, 6);
-        const uint32_t sV = smem_u32(smem + L::OFF_V + s * L::TILE);
         for (int t = 0; ok && t < 2; ++t) {
           ok = mbar_wait(&bar.p_full[t], j & 1, status, 5);
           if (!ok) break;
           tc_fence_after();
+          const uint32_t tOt = tmem + 256 + t * D, tPt = tmem + 128 * t;
           for (int ks = 0; ks < nu * 4; ++ks)
-            mma_ts(tmem + 256 + t * D, tmem + 128 * t + ks * 8, sdesc_sw128(sV + ks * 2048, 128 * 128, 1024),
-                   idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
+            mma_ts(tOt, tPt + ks * 8, dV + (uint64_t)ks * 128, idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
           mma_commit(&bar.pv_done[t]);
         }
         mma_commit(&bar.kv_empty[s]);
@@ -232,7 +233,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nu = meta & 15;
       const bool v0 = ((meta >> 4) >> qbit) & 1;
       const bool v1 = nu == 2 && (((meta >> 8) >> qbit) & 1);
-      // pass 1: maximum over the valid columns of this row
+      // Fast path (after the first valid tile): P against the running maximum
+      // in one pass over S, kept packed in registers; it is stored only if no
+      // P reached 2^8, i.e. no row's maximum grew past the lazy threshold.
+      bool done = false;
+      if (__all_sync(0xffffffffu, m > -INFINITY)) {
+        uint32_t pk[64];
+        float2 ls2 = make_float2(0.f, 0.f);
+        uint32_t pmax = 0u;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (c < 2 * nu && ((c < 2) ? v0 : v1)) {  // warp-uniform
+            uint32_t r[32];
+            tmem_ld32(tS + lane_off + c * 32, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              const float2 x = ffma2(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), scale_log2, -m);
+              const float2 p = make_float2(ex2f(x.x), ex2f(x.y));
+              ls2 = fadd2(ls2, p);
+              const uint32_t h2 = pack_f16(p.x, p.y);
+              pmax = hmax2u(pmax, h2);
+              pk[c * 16 + i / 2] = h2;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[c * 16 + i] = 0u;
+          }
+        }
+        // P >= 0, so fp16 bit patterns order like values; 0x5C00 is 256.0
+        const bool over = (pmax & 0xffffu) >= 0x5C00u || (pmax >> 16) >= 0x5C00u;
+        if (!__any_sync(0xffffffffu, over)) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            if (c < 2 * nu) tmem_st16(tS + lane_off + c * 16, &pk[c * 16]);
+          l += ls2.x + ls2.y;
+          done = true;
+        }
+      }
+      if (!done) {
+      // slow path, pass 1: maximum over the valid columns of this row
       float mt = -INFINITY;
       for (int c = 0; c < 2 * nu; ++c) {
         if (!((c < 2) ? v0 : v1)) continue;  // warp-uniform
@@ -240,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tS + lane_off + c * 32, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) mt = fmaxf(mt, fmaxf(__uint_as_float(r[i]), __uint_as_float(r[i + 1])));
+        for (int i = 0; i < 32; i += 2) mt = fmax3f(mt, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
       }
       mt *= scale_log2;
       // A row takes a new reference maximum only when it grows by more than
@@ -269,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         l *= alpha;
         m = m_new;
       }
-      // pass 2: P = exp2(s * scale_log2 - m) in fp16, two keys per column
+      // slow path, pass 2: P = exp2(s * scale_log2 - m) in fp16, two keys per column
       float2 ls = make_float2(0.f, 0.f);
       for (int c = 0; c < 2 * nu; ++c) {
         uint32_t pk[16];
@@ -291,6 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st16(tS + lane_off + c * 16, pk);
       }
       l += ls.x + ls.y;
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar.p_full[t]);

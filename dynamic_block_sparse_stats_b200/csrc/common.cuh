@@ -243,6 +243,14 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   d |= (uint64_t)2 << 61;
   return d;
 }
+// Offset (in the descriptor's 16-byte units) of the 16-element K slice kk of
+// a K-major SW128 tile whose 64-element column chunks are chunk_bytes apart.
+// Adding it to a descriptor is exact: shared-memory addresses stay below
+// 2^18, so the 14-bit address field never carries.
+__host__ __device__ constexpr uint64_t kslice16(int kk, int chunk_bytes) {
+  return (uint64_t)(((kk >> 2) * chunk_bytes + (kk & 3) * 32) >> 4);
+}
+
 // Instruction descriptor for kind::f16 with fp32 accumulation.
 //   bits 4-5 D format (1 = f32), 7-9 A format, 10-12 B format (0 = f16,
 //   1 = bf16; A and B always the same type), 15 A major (0 = K), 16 B major
@@ -263,6 +271,16 @@ __device__ __forceinline__ float ex2f(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t hmax2u(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
 __device__ __forceinline__ uint64_t f2u(float2 a) { return *reinterpret_cast<uint64_t *>(&a); }
 __device__ __forceinline__ float2 u2f(uint64_t a) { return *reinterpret_cast<float2 *>(&a); }

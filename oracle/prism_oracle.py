@@ -104,6 +104,16 @@ def zone_video_stats(Vh, T, H, W):
     return sig2, spatial, temporal
 
 
+def a2v_norm(hhat):
+    """a = ||h_hat||_2 per video token from the bridge output h_hat [N, C]
+    ([DIGEST] zone-guidance section: the vector length of each video
+    position's audio-to-video attention output is its audio injection
+    strength; [REVIEW] Method §1, a_{t,h,w} = ||h_hat_{t,h,w}||_2).
+    float64 from the given (bf16-rounded) values."""
+    h = np.asarray(hhat, dtype=np.float64)
+    return np.sqrt((h * h).sum(axis=1))
+
+
 def zone_a2v_stats(a, T, H, W):
     """Per-zone A2V-norm statistics from a [N] (float64), shared by all heads.
 
@@ -139,14 +149,16 @@ def shares(sig2):
     return out
 
 
-def variation_indicator(r, abar=None, vhat=None, eps=1e-6):
+def variation_indicator(r, abar=None, vhat=None, eps=1e-6, video=True, audio=True):
     """g_d(m) = r_{v,d}(m) + abar(m) * vhat_{a,d}(m) + eps  ([DIGEST]
     equation for g_d(m); [REVIEW] Method §1).  Layer 1 has no cached
     audio-to-video output, so only the video term is used ([DIGEST]
-    zone-guidance section)."""
-    if abar is None:
-        return r + eps
-    return r + abar[:, None] * vhat + eps
+    zone-guidance section).  video=False / audio=False drop a term, as in
+    the guidance ablation ([DIGEST] ablation section)."""
+    g = r if video else np.zeros_like(r)
+    if audio and abar is not None:
+        g = g + abar[:, None] * vhat
+    return g + eps
 
 
 def normalise_by_max(x):
@@ -169,14 +181,16 @@ def volumes(rho, tau128=0.5, tau256=0.25):
     return B, margin
 
 
-def lstar(g, B):
+def lstar(g, B, alpha=0.5):
     """Closed-form optimum of J = sum_d g_d (b_d^2 - 1) subject to
     prod_d b_d = B, in log2 space ([REVIEW] Method §2):
       l*_d = -1/2 log2 g_d + 1/3 (S + 1/2 sum_d' log2 g_d'),  S = log2 B.
+    alpha generalises the exponent of b*_d proportional to g_d^(-alpha)
+    (the mapping ablation of [DIGEST]; 1/2 is the Lagrange value).
     g: [..., 3], B: [...]."""
     lg = np.log2(g)
     S = np.log2(B.astype(np.float64))
-    return -0.5 * lg + (S[..., None] + 0.5 * lg.sum(axis=-1, keepdims=True)) / 3.0
+    return -alpha * lg + (S[..., None] + alpha * lg.sum(axis=-1, keepdims=True)) / 3.0
 
 
 def nearest_shape(ls, B):
@@ -274,12 +288,32 @@ def permutation(T, H, W, blocks):
     return perm
 
 
-def plan(V, a, T, H, W, tau128=0.5, tau256=0.25, eps=1e-6):
+def density_raw(spatial, temporal, abar_raw, mode=0):
+    """rho_raw(m) ([DIGEST] density section: the intra-zone spatial variance
+    plus the temporal frame-difference variance).  The density ablation of
+    [DIGEST] swaps it for the spatial term alone (mode 1), the temporal term
+    alone (2) or the zone's audio strength (3, the zone mean of a)."""
+    if mode == 1:
+        return spatial
+    if mode == 2:
+        return temporal
+    if mode == 3:
+        if abar_raw is None:
+            raise ValueError("density mode 3 needs the A2V norms")
+        return abar_raw
+    return spatial + temporal
+
+
+def plan(V, a, T, H, W, tau128=0.5, tau256=0.25, eps=1e-6, map_exponent=0.5, guidance=0, density=0):
     """Per-head plan ([DIGEST] overview: shapes and sparsity are computed per
-    head and per layer).  V: [N, heads, D] (bf16 values, any float dtype);
-    a: [N] or None (first layer)."""
+    head and per layer).  V: [N, heads, D] (bf16 values, any float dtype;
+    the guidance ablation of [DIGEST] also feeds K or Q here);
+    a: [N] or None (first layer).  map_exponent, guidance (bit 0 drops the
+    video term, bit 1 the A2V term) and density select the ablation
+    variants; their defaults are the method."""
     V = np.asarray(V)
     heads = V.shape[1]
+    abar = vhat = abar_raw = None
     if a is not None:
         abar_raw, sig2a = zone_a2v_stats(np.asarray(a, dtype=np.float64), T, H, W)
         abar = normalise_by_max(abar_raw)
@@ -288,10 +322,10 @@ def plan(V, a, T, H, W, tau128=0.5, tau256=0.25, eps=1e-6):
     for h in range(heads):
         sig2, spatial, temporal = zone_video_stats(V[:, h, :], T, H, W)
         r = shares(sig2)
-        g = variation_indicator(r, abar, vhat, eps) if a is not None else variation_indicator(r, eps=eps)
-        rho = normalise_by_max(spatial + temporal)
+        g = variation_indicator(r, abar, vhat, eps, video=not (guidance & 1), audio=not (guidance & 2))
+        rho = normalise_by_max(density_raw(spatial, temporal, abar_raw, density))
         B, vmargin = volumes(rho, tau128, tau256)
-        sid, smargin = nearest_shape(lstar(g, B), B)
+        sid, smargin = nearest_shape(lstar(g, B, map_exponent), B)
         blocks = head_blocks(T, H, W, sid)
         out.heads.append(HeadPlan(B, sid, g, rho, vmargin, smargin, blocks,
                                   permutation(T, H, W, blocks)))

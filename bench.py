@@ -2,6 +2,7 @@
 """Benchmark of the Prism dynamic block-sparse video self-attention layer.
 
 One step = one pass of the whole path over one synthetic layer:
+prism_a2v_norm (the A2V map from the previous layer's bridge output) ->
 prism_plan -> prism_select -> prism_attn_fwd -> prism_attn_bwd, on the
 native-2K training grid (T=56, H=96, W=160: 860,160 tokens, 24 heads,
 head_dim 128, bf16, Top-k 4%, Top-p 0.9) unless --workload says otherwise.
@@ -34,7 +35,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from dynamic_block_sparse_stats_b200 import _lib, api  # noqa: E402
-from dynamic_block_sparse_stats_b200.synth import WORKLOADS, make_inputs  # noqa: E402
+from dynamic_block_sparse_stats_b200.synth import WORKLOADS, make_bridge_output, make_inputs  # noqa: E402
 
 METRIC = "Prism sparse-attn fwd+bwd ms/layer & effective TFLOP/s at ~860K tokens"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -157,6 +158,8 @@ def kernel_rooflines(ktimes, P, D, N, h, nb, peaks, peak_src, steps):
         "block_mean": ("hbm", 4.0 * N * h * D, "GB/s", "one read of Q and K: 4*N*h*D bytes"),
         "block_score": ("alu", 2.0 * D * sum_nb2, "TFLOP/s", "2*D*sum_h Nb^2 fp32 FLOP (mul + add)"),
         "select_row": ("alu", None, None, "per-row radix selection over N_b scores"),
+        "a2v_norm": ("hbm", 2.0 * N * h * D + 4.0 * N, "GB/s",
+                     "one read of the bridge output (2*N*h*D bytes) + the fp32 norms (4*N)"),
     }
     out = {}
     for name, (n, ms) in ktimes.items():
@@ -221,6 +224,13 @@ def oracle_sample(w, inp, head=0, n_rows=2, seed=0):
     Kh = inp["K"][:, head:head + 1].float().cpu().numpy()
     a = inp["a"].cpu().numpy()
     dOh = inp["dO"][:, head:head + 1].float().cpu().numpy() if "dO" in inp else None
+    # the A2V norms of a row sample of a bridge output, scaled to all N rows
+    n_norm = min(w.N, 16384)
+    hs = make_bridge_output(inp["a"][:n_norm], w.heads * w.head_dim, seed=seed).float().cpu().numpy()
+    tn = time.perf_counter()
+    O.a2v_norm(hs)
+    norm_time = (time.perf_counter() - tn) * (w.N / n_norm)
+    del hs
     t0 = time.perf_counter()
     opl = O.plan(Vh, a, T, H, W)
     t1 = time.perf_counter()
@@ -241,9 +251,10 @@ def oracle_sample(w, inp, head=0, n_rows=2, seed=0):
     pairs_head = sum(int(hp.blocks[i, 4]) * int(hp.blocks[ids, 4].sum()) for (i, ids, _) in osel[0])
     P_total = pairs_head * w.heads
     attn_time = (t4 - t3) * (P_total / max(pairs_sample, 1))
-    layer_time = w.heads * ((t1 - t0) + (t2 - t1)) + attn_time
+    layer_time = norm_time + w.heads * ((t1 - t0) + (t2 - t1)) + attn_time
     threads = max([t.get("num_threads", 1) for t in threadpool_info()] + [1])
-    desc = (f"oracle plan+select of head {head} over the full {T}x{H}x{W} grid "
+    desc = (f"oracle A2V norms of {n_norm} bridge-output rows (x{w.N / n_norm:.1f}, {norm_time:.2f}s), "
+            f"plan+select of head {head} over the full {T}x{H}x{W} grid "
             f"({(t1 - t0):.2f}s + {(t2 - t1):.2f}s, x{w.heads} heads) and fwd"
             f"{'+bwd' if dOh is not None else ''} of {len(rows)} query blocks ({t4 - t3:.2f}s, "
             f"x{P_total / max(pairs_sample, 1):.0f} by computed pairs, the head's pairs x{w.heads} heads); "
@@ -252,15 +263,60 @@ def oracle_sample(w, inp, head=0, n_rows=2, seed=0):
 
 
 # ----------------------------------------------------------------------------- main arms
+def dense_sdpa(inp, w, backward, heads=1, iters=2):
+    """Dense bf16 attention (torch scaled_dot_product_attention) over the same
+    tokens on the same GPU, timed on `heads` of the layer's heads and scaled to
+    all of them (heads are independent and equal in cost).  The fastest
+    available backend is tried first; the one that ran is reported."""
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    import torch.nn.functional as F
+    N, D = w.N, w.head_dim
+    sub = [inp[k][:, :heads, :].permute(1, 0, 2).unsqueeze(0).contiguous() for k in ("Q", "K", "V")]
+    dO = inp["dO"][:, :heads, :].permute(1, 0, 2).unsqueeze(0).contiguous() if backward else None
+    stream = torch.cuda.current_stream()
+    for be in (SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION):
+        try:
+            q, k, v = (t.detach().requires_grad_(backward) for t in sub)
+
+            def run():
+                with sdpa_kernel(be):
+                    o = F.scaled_dot_product_attention(q, k, v)
+                    if backward:
+                        torch.autograd.grad(o, (q, k, v), dO)
+
+            run()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(iters):
+                run()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms_heads = e0.elapsed_time(e1) / iters
+            ms = ms_heads * w.heads / heads
+            flops = (4.0 + (10.0 if backward else 0.0)) * float(N) * N * D * w.heads
+            return {"backend": be.name, "ms_per_layer": ms, "TFLOPs": flops / (ms * 1e-3) / 1e12,
+                    "pass": "fwd+bwd" if backward else "fwd",
+                    "sample": f"{heads} of {w.heads} heads over all {N} tokens, x{w.heads // heads}",
+                    "iters": iters}
+        except RuntimeError as e:  # backend refuses the shape: try the next one
+            last = f"{be.name}: {str(e).splitlines()[0][:160]}"
+    return {"unavailable": last}
+
+
 def run_prism(args, w, rank, world, device):
     lib = _lib.load()
     p = api.params_for(w)
     inp = make_inputs(w, device, seed=rank_seed(rank))
     N, h, D = w.N, w.heads, w.head_dim
-    Q, K, V, a = inp["Q"], inp["K"], inp["V"], inp["a"]
+    Q, K, V = inp["Q"], inp["K"], inp["V"]
+    # the previous layer's bridge output, whose row norms are this layer's A2V map
+    hhat = make_bridge_output(inp["a"], h * D, seed=rank_seed(rank))
+    inp["hhat"] = hhat
     dO = inp.get("dO")
     backward = dO is not None
     # buffers reused by every step
+    a = api.a2v_norm(hhat)
     pl = api.plan(p, V, a)
     sel = api.select(p, pl, Q, K)
     sel = api.select(p, pl, Q, K, cap=int(sel.nnz * 1.1) + 1024)
@@ -277,6 +333,7 @@ def run_prism(args, w, rank, world, device):
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
+        api.a2v_norm(hhat, out=a)
         api.plan(p, V, a, out=pl)
         if ev is not None:
             ev[1].record(stream)
@@ -327,10 +384,10 @@ def run_prism(args, w, rank, world, device):
     # end to end through host buffers
     e2e = None
     if not args.no_e2e:
-        hin = {k: inp[k].cpu().pin_memory() for k in (["Q", "K", "V", "a"] + (["dO"] if backward else []))}
+        hin = {k: inp[k].cpu().pin_memory() for k in (["Q", "K", "V", "hhat"] + (["dO"] if backward else []))}
         outs = [O_] + (list(grads) if backward else [])
         hout = [torch.empty_like(t, device="cpu").pin_memory() for t in outs]
-        dev = {"Q": Q, "K": K, "V": V, "a": a, "dO": dO}
+        dev = {"Q": Q, "K": K, "V": V, "hhat": hhat, "dO": dO}
         h2d = sum(t.numel() * t.element_size() for t in hin.values())
         d2h = sum(t.numel() * t.element_size() for t in hout)
 
@@ -369,7 +426,8 @@ def run_prism(args, w, rank, world, device):
                 "traffic": stored_traffic(dom), "algorithmic": kd["algorithmic"],
                 "ms_per_launch": kd["ms_per_launch"]}
     peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
-    plan_bytes = N * h * D * 2 + N * 4
+    plan_bytes = N * h * D * 2 + N * 4        # the plan stage reads V and a; a2v_norm is in it too
+    plan_bytes += N * h * D * 2 + N * 4
     stage_roofline = {
         "plan_GBps": plan_bytes / (stage_ms["plan"] * 1e-3) / 1e9,
         "plan_frac_hbm": plan_bytes / (stage_ms["plan"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
@@ -384,6 +442,12 @@ def run_prism(args, w, rank, world, device):
         cpu = {"value": flops_or / layer_time / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": desc, "host_cpus": os.cpu_count(), "sample_wall_s": wall}
 
+    dense = None
+    if not args.no_dense:
+        dense = dense_sdpa(inp, w, backward)
+        if "ms_per_layer" in dense:
+            dense["speedup_of_prism_step"] = dense["ms_per_layer"] / ms
+
     density = P / (float(N) * N * h)
     line = {
         "metric": METRIC, "value": whole_job_rate(flops, world, ms_max) / 1e12, "unit": "TFLOP/s",
@@ -397,6 +461,7 @@ def run_prism(args, w, rank, world, device):
                    "pairs": P, "pair_density": density, "nnz_blocks": sel.nnz},
         "stage_ms": stage_ms, "stage_roofline": stage_roofline, "kernels": kernels,
         "clocks": clocks, "e2e": e2e, "gpu_launches": launches, "roofline": roofline, "cpu_baseline": cpu,
+        "dense_sdpa": dense,
     }
     return line
 
@@ -440,6 +505,7 @@ def main():
     ap.add_argument("--backward", action="store_true", help="time the backward on any workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense SDPA comparison")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

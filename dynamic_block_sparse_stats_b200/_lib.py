@@ -27,15 +27,16 @@ EXPORTS = (
     "prism_plan_workspace_size", "prism_plan", "prism_select_workspace_size", "prism_select",
     "prism_attn_workspace_size", "prism_attn_fwd", "prism_attn_bwd", "prism_workspace_status",
     "prism_last_error", "prism_version", "prism_kernel_launches", "prism_plan_noalloc",
-    "prism_kernel_timing", "prism_kernel_timing_read",
+    "prism_kernel_timing", "prism_kernel_timing_read", "prism_a2v_norm",
 )
-KERNEL_TIMING_IDS = 7
+KERNEL_TIMING_IDS = 8
 
 
 class PrismParams(C.Structure):
     _fields_ = [("T", C.c_int32), ("H", C.c_int32), ("W", C.c_int32), ("heads", C.c_int32),
                 ("head_dim", C.c_int32), ("tau128", C.c_float), ("tau256", C.c_float), ("eps", C.c_float),
-                ("topk_frac", C.c_float), ("topk_abs", C.c_int32), ("top_p", C.c_float), ("sm_scale", C.c_float)]
+                ("topk_frac", C.c_float), ("topk_abs", C.c_int32), ("top_p", C.c_float), ("sm_scale", C.c_float),
+                ("map_exponent", C.c_float), ("guidance", C.c_int32), ("density", C.c_int32)]
 
 
 class PrismPlan(C.Structure):
@@ -85,6 +86,7 @@ def load() -> C.CDLL:
         "prism_plan_noalloc": (C.c_int, [P(PrismParams), vp, vp, P(PrismPlan), st]),
         "prism_kernel_timing": (C.c_int, [C.c_int]),
         "prism_kernel_timing_read": (C.c_int, [C.c_int, P(C.c_int), P(C.c_double), P(C.c_char_p)]),
+        "prism_a2v_norm": (C.c_int, [vp, C.c_int64, C.c_int32, C.c_int64, vp, st]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)

@@ -17,9 +17,17 @@ from . import _lib
 from ._lib import PrismParams, PrismPlan, PrismSelect, check
 
 
+# guidance bits and density modes of the ablation variants (include/prism.h)
+GUIDE_NO_VIDEO, GUIDE_NO_A2V = 1, 2
+DENSITY_BOTH, DENSITY_SPATIAL, DENSITY_TEMPORAL, DENSITY_A2V = 0, 1, 2, 3
+
+
 def params(T, H, W, heads, head_dim, topk_frac=0.0, topk_abs=0, top_p=0.9, tau128=0.5, tau256=0.25,
-           eps=1e-6, sm_scale=0.0) -> PrismParams:
-    return PrismParams(T, H, W, heads, head_dim, tau128, tau256, eps, topk_frac, topk_abs, top_p, sm_scale)
+           eps=1e-6, sm_scale=0.0, map_exponent=0.0, guidance=0, density=0) -> PrismParams:
+    """Layer parameters; map_exponent 0 means the Lagrange value 1/2, and
+    guidance = density = 0 is the method as published."""
+    return PrismParams(T, H, W, heads, head_dim, tau128, tau256, eps, topk_frac, topk_abs, top_p, sm_scale,
+                       map_exponent, guidance, density)
 
 
 def params_for(w, **over) -> PrismParams:
@@ -52,6 +60,22 @@ def _check_tensor(t, name, dtype, shape):
 def _workspace(nbytes, device):
     # 256-byte alignment is guaranteed by the CUDA caching allocator
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def a2v_norm(hhat: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """prism_a2v_norm: ||h_hat||_2 of every row of the bf16 bridge output
+    h_hat [N, width] (rows may be strided; width a multiple of 8) -> fp32 [N],
+    the a2v_norm input of the next layer's plan."""
+    if not hhat.is_cuda or hhat.dtype != torch.bfloat16 or hhat.dim() != 2:
+        raise ValueError("hhat must be a 2-D bf16 CUDA tensor [N, width]")
+    if hhat.stride(1) != 1:
+        raise ValueError("hhat rows must be contiguous")
+    n, width = hhat.shape
+    out = out if out is not None else torch.empty((n,), dtype=torch.float32, device=hhat.device)
+    _check_tensor(out, "a2v_norm", torch.float32, (n,))
+    ld = hhat.stride(0) if n > 1 else width
+    check(_lib.load().prism_a2v_norm(_ptr(hhat), n, width, ld, _ptr(out), _stream(stream)))
+    return out
 
 
 @dataclass

@@ -57,6 +57,10 @@ static int check_params(const prism_params *p) {
   if (p->topk_abs < 0 || !(p->topk_frac >= 0.f) || !isfinite(p->topk_frac))
     return fail(PRISM_ERR_INVALID_ARG, "top-k must be non-negative");
   if (p->sm_scale < 0.f || !isfinite(p->sm_scale)) return fail(PRISM_ERR_INVALID_ARG, "sm_scale must be >= 0");
+  if (!(p->map_exponent >= 0.f && p->map_exponent <= 8.f))
+    return fail(PRISM_ERR_INVALID_ARG, "map_exponent must lie in [0, 8] (0 selects 1/2)");
+  if (p->guidance < 0 || p->guidance > 3) return fail(PRISM_ERR_INVALID_ARG, "guidance must be 0..3");
+  if (p->density < 0 || p->density > 3) return fail(PRISM_ERR_INVALID_ARG, "density must be 0..3");
   return PRISM_OK;
 }
 
@@ -74,10 +78,11 @@ static int check_ws(void *ws, size_t bytes, size_t need) {
 }
 
 // Argument checks of prism_plan, for other entry points that plan the same way.
-int check_plan_call(const prism_params *p, const uint16_t *V, const prism_plan_t *out) {
+int check_plan_call(const prism_params *p, const uint16_t *V, const float *a2v_norm, const prism_plan_t *out) {
   int rc;
   if ((rc = check_params(p)) != PRISM_OK) return rc;
   if (!V) return fail(PRISM_ERR_INVALID_ARG, "V is NULL");
+  if (p->density == 3 && !a2v_norm) return fail(PRISM_ERR_INVALID_ARG, "density 3 (A2V strength) needs a2v_norm");
   return check_plan(out);
 }
 
@@ -105,9 +110,7 @@ size_t prism_plan_workspace_size(const prism_params *p) {
 int prism_plan(const prism_params *p, const uint16_t *V, const float *a2v_norm, const prism_plan_t *out,
                void *workspace, size_t ws_bytes, prism_stream_t stream) {
   int rc;
-  if ((rc = check_params(p)) != PRISM_OK) return rc;
-  if (!V) return fail(PRISM_ERR_INVALID_ARG, "V is NULL");
-  if ((rc = check_plan(out)) != PRISM_OK) return rc;
+  if ((rc = check_plan_call(p, V, a2v_norm, out)) != PRISM_OK) return rc;
   if ((rc = check_ws(workspace, ws_bytes, plan_ws_bytes(*p))) != PRISM_OK) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(workspace, 0, kWsHeader, st);

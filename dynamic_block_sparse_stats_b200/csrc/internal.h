@@ -67,6 +67,7 @@ enum KernelTimingId {
   KT_ATTN_FWD,
   KT_ATTN_DKDV,
   KT_ATTN_DQ,
+  KT_A2V_NORM,
   KT_COUNT
 };
 // Records an event on `st` at construction and at destruction when timing is
@@ -82,7 +83,7 @@ class KernelTimer {
 };
 
 // api.cu: prism_plan's argument checks; error reporting for prism_last_error
-int check_plan_call(const prism_params *p, const uint16_t *V, const prism_plan_t *out);
+int check_plan_call(const prism_params *p, const uint16_t *V, const float *a2v_norm, const prism_plan_t *out);
 int report_error(int code, const char *msg);
 void clear_error();
 

@@ -247,7 +247,9 @@ __device__ __forceinline__ double block_max_d(double v, double *sh) {
 __global__ void __launch_bounds__(1024) plan_finalize_kernel(const double *__restrict__ vstats,
                                                              const double *__restrict__ astats, int Z, int T,
                                                              int H, int W, int heads, int NB, float tau128,
-                                                             float tau256, float eps, uint8_t *__restrict__ zone_shape,
+                                                             float tau256, float eps, float map_exponent,
+                                                             int guidance, int density,
+                                                             uint8_t *__restrict__ zone_shape,
                                                              double *__restrict__ zone_g,
                                                              double *__restrict__ zone_rho,
                                                              int32_t *__restrict__ n_blocks,
@@ -259,9 +261,18 @@ __global__ void __launch_bounds__(1024) plan_finalize_kernel(const double *__res
   const int h = blockIdx.x;
   const double *vs = vstats + (size_t)h * Z * 5;
 
+  // rho_raw(m) of the chosen density variant (0: spatial + temporal terms)
+  auto rho_raw = [&](int m) -> double {
+    switch (density) {
+      case 1: return vs[m * 5 + 3];
+      case 2: return vs[m * 5 + 4];
+      case 3: return astats[m * 4 + 0];
+      default: return vs[m * 5 + 3] + vs[m * 5 + 4];
+    }
+  };
   double mx = 0.0, ma = 0.0;
   for (int m = threadIdx.x; m < Z; m += blockDim.x) {
-    mx = max(mx, vs[m * 5 + 3] + vs[m * 5 + 4]);
+    mx = max(mx, rho_raw(m));
     if (astats) ma = max(ma, astats[m * 4 + 0]);
   }
   const double rho_max = block_max_d(mx, sh);
@@ -279,21 +290,24 @@ __global__ void __launch_bounds__(1024) plan_finalize_kernel(const double *__res
       const double sv = s[0] + s[1] + s[2];
       double r[3];
       for (int d = 0; d < 3; ++d) r[d] = sv > 0.0 ? s[d] / sv : (1.0 / 3.0);
+      // g_d = r_{v,d} + abar * vhat_{a,d} + eps, less the terms the guidance variant drops
       double g[3];
-      if (astats) {
+      for (int d = 0; d < 3; ++d) g[d] = (guidance & 1) ? 0.0 : r[d];
+      if (astats && !(guidance & 2)) {
         const double *as = astats + (size_t)m * 4;
         const double abar = a_max > 0.0 ? as[0] / a_max : 0.0;
         const double sa = as[1] + as[2] + as[3];
-        for (int d = 0; d < 3; ++d) g[d] = r[d] + abar * (sa > 0.0 ? as[1 + d] / sa : (1.0 / 3.0)) + e;
-      } else {
-        for (int d = 0; d < 3; ++d) g[d] = r[d] + e;
+        for (int d = 0; d < 3; ++d) g[d] = g[d] + abar * (sa > 0.0 ? as[1 + d] / sa : (1.0 / 3.0));
       }
-      const double rho = rho_max > 0.0 ? (s[3] + s[4]) / rho_max : 0.0;
+      for (int d = 0; d < 3; ++d) g[d] = g[d] + e;
+      const double rho = rho_max > 0.0 ? rho_raw(m) / rho_max : 0.0;
       vol = rho >= t128 ? 64 : (rho >= t256 ? 128 : 256);
       const double S = vol == 64 ? 6.0 : (vol == 128 ? 7.0 : 8.0);
+      // l*_d for b*_d proportional to g_d^(-alpha); alpha = 1/2 is the Lagrange optimum of J
+      const double alpha = map_exponent > 0.f ? (double)map_exponent : 0.5;
       const double lg0 = log2(g[0]), lg1 = log2(g[1]), lg2 = log2(g[2]);
-      const double shift = (S + 0.5 * (lg0 + lg1 + lg2)) / 3.0;
-      const double l0 = -0.5 * lg0 + shift, l1 = -0.5 * lg1 + shift, l2 = -0.5 * lg2 + shift;
+      const double shift = (S + alpha * (lg0 + lg1 + lg2)) / 3.0;
+      const double l0 = -alpha * lg0 + shift, l1 = -alpha * lg1 + shift, l2 = -alpha * lg2 + shift;
       double best = 1.0e300;
       for (int c = 0; c < 16; ++c) {
         if (c_shapes.vol[c] != vol) continue;
@@ -419,7 +433,8 @@ cudaError_t launch_plan(const prism_params &p, const uint16_t *V, const float *a
   }
   if (a) zone_a2v_stats_kernel<<<Z, 64, 0, st>>>(a, p.T, p.H, p.W, astats);
   plan_finalize_kernel<<<p.heads, 1024, 0, st>>>(vstats, a ? astats : nullptr, Z, p.T, p.H, p.W, p.heads, NB,
-                                                 p.tau128, p.tau256, p.eps, out.zone_shape, out.zone_g,
+                                                 p.tau128, p.tau256, p.eps, p.map_exponent, p.guidance,
+                                                 p.density, out.zone_shape, out.zone_g,
                                                  out.zone_rho, out.n_blocks, out.blocks, zone_first);
   dim3 g3((N + 255) / 256, p.heads);
   perm_kernel<<<g3, 256, 0, st>>>(out.zone_shape, p.T, p.H, p.W, Z, out.perm, out.inv_perm);

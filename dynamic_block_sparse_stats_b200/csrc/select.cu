@@ -142,10 +142,15 @@ __global__ void __launch_bounds__(256) block_score_kernel(const float *__restric
 // ---------------------------------------------------------------------------
 // K5b: hybrid selection of one query block (row).  Scores become ordered
 // uint32 keys (larger score -> larger key).  e_j = exp(s_j - max) in fp32 from
-// the exact float64 difference; Top-p sums in float64.  A most-significant-
-// byte radix descent over the keys finds the Top-p crossing key and the
-// Top-k threshold without sorting; the kept ids are emitted in ascending
-// order into the row's own scratch, and the count into counts[i].
+// the exact float64 difference, then quantised to an integer multiple of
+// 2^-qb (qb chosen so that the row's total fits 62 bits; quantum <= 2^-48 at
+// the 2K grid).  Top-p sums are exact integer sums of those, so the crossing
+// does not depend on the order of the atomic additions: the selection is
+// deterministic.  With p >= 1 every block is kept (in exact arithmetic the
+// cumulative probability reaches 1 only at the last block).  A
+// most-significant-byte radix descent over the keys finds the Top-p crossing
+// key and the Top-k threshold without sorting; the kept ids are emitted in
+// ascending order into the row's own scratch, and the count into counts[i].
 // ---------------------------------------------------------------------------
 constexpr int kSelThreads = 512;
 
@@ -165,30 +170,35 @@ __device__ __forceinline__ float score_weight(float s, double m) {
   return fmaf(ex, xl, ex);  // exp(xh) * (1 + xl)
 }
 
+// quantised weight: round(e * 2^qb), e in [0, 1]
+__device__ __forceinline__ unsigned long long quant_weight(float e, double qscale) {
+  return __double2ull_rn((double)e * qscale);
+}
+
 struct SelShared {
   int hcnt[256];
-  double hsum[256];
+  unsigned long long hsum[256];
   int wtot[kSelThreads / 32];
   int wtot2[kSelThreads / 32];
-  double dred[kSelThreads / 32];
+  unsigned long long zred[kSelThreads / 32];
   uint32_t ured[kSelThreads / 32];
   // descent state broadcast
   uint32_t prefix;
   int found;
   int cabove;
-  double sabove;
+  unsigned long long sabove;
 };
 
 // Descending scan of the 256-bucket histogram by warp 0.  Finds the first
 // bucket (from the top) where `above + running >= target` (sum mode) or
 // `cabove + running count >= target_n` (count mode).  Returns bucket or -1.
-__device__ void bucket_descent(SelShared &sh, bool by_sum, double target, int target_n, int shift) {
+__device__ void bucket_descent(SelShared &sh, bool by_sum, unsigned long long target, int target_n, int shift) {
   const int lane = threadIdx.x & 31;
   // lane l owns buckets 255-8l ... 255-8l-7 (descending)
   int c[8];
-  double s[8];
+  unsigned long long s[8];
   int csum = 0;
-  double ssum = 0.0;
+  unsigned long long ssum = 0;
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     const int b = 255 - 8 * lane - k;
@@ -198,11 +208,11 @@ __device__ void bucket_descent(SelShared &sh, bool by_sum, double target, int ta
     ssum += s[k];
   }
   int cex = csum;
-  double sex = ssum;
+  unsigned long long sex = ssum;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int yc = __shfl_up_sync(0xffffffffu, cex, o);
-    const double ys = __shfl_up_sync(0xffffffffu, sex, o);
+    const unsigned long long ys = __shfl_up_sync(0xffffffffu, sex, o);
     if (lane >= o) {
       cex += yc;
       sex += ys;
@@ -211,10 +221,10 @@ __device__ void bucket_descent(SelShared &sh, bool by_sum, double target, int ta
   cex -= csum;  // exclusive
   sex -= ssum;
   int hit = -1, hc = 0;
-  double hs = 0.0;
+  unsigned long long hs = 0;
   {
     int rc = cex;
-    double rs = sex;
+    unsigned long long rs = sex;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const bool reach = by_sum ? (sh.sabove + rs + s[k] >= target) : (sh.cabove + rc + c[k] >= target_n);
@@ -302,18 +312,20 @@ __global__ void __launch_bounds__(kSelThreads) select_row_kernel(float *__restri
   for (int w = 0; w < kSelThreads / 32; ++w) kmax = max(kmax, sh.ured[w]);
   const double m = (double)key_score(kmax);
 
-  // 2. weights and their total
-  double zp = 0.0;
+  // 2. weights, quantised to multiples of 2^-qb, and their exact total
+  const int qb = 62 - (32 - __clz(nb));  // nb < 2^(32 - clz(nb)), so the total stays below 2^62
+  const double qscale = ldexp(1.0, qb);
+  unsigned long long zp = 0;
   for (int j = tid; j < nb; j += kSelThreads) {
     const float e = score_weight(key_score(key[j]), m);
     ev[j] = e;
-    zp += (double)e;
+    zp += quant_weight(e, qscale);
   }
   zp = warp_sum(zp);
-  if (lane == 0) sh.dred[warp] = zp;
+  if (lane == 0) sh.zred[warp] = zp;
   __syncthreads();
-  double Z = 0.0;
-  for (int w = 0; w < kSelThreads / 32; ++w) Z += sh.dred[w];
+  unsigned long long Z = 0;
+  for (int w = 0; w < kSelThreads / 32; ++w) Z += sh.zred[w];
 
   // 3. counts: k and n_p
   int k;
@@ -321,17 +333,31 @@ __global__ void __launch_bounds__(kSelThreads) select_row_kernel(float *__restri
     k = min(nb, topk_abs);
   else
     k = min(nb, max(1, (int)ceil((double)topk_frac * (double)nb)));
-  const double target = (double)top_p * Z;
+  // target = ceil(p * Z) exactly: p = pm * 2^(e2 - 24) with a 24-bit integer pm
+  unsigned long long target = 0;
+  if (top_p > 0.0f && top_p < 1.0f) {
+    int e2;
+    const float mant = frexpf(top_p, &e2);
+    const unsigned long long pm = (unsigned long long)ldexpf(mant, 24);
+    const unsigned __int128 prod = (unsigned __int128)pm * Z;
+    const int rs = 24 - e2;  // >= 24 for p < 1
+    if (rs >= 127)
+      target = prod != 0 ? 1ull : 0ull;
+    else
+      target = (unsigned long long)((prod + (((unsigned __int128)1 << rs) - 1)) >> rs);
+  }
 
   int n_p = 0;
   uint32_t thr = 0;
   int need = 0;
   bool have_thr = false;
-  if (top_p > 0.0f) {
+  if (top_p >= 1.0f) {
+    n_p = nb;
+  } else if (top_p > 0.0f) {
     if (tid == 0) {
       sh.prefix = 0;
       sh.cabove = 0;
-      sh.sabove = 0.0;
+      sh.sabove = 0;
       sh.found = 1;
     }
     __syncthreads();
@@ -341,7 +367,7 @@ __global__ void __launch_bounds__(kSelThreads) select_row_kernel(float *__restri
       const int shift = 24 - 8 * level;
       for (int b = tid; b < 256; b += kSelThreads) {
         sh.hcnt[b] = 0;
-        sh.hsum[b] = 0.0;
+        sh.hsum[b] = 0;
       }
       __syncthreads();
       const uint32_t prefix = sh.prefix;
@@ -350,7 +376,7 @@ __global__ void __launch_bounds__(kSelThreads) select_row_kernel(float *__restri
         if ((u & pmask) == prefix) {
           const int b = (u >> shift) & 255;
           atomicAdd(&sh.hcnt[b], 1);
-          atomicAdd(&sh.hsum[b], (double)ev[j]);
+          atomicAdd(&sh.hsum[b], quant_weight(ev[j], qscale));
         }
       }
       __syncthreads();
@@ -363,16 +389,16 @@ __global__ void __launch_bounds__(kSelThreads) select_row_kernel(float *__restri
       pmask |= 0xffu << shift;
     }
     if (!ok) {
-      n_p = nb;  // the cumulative sum never reaches p (rounding, p >= 1)
+      n_p = nb;  // cannot happen for p < 1 (target <= Z); kept as a safe bound
     } else {
+      // every key of the final bucket is the same score, hence the same weight
       const uint32_t ustar = sh.prefix;
       const int cstar = sh.hcnt[ustar & 255];
-      const double estar = (double)score_weight(key_score(ustar), m);
-      const double sab = sh.sabove;
-      int q = (int)ceil((target - sab) / estar);
+      const unsigned long long estar = quant_weight(score_weight(key_score(ustar), m), qscale);
+      const unsigned long long sab = sh.sabove;
+      int q = 1;
+      if (estar > 0 && target > sab) q = (int)min((unsigned long long)cstar, (target - sab + estar - 1) / estar);
       q = max(1, min(q, cstar));
-      while (q > 1 && sab + (double)(q - 1) * estar >= target) --q;
-      while (q < cstar && sab + (double)q * estar < target) ++q;
       n_p = sh.cabove + q;
       thr = ustar;
       need = q;
@@ -386,7 +412,7 @@ __global__ void __launch_bounds__(kSelThreads) select_row_kernel(float *__restri
     if (tid == 0) {
       sh.prefix = 0;
       sh.cabove = 0;
-      sh.sabove = 0.0;
+      sh.sabove = 0;
       sh.found = 1;
     }
     __syncthreads();
@@ -395,7 +421,7 @@ __global__ void __launch_bounds__(kSelThreads) select_row_kernel(float *__restri
       const int shift = 24 - 8 * level;
       for (int b = tid; b < 256; b += kSelThreads) {
         sh.hcnt[b] = 0;
-        sh.hsum[b] = 0.0;
+        sh.hsum[b] = 0;
       }
       __syncthreads();
       const uint32_t prefix = sh.prefix;
@@ -404,7 +430,7 @@ __global__ void __launch_bounds__(kSelThreads) select_row_kernel(float *__restri
         if ((u & pmask) == prefix) atomicAdd(&sh.hcnt[(u >> shift) & 255], 1);
       }
       __syncthreads();
-      if (warp == 0) bucket_descent(sh, false, 0.0, n, shift);
+      if (warp == 0) bucket_descent(sh, false, 0ull, n, shift);
       __syncthreads();
       pmask |= 0xffu << shift;
     }

@@ -9,7 +9,7 @@ namespace prism {
 namespace {
 
 const char *const kNames[KT_COUNT] = {"zone_video_stats", "block_mean", "block_score", "select_row",
-                                      "attn_fwd",         "attn_bwd_dkdv", "attn_bwd_dq"};
+                                      "attn_fwd",         "attn_bwd_dkdv", "attn_bwd_dq", "a2v_norm"};
 
 struct Rec {
   cudaEvent_t a, b;

@@ -87,7 +87,7 @@ WORKLOADS = {
 }
 
 # tensor ids used as generator streams
-_ID_VBG, _ID_VREG, _ID_F, _ID_N1, _ID_N2, _ID_ANOISE, _ID_DO, _ID_LAYOUT = range(1, 9)
+_ID_VBG, _ID_VREG, _ID_F, _ID_N1, _ID_N2, _ID_ANOISE, _ID_DO, _ID_LAYOUT, _ID_HHAT = range(1, 10)
 _CHUNK = 256  # channels per generation chunk (fixed, so bits do not depend on memory)
 
 
@@ -300,4 +300,21 @@ def make_inputs(w: Workload | str, device="cpu", seed: int = 0, with_grad: bool 
     if with_grad:
         out["dO"] = torch.randn((N, h, D), generator=_gen(device, seed, _ID_DO),
                                 device=device).to(torch.bfloat16)
+    return out
+
+
+def make_bridge_output(a: torch.Tensor, width: int, seed: int = 0) -> torch.Tensor:
+    """A stand-in for a layer's audio-to-video bridge output h_hat, bf16
+    [N, width] on a's device: row n is (a[n] / sqrt(width)) * z_n with z_n
+    i.i.d. N(0, 1), so its length is a[n] up to chi-distribution spread
+    (relative ~ 1/sqrt(2 width)).  The norms of its rows carry the A2V map
+    of the workload; nothing here computes them."""
+    N = a.numel()
+    out = torch.empty((N, width), dtype=torch.bfloat16, device=a.device)
+    scale = (a.float() / math.sqrt(width)).view(N, 1)
+    for c0 in range(0, width, _CHUNK):
+        c1 = min(width, c0 + _CHUNK)
+        z = torch.randn((N, c1 - c0), generator=_gen(a.device, seed, _ID_HHAT, c0 // _CHUNK), device=a.device)
+        out[:, c0:c1] = (scale * z).to(torch.bfloat16)
+        del z
     return out

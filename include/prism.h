@@ -74,6 +74,22 @@ typedef enum prism_status {
  *                  benchmark grids).
  *   sm_scale       attention scale; 0 selects 1/sqrt(head_dim).  The same
  *                  scale multiplies the block scores.
+ *
+ * Ablation variants (digest, section on the shape, guidance and sparsity
+ * ablations).  Zero in all three fields is the method as published; the
+ * pages' Top-k-only and Top-p-only settings need no field: top_p = 0 keeps
+ * the Top-k prefix alone, and topk_frac = topk_abs = 0 (k = 1) leaves Top-p.
+ *   map_exponent   a in b*_d proportional to g_d^(-a):
+ *                  l*_d = -a log2 g_d + (S + a sum_d' log2 g_d')/3.  0 selects
+ *                  the Lagrange value 1/2.  Any value in (0, 8].  (a = 0, the
+ *                  isotropic mapping, is guidance = 3.)
+ *   guidance       bit 0 drops the video term r_{v,d} from g_d, bit 1 drops
+ *                  the A2V term abar*vhat_{a,d}.  guidance = 3 leaves
+ *                  g_d = eps: isotropic shapes.
+ *   density        what rho_raw(m) is: 0 spatial + temporal terms (the
+ *                  method), 1 the spatial term only, 2 the temporal term
+ *                  only, 3 the zone's A2V strength (zone mean of a2v_norm;
+ *                  the heads then share rho; needs a2v_norm).
  */
 typedef struct prism_params {
   int32_t T, H, W;
@@ -83,6 +99,9 @@ typedef struct prism_params {
   int32_t topk_abs;
   float top_p;
   float sm_scale;
+  float map_exponent;
+  int32_t guidance;
+  int32_t density;
 } prism_params;
 
 /*
@@ -114,6 +133,27 @@ typedef struct prism_plan_t {
   int32_t *inv_perm;
 } prism_plan_t;
 
+/*
+ * prism_a2v_norm -- the A2V guidance signal a = ||h_hat||_2 per video token
+ * (digest, section on the zone guidance signals: the length of each video
+ * position's audio-to-video cross-attention output; review, Method
+ * section 1, a_{t,h,w} = ||h_hat_{t,h,w}||_2).  Run it on a layer's bridge
+ * output; the next layer's prism_plan takes the result as a2v_norm.
+ *   hhat      bf16 [n][ld] device rows (natural token order); only the first
+ *             `width` elements of each row are read.  16-byte aligned.
+ *   n         number of video tokens (rows), >= 0; 0 launches nothing.
+ *   width     channels per row (the bridge output width, e.g. heads *
+ *             head_dim), a positive multiple of 8, at most 2^20.
+ *   ld        row stride in elements, a multiple of 8, >= width.
+ *   a2v_norm  fp32 [n] device output.
+ * Squares of the bf16 inputs are exact in fp32; they are summed in fp32
+ * (eight partial sums per lane, then a fixed tree), deterministically, and
+ * the square root is the correctly rounded sqrtf.
+ * Returns PRISM_OK, PRISM_ERR_INVALID_ARG or PRISM_ERR_CUDA.
+ */
+int prism_a2v_norm(const uint16_t *hhat, int64_t n, int32_t width, int64_t ld, float *a2v_norm,
+                   prism_stream_t stream);
+
 /* Bytes of workspace prism_plan needs (0 on invalid params). */
 size_t prism_plan_workspace_size(const prism_params *p);
 
@@ -129,8 +169,9 @@ size_t prism_plan_workspace_size(const prism_params *p);
  *   + eps; l*_d closed form; nearest candidate in log2 space.
  *   V         bf16 [N][heads][head_dim].
  *   a2v_norm  fp32 [N] norm of the previous layer's audio-to-video
- *             attention output per video token, or NULL for the first
- *             layer (video guidance only).
+ *             attention output per video token (prism_a2v_norm computes
+ *             it), or NULL for the first layer (video guidance only).
+ *             Required when p->density == 3.
  *   out       arrays to fill (see prism_plan_t).
  *   workspace, ws_bytes  at least prism_plan_workspace_size(p) bytes.
  * Returns PRISM_OK, PRISM_ERR_INVALID_ARG, PRISM_ERR_UNSUPPORTED,

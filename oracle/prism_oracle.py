@@ -391,7 +391,10 @@ def hybrid_select_row(s_row, k, p):
     P_i = softmax(s_i) computed in float64 from the fp32 scores.  Order:
     score descending, then index ascending.  READING: "passes" means >= and
     the crossing block is included.  Both sets are prefixes of one order, so
-    the union is the prefix of length max(k, n_p).
+    the union is the prefix of length max(k, n_p).  With p >= 1 every block
+    is kept: every P_ij is positive, so in exact arithmetic the cumulative
+    probability reaches 1 only with the last block (float64 rounding of the
+    running sum must not cut that tail short).
 
     Returns (sorted ids, info) with info = n, k, n_p and the decision
     margins: the score gap at the prefix boundary and the distance of the
@@ -407,6 +410,8 @@ def hybrid_select_row(s_row, k, p):
     target = float(np.float32(p)) * Z
     if p <= 0:
         n_p = 0
+    elif p >= 1:
+        n_p = nb
     else:
         hit = np.nonzero(csum >= target)[0]
         n_p = int(hit[0]) + 1 if hit.size else nb

@@ -40,3 +40,33 @@ def to_np(t):
 def csr_rows(row_ptr, col, NB, h, i):
     r = h * NB + i
     return col[row_ptr[r]:row_ptr[r + 1]]
+
+
+def compare_plan(w, pl, ref, heads):
+    """Library plan vs oracle plan (heads[k] of the library = ref.heads[k]).
+    Statistic values within fp32-partial-sum rounding; shapes, block table
+    and permutation bit-exact except at decisions whose oracle margin is
+    <= TIE.  Returns the number of zone decisions excluded at ties."""
+    shapes, g, rho = to_np(pl.zone_shape), to_np(pl.zone_g), to_np(pl.zone_rho)
+    nblk, blocks, perm, inv = to_np(pl.n_blocks), to_np(pl.blocks), to_np(pl.perm), to_np(pl.inv_perm)
+    excluded = 0
+    for k, h in enumerate(heads):
+        hp = ref.heads[k]
+        np.testing.assert_allclose(rho[h], hp.rho, rtol=1e-6, atol=1e-12)
+        np.testing.assert_allclose(g[h], hp.g, rtol=1e-6, atol=1e-12)
+        diff = shapes[h] != hp.shape
+        tie = (hp.vol_margin <= TIE) | (hp.shape_margin <= TIE)
+        assert not (diff & ~tie).any(), f"head {h}: shape differs outside ties at zones {np.nonzero(diff & ~tie)}"
+        excluded += int((diff & tie).sum())
+        if diff.any():
+            continue
+        nb = hp.blocks.shape[0]
+        assert nblk[h] == nb
+        got = blocks[h, :nb]
+        np.testing.assert_array_equal(got[:, 0], hp.blocks[:, 5])
+        np.testing.assert_array_equal(got[:, 1], hp.blocks[:, 4])
+        np.testing.assert_array_equal(got[:, 2], (hp.blocks[:, 0] * w.H + hp.blocks[:, 1]) * w.W + hp.blocks[:, 2])
+        np.testing.assert_array_equal(got[:, 3], hp.blocks[:, 3])
+        np.testing.assert_array_equal(perm[h], hp.perm)
+        np.testing.assert_array_equal(inv[h][perm[h]], np.arange(w.N))
+    return excluded

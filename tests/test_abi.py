@@ -30,7 +30,7 @@ def test_library_loads_and_exports_every_symbol():
 
 
 def test_struct_layouts_match_header():
-    assert C.sizeof(_lib.PrismParams) == 12 * 4
+    assert C.sizeof(_lib.PrismParams) == 15 * 4
     assert C.sizeof(_lib.PrismPlan) == 7 * 8
     assert C.sizeof(_lib.PrismSelect) == 6 * 8
 
@@ -41,6 +41,10 @@ def test_struct_layouts_match_header():
     (dict(heads=0), _lib.PRISM_ERR_INVALID_ARG),
     (dict(top_p=-0.5), _lib.PRISM_ERR_INVALID_ARG),
     (dict(tau128=0.1, tau256=0.2), _lib.PRISM_ERR_INVALID_ARG),
+    (dict(map_exponent=-1.0), _lib.PRISM_ERR_INVALID_ARG),
+    (dict(map_exponent=9.0), _lib.PRISM_ERR_INVALID_ARG),
+    (dict(guidance=4), _lib.PRISM_ERR_INVALID_ARG),
+    (dict(density=4), _lib.PRISM_ERR_INVALID_ARG),
 ])
 def test_invalid_params_are_rejected_before_any_cuda_call(bad, code):
     lib = _lib.load()
@@ -52,6 +56,15 @@ def test_invalid_params_are_rejected_before_any_cuda_call(bad, code):
     rc = lib.prism_plan(C.byref(p), C.c_void_p(8), None, C.byref(plan), C.c_void_p(256), 1 << 20, None)
     assert rc == code
     assert lib.prism_last_error().decode()
+
+
+def test_a2v_density_without_norms_is_rejected():
+    lib = _lib.load()
+    p = api.params(8, 16, 16, 1, 64, topk_abs=2, density=api.DENSITY_A2V)
+    plan = _lib.PrismPlan(8, 8, 8, 8, 8, 8, 8)
+    rc = lib.prism_plan(C.byref(p), C.c_void_p(8), None, C.byref(plan), C.c_void_p(256), 1 << 20, None)
+    assert rc == _lib.PRISM_ERR_INVALID_ARG and "a2v_norm" in lib.prism_last_error().decode()
+    assert lib.prism_plan_noalloc(C.byref(p), C.c_void_p(8), None, C.byref(plan), None) == _lib.PRISM_ERR_INVALID_ARG
 
 
 def test_null_pointers_and_short_workspace_are_rejected():
@@ -80,3 +93,16 @@ def test_workspace_sizes_grow_with_the_grid():
     for f in (lib.prism_plan_workspace_size, lib.prism_select_workspace_size):
         assert 0 < f(C.byref(small)) < f(C.byref(big))
     assert lib.prism_attn_workspace_size(C.byref(big), 0) >= 3 * 860160 * 24 * 128 * 2
+
+
+def test_a2v_norm_argument_checks_need_no_gpu():
+    lib = _lib.load()
+    ok = C.c_void_p(256)
+    assert lib.prism_a2v_norm(ok, 0, 3072, 3072, ok, None) == _lib.PRISM_OK        # n = 0: nothing to do
+    assert lib.prism_a2v_norm(ok, -1, 3072, 3072, ok, None) == _lib.PRISM_ERR_INVALID_ARG
+    assert lib.prism_a2v_norm(ok, 4, 12, 16, ok, None) == _lib.PRISM_ERR_INVALID_ARG   # width % 8
+    assert lib.prism_a2v_norm(ok, 4, 64, 56, ok, None) == _lib.PRISM_ERR_INVALID_ARG   # ld < width
+    assert lib.prism_a2v_norm(ok, 4, 64, 68, ok, None) == _lib.PRISM_ERR_INVALID_ARG   # ld % 8
+    assert lib.prism_a2v_norm(C.c_void_p(264), 4, 64, 64, ok, None) == _lib.PRISM_ERR_INVALID_ARG  # alignment
+    assert lib.prism_a2v_norm(None, 4, 64, 64, ok, None) == _lib.PRISM_ERR_INVALID_ARG
+    assert "prism_a2v_norm" in lib.prism_last_error().decode()

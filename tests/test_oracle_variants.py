@@ -197,3 +197,5 @@ def test_topk_only_and_topp_only_rows():
             c += w[order[n]]
             n += 1
         assert sorted(kept) == sorted(order[:n])
+        kept, _ = O.hybrid_select_row(s, 1, 1.0)                 # p = 1 keeps every block
+        assert sorted(kept) == list(range(nb))

@@ -10,17 +10,19 @@
 //   dS = P (dP - Delta), dQ = scale dS K, dK = scale dS^T Q, dV = P^T dO.
 //
 // Two kernels, no atomics (deterministic):
-//   dq_kernel    one CTA per 128-query tile; walks the CSR like the forward:
-//                S = Q K^T, dP = dO V^T (TMEM), dS -> TMEM (fp16),
-//                dQ += dS K (TS MMA).
-//   dkdv_kernel  one CTA per 128-key tile; walks the transpose (CSC):
-//                S^T = K Q^T, dP^T = V dO^T (TMEM), P^T and dS^T -> TMEM
-//                (fp16), dV += P^T dO, dK += dS^T Q (TS MMAs).
+//   dq_kernel    one CTA per 128-query tile; walks the CSR like the forward,
+//                two key units (128 keys) per step: S = Q K^T and dP = dO V^T
+//                (TMEM, S double buffered), dS -> TMEM (fp16), dQ += dS K
+//                (TS MMA).
+//   dkdv_kernel  one CTA per 128-key tile; walks the transpose (CSC), two
+//                query units per step: S^T = K Q^T, dP^T = V dO^T (TMEM),
+//                P^T and dS^T -> TMEM (fp16), dV += P^T dO, dK += dS^T Q (TS
+//                MMAs); the softmax of a step overlaps its dP^T product and
+//                dS^T overlaps the dV product.
 // Operands are fp16 (exact conversions of the bf16 inputs, see the forward).
 // Roles: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer, warps 4-11
-// two compute warpgroups (one thread per TMEM lane), each taking one 32-token
-// half of every 64-token step.  Steps alternate between two TMEM buffer
-// pairs, so the compute of a step overlaps the MMAs of the next.
+// two compute warpgroups (one thread per TMEM lane), each taking one of the
+// step's two 64-token units.
 #include "attn_walk.cuh"
 
 namespace prism {
@@ -76,12 +78,21 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const int32_t *__restrict
 }
 
 // ---------------------------------------------------------------------------
-// Shared pieces of the two kernels.  Both walk 64-token units of the
-// streamed side, one unit per step, alternating between two TMEM buffer
-// pairs so the compute of step i overlaps the MMAs of step i+1; the two
-// compute warpgroups split each step's 64 columns.
+// Shared pieces of the two kernels.  Both walk the streamed side's 64-token
+// units in pairs: one step is up to 128 streamed tokens, so every S-like
+// product is a full-width M=128, N=128 tcgen05.mma (narrower products run
+// the tensor pipe at a fraction of its rate).  The two compute warpgroups
+// share the TMEM lanes (one thread per row of the CTA's tile) and split a
+// step by unit: warpgroup g takes the step's unit g (fp32 columns
+// [64g, 64g+64) of a product).  Each writes its fp16 results, packed two per
+// column, into the first 32 columns of its own range, so neither overwrites
+// columns the other may still be reading.  The TS MMA's 16-wide K slice ks
+// therefore starts at column pk_col(ks).
 // ---------------------------------------------------------------------------
-constexpr int NS = 4;  // ring depth (steps of one 64-token unit)
+constexpr int NS = 2;  // ring depth (steps of up to two 64-token units)
+constexpr int kPolyPairs = 4;  // of every 16 column pairs, this many take exp2_poly2
+
+__host__ __device__ constexpr uint32_t pk_col(int ks) { return (uint32_t)((ks >> 2) * 64 + (ks & 3) * 8); }
 
 template <int D>
 __device__ __forceinline__ void store_row(void *out, bool fp32, size_t off, const uint32_t (&o)[32], float mul) {
@@ -102,32 +113,48 @@ __device__ __forceinline__ void store_row(void *out, bool fp32, size_t off, cons
   }
 }
 
+// P = 2^(s * scale_log2 - lse2) for 32 fp32 scores; a share of the
+// exponentials on the FMA pipe.  neg_lse2(k) gives -lse2 of column k's pair
+// partner (per column for dK/dV, one value per row for dQ).
+template <typename F>
+__device__ __forceinline__ void softmax_p32(const uint32_t (&sv)[32], float scale_log2, F neg_lse2, float *pf) {
+#pragma unroll
+  for (int k = 0; k < 32; k += 2) {
+    const float2 x = ffma2(make_float2(__uint_as_float(sv[k]), __uint_as_float(sv[k + 1])),
+                           make_float2(scale_log2, scale_log2), neg_lse2(k));
+    const float2 p = k < 2 * kPolyPairs ? exp2_poly2(x) : make_float2(ex2f(x.x), ex2f(x.y));
+    pf[k] = p.x;
+    pf[k + 1] = p.y;
+  }
+}
+
 // ---------------------------------------------------------------------------
-// dQ kernel: one CTA per 128-query tile; steps over the key units of the
-// union of its rows' selections.
-//   TMEM: dQ [0, D); step buffer b: S at 128+128b, dP (then dS) at 192+128b.
+// dQ kernel: one CTA per 128-query tile; steps over pairs of the key units of
+// the union of its rows' selections.
+//   TMEM: dQ [0, 128); dP [128, 256); S in buffer b at [256 + 128b, +128),
+//   dS packed into the same columns.
 // ---------------------------------------------------------------------------
 template <int D>
 struct DqSmem {
   static constexpr int CHUNKS = D / 64;
   static constexpr int TILE = 128 * D * 2;  // 128 rows of fp16
-  static constexpr int UNIT = 64 * D * 2;   // 64 rows
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_DO = OFF_Q + TILE;
   static constexpr int OFF_K = OFF_DO + TILE;
-  static constexpr int OFF_V = OFF_K + NS * UNIT;
-  static constexpr int OFF_BAR = OFF_V + NS * UNIT;
+  static constexpr int OFF_V = OFF_K + NS * TILE;
+  static constexpr int OFF_BAR = OFF_V + NS * TILE;
   static constexpr int BYTES = OFF_BAR + 256;
 };
 
 struct DqBars {
   uint64_t qdo_full;
   uint64_t k_full[NS], v_full[NS], kv_empty[NS];
-  uint64_t s_full[2], dp_full[2], ds_ready[2], dq_done[2];
+  uint64_t s_full[2], ds_ready[2], dq_done[2];
+  uint64_t dp_full, dp_free;
   uint64_t fin;  // single use: every MMA of the tile has completed
-  int mask[NS];
+  int meta[NS];  // units | mask_a << 4 | mask_b << 8 (bit = 64-row half of the tile)
   uint32_t tmem_base;
-  int nsteps, abort;
+  int nsteps, nunits, abort;
 };
 
 template <int D>
@@ -160,12 +187,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bar.s_full[b], 1);
-      mbar_init(&bar.dp_full[b], 1);
       mbar_init(&bar.ds_ready[b], 256);
       mbar_init(&bar.dq_done[b], 1);
     }
+    mbar_init(&bar.dp_full, 1);
+    mbar_init(&bar.dp_free, 256);
     mbar_init(&bar.fin, 1);
-    bar.nsteps = tile_units[(size_t)h * (N / 128) + tile];
+    bar.nunits = tile_units[(size_t)h * (N / 128) + tile];
+    bar.nsteps = (bar.nunits + 1) >> 1;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -176,10 +205,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bar.tmem_base;
-  const int nsteps = bar.nsteps;
-  const uint32_t tQ = tmem;
+  const int nsteps = bar.nsteps, nunits = bar.nunits;
+  const uint32_t tQacc = tmem, tdP = tmem + 128;
 
   if (warp == 0) {
+    // ------------------------------------------------------------ producer
     const int blk[2] = {unit_block[(size_t)h * NB + 2 * tile], unit_block[(size_t)h * NB + 2 * tile + 1]};
     UnitWalk<2> w;
     walk_init<2>(w, blk, 2, row_ptr, h * NB);
@@ -193,70 +223,84 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int j = 0; j < nsteps; ++j) {
       const int s = j % NS;
-      uint32_t u;
-      int m;
-      walk_next<2>(w, col, blocks_h, u, m);
-      u = min(u, (uint32_t)(NB - 1));  // a well-formed walk never clamps
+      uint32_t ua, ub = 0;
+      int ma, mb = 0, nu = 1;
+      walk_next<2>(w, col, blocks_h, ua, ma);
+      if (2 * j + 2 <= nunits) {
+        walk_next<2>(w, col, blocks_h, ub, mb);
+        nu = 2;
+      }
+      ua = min(ua, (uint32_t)(NB - 1));  // a well-formed walk never clamps
+      ub = min(ub, (uint32_t)(NB - 1));
       if (lane == 0) {
         bool ok = true;
         if (j >= NS) ok = mbar_wait(&bar.kv_empty[s], ((j / NS) - 1) & 1, status, 21);
         if (!ok) bar.abort = 1;
         if (ok) {
-          bar.mask[s] = m;
-          mbar_arrive_expect_tx(&bar.k_full[s], L::UNIT);
+          bar.meta[s] = nu | (ma << 4) | (mb << 8);
+          uint8_t *ks = smem + L::OFF_K + s * L::TILE;
+          uint8_t *vs = smem + L::OFF_V + s * L::TILE;
+          mbar_arrive_expect_tx(&bar.k_full[s], nu * 64 * D * 2);
 #pragma unroll
-          for (int c = 0; c < L::CHUNKS; ++c)
-            tma_load_2d(smem + L::OFF_K + s * L::UNIT + c * (64 * 128), &mapK, &bar.k_full[s], c * 64,
-                        h * N + (int)u * 64);
-          mbar_arrive_expect_tx(&bar.v_full[s], L::UNIT);
+          for (int c = 0; c < L::CHUNKS; ++c) {
+            tma_load_2d(ks + c * (128 * 128), &mapK, &bar.k_full[s], c * 64, h * N + (int)ua * 64);
+            if (nu == 2) tma_load_2d(ks + c * (128 * 128) + 64 * 128, &mapK, &bar.k_full[s], c * 64, h * N + (int)ub * 64);
+          }
+          mbar_arrive_expect_tx(&bar.v_full[s], nu * 64 * D * 2);
 #pragma unroll
-          for (int c = 0; c < L::CHUNKS; ++c)
-            tma_load_2d(smem + L::OFF_V + s * L::UNIT + c * (64 * 128), &mapV, &bar.v_full[s], c * 64,
-                        h * N + (int)u * 64);
+          for (int c = 0; c < L::CHUNKS; ++c) {
+            tma_load_2d(vs + c * (128 * 128), &mapV, &bar.v_full[s], c * 64, h * N + (int)ua * 64);
+            if (nu == 2) tma_load_2d(vs + c * (128 * 128) + 64 * 128, &mapV, &bar.v_full[s], c * 64, h * N + (int)ub * 64);
+          }
         }
       }
       __syncwarp();
       if (*reinterpret_cast<volatile int *>(&bar.abort)) break;
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t id64 = idesc_f16(128, 64, 0), id_dq = idesc_f16(128, D, 1);
+      const uint32_t id_full = idesc_f16(128, 128, 0), id_half = idesc_f16(128, 64, 0);
+      const uint32_t id_acc = idesc_f16(128, D, 1);
       const uint64_t dQd = sdesc_sw128(smem_u32(smem + L::OFF_Q), 16, 1024);
       const uint64_t dDOd = sdesc_sw128(smem_u32(smem + L::OFF_DO), 16, 1024);
       bool ok = mbar_wait(&bar.qdo_full, 0, status, 22);
       tc_fence_after();
       for (int i = 0; ok && i <= nsteps; ++i) {
-        if (i < nsteps) {  // S_i = Q K_i^T, dP_i = dO V_i^T into buffer i&1
+        if (i < nsteps) {  // S_i = Q K_i^T into buffer i&1, dP_i = dO V_i^T
           const int s = i % NS, b = i & 1;
-          const uint32_t tS = tmem + 128 + 128 * b, tP = tS + 64;
           ok = mbar_wait(&bar.k_full[s], (i / NS) & 1, status, 24);
-          if (!ok) break;
-          tc_fence_after();
-          const uint64_t dK = sdesc_sw128(smem_u32(smem + L::OFF_K + s * L::UNIT), 16, 1024);
-          const uint64_t dV = sdesc_sw128(smem_u32(smem + L::OFF_V + s * L::UNIT), 16, 1024);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tS, dQd + kslice16(kk, 128 * 128), dK + kslice16(kk, 64 * 128), id64, kk > 0 ? 1u : 0u);
-          mma_commit(&bar.s_full[b]);
-          ok = mbar_wait(&bar.v_full[s], (i / NS) & 1, status, 25);
           if (ok && i >= 2) ok = mbar_wait(&bar.dq_done[b], ((i - 2) >> 1) & 1, status, 26);
           if (!ok) break;
           tc_fence_after();
+          const int nu = bar.meta[s] & 15;  // written before the stage's K arrived
+          const uint32_t id = nu == 2 ? id_full : id_half;
+          const uint64_t dK = sdesc_sw128(smem_u32(smem + L::OFF_K + s * L::TILE), 16, 1024);
+          const uint64_t dV = sdesc_sw128(smem_u32(smem + L::OFF_V + s * L::TILE), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tP, dDOd + kslice16(kk, 128 * 128), dV + kslice16(kk, 64 * 128), id64, kk > 0 ? 1u : 0u);
-          mma_commit(&bar.dp_full[b]);
+            mma_ss(tmem + 256 + 128 * b, dQd + kslice16(kk, 128 * 128), dK + kslice16(kk, 128 * 128), id,
+                   kk > 0 ? 1u : 0u);
+          mma_commit(&bar.s_full[b]);
+          ok = mbar_wait(&bar.v_full[s], (i / NS) & 1, status, 25);
+          if (ok && i >= 1) ok = mbar_wait(&bar.dp_free, (i - 1) & 1, status, 27);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tdP, dDOd + kslice16(kk, 128 * 128), dV + kslice16(kk, 128 * 128), id, kk > 0 ? 1u : 0u);
+          mma_commit(&bar.dp_full);
         }
         if (i >= 1) {  // dQ += dS_{i-1} K_{i-1}
           const int jj = i - 1, s = jj % NS, b = jj & 1;
-          const uint32_t tP = tmem + 192 + 128 * b;
+          const int nu = bar.meta[s] & 15;
           ok = mbar_wait(&bar.ds_ready[b], (jj >> 1) & 1, status, 23);
           if (!ok) break;
           tc_fence_after();
-          const uint64_t dKmn = sdesc_sw128(smem_u32(smem + L::OFF_K + s * L::UNIT), 64 * 128, 1024);
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_ts(tQ, tP + ks * 8, dKmn + (uint64_t)ks * 128, id_dq, (jj > 0 || ks > 0) ? 1u : 0u);
+          const uint64_t dKmn = sdesc_sw128(smem_u32(smem + L::OFF_K + s * L::TILE), 128 * 128, 1024);
+          for (int ks = 0; ks < 4 * nu; ++ks)
+            mma_ts(tQacc, tmem + 256 + 128 * b + pk_col(ks), dKmn + (uint64_t)ks * 128, id_acc,
+                   (jj > 0 || ks > 0) ? 1u : 0u);
           mma_commit(&bar.dq_done[b]);
           mma_commit(&bar.kv_empty[s]);
         }
@@ -266,50 +310,70 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    const int g = (warp - 4) >> 2;  // warpgroup: 32-key chunk g of every step
+    // ------------------------------------------------------------ compute
+    const int g = (warp - 4) >> 2;  // warpgroup: key unit g of every step
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const int half = row >> 6;  // warp-uniform
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const size_t prow = (size_t)h * N + (size_t)tile * 128 + row;
     const float lse2 = lse2p[prow], dl = deltap[prow];
+    const auto row_lse = [lse2](int) { return make_float2(-lse2, -lse2); };
     bool ok = true;
     for (int i = 0; i < nsteps; ++i) {
-      const int b = i & 1, ph = (i >> 1) & 1;
-      const uint32_t tS = tmem + 128 + 128 * b, tP = tS + 64;
-      ok = mbar_wait_warp(&bar.s_full[b], ph, status, 27);
-      if (ok) ok = mbar_wait_warp(&bar.dp_full[b], ph, status, 28);
+      const int b = i & 1, s = i % NS;
+      const uint32_t tS = tmem + 256 + 128 * b + 64 * g;
+      ok = mbar_wait_warp(&bar.s_full[b], (i >> 1) & 1, status, 28);
       if (!ok) break;
       tc_fence_after();
-      const bool valid = (bar.mask[i % NS] >> half) & 1;
-      uint32_t pk[16];
+      const int meta = bar.meta[s];
+      const bool active = g < (meta & 15);
+      const bool valid = active && (((meta >> (4 + 4 * g)) >> half) & 1);  // warp-uniform
+      float pf[64];
       if (valid) {
-        uint32_t sv[32], dv[32];
-        tmem_ld32(tS + lane_off + g * 32, sv);
-        tmem_ld32(tP + lane_off + g * 32, dv);
-        tmem_wait_ld();
 #pragma unroll
-        for (int k = 0; k < 32; k += 2) {
-          const float2 x = ffma2(make_float2(__uint_as_float(sv[k]), __uint_as_float(sv[k + 1])), scale_log2, -lse2);
-          const float2 p = make_float2(ex2f(x.x), ex2f(x.y));
-          const float2 d = fmul2(p, fsub2(make_float2(__uint_as_float(dv[k]), __uint_as_float(dv[k + 1])),
-                                          make_float2(dl, dl)));
-          pk[k / 2] = pack_f16(d.x, d.y);
+        for (int c = 0; c < 2; ++c) {
+          uint32_t sv[32];
+          tmem_ld32(tS + lane_off + 32 * c, sv);
+          tmem_wait_ld();
+          softmax_p32(sv, scale_log2, row_lse, pf + 32 * c);
         }
-      } else {
-#pragma unroll
-        for (int k = 0; k < 16; ++k) pk[k] = 0u;
       }
-      tmem_st16(tP + lane_off + g * 16, pk);
+      ok = mbar_wait_warp(&bar.dp_full, i & 1, status, 29);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[16];
+        if (valid) {
+          uint32_t dv[32];
+          tmem_ld32(tdP + lane_off + 64 * g + 32 * c, dv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; k += 2) {
+            const float2 d = fmul2(make_float2(pf[32 * c + k], pf[32 * c + k + 1]),
+                                   fsub2(make_float2(__uint_as_float(dv[k]), __uint_as_float(dv[k + 1])),
+                                         make_float2(dl, dl)));
+            pk[k / 2] = pack_f16(d.x, d.y);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) pk[k] = 0u;
+        }
+        if (c == 1) {  // every read of dP_i is done: the next dP may overwrite it
+          tc_fence_before();
+          mbar_arrive(&bar.dp_free);
+        }
+        if (active) tmem_st16(tS + lane_off + 16 * c, pk);
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar.ds_ready[b]);
     }
-    // A parity wait on dq_done could match an older phase for the warpgroup
-    // that did not run the step before the last; the single-use barrier
-    // cannot.
+    // A parity wait on dq_done could match an older phase; the single-use
+    // barrier cannot.
     ok = __all_sync(0xffffffffu, ok);
-    if (ok && nsteps > 0) ok = mbar_wait_warp(&bar.fin, 0, status, 29);
+    if (ok && nsteps > 0) ok = mbar_wait_warp(&bar.fin, 0, status, 30);
     if (ok) {
       tc_fence_after();
       const int n = perm[prow];
@@ -318,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = g * (D / 2); c < (g + 1) * (D / 2); c += 32) {
         uint32_t o[32];
         if (nsteps > 0) {
-          tmem_ld32(tQ + lane_off + c, o);
+          tmem_ld32(tQacc + lane_off + c, o);
           tmem_wait_ld();
         } else {
 #pragma unroll
@@ -339,33 +403,32 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// dK/dV kernel: one CTA per 128-key tile; steps over the query units of the
-// union of its blocks' columns (the transpose of the selection).
-//   TMEM: dV [0, D), dK [128, 128+D); step buffer b: S^T (then P^T) at
-//   256+128b, dP^T (then dS^T) at 320+128b.
+// dK/dV kernel: one CTA per 128-key tile; steps over pairs of the query units
+// of the union of its blocks' columns (the transpose of the selection).
+//   TMEM: dV [0, 128), dK [128, 256), S^T [256, 384) (P^T packed into it),
+//   dP^T [384, 512) (dS^T packed into it).
 // ---------------------------------------------------------------------------
 template <int D>
 struct KvSmem {
   static constexpr int CHUNKS = D / 64;
   static constexpr int TILE = 128 * D * 2;
-  static constexpr int UNIT = 64 * D * 2;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + TILE;
-  static constexpr int OFF_Q = OFF_V + TILE;                // ring of query units
-  static constexpr int OFF_DO = OFF_Q + NS * UNIT;          // ring of dO units
-  static constexpr int OFF_STAT = OFF_DO + NS * UNIT;       // [NS][2][64] floats: lse2, delta
-  static constexpr int OFF_BAR = OFF_STAT + NS * 2 * 64 * 4;
+  static constexpr int OFF_Q = OFF_V + TILE;                // ring of query-unit pairs
+  static constexpr int OFF_DO = OFF_Q + NS * TILE;          // ring of dO-unit pairs
+  static constexpr int OFF_STAT = OFF_DO + NS * TILE;       // [NS][lse2 128, delta 128] floats
+  static constexpr int OFF_BAR = OFF_STAT + NS * 256 * 4;
   static constexpr int BYTES = OFF_BAR + 256;
 };
 
 struct KvBars {
   uint64_t kv_full;
   uint64_t q_full[NS], q_empty[NS];
-  uint64_t s_full[2], dp_full[2], ds_ready[2], dv_done[2], dk_done[2];
+  uint64_t s_full, dp_full, p_ready, ds_ready, dv_done, dk_done;
   uint64_t fin;  // single use: every MMA of the tile has completed
-  int mask[NS];
+  int meta[NS];  // units | mask_a << 4 | mask_b << 8 (bit = 64-row half of the key tile)
   uint32_t tmem_base;
-  int nsteps, abort;
+  int nsteps, nunits, abort;
 };
 
 template <int D>
@@ -397,15 +460,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar.q_full[s], 1);
       mbar_init(&bar.q_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bar.s_full[b], 1);
-      mbar_init(&bar.dp_full[b], 1);
-      mbar_init(&bar.ds_ready[b], 256);
-      mbar_init(&bar.dv_done[b], 1);
-      mbar_init(&bar.dk_done[b], 1);
-    }
+    mbar_init(&bar.s_full, 1);
+    mbar_init(&bar.dp_full, 1);
+    mbar_init(&bar.p_ready, 256);
+    mbar_init(&bar.ds_ready, 256);
+    mbar_init(&bar.dv_done, 1);
+    mbar_init(&bar.dk_done, 1);
     mbar_init(&bar.fin, 1);
-    bar.nsteps = tile_units[(size_t)h * (N / 128) + tile];
+    bar.nunits = tile_units[(size_t)h * (N / 128) + tile];
+    bar.nsteps = (bar.nunits + 1) >> 1;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -416,10 +479,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bar.tmem_base;
-  const int nsteps = bar.nsteps;
-  const uint32_t tV = tmem, tK = tmem + 128;
+  const int nsteps = bar.nsteps, nunits = bar.nunits;
+  const uint32_t tV = tmem, tK = tmem + 128, tS = tmem + 256, tP = tmem + 384;
 
   if (warp == 0) {
+    // ------------------------------------------------------------ producer
     const int blk[2] = {unit_block[(size_t)h * NB + 2 * tile], unit_block[(size_t)h * NB + 2 * tile + 1]};
     UnitWalk<2> w;
     walk_init<2>(w, blk, 2, col_ptr, h * NB);
@@ -433,138 +497,181 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int j = 0; j < nsteps; ++j) {
       const int s = j % NS;
-      uint32_t u;
-      int m;
-      walk_next<2>(w, rowidx, blocks_h, u, m);
-      u = min(u, (uint32_t)(NB - 1));
+      uint32_t ua, ub = 0;
+      int ma, mb = 0, nu = 1;
+      walk_next<2>(w, rowidx, blocks_h, ua, ma);
+      if (2 * j + 2 <= nunits) {
+        walk_next<2>(w, rowidx, blocks_h, ub, mb);
+        nu = 2;
+      }
+      ua = min(ua, (uint32_t)(NB - 1));
+      ub = min(ub, (uint32_t)(NB - 1));
       if (lane == 0) {
         bool ok = true;
         if (j >= NS) ok = mbar_wait(&bar.q_empty[s], ((j / NS) - 1) & 1, status, 41);
         if (!ok) bar.abort = 1;
         if (ok) {
-          bar.mask[s] = m;
-          mbar_arrive_expect_tx(&bar.q_full[s], 2 * L::UNIT + 2 * 64 * 4);
+          bar.meta[s] = nu | (ma << 4) | (mb << 8);
+          uint8_t *qs = smem + L::OFF_Q + s * L::TILE;
+          uint8_t *os = smem + L::OFF_DO + s * L::TILE;
+          float *st = stat + s * 256;
+          mbar_arrive_expect_tx(&bar.q_full[s], nu * (2 * 64 * D * 2 + 2 * 64 * 4));
 #pragma unroll
           for (int c = 0; c < L::CHUNKS; ++c) {
-            tma_load_2d(smem + L::OFF_Q + s * L::UNIT + c * (64 * 128), &mapQ, &bar.q_full[s], c * 64,
-                        h * N + (int)u * 64);
-            tma_load_2d(smem + L::OFF_DO + s * L::UNIT + c * (64 * 128), &mapDO, &bar.q_full[s], c * 64,
-                        h * N + (int)u * 64);
+            tma_load_2d(qs + c * (128 * 128), &mapQ, &bar.q_full[s], c * 64, h * N + (int)ua * 64);
+            tma_load_2d(os + c * (128 * 128), &mapDO, &bar.q_full[s], c * 64, h * N + (int)ua * 64);
+            if (nu == 2) {
+              tma_load_2d(qs + c * (128 * 128) + 64 * 128, &mapQ, &bar.q_full[s], c * 64, h * N + (int)ub * 64);
+              tma_load_2d(os + c * (128 * 128) + 64 * 128, &mapDO, &bar.q_full[s], c * 64, h * N + (int)ub * 64);
+            }
           }
-          bulk_load(stat + s * 128, lse2p + (size_t)h * N + (size_t)u * 64, 256, &bar.q_full[s]);
-          bulk_load(stat + s * 128 + 64, deltap + (size_t)h * N + (size_t)u * 64, 256, &bar.q_full[s]);
+          bulk_load(st, lse2p + (size_t)h * N + (size_t)ua * 64, 256, &bar.q_full[s]);
+          bulk_load(st + 128, deltap + (size_t)h * N + (size_t)ua * 64, 256, &bar.q_full[s]);
+          if (nu == 2) {
+            bulk_load(st + 64, lse2p + (size_t)h * N + (size_t)ub * 64, 256, &bar.q_full[s]);
+            bulk_load(st + 192, deltap + (size_t)h * N + (size_t)ub * 64, 256, &bar.q_full[s]);
+          }
         }
       }
       __syncwarp();
       if (*reinterpret_cast<volatile int *>(&bar.abort)) break;
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t id64 = idesc_f16(128, 64, 0), id_acc = idesc_f16(128, D, 1);
+      const uint32_t id_full = idesc_f16(128, 128, 0), id_half = idesc_f16(128, 64, 0);
+      const uint32_t id_acc = idesc_f16(128, D, 1);
       const uint64_t dKd = sdesc_sw128(smem_u32(smem + L::OFF_K), 16, 1024);
       const uint64_t dVd = sdesc_sw128(smem_u32(smem + L::OFF_V), 16, 1024);
       bool ok = mbar_wait(&bar.kv_full, 0, status, 42);
       tc_fence_after();
-      for (int i = 0; ok && i <= nsteps; ++i) {
-        if (i < nsteps) {  // S^T_i = K Q_i^T, dP^T_i = V dO_i^T into buffer i&1
-          const int s = i % NS, b = i & 1;
-          const uint32_t tS = tmem + 256 + 128 * b, tP = tS + 64;
-          ok = mbar_wait(&bar.q_full[s], (i / NS) & 1, status, 44);
-          if (ok && i >= 2) ok = mbar_wait(&bar.dv_done[b], ((i - 2) >> 1) & 1, status, 45);
-          if (!ok) break;
-          tc_fence_after();
-          const uint64_t dQs = sdesc_sw128(smem_u32(smem + L::OFF_Q + s * L::UNIT), 16, 1024);
-          const uint64_t dDOs = sdesc_sw128(smem_u32(smem + L::OFF_DO + s * L::UNIT), 16, 1024);
+      for (int i = 0; ok && i < nsteps; ++i) {
+        const int s = i % NS;
+        ok = mbar_wait(&bar.q_full[s], (i / NS) & 1, status, 44);
+        // S^T and dP^T reuse the columns the previous step's dV and dK read P^T and dS^T from
+        if (ok && i >= 1) ok = mbar_wait(&bar.dv_done, (i - 1) & 1, status, 45);
+        if (!ok) break;
+        tc_fence_after();
+        const int nu = bar.meta[s] & 15;  // written before the stage's Q arrived
+        const uint32_t id = nu == 2 ? id_full : id_half;
+        const uint64_t dQs = sdesc_sw128(smem_u32(smem + L::OFF_Q + s * L::TILE), 16, 1024);
+        const uint64_t dDOs = sdesc_sw128(smem_u32(smem + L::OFF_DO + s * L::TILE), 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tS, dKd + kslice16(kk, 128 * 128), dQs + kslice16(kk, 64 * 128), id64, kk > 0 ? 1u : 0u);
-          mma_commit(&bar.s_full[b]);
-          if (i >= 2) ok = mbar_wait(&bar.dk_done[b], ((i - 2) >> 1) & 1, status, 46);
-          if (!ok) break;
-          tc_fence_after();
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tS, dKd + kslice16(kk, 128 * 128), dQs + kslice16(kk, 128 * 128), id, kk > 0 ? 1u : 0u);
+        mma_commit(&bar.s_full);
+        if (i >= 1) ok = mbar_wait(&bar.dk_done, (i - 1) & 1, status, 46);
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tP, dVd + kslice16(kk, 128 * 128), dDOs + kslice16(kk, 64 * 128), id64, kk > 0 ? 1u : 0u);
-          mma_commit(&bar.dp_full[b]);
-        }
-        if (i >= 1) {  // dV += P^T dO, dK += dS^T Q  (step i-1)
-          const int jj = i - 1, s = jj % NS, b = jj & 1;
-          const uint32_t tS = tmem + 256 + 128 * b, tP = tS + 64;
-          ok = mbar_wait(&bar.ds_ready[b], (jj >> 1) & 1, status, 43);
-          if (!ok) break;
-          tc_fence_after();
-          const uint64_t dQmn = sdesc_sw128(smem_u32(smem + L::OFF_Q + s * L::UNIT), 64 * 128, 1024);
-          const uint64_t dDOmn = sdesc_sw128(smem_u32(smem + L::OFF_DO + s * L::UNIT), 64 * 128, 1024);
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_ts(tV, tS + ks * 8, dDOmn + (uint64_t)ks * 128, id_acc, (jj > 0 || ks > 0) ? 1u : 0u);
-          mma_commit(&bar.dv_done[b]);
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_ts(tK, tP + ks * 8, dQmn + (uint64_t)ks * 128, id_acc, (jj > 0 || ks > 0) ? 1u : 0u);
-          mma_commit(&bar.dk_done[b]);
-          mma_commit(&bar.q_empty[s]);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tP, dVd + kslice16(kk, 128 * 128), dDOs + kslice16(kk, 128 * 128), id, kk > 0 ? 1u : 0u);
+        mma_commit(&bar.dp_full);
+        // dV += P^T dO, dK += dS^T Q
+        const uint64_t dQmn = sdesc_sw128(smem_u32(smem + L::OFF_Q + s * L::TILE), 128 * 128, 1024);
+        const uint64_t dDOmn = sdesc_sw128(smem_u32(smem + L::OFF_DO + s * L::TILE), 128 * 128, 1024);
+        ok = mbar_wait(&bar.p_ready, i & 1, status, 43);
+        if (!ok) break;
+        tc_fence_after();
+        for (int ks = 0; ks < 4 * nu; ++ks)
+          mma_ts(tV, tS + pk_col(ks), dDOmn + (uint64_t)ks * 128, id_acc, (i > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(&bar.dv_done);
+        ok = mbar_wait(&bar.ds_ready, i & 1, status, 47);
+        if (!ok) break;
+        tc_fence_after();
+        for (int ks = 0; ks < 4 * nu; ++ks)
+          mma_ts(tK, tP + pk_col(ks), dQmn + (uint64_t)ks * 128, id_acc, (i > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(&bar.dk_done);
+        mma_commit(&bar.q_empty[s]);
       }
       if (ok && nsteps > 0) mma_commit(&bar.fin);
       if (!ok) bar.abort = 1;
     }
     __syncwarp();
   } else if (warp >= 4) {
-    const int g = (warp - 4) >> 2;   // warpgroup: 32-query chunk g of every step
+    // ------------------------------------------------------------ compute
+    const int g = (warp - 4) >> 2;   // warpgroup: query unit g of every step
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;  // key row of the tile
     const int half = row >> 6;       // warp-uniform
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     bool ok = true;
     for (int i = 0; i < nsteps; ++i) {
-      const int b = i & 1, ph = (i >> 1) & 1, s = i % NS;
-      const uint32_t tS = tmem + 256 + 128 * b, tP = tS + 64;
-      ok = mbar_wait_warp(&bar.s_full[b], ph, status, 47);
-      if (ok) ok = mbar_wait_warp(&bar.dp_full[b], ph, status, 48);
+      const int s = i % NS;
+      ok = mbar_wait_warp(&bar.s_full, i & 1, status, 48);
       // the stage's statistics were written by the async proxy: observe the
       // stage's own barrier (already complete; the stage cannot be refilled
       // before this step releases it) so those writes are visible here
       if (ok) ok = mbar_wait_warp(&bar.q_full[s], (i / NS) & 1, status, 50);
       if (!ok) break;
       tc_fence_after();
-      const bool valid = (bar.mask[s] >> half) & 1;
-      const float4 *l2 = reinterpret_cast<const float4 *>(stat + s * 128 + g * 32);
-      const float4 *dl = reinterpret_cast<const float4 *>(stat + s * 128 + 64 + g * 32);
-      uint32_t pp[16], pd[16];
-      if (valid) {
-        uint32_t sv[32], dv[32];
-        tmem_ld32(tS + lane_off + g * 32, sv);
-        tmem_ld32(tP + lane_off + g * 32, dv);
-        tmem_wait_ld();
+      const int meta = bar.meta[s];
+      const bool active = g < (meta & 15);
+      const bool valid = active && (((meta >> (4 + 4 * g)) >> half) & 1);  // warp-uniform
+      const float *st = stat + s * 256 + 64 * g;
+      float pf[64];
 #pragma unroll
-        for (int k4 = 0; k4 < 8; ++k4) {
-          const float4 lq = l2[k4], dq = dl[k4];
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[16];
+        if (valid) {
+          uint32_t sv[32];
+          float nl[32];
+          tmem_ld32(tS + lane_off + 64 * g + 32 * c, sv);
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int k = 4 * k4 + 2 * u;
-            const float2 lm = u ? make_float2(-lq.z, -lq.w) : make_float2(-lq.x, -lq.y);
-            const float2 dd = u ? make_float2(dq.z, dq.w) : make_float2(dq.x, dq.y);
-            const float2 x = ffma2(make_float2(__uint_as_float(sv[k]), __uint_as_float(sv[k + 1])),
-                                   make_float2(scale_log2, scale_log2), lm);
-            const float2 p = make_float2(ex2f(x.x), ex2f(x.y));
-            const float2 d = fmul2(p, fsub2(make_float2(__uint_as_float(dv[k]), __uint_as_float(dv[k + 1])), dd));
-            pp[k / 2] = pack_f16(p.x, p.y);
-            pd[k / 2] = pack_f16(d.x, d.y);
+          for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 lq = reinterpret_cast<const float4 *>(st + 32 * c)[k4];
+            nl[4 * k4] = -lq.x;
+            nl[4 * k4 + 1] = -lq.y;
+            nl[4 * k4 + 2] = -lq.z;
+            nl[4 * k4 + 3] = -lq.w;
           }
-        }
-      } else {
+          tmem_wait_ld();
+          softmax_p32(sv, scale_log2, [&nl](int k) { return make_float2(nl[k], nl[k + 1]); }, pf + 32 * c);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) pp[k] = pd[k] = 0u;
+          for (int k = 0; k < 32; k += 2) pk[k / 2] = pack_f16(pf[32 * c + k], pf[32 * c + k + 1]);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) pk[k] = 0u;
+        }
+        if (active) tmem_st16(tS + lane_off + 64 * g + 16 * c, pk);
       }
-      tmem_st16(tS + lane_off + g * 16, pp);
-      tmem_st16(tP + lane_off + g * 16, pd);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar.ds_ready[b]);
+      mbar_arrive(&bar.p_ready);
+      ok = mbar_wait_warp(&bar.dp_full, i & 1, status, 49);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[16];
+        if (valid) {
+          uint32_t dv[32];
+          tmem_ld32(tP + lane_off + 64 * g + 32 * c, dv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 dq = reinterpret_cast<const float4 *>(st + 128 + 32 * c)[k4];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int k = 4 * k4 + 2 * u;
+              const float2 dd = u ? make_float2(dq.z, dq.w) : make_float2(dq.x, dq.y);
+              const float2 d = fmul2(make_float2(pf[32 * c + k], pf[32 * c + k + 1]),
+                                     fsub2(make_float2(__uint_as_float(dv[k]), __uint_as_float(dv[k + 1])), dd));
+              pk[k / 2] = pack_f16(d.x, d.y);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) pk[k] = 0u;
+        }
+        if (active) tmem_st16(tP + lane_off + 64 * g + 16 * c, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar.ds_ready);
     }
     ok = __all_sync(0xffffffffu, ok);
-    if (ok && nsteps > 0) ok = mbar_wait_warp(&bar.fin, 0, status, 49);
+    if (ok && nsteps > 0) ok = mbar_wait_warp(&bar.fin, 0, status, 51);
     if (ok) {
       tc_fence_after();
       const size_t prow = (size_t)h * N + (size_t)tile * 128 + row;

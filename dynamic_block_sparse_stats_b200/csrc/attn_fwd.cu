@@ -13,15 +13,20 @@
 // their selections and masks each key unit per row half.  Keys are streamed
 // as tiles of two 64-token units (any two units of the walk).
 //
-// Roles (192 threads):
-//   warp 0      TMA producer: Q once, then K and V units into a 2-stage ring.
+// Roles (384 threads, two 128-row query tiles t = 0, 1 per CTA):
+//   warp 0      TMA producer: Q once, then per key tile j the K tile j and
+//               the V tile j-1 into two 2-stage rings (K runs one ahead).
 //   warp 1      allocates TMEM; lane 0 issues tcgen05.mma:
-//                 S[b] = Q K^T  (SS, fp32 in TMEM, double buffered)
-//                 O   += P V    (TS: P is read from TMEM where S[b] was)
-//   warps 2-5   softmax, one thread per query row: reads S[b], online max
-//               with lazy rescaling of O (only when the max grows by more
-//               than 2^8), writes P as fp16 into TMEM, and finally
-//               normalises O and scatters it to natural token order.
+//                 S_t = Q_t K^T  (SS, fp32 in TMEM)
+//                 O_t += P_t V   (TS: P_t is read from TMEM where S_t was)
+//               in the order PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): each
+//               tile's next S waits only for its own PV, so the softmax of
+//               one tile runs while the tensor pipe works for the other.
+//   warps 4-11  two softmax warpgroups (tile t = warpgroup), one thread per
+//               query row: reads S_t, online max with lazy rescaling of O_t
+//               (only when the max grows by more than 2^8), writes P_t as
+//               fp16 into TMEM, and finally normalises O_t and scatters it
+//               to natural token order.
 #include "attn_walk.cuh"
 
 namespace prism {
@@ -34,6 +39,7 @@ constexpr int NSTAGE = 2;        // K/V ring depth
 constexpr int kThreads = 384;    // 12 warps
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (factor 256)
+constexpr int kPolyPairs = 0;         // of every 16 column pairs, this many take exp2_poly2 (none: measured slower here)
 
 template <int D>
 struct Smem {
@@ -46,15 +52,19 @@ struct Smem {
   static constexpr int BYTES = OFF_BAR + 256;
 };
 
+constexpr int NMETA = 4;  // ring of per-key-tile descriptors
+
 struct Bars {
   uint64_t q_full;
-  uint64_t k_full[NSTAGE];
-  uint64_t v_full[NSTAGE];
-  uint64_t kv_empty[NSTAGE];
+  uint64_t k_full[NSTAGE], k_empty[NSTAGE];
+  uint64_t v_full[NSTAGE], v_empty[NSTAGE];
   uint64_t s_full[2];   // per query tile
   uint64_t p_full[2];
   uint64_t pv_done[2];
-  int meta[NSTAGE];     // units | maskA << 4 | maskB << 8  (masks: bit = 64-row quarter)
+  // per key tile j, slot j % NMETA: units | maskA << 4 | maskB << 8 (masks:
+  // bit = 64-row quarter).  Written with K(j); slot j is rewritten for tile
+  // j + 4 only after both softmax warpgroups have finished tile j.
+  int meta[NMETA];
   uint32_t tmem_base;
   int ntiles;
   int nunits;
@@ -87,8 +97,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar.q_full, 1);
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(&bar.k_full[s], 1);
+      mbar_init(&bar.k_empty[s], 1);
       mbar_init(&bar.v_full[s], 1);
-      mbar_init(&bar.kv_empty[s], 1);
+      mbar_init(&bar.v_empty[s], 1);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bar.s_full[t], 1);
@@ -130,40 +141,58 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(smem + L::OFF_Q + t * L::TILE + c * (128 * 128), &mapQ, &bar.q_full, c * 64,
                       h * N + quad * BQ + t * 128);
     }
-    for (int j = 0; j < ntiles; ++j) {
-      const int s = j % NSTAGE;
-      uint32_t ua, ub = 0;
-      int ma, mb = 0, nu = 1;
-      walk_next<4>(w, col, blocks_h, ua, ma);
-      if (2 * j + 2 <= nunits) {
-        walk_next<4>(w, col, blocks_h, ub, mb);
-        nu = 2;
+    // iteration j loads K(j) and V(j-1): the next S needs K one tile before
+    // the PV that needs V
+    uint32_t pa = 0, pb = 0;  // units of tile j-1, for its V
+    int pnu = 0;
+    for (int j = 0; j <= ntiles; ++j) {
+      uint32_t ua = 0, ub = 0;
+      int ma = 0, mb = 0, nu = 1;
+      if (j < ntiles) {
+        walk_next<4>(w, col, blocks_h, ua, ma);
+        if (2 * j + 2 <= nunits) {
+          walk_next<4>(w, col, blocks_h, ub, mb);
+          nu = 2;
+        }
+        ua = min(ua, (uint32_t)(NB - 1));  // a well-formed walk never clamps
+        ub = min(ub, (uint32_t)(NB - 1));
       }
-      ua = min(ua, (uint32_t)(NB - 1));  // a well-formed walk never clamps
-      ub = min(ub, (uint32_t)(NB - 1));
       if (lane == 0) {
         bool ok = true;
-        if (j >= NSTAGE) ok = mbar_wait(&bar.kv_empty[s], ((j / NSTAGE) - 1) & 1, status, 1);
-        if (!ok) bar.abort = 1;
-        if (ok) {
-          bar.meta[s] = nu | (ma << 4) | (mb << 8);
-          uint8_t *ks = smem + L::OFF_K + s * L::TILE;
-          uint8_t *vs = smem + L::OFF_V + s * L::TILE;
-          const int bytes = nu * 64 * D * 2;
-          mbar_arrive_expect_tx(&bar.k_full[s], bytes);
+        if (j < ntiles) {
+          const int s = j % NSTAGE;
+          if (j >= NSTAGE) ok = mbar_wait(&bar.k_empty[s], ((j / NSTAGE) - 1) & 1, status, 1);
+          if (ok) {
+            bar.meta[j % NMETA] = nu | (ma << 4) | (mb << 8);
+            uint8_t *ks = smem + L::OFF_K + s * L::TILE;
+            mbar_arrive_expect_tx(&bar.k_full[s], nu * 64 * D * 2);
 #pragma unroll
-          for (int c = 0; c < L::CHUNKS; ++c) {
-            tma_load_2d(ks + c * (128 * 128), &mapK, &bar.k_full[s], c * 64, h * N + (int)ua * 64);
-            if (nu == 2) tma_load_2d(ks + c * (128 * 128) + 64 * 128, &mapK, &bar.k_full[s], c * 64, h * N + (int)ub * 64);
-          }
-          mbar_arrive_expect_tx(&bar.v_full[s], bytes);
-#pragma unroll
-          for (int c = 0; c < L::CHUNKS; ++c) {
-            tma_load_2d(vs + c * (128 * 128), &mapV, &bar.v_full[s], c * 64, h * N + (int)ua * 64);
-            if (nu == 2) tma_load_2d(vs + c * (128 * 128) + 64 * 128, &mapV, &bar.v_full[s], c * 64, h * N + (int)ub * 64);
+            for (int c = 0; c < L::CHUNKS; ++c) {
+              tma_load_2d(ks + c * (128 * 128), &mapK, &bar.k_full[s], c * 64, h * N + (int)ua * 64);
+              if (nu == 2)
+                tma_load_2d(ks + c * (128 * 128) + 64 * 128, &mapK, &bar.k_full[s], c * 64, h * N + (int)ub * 64);
+            }
           }
         }
+        if (ok && j >= 1) {
+          const int jv = j - 1, s = jv % NSTAGE;
+          if (jv >= NSTAGE) ok = mbar_wait(&bar.v_empty[s], ((jv / NSTAGE) - 1) & 1, status, 10);
+          if (ok) {
+            uint8_t *vs = smem + L::OFF_V + s * L::TILE;
+            mbar_arrive_expect_tx(&bar.v_full[s], pnu * 64 * D * 2);
+#pragma unroll
+            for (int c = 0; c < L::CHUNKS; ++c) {
+              tma_load_2d(vs + c * (128 * 128), &mapV, &bar.v_full[s], c * 64, h * N + (int)pa * 64);
+              if (pnu == 2)
+                tma_load_2d(vs + c * (128 * 128) + 64 * 128, &mapV, &bar.v_full[s], c * 64, h * N + (int)pb * 64);
+            }
+          }
+        }
+        if (!ok) bar.abort = 1;
       }
+      pa = ua;
+      pb = ub;
+      pnu = nu;
       __syncwarp();
       if (*reinterpret_cast<volatile int *>(&bar.abort)) break;
     }
@@ -175,31 +204,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_o = idesc_f16(128, D, 1);
       const uint64_t dQ0 = sdesc_sw128(smem_u32(smem + L::OFF_Q), 16, 1024);
       const uint64_t dQ1 = sdesc_sw128(smem_u32(smem + L::OFF_Q + L::TILE), 16, 1024);
-      bool ok = mbar_wait(&bar.q_full, 0, status, 2);
-      tc_fence_after();
-      for (int j = 0; ok && j < ntiles; ++j) {
-        const int s = j % NSTAGE;
-        ok = mbar_wait(&bar.k_full[s], (j / NSTAGE) & 1, status, 3);
-        if (!ok) break;
-        tc_fence_after();
-        const int nu = bar.meta[s] & 15;
+      // S_t(jj) = Q_t K(jj)^T into S_t's columns; K(jj) is in stage jj % NSTAGE
+      auto issue_s = [&](int t, int jj) {
+        const int nu = bar.meta[jj % NMETA] & 15;
         const uint32_t idesc_s = nu == 2 ? idesc_s_full : idesc_s_half;
-        const uint64_t dK = sdesc_sw128(smem_u32(smem + L::OFF_K + s * L::TILE), 16, 1024);
-        const uint64_t dV = sdesc_sw128(smem_u32(smem + L::OFF_V + s * L::TILE), 128 * 128, 1024);
-        for (int t = 0; t < 2; ++t) {
-          // S_t is free once the PV of the previous key tile read its P
-          if (j >= 1) ok = mbar_wait(&bar.pv_done[t], (j - 1) & 1, status, 4);
-          if (!ok) break;
-          tc_fence_after();
-          const uint64_t dQt = t ? dQ1 : dQ0;
+        const uint64_t dK = sdesc_sw128(smem_u32(smem + L::OFF_K + (jj % NSTAGE) * L::TILE), 16, 1024);
+        const uint64_t dQt = t ? dQ1 : dQ0;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + 128 * t, dQt + kslice16(kk, 128 * 128), dK + kslice16(kk, 128 * 128), idesc_s,
-                   kk > 0 ? 1u : 0u);
-          mma_commit(&bar.s_full[t]);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + 128 * t, dQt + kslice16(kk, 128 * 128), dK + kslice16(kk, 128 * 128), idesc_s,
+                 kk > 0 ? 1u : 0u);
+        mma_commit(&bar.s_full[t]);
+      };
+      bool ok = mbar_wait(&bar.q_full, 0, status, 2);
+      if (ok && ntiles > 0) ok = mbar_wait(&bar.k_full[0], 0, status, 3);
+      if (ok && ntiles > 0) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        mma_commit(&bar.k_empty[0]);
+      }
+      for (int j = 0; ok && j < ntiles; ++j) {
+        const int sv = j % NSTAGE;
+        const int nu = bar.meta[j % NMETA] & 15;
+        const bool next = j + 1 < ntiles;
+        ok = mbar_wait(&bar.v_full[sv], (j / NSTAGE) & 1, status, 6);
+        if (ok && next) ok = mbar_wait(&bar.k_full[(j + 1) % NSTAGE], ((j + 1) / NSTAGE) & 1, status, 3);
         if (!ok) break;
-        ok = mbar_wait(&bar.v_full[s], (j / NSTAGE) & 1, status, 6);
+        const uint64_t dV = sdesc_sw128(smem_u32(smem + L::OFF_V + sv * L::TILE), 128 * 128, 1024);
         for (int t = 0; ok && t < 2; ++t) {
           ok = mbar_wait(&bar.p_full[t], j & 1, status, 5);
           if (!ok) break;
@@ -208,8 +240,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int ks = 0; ks < nu * 4; ++ks)
             mma_ts(tOt, tPt + ks * 8, dV + (uint64_t)ks * 128, idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
           mma_commit(&bar.pv_done[t]);
+          if (t == 1) mma_commit(&bar.v_empty[sv]);
+          if (next) {
+            // S_t(j+1) overwrites the columns PV_t(j) reads P_t from
+            ok = mbar_wait(&bar.pv_done[t], j & 1, status, 4);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(t, j + 1);
+            if (t == 1) mma_commit(&bar.k_empty[(j + 1) % NSTAGE]);
+          }
         }
-        mma_commit(&bar.kv_empty[s]);
       }
       if (!ok) bar.abort = 1;
     }
@@ -225,11 +265,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
-      const int s = j % NSTAGE;
       ok = mbar_wait_warp(&bar.s_full[t], j & 1, status, 7);
       if (!ok) break;
       tc_fence_after();
-      const int meta = bar.meta[s];
+      const int meta = bar.meta[j % NMETA];
       const int nu = meta & 15;
       const bool v0 = ((meta >> 4) >> qbit) & 1;
       const bool v1 = nu == 2 && (((meta >> 8) >> qbit) & 1);
@@ -250,7 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
               const float2 x = ffma2(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), scale_log2, -m);
-              const float2 p = make_float2(ex2f(x.x), ex2f(x.y));
+              // a share of the exponentials on the FMA pipe, the rest on MUFU
+              const float2 p = i < 2 * kPolyPairs ? exp2_poly2(x) : make_float2(ex2f(x.x), ex2f(x.y));
               ls2 = fadd2(ls2, p);
               const uint32_t h2 = pack_f16(p.x, p.y);
               pmax = hmax2u(pmax, h2);

@@ -272,6 +272,23 @@ __device__ __forceinline__ float ex2f(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// 2^x on the FMA pipe, for a share of the softmax exponentials (the MUFU unit
+// is otherwise as busy as the tensor pipe).  Cody-Waite style range
+// reduction x = n + f, n = floor(x), f in [0, 1): n comes from adding
+// 1.5 * 2^23 with rounding toward -inf, 2^f from a degree-3 polynomial whose
+// coefficients are a minimax fit of 2^f on [0, 1) in relative error
+// (computed here by linear programming; max relative error 7.5e-5 in fp32,
+// below half an fp16 ulp), and 2^n is added to the exponent field.
+// x is clamped to [-125, 64]: below, the result is far under the smallest
+// fp16 subnormal; above, it is +inf after fp16 conversion like the MUFU
+// result it replaces.
+__device__ __forceinline__ float2 fadd2_rm(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rm.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<uint64_t *>(&a)), "l"(*reinterpret_cast<uint64_t *>(&b)));
+  return *reinterpret_cast<float2 *>(&d);
+}
 __device__ __forceinline__ float fmax3f(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -307,6 +324,23 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
   uint64_t d;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
   return u2f(d);
+}
+// 2^x for a pair, on the FMA pipe (see fadd2_rm above for the method)
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.9999251961708069f, c1 = 0.6958335638046265f, c2 = 0.22606714069843292f,
+                  c3 = 0.07802452892065048f;
+  x.x = fminf(fmaxf(x.x, -125.0f), 64.0f);
+  x.y = fminf(fmaxf(x.y, -125.0f), 64.0f);
+  const float2 t = fadd2_rm(x, make_float2(kMagic, kMagic));    // floor(x) + 1.5 * 2^23, exactly
+  const float2 f = fsub2(x, fsub2(t, make_float2(kMagic, kMagic)));
+  float2 p = ffma2(f, make_float2(c3, c3), make_float2(c2, c2));
+  p = ffma2(p, f, make_float2(c1, c1));
+  p = ffma2(p, f, make_float2(c0, c0));
+  // the low mantissa bits of t hold floor(x) (two's complement); shifted
+  // into the exponent field they scale p by 2^floor(x)
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
 // ---------------------------------------------------------------------------

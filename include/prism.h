@@ -337,6 +337,16 @@ int prism_kernel_timing_read(int id, int *launches, double *total_ms,
 /* Library version, "major.minor.patch". */
 const char *prism_version(void);
 
+/*
+ * prism_diag_exp2 -- diagnostics.  Evaluates, for n fp32 inputs x (device
+ * memory), the two exponentials prism_attn_fwd uses for softmax weights:
+ * y_poly = 2^x from the FMA-pipe polynomial (x clamped to [-125, 64];
+ * relative error at most 7.5e-5, below half an fp16 ulp) and y_mufu = 2^x
+ * from the MUFU instruction.  Outputs are fp32 device arrays of n entries.
+ * Returns PRISM_OK, PRISM_ERR_INVALID_ARG or PRISM_ERR_CUDA.
+ */
+int prism_diag_exp2(const float *x, float *y_poly, float *y_mufu, int64_t n, prism_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

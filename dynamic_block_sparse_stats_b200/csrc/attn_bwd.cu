@@ -12,8 +12,8 @@
 // Two kernels, no atomics (deterministic):
 //   dq_kernel    one CTA per 128-query tile; walks the CSR like the forward,
 //                two key units (128 keys) per step: S = Q K^T and dP = dO V^T
-//                (TMEM, S double buffered), dS -> TMEM (fp16), dQ += dS K
-//                (TS MMA).
+//                with Q and dO held in TMEM (TS MMAs), dS -> TMEM (fp16),
+//                dQ += dS K (TS MMA).
 //   dkdv_kernel  one CTA per 128-key tile; walks the transpose (CSC), two
 //                query units per step: S^T = K Q^T, dP^T = V dO^T (TMEM),
 //                P^T and dS^T -> TMEM (fp16), dV += P^T dO, dK += dS^T Q (TS
@@ -131,36 +131,39 @@ __device__ __forceinline__ void softmax_p32(const uint32_t (&sv)[32], float scal
 // ---------------------------------------------------------------------------
 // dQ kernel: one CTA per 128-query tile; steps over pairs of the key units of
 // the union of its rows' selections.
-//   TMEM: dQ [0, 128); dP [128, 256); S in buffer b at [256 + 128b, +128),
-//   dS packed into the same columns.
+//   TMEM: dQ [0, 128); Q and dO as fp16 MMA operands [128, 192) and
+//   [192, 256) (loaded once, so S and dP are TS products that read only K
+//   and V from shared memory); S [256, 384); dP [384, 512), dS packed into
+//   the dP columns.
+//   Per step the MMA issue order is S(i+1), dQ(i), dP(i+1): the next S runs
+//   while the compute warps turn dP(i) into dS(i).
 // ---------------------------------------------------------------------------
+constexpr int NSQ = 3;  // K/V ring depth of the dQ kernel
+
 template <int D>
 struct DqSmem {
   static constexpr int CHUNKS = D / 64;
   static constexpr int TILE = 128 * D * 2;  // 128 rows of fp16
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_DO = OFF_Q + TILE;
-  static constexpr int OFF_K = OFF_DO + TILE;
-  static constexpr int OFF_V = OFF_K + NS * TILE;
-  static constexpr int OFF_BAR = OFF_V + NS * TILE;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + NSQ * TILE;
+  static constexpr int OFF_BAR = OFF_V + NSQ * TILE;
   static constexpr int BYTES = OFF_BAR + 256;
 };
 
 struct DqBars {
-  uint64_t qdo_full;
-  uint64_t k_full[NS], v_full[NS], kv_empty[NS];
-  uint64_t s_full[2], ds_ready[2], dq_done[2];
-  uint64_t dp_full, dp_free;
+  uint64_t k_full[NSQ], v_full[NSQ], k_empty[NSQ], v_empty[NSQ];
+  uint64_t qdo_ready;  // Q and dO are in TMEM (256 arrivals)
+  uint64_t s_full, s_free, dp_full, ds_ready, dq_done;
   uint64_t fin;  // single use: every MMA of the tile has completed
-  int meta[NS];  // units | mask_a << 4 | mask_b << 8 (bit = 64-row half of the tile)
+  int meta[NSQ];  // units | mask_a << 4 | mask_b << 8 (bit = 64-row half of the tile)
   uint32_t tmem_base;
   int nsteps, nunits, abort;
 };
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    dq_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapDO,
-              const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
+    dq_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
+              const uint16_t *__restrict__ Qp, const uint16_t *__restrict__ dOp,
               const int32_t *__restrict__ row_ptr, const int32_t *__restrict__ col, const int32_t *__restrict__ blocks,
               const int32_t *__restrict__ unit_block, const int32_t *__restrict__ tile_units,
               const int32_t *__restrict__ perm, const float *__restrict__ lse2p, const float *__restrict__ deltap,
@@ -179,19 +182,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (bar.abort) return;
   if (threadIdx.x == 0) {
-    mbar_init(&bar.qdo_full, 1);
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < NSQ; ++s) {
       mbar_init(&bar.k_full[s], 1);
       mbar_init(&bar.v_full[s], 1);
-      mbar_init(&bar.kv_empty[s], 1);
+      mbar_init(&bar.k_empty[s], 1);
+      mbar_init(&bar.v_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bar.s_full[b], 1);
-      mbar_init(&bar.ds_ready[b], 256);
-      mbar_init(&bar.dq_done[b], 1);
-    }
+    mbar_init(&bar.qdo_ready, 256);
+    mbar_init(&bar.s_full, 1);
+    mbar_init(&bar.s_free, 256);
     mbar_init(&bar.dp_full, 1);
-    mbar_init(&bar.dp_free, 256);
+    mbar_init(&bar.ds_ready, 256);
+    mbar_init(&bar.dq_done, 1);
     mbar_init(&bar.fin, 1);
     bar.nunits = tile_units[(size_t)h * (N / 128) + tile];
     bar.nsteps = (bar.nunits + 1) >> 1;
@@ -206,23 +208,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bar.tmem_base;
   const int nsteps = bar.nsteps, nunits = bar.nunits;
-  const uint32_t tQacc = tmem, tdP = tmem + 128;
+  const uint32_t tQacc = tmem, tQ16 = tmem + 128, tdO16 = tmem + 192, tS = tmem + 256, tdP = tmem + 384;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     const int blk[2] = {unit_block[(size_t)h * NB + 2 * tile], unit_block[(size_t)h * NB + 2 * tile + 1]};
     UnitWalk<2> w;
     walk_init<2>(w, blk, 2, row_ptr, h * NB);
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&bar.qdo_full, 2 * L::TILE);
-#pragma unroll
-      for (int c = 0; c < L::CHUNKS; ++c) {
-        tma_load_2d(smem + L::OFF_Q + c * (128 * 128), &mapQ, &bar.qdo_full, c * 64, h * N + tile * 128);
-        tma_load_2d(smem + L::OFF_DO + c * (128 * 128), &mapDO, &bar.qdo_full, c * 64, h * N + tile * 128);
-      }
-    }
     for (int j = 0; j < nsteps; ++j) {
-      const int s = j % NS;
+      const int s = j % NSQ;
       uint32_t ua, ub = 0;
       int ma, mb = 0, nu = 1;
       walk_next<2>(w, col, blocks_h, ua, ma);
@@ -234,18 +228,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       ub = min(ub, (uint32_t)(NB - 1));
       if (lane == 0) {
         bool ok = true;
-        if (j >= NS) ok = mbar_wait(&bar.kv_empty[s], ((j / NS) - 1) & 1, status, 21);
-        if (!ok) bar.abort = 1;
+        if (j >= NSQ) ok = mbar_wait(&bar.k_empty[s], ((j / NSQ) - 1) & 1, status, 21);
         if (ok) {
           bar.meta[s] = nu | (ma << 4) | (mb << 8);
           uint8_t *ks = smem + L::OFF_K + s * L::TILE;
-          uint8_t *vs = smem + L::OFF_V + s * L::TILE;
           mbar_arrive_expect_tx(&bar.k_full[s], nu * 64 * D * 2);
 #pragma unroll
           for (int c = 0; c < L::CHUNKS; ++c) {
             tma_load_2d(ks + c * (128 * 128), &mapK, &bar.k_full[s], c * 64, h * N + (int)ua * 64);
             if (nu == 2) tma_load_2d(ks + c * (128 * 128) + 64 * 128, &mapK, &bar.k_full[s], c * 64, h * N + (int)ub * 64);
           }
+        }
+        if (ok && j >= NSQ) ok = mbar_wait(&bar.v_empty[s], ((j / NSQ) - 1) & 1, status, 20);
+        if (ok) {
+          uint8_t *vs = smem + L::OFF_V + s * L::TILE;
           mbar_arrive_expect_tx(&bar.v_full[s], nu * 64 * D * 2);
 #pragma unroll
           for (int c = 0; c < L::CHUNKS; ++c) {
@@ -253,6 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (nu == 2) tma_load_2d(vs + c * (128 * 128) + 64 * 128, &mapV, &bar.v_full[s], c * 64, h * N + (int)ub * 64);
           }
         }
+        if (!ok) bar.abort = 1;
       }
       __syncwarp();
       if (*reinterpret_cast<volatile int *>(&bar.abort)) break;
@@ -262,48 +259,55 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t id_full = idesc_f16(128, 128, 0), id_half = idesc_f16(128, 64, 0);
       const uint32_t id_acc = idesc_f16(128, D, 1);
-      const uint64_t dQd = sdesc_sw128(smem_u32(smem + L::OFF_Q), 16, 1024);
-      const uint64_t dDOd = sdesc_sw128(smem_u32(smem + L::OFF_DO), 16, 1024);
-      bool ok = mbar_wait(&bar.qdo_full, 0, status, 22);
+      // S(i) = Q K_i^T (TS); waits for the stage's K and for the compute warps
+      // to have read S(i-1)
+      auto issue_s = [&](int i) -> bool {
+        const int s = i % NSQ;
+        bool ok = mbar_wait(&bar.k_full[s], (i / NSQ) & 1, status, 24);
+        if (ok && i >= 1) ok = mbar_wait(&bar.s_free, (i - 1) & 1, status, 26);
+        if (!ok) return false;
+        tc_fence_after();
+        const int nu = bar.meta[s] & 15;  // written before the stage's K arrived
+        const uint64_t dK = sdesc_sw128(smem_u32(smem + L::OFF_K + s * L::TILE), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ts(tS, tQ16 + kk * 8, dK + kslice16(kk, 128 * 128), nu == 2 ? id_full : id_half, kk > 0 ? 1u : 0u);
+        mma_commit(&bar.s_full);
+        return true;
+      };
+      // dP(i) = dO V_i^T (TS) into the dP columns, free once dQ(i-1) read dS(i-1)
+      auto issue_dp = [&](int i) -> bool {
+        const int s = i % NSQ;
+        bool ok = mbar_wait(&bar.v_full[s], (i / NSQ) & 1, status, 25);
+        if (ok && i >= 1) ok = mbar_wait(&bar.dq_done, (i - 1) & 1, status, 27);
+        if (!ok) return false;
+        tc_fence_after();
+        const int nu = bar.meta[s] & 15;
+        const uint64_t dV = sdesc_sw128(smem_u32(smem + L::OFF_V + s * L::TILE), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ts(tdP, tdO16 + kk * 8, dV + kslice16(kk, 128 * 128), nu == 2 ? id_full : id_half, kk > 0 ? 1u : 0u);
+        mma_commit(&bar.dp_full);
+        mma_commit(&bar.v_empty[s]);
+        return true;
+      };
+      bool ok = mbar_wait(&bar.qdo_ready, 0, status, 22);
       tc_fence_after();
-      for (int i = 0; ok && i <= nsteps; ++i) {
-        if (i < nsteps) {  // S_i = Q K_i^T into buffer i&1, dP_i = dO V_i^T
-          const int s = i % NS, b = i & 1;
-          ok = mbar_wait(&bar.k_full[s], (i / NS) & 1, status, 24);
-          if (ok && i >= 2) ok = mbar_wait(&bar.dq_done[b], ((i - 2) >> 1) & 1, status, 26);
-          if (!ok) break;
-          tc_fence_after();
-          const int nu = bar.meta[s] & 15;  // written before the stage's K arrived
-          const uint32_t id = nu == 2 ? id_full : id_half;
-          const uint64_t dK = sdesc_sw128(smem_u32(smem + L::OFF_K + s * L::TILE), 16, 1024);
-          const uint64_t dV = sdesc_sw128(smem_u32(smem + L::OFF_V + s * L::TILE), 16, 1024);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + 256 + 128 * b, dQd + kslice16(kk, 128 * 128), dK + kslice16(kk, 128 * 128), id,
-                   kk > 0 ? 1u : 0u);
-          mma_commit(&bar.s_full[b]);
-          ok = mbar_wait(&bar.v_full[s], (i / NS) & 1, status, 25);
-          if (ok && i >= 1) ok = mbar_wait(&bar.dp_free, (i - 1) & 1, status, 27);
-          if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tdP, dDOd + kslice16(kk, 128 * 128), dV + kslice16(kk, 128 * 128), id, kk > 0 ? 1u : 0u);
-          mma_commit(&bar.dp_full);
-        }
-        if (i >= 1) {  // dQ += dS_{i-1} K_{i-1}
-          const int jj = i - 1, s = jj % NS, b = jj & 1;
-          const int nu = bar.meta[s] & 15;
-          ok = mbar_wait(&bar.ds_ready[b], (jj >> 1) & 1, status, 23);
-          if (!ok) break;
-          tc_fence_after();
-          const uint64_t dKmn = sdesc_sw128(smem_u32(smem + L::OFF_K + s * L::TILE), 128 * 128, 1024);
-          for (int ks = 0; ks < 4 * nu; ++ks)
-            mma_ts(tQacc, tmem + 256 + 128 * b + pk_col(ks), dKmn + (uint64_t)ks * 128, id_acc,
-                   (jj > 0 || ks > 0) ? 1u : 0u);
-          mma_commit(&bar.dq_done[b]);
-          mma_commit(&bar.kv_empty[s]);
-        }
+      if (ok && nsteps > 0) ok = issue_s(0) && issue_dp(0);
+      for (int i = 0; ok && i < nsteps; ++i) {
+        if (i + 1 < nsteps && !(ok = issue_s(i + 1))) break;
+        // dQ += dS(i) K(i)
+        const int s = i % NSQ;
+        ok = mbar_wait(&bar.ds_ready, i & 1, status, 23);
+        if (!ok) break;
+        tc_fence_after();
+        const int nu = bar.meta[s] & 15;
+        const uint64_t dKmn = sdesc_sw128(smem_u32(smem + L::OFF_K + s * L::TILE), 128 * 128, 1024);
+        for (int ks = 0; ks < 4 * nu; ++ks)
+          mma_ts(tQacc, tdP + pk_col(ks), dKmn + (uint64_t)ks * 128, id_acc, (i > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(&bar.dq_done);
+        mma_commit(&bar.k_empty[s]);
+        if (i + 1 < nsteps && !(ok = issue_dp(i + 1))) break;
       }
       if (ok && nsteps > 0) mma_commit(&bar.fin);
       if (!ok) bar.abort = 1;
@@ -319,11 +323,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t prow = (size_t)h * N + (size_t)tile * 128 + row;
     const float lse2 = lse2p[prow], dl = deltap[prow];
     const auto row_lse = [lse2](int) { return make_float2(-lse2, -lse2); };
+    // Q and dO rows into TMEM as fp16 operands (two elements per column):
+    // warpgroup g stores elements [g D/2, (g+1) D/2) of the row
+    {
+      const uint4 *qs = reinterpret_cast<const uint4 *>(Qp + prow * D + (D / 2) * g);
+      const uint4 *os = reinterpret_cast<const uint4 *>(dOp + prow * D + (D / 2) * g);
+      uint32_t q[32], o[32];
+#pragma unroll
+      for (int v = 0; v < D / 16; ++v) {
+        const uint4 a = __ldg(qs + v), b = __ldg(os + v);
+        q[4 * v] = a.x, q[4 * v + 1] = a.y, q[4 * v + 2] = a.z, q[4 * v + 3] = a.w;
+        o[4 * v] = b.x, o[4 * v + 1] = b.y, o[4 * v + 2] = b.z, o[4 * v + 3] = b.w;
+      }
+      if (D == 128) {
+        tmem_st32(tQ16 + lane_off + 32 * g, q);
+        tmem_st32(tdO16 + lane_off + 32 * g, o);
+      } else {
+        tmem_st16(tQ16 + lane_off + 16 * g, q);
+        tmem_st16(tdO16 + lane_off + 16 * g, o);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar.qdo_ready);
+    }
     bool ok = true;
     for (int i = 0; i < nsteps; ++i) {
-      const int b = i & 1, s = i % NS;
-      const uint32_t tS = tmem + 256 + 128 * b + 64 * g;
-      ok = mbar_wait_warp(&bar.s_full[b], (i >> 1) & 1, status, 28);
+      const int s = i % NSQ;
+      ok = mbar_wait_warp(&bar.s_full, i & 1, status, 28);
       if (!ok) break;
       tc_fence_after();
       const int meta = bar.meta[s];
@@ -331,28 +357,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = active && (((meta >> (4 + 4 * g)) >> half) & 1);  // warp-uniform
       float pf[64];
       if (valid) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t sv[32];
-          tmem_ld32(tS + lane_off + 32 * c, sv);
-          tmem_wait_ld();
-          softmax_p32(sv, scale_log2, row_lse, pf + 32 * c);
-        }
+        uint32_t sv[2][32];
+        tmem_ld32(tS + lane_off + 64 * g, sv[0]);
+        tmem_ld32(tS + lane_off + 64 * g + 32, sv[1]);
+        tmem_wait_ld();
+        softmax_p32(sv[0], scale_log2, row_lse, pf);
+        softmax_p32(sv[1], scale_log2, row_lse, pf + 32);
       }
+      tc_fence_before();
+      mbar_arrive(&bar.s_free);  // S(i) read: S(i+1) may overwrite it
       ok = mbar_wait_warp(&bar.dp_full, i & 1, status, 29);
       if (!ok) break;
       tc_fence_after();
+      uint32_t dv[2][32];
+      if (valid) tmem_ld32(tdP + lane_off + 64 * g, dv[0]);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t pk[16];
         if (valid) {
-          uint32_t dv[32];
-          tmem_ld32(tdP + lane_off + 64 * g + 32 * c, dv);
-          tmem_wait_ld();
+          tmem_wait_ld_r(dv[c]);
+          if (c == 0) tmem_ld32(tdP + lane_off + 64 * g + 32, dv[1]);
 #pragma unroll
           for (int k = 0; k < 32; k += 2) {
             const float2 d = fmul2(make_float2(pf[32 * c + k], pf[32 * c + k + 1]),
-                                   fsub2(make_float2(__uint_as_float(dv[k]), __uint_as_float(dv[k + 1])),
+                                   fsub2(make_float2(__uint_as_float(dv[c][k]), __uint_as_float(dv[c][k + 1])),
                                          make_float2(dl, dl)));
             pk[k / 2] = pack_f16(d.x, d.y);
           }
@@ -360,18 +388,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < 16; ++k) pk[k] = 0u;
         }
-        if (c == 1) {  // every read of dP_i is done: the next dP may overwrite it
-          tc_fence_before();
-          mbar_arrive(&bar.dp_free);
-        }
-        if (active) tmem_st16(tS + lane_off + 16 * c, pk);
+        // dS goes into the first half of this warpgroup's own dP columns,
+        // below the chunk-1 values still loading
+        if (active) tmem_st16(tdP + lane_off + 64 * g + 16 * c, pk);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar.ds_ready[b]);
+      mbar_arrive(&bar.ds_ready);
     }
-    // A parity wait on dq_done could match an older phase; the single-use
-    // barrier cannot.
     ok = __all_sync(0xffffffffu, ok);
     if (ok && nsteps > 0) ok = mbar_wait_warp(&bar.fin, 0, status, 30);
     if (ok) {
@@ -610,30 +634,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = active && (((meta >> (4 + 4 * g)) >> half) & 1);  // warp-uniform
       const float *st = stat + s * 256 + 64 * g;
       float pf[64];
+      // P^T: 32-column chunks of S^T, chunk 1 loading while chunk 0 is computed
+      {
+        uint32_t sv[2][32];
+        if (valid) tmem_ld32(tS + lane_off + 64 * g, sv[0]);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t pk[16];
-        if (valid) {
-          uint32_t sv[32];
-          float nl[32];
-          tmem_ld32(tS + lane_off + 64 * g + 32 * c, sv);
+        for (int c = 0; c < 2; ++c) {
+          uint32_t pk[16];
+          if (valid) {
+            tmem_wait_ld_r(sv[c]);
+            if (c == 0) tmem_ld32(tS + lane_off + 64 * g + 32, sv[1]);
+            const float *lq = st + 32 * c;
+            softmax_p32(sv[c], scale_log2,
+                        [lq](int k) {
+                          const float2 v = *reinterpret_cast<const float2 *>(lq + k);
+                          return make_float2(-v.x, -v.y);
+                        },
+                        pf + 32 * c);
 #pragma unroll
-          for (int k4 = 0; k4 < 8; ++k4) {
-            const float4 lq = reinterpret_cast<const float4 *>(st + 32 * c)[k4];
-            nl[4 * k4] = -lq.x;
-            nl[4 * k4 + 1] = -lq.y;
-            nl[4 * k4 + 2] = -lq.z;
-            nl[4 * k4 + 3] = -lq.w;
+            for (int k = 0; k < 32; k += 2) pk[k / 2] = pack_f16(pf[32 * c + k], pf[32 * c + k + 1]);
+          } else {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) pk[k] = 0u;
           }
-          tmem_wait_ld();
-          softmax_p32(sv, scale_log2, [&nl](int k) { return make_float2(nl[k], nl[k + 1]); }, pf + 32 * c);
-#pragma unroll
-          for (int k = 0; k < 32; k += 2) pk[k / 2] = pack_f16(pf[32 * c + k], pf[32 * c + k + 1]);
-        } else {
-#pragma unroll
-          for (int k = 0; k < 16; ++k) pk[k] = 0u;
+          // chunk c's P^T goes to [16c, 16c+16) of this warpgroup's columns,
+          // below the chunk-1 scores still loading
+          if (active) tmem_st16(tS + lane_off + 64 * g + 16 * c, pk);
         }
-        if (active) tmem_st16(tS + lane_off + 64 * g + 16 * c, pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -641,30 +668,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = mbar_wait_warp(&bar.dp_full, i & 1, status, 49);
       if (!ok) break;
       tc_fence_after();
+      {
+        uint32_t dv[2][32];
+        if (valid) tmem_ld32(tP + lane_off + 64 * g, dv[0]);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t pk[16];
-        if (valid) {
-          uint32_t dv[32];
-          tmem_ld32(tP + lane_off + 64 * g + 32 * c, dv);
-          tmem_wait_ld();
+        for (int c = 0; c < 2; ++c) {
+          uint32_t pk[16];
+          if (valid) {
+            tmem_wait_ld_r(dv[c]);
+            if (c == 0) tmem_ld32(tP + lane_off + 64 * g + 32, dv[1]);
 #pragma unroll
-          for (int k4 = 0; k4 < 8; ++k4) {
-            const float4 dq = reinterpret_cast<const float4 *>(st + 128 + 32 * c)[k4];
+            for (int k4 = 0; k4 < 8; ++k4) {
+              const float4 dq = reinterpret_cast<const float4 *>(st + 128 + 32 * c)[k4];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int k = 4 * k4 + 2 * u;
-              const float2 dd = u ? make_float2(dq.z, dq.w) : make_float2(dq.x, dq.y);
-              const float2 d = fmul2(make_float2(pf[32 * c + k], pf[32 * c + k + 1]),
-                                     fsub2(make_float2(__uint_as_float(dv[k]), __uint_as_float(dv[k + 1])), dd));
-              pk[k / 2] = pack_f16(d.x, d.y);
+              for (int u = 0; u < 2; ++u) {
+                const int k = 4 * k4 + 2 * u;
+                const float2 dd = u ? make_float2(dq.z, dq.w) : make_float2(dq.x, dq.y);
+                const float2 d = fmul2(make_float2(pf[32 * c + k], pf[32 * c + k + 1]),
+                                       fsub2(make_float2(__uint_as_float(dv[c][k]), __uint_as_float(dv[c][k + 1])),
+                                             dd));
+                pk[k / 2] = pack_f16(d.x, d.y);
+              }
             }
-          }
-        } else {
+          } else {
 #pragma unroll
-          for (int k = 0; k < 16; ++k) pk[k] = 0u;
+            for (int k = 0; k < 16; ++k) pk[k] = 0u;
+          }
+          if (active) tmem_st16(tP + lane_off + 64 * g + 16 * c, pk);
         }
-        if (active) tmem_st16(tP + lane_off + 64 * g + 16 * c, pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -752,10 +783,8 @@ static cudaError_t run_bwd(const prism_params &p, const prism_plan_t &plan, cons
                            const BwdWs &w, void *dQ, void *dK, void *dV, int grad_fp32, cudaStream_t st) {
   const int N = p.T * p.H * p.W;
   const long long rows = (long long)p.heads * N;
-  CUtensorMap mQ128, mDO128, mK64, mV64, mQ64, mDO64, mK128, mV128;  // box rows 128 or 64
+  CUtensorMap mK64, mV64, mQ64, mDO64, mK128, mV128;  // box rows 128 or 64
   cudaError_t e;
-  if ((e = make_rows_map(&mQ128, w.Qp, rows, D, 128)) != cudaSuccess) return e;
-  if ((e = make_rows_map(&mDO128, w.dOp, rows, D, 128)) != cudaSuccess) return e;
   if ((e = make_rows_map(&mK64, w.Kp, rows, D, 64)) != cudaSuccess) return e;
   if ((e = make_rows_map(&mV64, w.Vp, rows, D, 64)) != cudaSuccess) return e;
   if ((e = make_rows_map(&mQ64, w.Qp, rows, D, 64)) != cudaSuccess) return e;
@@ -777,7 +806,7 @@ static cudaError_t run_bwd(const prism_params &p, const prism_plan_t &plan, cons
   cudaFuncSetAttribute(bwd::dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, s2);
   {
   KernelTimer kt_(KT_ATTN_DQ, st);
-  bwd::dq_kernel<D><<<grid, bwd::kThreads, s2, st>>>(mQ128, mDO128, mK64, mV64, sel.row_ptr, sel.col, plan.blocks,
+  bwd::dq_kernel<D><<<grid, bwd::kThreads, s2, st>>>(mK64, mV64, w.Qp, w.dOp, sel.row_ptr, sel.col, plan.blocks,
                                                      w.unit_block, w.tu_q, plan.perm, w.lse2p, w.deltap, dQ,
                                                      grad_fp32, N, p.heads, scale_log2, scale, &w.hdr->status);
   }

@@ -280,12 +280,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pk[64];
         float2 ls2 = make_float2(0.f, 0.f);
         uint32_t pmax = 0u;
+        // 32-column chunks of S; chunk c+1 loads while chunk c is computed
+        const bool cv[4] = {v0, v0, nu == 2 && v1, nu == 2 && v1};  // warp-uniform
+        uint32_t rr[2][32];
+        if (cv[0]) tmem_ld32(tS + lane_off, rr[0]);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          if (c < 2 * nu && ((c < 2) ? v0 : v1)) {  // warp-uniform
-            uint32_t r[32];
-            tmem_ld32(tS + lane_off + c * 32, r);
-            tmem_wait_ld();
+          uint32_t(&r)[32] = rr[c & 1];
+          if (cv[c]) tmem_wait_ld_r(r);
+          if (c + 1 < 4 && cv[c + 1]) tmem_ld32(tS + lane_off + (c + 1) * 32, rr[(c + 1) & 1]);
+          if (cv[c]) {
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
               const float2 x = ffma2(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), scale_log2, -m);

@@ -28,6 +28,7 @@ EXPORTS = (
     "prism_attn_workspace_size", "prism_attn_fwd", "prism_attn_bwd", "prism_workspace_status",
     "prism_last_error", "prism_version", "prism_kernel_launches", "prism_plan_noalloc",
     "prism_kernel_timing", "prism_kernel_timing_read", "prism_a2v_norm", "prism_diag_exp2",
+    "prism_diag_wait_timeout",
 )
 KERNEL_TIMING_IDS = 8
 
@@ -88,6 +89,7 @@ def load() -> C.CDLL:
         "prism_kernel_timing_read": (C.c_int, [C.c_int, P(C.c_int), P(C.c_double), P(C.c_char_p)]),
         "prism_a2v_norm": (C.c_int, [vp, C.c_int64, C.c_int32, C.c_int64, vp, st]),
         "prism_diag_exp2": (C.c_int, [vp, vp, vp, C.c_int64, st]),
+        "prism_diag_wait_timeout": (C.c_int, [vp, sz, C.c_int64, st]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)

@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const int32_t *__restrict
 // therefore starts at column pk_col(ks).
 // ---------------------------------------------------------------------------
 constexpr int NS = 2;  // ring depth (steps of up to two 64-token units)
-constexpr int kPolyPairs = 4;  // of every 16 column pairs, this many take exp2_poly2
+constexpr int kPolyPairs = 0;  // of every 16 column pairs, this many take exp2_poly2 (none: measured no faster)
 
 __host__ __device__ constexpr uint32_t pk_col(int ks) { return (uint32_t)((ks >> 2) * 64 + (ks & 3) * 8); }
 
@@ -634,33 +634,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = active && (((meta >> (4 + 4 * g)) >> half) & 1);  // warp-uniform
       const float *st = stat + s * 256 + 64 * g;
       float pf[64];
-      // P^T: 32-column chunks of S^T, chunk 1 loading while chunk 0 is computed
-      {
-        uint32_t sv[2][32];
-        if (valid) tmem_ld32(tS + lane_off + 64 * g, sv[0]);
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t pk[16];
-          if (valid) {
-            tmem_wait_ld_r(sv[c]);
-            if (c == 0) tmem_ld32(tS + lane_off + 64 * g + 32, sv[1]);
-            const float *lq = st + 32 * c;
-            softmax_p32(sv[c], scale_log2,
-                        [lq](int k) {
-                          const float2 v = *reinterpret_cast<const float2 *>(lq + k);
-                          return make_float2(-v.x, -v.y);
-                        },
-                        pf + 32 * c);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[16];
+        if (valid) {
+          uint32_t sv[32];
+          float nl[32];
+          tmem_ld32(tS + lane_off + 64 * g + 32 * c, sv);
 #pragma unroll
-            for (int k = 0; k < 32; k += 2) pk[k / 2] = pack_f16(pf[32 * c + k], pf[32 * c + k + 1]);
-          } else {
-#pragma unroll
-            for (int k = 0; k < 16; ++k) pk[k] = 0u;
+          for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 lq = reinterpret_cast<const float4 *>(st + 32 * c)[k4];
+            nl[4 * k4] = -lq.x;
+            nl[4 * k4 + 1] = -lq.y;
+            nl[4 * k4 + 2] = -lq.z;
+            nl[4 * k4 + 3] = -lq.w;
           }
-          // chunk c's P^T goes to [16c, 16c+16) of this warpgroup's columns,
-          // below the chunk-1 scores still loading
-          if (active) tmem_st16(tS + lane_off + 64 * g + 16 * c, pk);
+          tmem_wait_ld();
+          softmax_p32(sv, scale_log2, [&nl](int k) { return make_float2(nl[k], nl[k + 1]); }, pf + 32 * c);
+#pragma unroll
+          for (int k = 0; k < 32; k += 2) pk[k / 2] = pack_f16(pf[32 * c + k], pf[32 * c + k + 1]);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) pk[k] = 0u;
         }
+        if (active) tmem_st16(tS + lane_off + 64 * g + 16 * c, pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -668,34 +665,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = mbar_wait_warp(&bar.dp_full, i & 1, status, 49);
       if (!ok) break;
       tc_fence_after();
-      {
-        uint32_t dv[2][32];
-        if (valid) tmem_ld32(tP + lane_off + 64 * g, dv[0]);
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t pk[16];
-          if (valid) {
-            tmem_wait_ld_r(dv[c]);
-            if (c == 0) tmem_ld32(tP + lane_off + 64 * g + 32, dv[1]);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[16];
+        if (valid) {
+          uint32_t dv[32];
+          tmem_ld32(tP + lane_off + 64 * g + 32 * c, dv);
+          tmem_wait_ld();
 #pragma unroll
-            for (int k4 = 0; k4 < 8; ++k4) {
-              const float4 dq = reinterpret_cast<const float4 *>(st + 128 + 32 * c)[k4];
+          for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 dq = reinterpret_cast<const float4 *>(st + 128 + 32 * c)[k4];
 #pragma unroll
-              for (int u = 0; u < 2; ++u) {
-                const int k = 4 * k4 + 2 * u;
-                const float2 dd = u ? make_float2(dq.z, dq.w) : make_float2(dq.x, dq.y);
-                const float2 d = fmul2(make_float2(pf[32 * c + k], pf[32 * c + k + 1]),
-                                       fsub2(make_float2(__uint_as_float(dv[c][k]), __uint_as_float(dv[c][k + 1])),
-                                             dd));
-                pk[k / 2] = pack_f16(d.x, d.y);
-              }
+            for (int u = 0; u < 2; ++u) {
+              const int k = 4 * k4 + 2 * u;
+              const float2 dd = u ? make_float2(dq.z, dq.w) : make_float2(dq.x, dq.y);
+              const float2 d = fmul2(make_float2(pf[32 * c + k], pf[32 * c + k + 1]),
+                                     fsub2(make_float2(__uint_as_float(dv[k]), __uint_as_float(dv[k + 1])), dd));
+              pk[k / 2] = pack_f16(d.x, d.y);
             }
-          } else {
-#pragma unroll
-            for (int k = 0; k < 16; ++k) pk[k] = 0u;
           }
-          if (active) tmem_st16(tP + lane_off + 64 * g + 16 * c, pk);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) pk[k] = 0u;
         }
+        if (active) tmem_st16(tP + lane_off + 64 * g + 16 * c, pk);
       }
       tmem_wait_st();
       tc_fence_before();

@@ -347,6 +347,20 @@ const char *prism_version(void);
  */
 int prism_diag_exp2(const float *x, float *y_poly, float *y_mufu, int64_t n, prism_stream_t stream);
 
+/*
+ * prism_diag_wait_timeout -- diagnostics: exercises the failure path of the
+ * kernels' bounded waits without any fault.  Clears the workspace header,
+ * then runs one warp that waits on an mbarrier nothing completes; after
+ * limit_cycles SM cycles (at most 1e9) it gives up and records
+ * PRISM_ERR_TIMEOUT in the workspace status word, as any library kernel does
+ * when one of its waits runs out.  prism_workspace_status(workspace) then
+ * returns PRISM_ERR_TIMEOUT, and the context stays usable.
+ *   workspace  device memory of at least 256 bytes, 256-byte aligned.
+ * Returns PRISM_OK (the kernel was enqueued), PRISM_ERR_INVALID_ARG or
+ * PRISM_ERR_CUDA.
+ */
+int prism_diag_wait_timeout(void *workspace, size_t ws_bytes, int64_t limit_cycles, prism_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

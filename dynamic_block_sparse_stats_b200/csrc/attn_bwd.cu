@@ -154,7 +154,8 @@ struct DqBars {
   uint64_t k_full[NSQ], v_full[NSQ], k_empty[NSQ], v_empty[NSQ];
   uint64_t qdo_ready;  // Q and dO are in TMEM (256 arrivals)
   uint64_t s_full, s_free, dp_full, ds_ready, dq_done;
-  uint64_t fin;  // single use: every MMA of the tile has completed
+  uint64_t fin;    // single use: every MMA of the tile has completed
+  uint64_t drain;  // single use: the MMA thread's in-flight products after an abort
   int meta[NSQ];  // units | mask_a << 4 | mask_b << 8 (bit = 64-row half of the tile)
   uint32_t tmem_base;
   int nsteps, nunits, abort;
@@ -195,6 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar.ds_ready, 256);
     mbar_init(&bar.dq_done, 1);
     mbar_init(&bar.fin, 1);
+    mbar_init(&bar.drain, 1);
     bar.nunits = tile_units[(size_t)h * (N / 128) + tile];
     bar.nsteps = (bar.nunits + 1) >> 1;
     fence_barrier_init();
@@ -215,6 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int blk[2] = {unit_block[(size_t)h * NB + 2 * tile], unit_block[(size_t)h * NB + 2 * tile + 1]};
     UnitWalk<2> w;
     walk_init<2>(w, blk, 2, row_ptr, h * NB);
+    int k_issued = 0, v_issued = 0;
     for (int j = 0; j < nsteps; ++j) {
       const int s = j % NSQ;
       uint32_t ua, ub = 0;
@@ -238,6 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(ks + c * (128 * 128), &mapK, &bar.k_full[s], c * 64, h * N + (int)ua * 64);
             if (nu == 2) tma_load_2d(ks + c * (128 * 128) + 64 * 128, &mapK, &bar.k_full[s], c * 64, h * N + (int)ub * 64);
           }
+          ++k_issued;
         }
         if (ok && j >= NSQ) ok = mbar_wait(&bar.v_empty[s], ((j / NSQ) - 1) & 1, status, 20);
         if (ok) {
@@ -248,11 +252,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(vs + c * (128 * 128), &mapV, &bar.v_full[s], c * 64, h * N + (int)ua * 64);
             if (nu == 2) tma_load_2d(vs + c * (128 * 128) + 64 * 128, &mapV, &bar.v_full[s], c * 64, h * N + (int)ub * 64);
           }
+          ++v_issued;
         }
         if (!ok) bar.abort = 1;
       }
       __syncwarp();
       if (*reinterpret_cast<volatile int *>(&bar.abort)) break;
+    }
+    if (lane == 0) {  // no copy may still be writing when the CTA leaves
+      drain_loads(bar.k_full, NSQ, k_issued, status, 31);
+      drain_loads(bar.v_full, NSQ, v_issued, status, 32);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -310,7 +319,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (i + 1 < nsteps && !(ok = issue_dp(i + 1))) break;
       }
       if (ok && nsteps > 0) mma_commit(&bar.fin);
-      if (!ok) bar.abort = 1;
+      if (!ok) {
+        bar.abort = 1;
+        mma_drain(&bar.drain, status, 33);
+      }
     }
     __syncwarp();
   } else if (warp >= 4) {
@@ -449,8 +461,9 @@ struct KvBars {
   uint64_t kv_full;
   uint64_t q_full[NS], q_empty[NS];
   uint64_t s_full, dp_full, p_ready, ds_ready, dv_done, dk_done;
-  uint64_t fin;  // single use: every MMA of the tile has completed
-  int meta[NS];  // units | mask_a << 4 | mask_b << 8 (bit = 64-row half of the key tile)
+  uint64_t fin;    // single use: every MMA of the tile has completed
+  uint64_t drain;  // single use: the MMA thread's in-flight products after an abort
+  int meta[NS];    // units | mask_a << 4 | mask_b << 8 (bit = 64-row half of the key tile)
   uint32_t tmem_base;
   int nsteps, nunits, abort;
 };
@@ -491,6 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar.dv_done, 1);
     mbar_init(&bar.dk_done, 1);
     mbar_init(&bar.fin, 1);
+    mbar_init(&bar.drain, 1);
     bar.nunits = tile_units[(size_t)h * (N / 128) + tile];
     bar.nsteps = (bar.nunits + 1) >> 1;
     fence_barrier_init();
@@ -511,6 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int blk[2] = {unit_block[(size_t)h * NB + 2 * tile], unit_block[(size_t)h * NB + 2 * tile + 1]};
     UnitWalk<2> w;
     walk_init<2>(w, blk, 2, col_ptr, h * NB);
+    int q_issued = 0;
     if (lane == 0) {
       mbar_arrive_expect_tx(&bar.kv_full, 2 * L::TILE);
 #pragma unroll
@@ -555,10 +570,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_load(st + 64, lse2p + (size_t)h * N + (size_t)ub * 64, 256, &bar.q_full[s]);
             bulk_load(st + 192, deltap + (size_t)h * N + (size_t)ub * 64, 256, &bar.q_full[s]);
           }
+          ++q_issued;
         }
       }
       __syncwarp();
       if (*reinterpret_cast<volatile int *>(&bar.abort)) break;
+    }
+    if (lane == 0) {  // no copy may still be writing when the CTA leaves
+      drain_loads(&bar.kv_full, 1, 1, status, 52);
+      drain_loads(bar.q_full, NS, q_issued, status, 53);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -609,7 +629,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&bar.q_empty[s]);
       }
       if (ok && nsteps > 0) mma_commit(&bar.fin);
-      if (!ok) bar.abort = 1;
+      if (!ok) {
+        bar.abort = 1;
+        mma_drain(&bar.drain, status, 54);
+      }
     }
     __syncwarp();
   } else if (warp >= 4) {

@@ -61,6 +61,7 @@ struct Bars {
   uint64_t s_full[2];   // per query tile
   uint64_t p_full[2];
   uint64_t pv_done[2];
+  uint64_t drain;  // single use: the MMA thread's in-flight products after an abort
   // per key tile j, slot j % NMETA: units | maskA << 4 | maskB << 8 (masks:
   // bit = 64-row quarter).  Written with K(j); slot j is rewritten for tile
   // j + 4 only after both softmax warpgroups have finished tile j.
@@ -106,6 +107,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar.p_full[t], 128);
       mbar_init(&bar.pv_done[t], 1);
     }
+    mbar_init(&bar.drain, 1);
     bar.nunits = tile_units[(size_t)h * (N / BQ) + quad];
     bar.ntiles = (bar.nunits + 1) >> 1;
     bar.abort = 0;
@@ -145,6 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the PV that needs V
     uint32_t pa = 0, pb = 0;  // units of tile j-1, for its V
     int pnu = 0;
+    int k_issued = 0, v_issued = 0;
     for (int j = 0; j <= ntiles; ++j) {
       uint32_t ua = 0, ub = 0;
       int ma = 0, mb = 0, nu = 1;
@@ -172,6 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (nu == 2)
                 tma_load_2d(ks + c * (128 * 128) + 64 * 128, &mapK, &bar.k_full[s], c * 64, h * N + (int)ub * 64);
             }
+            ++k_issued;
           }
         }
         if (ok && j >= 1) {
@@ -186,6 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (pnu == 2)
                 tma_load_2d(vs + c * (128 * 128) + 64 * 128, &mapV, &bar.v_full[s], c * 64, h * N + (int)pb * 64);
             }
+            ++v_issued;
           }
         }
         if (!ok) bar.abort = 1;
@@ -195,6 +200,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       pnu = nu;
       __syncwarp();
       if (*reinterpret_cast<volatile int *>(&bar.abort)) break;
+    }
+    if (lane == 0) {  // no copy may still be writing when the CTA leaves
+      drain_loads(bar.k_full, NSTAGE, k_issued, status, 11);
+      drain_loads(bar.v_full, NSTAGE, v_issued, status, 12);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -251,7 +260,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (!ok) bar.abort = 1;
+      if (!ok) {
+        bar.abort = 1;
+        mma_drain(&bar.drain, status, 13);
+      }
     }
     __syncwarp();
   } else if (warp >= 4) {

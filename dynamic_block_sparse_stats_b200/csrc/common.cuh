@@ -121,6 +121,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *s
   return true;
 }
 
+// Before a CTA leaves: wait (bounded) for the last `nstage` loads a producer
+// issued into a ring of `nstage` full barriers (load j went to barrier
+// j % nstage, completing its phase j / nstage), so that no copy still writes
+// into shared memory the CTA gives back.  After a normal run they are long
+// complete.
+__device__ __forceinline__ void drain_loads(uint64_t *full, int nstage, int issued, int *status, int where) {
+  for (int j = issued > nstage ? issued - nstage : 0; j < issued; ++j)
+    mbar_wait(&full[j % nstage], (uint32_t)((j / nstage) & 1), status, where);
+}
+
 // Bounded wait whose outcome is the same for every lane of the warp, so that
 // the .sync.aligned tcgen05 instructions that follow stay convergent.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, int *status, int where) {
@@ -192,6 +202,13 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                : "memory");
+}
+// After an abort: wait (bounded) for this thread's MMAs still in flight, so
+// that the CTA does not free TMEM under them.  `bar` is a fresh barrier
+// (count 1) used for nothing else.
+__device__ __forceinline__ void mma_drain(uint64_t *bar, int *status, int where) {
+  mma_commit(bar);
+  mbar_wait(bar, 0, status, where);
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }

@@ -64,10 +64,17 @@ static int check_params(const prism_params *p) {
   return PRISM_OK;
 }
 
+// The kernels move tensor rows in 16-byte vectors (and the plan table in
+// int4 rows), so every such pointer must be 16-byte aligned.
+static int check_aligned16(const void *ptr, const char *name) {
+  if (reinterpret_cast<uintptr_t>(ptr) % 16) return fail(PRISM_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return PRISM_OK;
+}
+
 static int check_plan(const prism_plan_t *pl) {
   if (!pl || !pl->zone_shape || !pl->n_blocks || !pl->blocks || !pl->perm)
     return fail(PRISM_ERR_INVALID_ARG, "plan arrays (zone_shape, n_blocks, blocks, perm) must be non-NULL");
-  return PRISM_OK;
+  return check_aligned16(pl->blocks, "plan blocks");
 }
 
 static int check_ws(void *ws, size_t bytes, size_t need) {
@@ -82,6 +89,7 @@ int check_plan_call(const prism_params *p, const uint16_t *V, const float *a2v_n
   int rc;
   if ((rc = check_params(p)) != PRISM_OK) return rc;
   if (!V) return fail(PRISM_ERR_INVALID_ARG, "V is NULL");
+  if ((rc = check_aligned16(V, "V")) != PRISM_OK) return rc;
   if (p->density == 3 && !a2v_norm) return fail(PRISM_ERR_INVALID_ARG, "density 3 (A2V strength) needs a2v_norm");
   return check_plan(out);
 }
@@ -130,6 +138,7 @@ int prism_select(const prism_params *p, const prism_plan_t *plan, const uint16_t
   int rc;
   if ((rc = check_params(p)) != PRISM_OK) return rc;
   if (!Q || !K) return fail(PRISM_ERR_INVALID_ARG, "Q or K is NULL");
+  if ((rc = check_aligned16(Q, "Q")) != PRISM_OK || (rc = check_aligned16(K, "K")) != PRISM_OK) return rc;
   if ((rc = check_plan(plan)) != PRISM_OK) return rc;
   if (!out || !out->row_ptr || !out->col || out->cap < 0)
     return fail(PRISM_ERR_INVALID_ARG, "select output (row_ptr, col, cap) invalid");
@@ -163,6 +172,12 @@ int prism_attn_fwd(const prism_params *p, const prism_plan_t *plan, const prism_
   int rc;
   if ((rc = check_params(p)) != PRISM_OK) return rc;
   if (!Q || !K || !V || !O || !lse) return fail(PRISM_ERR_INVALID_ARG, "Q, K, V, O or lse is NULL");
+  {
+    const void *ptrs[5] = {Q, K, V, O, O_res};
+    const char *names[5] = {"Q", "K", "V", "O", "O_res"};
+    for (int k = 0; k < 5; ++k)
+      if ((rc = check_aligned16(ptrs[k], names[k])) != PRISM_OK) return rc;
+  }
   if ((rc = check_plan(plan)) != PRISM_OK) return rc;
   if (!sel || !sel->row_ptr || !sel->col) return fail(PRISM_ERR_INVALID_ARG, "selection is NULL");
   if ((rc = check_ws(workspace, ws_bytes, attn_fwd_ws_bytes(*p))) != PRISM_OK) return rc;
@@ -182,6 +197,12 @@ int prism_attn_bwd(const prism_params *p, const prism_plan_t *plan, const prism_
   if ((rc = check_params(p)) != PRISM_OK) return rc;
   if (!Q || !K || !V || !O || !dO || !lse || !dQ || !dK || !dV)
     return fail(PRISM_ERR_INVALID_ARG, "a tensor argument is NULL");
+  {
+    const void *ptrs[9] = {Q, K, V, O, O_res, dO, dQ, dK, dV};
+    const char *names[9] = {"Q", "K", "V", "O", "O_res", "dO", "dQ", "dK", "dV"};
+    for (int k = 0; k < 9; ++k)
+      if ((rc = check_aligned16(ptrs[k], names[k])) != PRISM_OK) return rc;
+  }
   if ((rc = check_plan(plan)) != PRISM_OK) return rc;
   if (!sel || !sel->row_ptr || !sel->col || !sel->col_ptr || !sel->row)
     return fail(PRISM_ERR_INVALID_ARG, "selection with its transpose (col_ptr, row) is required");

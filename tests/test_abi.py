@@ -61,29 +61,29 @@ def test_invalid_params_are_rejected_before_any_cuda_call(bad, code):
 def test_a2v_density_without_norms_is_rejected():
     lib = _lib.load()
     p = api.params(8, 16, 16, 1, 64, topk_abs=2, density=api.DENSITY_A2V)
-    plan = _lib.PrismPlan(8, 8, 8, 8, 8, 8, 8)
-    rc = lib.prism_plan(C.byref(p), C.c_void_p(8), None, C.byref(plan), C.c_void_p(256), 1 << 20, None)
+    plan = _lib.PrismPlan(256, 256, 256, 256, 256, 256, 256)
+    rc = lib.prism_plan(C.byref(p), C.c_void_p(256), None, C.byref(plan), C.c_void_p(256), 1 << 20, None)
     assert rc == _lib.PRISM_ERR_INVALID_ARG and "a2v_norm" in lib.prism_last_error().decode()
-    assert lib.prism_plan_noalloc(C.byref(p), C.c_void_p(8), None, C.byref(plan), None) == _lib.PRISM_ERR_INVALID_ARG
+    assert lib.prism_plan_noalloc(C.byref(p), C.c_void_p(256), None, C.byref(plan), None) == _lib.PRISM_ERR_INVALID_ARG
 
 
 def test_null_pointers_and_short_workspace_are_rejected():
     lib = _lib.load()
     p = api.params(8, 16, 16, 1, 64, topk_abs=2)
-    plan = _lib.PrismPlan(8, 8, 8, 8, 8, 8, 8)
+    plan = _lib.PrismPlan(256, 256, 256, 256, 256, 256, 256)
     assert lib.prism_plan(C.byref(p), None, None, C.byref(plan), C.c_void_p(256), 1 << 20, None) == \
         _lib.PRISM_ERR_INVALID_ARG
     need = lib.prism_plan_workspace_size(C.byref(p))
     assert need > 256
-    rc = lib.prism_plan(C.byref(p), C.c_void_p(8), None, C.byref(plan), C.c_void_p(256), need - 1, None)
+    rc = lib.prism_plan(C.byref(p), C.c_void_p(256), None, C.byref(plan), C.c_void_p(256), need - 1, None)
     assert rc == _lib.PRISM_ERR_CAPACITY and "need" in lib.prism_last_error().decode()
-    rc = lib.prism_plan(C.byref(p), C.c_void_p(8), None, C.byref(plan), C.c_void_p(264), need, None)
+    rc = lib.prism_plan(C.byref(p), C.c_void_p(256), None, C.byref(plan), C.c_void_p(264), need, None)
     assert rc == _lib.PRISM_ERR_INVALID_ARG  # misaligned workspace
-    sel = _lib.PrismSelect(8, 8, 10, 0, 8, None)  # col_ptr without row
-    assert lib.prism_select(C.byref(p), C.byref(plan), C.c_void_p(8), C.c_void_p(8), C.byref(sel),
+    sel = _lib.PrismSelect(256, 256, 10, 0, 256, None)  # col_ptr without row
+    assert lib.prism_select(C.byref(p), C.byref(plan), C.c_void_p(256), C.c_void_p(256), C.byref(sel),
                             C.c_void_p(256), 1 << 30, None) == _lib.PRISM_ERR_INVALID_ARG
-    assert lib.prism_attn_bwd(C.byref(p), C.byref(plan), C.byref(_lib.PrismSelect(8, 8, 10, 0, None, None)),
-                              *([C.c_void_p(8)] * 10), 0, C.c_void_p(256), 1 << 30, None) == _lib.PRISM_ERR_INVALID_ARG
+    assert lib.prism_attn_bwd(C.byref(p), C.byref(plan), C.byref(_lib.PrismSelect(256, 256, 10, 0, None, None)),
+                              *([C.c_void_p(256)] * 10), 0, C.c_void_p(256), 1 << 30, None) == _lib.PRISM_ERR_INVALID_ARG
 
 
 def test_workspace_sizes_grow_with_the_grid():
@@ -106,3 +106,28 @@ def test_a2v_norm_argument_checks_need_no_gpu():
     assert lib.prism_a2v_norm(C.c_void_p(264), 4, 64, 64, ok, None) == _lib.PRISM_ERR_INVALID_ARG  # alignment
     assert lib.prism_a2v_norm(None, 4, 64, 64, ok, None) == _lib.PRISM_ERR_INVALID_ARG
     assert "prism_a2v_norm" in lib.prism_last_error().decode()
+
+
+def test_misaligned_tensor_pointers_are_rejected_before_any_cuda_call():
+    """The kernels move rows in 16-byte vectors: a pointer off that grid is an
+    argument error, reported before anything is launched."""
+    lib = _lib.load()
+    p = api.params(8, 16, 16, 1, 64, topk_abs=2)
+    plan = _lib.PrismPlan(256, 256, 256, 256, 256, 256, 256)
+    ws = C.c_void_p(256)
+    rc = lib.prism_plan(C.byref(p), C.c_void_p(8), None, C.byref(plan), ws, 1 << 20, None)
+    assert rc == _lib.PRISM_ERR_INVALID_ARG and "V" in lib.prism_last_error().decode()
+    bad_plan = _lib.PrismPlan(256, 256, 256, 256, 264, 256, 256)     # blocks off by 8 bytes
+    rc = lib.prism_plan(C.byref(p), C.c_void_p(256), None, C.byref(bad_plan), ws, 1 << 20, None)
+    assert rc == _lib.PRISM_ERR_INVALID_ARG and "blocks" in lib.prism_last_error().decode()
+    sel = _lib.PrismSelect(256, 256, 10, 0, 256, 256)
+    rc = lib.prism_select(C.byref(p), C.byref(plan), C.c_void_p(256), C.c_void_p(258), C.byref(sel), ws, 1 << 30,
+                          None)
+    assert rc == _lib.PRISM_ERR_INVALID_ARG and "K" in lib.prism_last_error().decode()
+    a = [C.c_void_p(256)] * 5
+    rc = lib.prism_attn_fwd(C.byref(p), C.byref(plan), C.byref(sel), a[0], a[1], C.c_void_p(264), a[3], a[4],
+                            C.c_void_p(256), ws, 1 << 40, None)
+    assert rc == _lib.PRISM_ERR_INVALID_ARG and "V" in lib.prism_last_error().decode()
+    rc = lib.prism_attn_bwd(C.byref(p), C.byref(plan), C.byref(sel), *[C.c_void_p(256)] * 5, C.c_void_p(256),
+                            C.c_void_p(256), C.c_void_p(256), C.c_void_p(260), C.c_void_p(256), 1, ws, 1 << 40, None)
+    assert rc == _lib.PRISM_ERR_INVALID_ARG and "dK" in lib.prism_last_error().decode()

@@ -22,7 +22,9 @@
  *   Sizes.  Z = (T/8)(H/8)(W/8) zones; NB = N/64 is the most blocks a head
  *     can have (every zone at B = 64).
  *   Memory.  Every pointer argument is DEVICE memory unless stated
- *     otherwise.  The caller allocates and owns every buffer, including the
+ *     otherwise.  Tensor pointers (Q, K, V, O, O_res, dO, dQ, dK, dV, the
+ *     bridge output of prism_a2v_norm) and the plan's block table must be
+ *     16-byte aligned; a misaligned one is PRISM_ERR_INVALID_ARG.  The caller allocates and owns every buffer, including the
  *     workspaces sized by the *_workspace_size() queries; the library never
  *     allocates device memory.  Workspaces must be 256-byte aligned and may
  *     not be shared by calls that run concurrently.

@@ -12,8 +12,10 @@ head_dim 128, bf16, Top-k 4%, Top-p 0.9) unless --workload says otherwise.
 Prints one JSON line (rank 0).  `value` is the effective TFLOP/s of the whole
 step over all ranks, counting only the computed blocks: (4 + 10) * P * D per
 layer, P = number of computed (query, key) token pairs.  Multi-GPU runs are
-weak scaling: every rank runs its own independent layer (seeded by rank);
-ranks exchange nothing but the timing barrier.
+weak scaling by default: every rank runs its own independent layer (seeded by
+rank).  With --shard heads the ranks split one layer's heads instead (strong
+scaling).  Either way the ranks exchange nothing on the path, only the timing
+barrier and the max/sum of their measurements.
 """
 from __future__ import annotations
 
@@ -112,6 +114,24 @@ def max_over_ranks(x: float, world: int, device=None) -> float:
 def whole_job_rate(units_per_rank: float, world: int, ms_max: float) -> float:
     """Units processed by all ranks per second, timed by the slowest rank."""
     return world * units_per_rank / (ms_max * 1e-3)
+
+
+def head_range(rank: int, world: int, heads: int) -> tuple[int, int]:
+    """Contiguous, balanced share of a layer's heads for one rank (the path
+    has no cross-head exchange: plan, selection and attention are per head,
+    and the A2V map is per token, so each rank recomputes it)."""
+    base, extra = divmod(heads, world)
+    h0 = rank * base + min(rank, extra)
+    return h0, h0 + base + (1 if rank < extra else 0)
+
+
+def sum_over_ranks(x: float, world: int, device=None) -> float:
+    """Sum of a per-rank count over all ranks (measurement only)."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
 
 
 # ----------------------------------------------------------------------------- flops
@@ -306,12 +326,25 @@ def dense_sdpa(inp, w, backward, heads=1, iters=2):
 
 def run_prism(args, w, rank, world, device):
     lib = _lib.load()
-    p = api.params_for(w)
-    inp = make_inputs(w, device, seed=rank_seed(rank))
+    heads_mode = args.shard == "heads" and world > 1
+    if heads_mode and world > w.heads:
+        raise SystemExit(f"--shard heads needs at most {w.heads} ranks")
+    # layers: every rank its own layer (weak); heads: one layer, heads split over ranks (strong)
+    inp = make_inputs(w, device, seed=0 if heads_mode else rank_seed(rank))
     N, h, D = w.N, w.heads, w.head_dim
+    h0, h1 = head_range(rank, world, h) if heads_mode else (0, h)
+    if heads_mode:
+        for k in ("Q", "K", "V", "dO"):
+            if k in inp:
+                inp[k] = inp[k][:, h0:h1].contiguous()
+        import dataclasses
+        w = dataclasses.replace(w, heads=h1 - h0)
+        h = h1 - h0
+    p = api.params_for(w)
     Q, K, V = inp["Q"], inp["K"], inp["V"]
     # the previous layer's bridge output, whose row norms are this layer's A2V map
-    hhat = make_bridge_output(inp["a"], h * D, seed=rank_seed(rank))
+    hhat = make_bridge_output(inp["a"], (w.heads if not heads_mode else WORKLOADS[args.workload].heads) * D,
+                              seed=0 if heads_mode else rank_seed(rank))
     inp["hhat"] = hhat
     dO = inp.get("dO")
     backward = dO is not None
@@ -353,6 +386,8 @@ def run_prism(args, w, rank, world, device):
     torch.cuda.synchronize()
     P = computed_pairs(p, pl, sel)
     flops_fwd, flops_bwd = 4.0 * P * D, (10.0 * P * D if backward else 0.0)
+    # whole-job work: the sum of every rank's computed pairs (own layer, or own heads)
+    total_flops = sum_over_ranks(flops_fwd + flops_bwd, world, device)
     flops = flops_fwd + flops_bwd
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(args.steps)]
@@ -411,7 +446,7 @@ def run_prism(args, w, rank, world, device):
         e1.record(stream)
         torch.cuda.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1) / ksteps, world, device)
-        e2e = {"value": whole_job_rate(flops, world, ems) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": total_flops / (ems * 1e-3) / 1e12, "unit": "TFLOP/s",
                "ms_per_step": ems, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": ksteps}
         del hin, hout
@@ -443,20 +478,23 @@ def run_prism(args, w, rank, world, device):
                "sample": desc, "host_cpus": os.cpu_count(), "sample_wall_s": wall}
 
     dense = None
-    if not args.no_dense:
+    if not args.no_dense and world == 1:
         dense = dense_sdpa(inp, w, backward)
         if "ms_per_layer" in dense:
             dense["speedup_of_prism_step"] = dense["ms_per_layer"] / ms
 
     density = P / (float(N) * N * h)
     line = {
-        "metric": METRIC, "value": whole_job_rate(flops, world, ms_max) / 1e12, "unit": "TFLOP/s",
+        "metric": METRIC, "value": total_flops / (ms_max * 1e-3) / 1e12, "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "strong" if heads_mode else "weak", "vs_baseline": None,
+        "dtype": "bf16",
         "data": "synthetic (seeded generator; stands in for the pages' 2K-Bench latents)",
-        "config": {"workload": w.name, "T": w.T, "H": w.H, "W": w.W, "tokens": N, "heads": h, "head_dim": D,
+        "config": {"workload": w.name, "T": w.T, "H": w.H, "W": w.W, "tokens": N,
+                   "heads": WORKLOADS[args.workload].heads, "heads_per_rank": h, "head_dim": D,
                    "topk_frac": w.topk_frac, "top_p": w.top_p, "backward": backward,
-                   "parallelism": f"weak x{world} (independent layers, no collectives)",
+                   "parallelism": (f"heads split over {world} ranks (this rank {h0}-{h1 - 1}), no collectives on the path"
+                                   if heads_mode else f"weak x{world} (independent layers, no collectives)"),
                    "l2": "inputs larger than L2 (each bf16 tensor %.2f GB)" % (N * h * D * 2 / 1e9),
                    "pairs": P, "pair_density": density, "nnz_blocks": sel.nnz},
         "stage_ms": stage_ms, "stage_roofline": stage_roofline, "kernels": kernels,
@@ -506,6 +544,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense SDPA comparison")
+    ap.add_argument("--shard", choices=["layers", "heads"], default="layers",
+                    help="N>1: every rank its own layer (weak scaling, default) or one layer's heads split "
+                         "over the ranks (strong scaling); neither exchanges data on the path")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

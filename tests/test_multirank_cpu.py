@@ -52,3 +52,57 @@ def test_single_rank_is_identity():
     import bench
     assert bench.max_over_ranks(3.0, 1) == 3.0
     assert bench.whole_job_rate(10.0, 1, 1000.0) == 10.0
+
+
+def _heads_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import bench
+        h0, h1 = bench.head_range(rank, world, 24)
+        pairs = 1000.0 * (h1 - h0)                  # this rank's computed pairs
+        total = bench.sum_over_ranks(pairs, world)
+        q.put((rank, h0, h1, total))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_head_sharding_splits_a_layer_and_sums_its_work():
+    """--shard heads: the ranks' head ranges tile the layer's heads exactly,
+    and the whole-job work is the sum of the ranks' own work."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_heads_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [(o[1], o[2]) for o in out] == [(0, 12), (12, 24)]
+    assert all(o[3] == 24000.0 for o in out)
+
+
+def test_heads_are_independent_in_the_oracle():
+    """The reason head sharding needs no exchange: planning and selection of a
+    subset of heads equal the same heads of the full layer (the A2V map is per
+    token and shared)."""
+    import numpy as np
+    from oracle import prism_oracle as O
+    rng = np.random.default_rng(0)
+    T, H, W = 8, 16, 16
+    N = T * H * W
+    V = rng.normal(size=(N, 4, 8)) * rng.uniform(0.3, 3, size=(N, 4, 1))
+    Q, K = rng.normal(size=(N, 4, 8)), rng.normal(size=(N, 4, 8))
+    a = np.abs(rng.normal(size=N))
+    full = O.plan(V, a, T, H, W)
+    part = O.plan(V[:, 2:4], a, T, H, W)
+    for k in range(2):
+        assert np.array_equal(full.heads[2 + k].perm, part.heads[k].perm)
+        assert np.array_equal(full.heads[2 + k].g, part.heads[k].g)
+    s_full = O.select(Q, K, full, 0.1, 0, 0.9, heads=[2, 3])
+    s_part = O.select(Q[:, 2:4], K[:, 2:4], part, 0.1, 0, 0.9)
+    for a_, b_ in zip(s_full, s_part):
+        assert all(np.array_equal(x[1], y[1]) for x, y in zip(a_, b_))

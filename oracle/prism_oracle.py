@@ -23,8 +23,8 @@ Sources, cited by page title and section:
             (B(m), tau_128, tau_256, closed form l*_d, nearest candidate in
             log2 space), section 3 (S_i = Top-k(P_i,k) U Top-p(P_i,p)).
 
-Readings of points the pages leave open are marked READING and collected in
-the design doc's list of readings.
+Readings of points the pages leave open are marked READING where they are
+applied; each states the choice and why.
 
 Parity status: every function below is pinned by a ``-m "not gpu"`` test
 (closed forms, invariants, brute force, independent dense formulations).

@@ -589,44 +589,57 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dVd = sdesc_sw128(smem_u32(smem + L::OFF_V), 16, 1024);
       bool ok = mbar_wait(&bar.kv_full, 0, status, 42);
       tc_fence_after();
-      for (int i = 0; ok && i < nsteps; ++i) {
-        const int s = i % NS;
-        ok = mbar_wait(&bar.q_full[s], (i / NS) & 1, status, 44);
-        // S^T and dP^T reuse the columns the previous step's dV and dK read P^T and dS^T from
-        if (ok && i >= 1) ok = mbar_wait(&bar.dv_done, (i - 1) & 1, status, 45);
-        if (!ok) break;
-        tc_fence_after();
-        const int nu = bar.meta[s] & 15;  // written before the stage's Q arrived
-        const uint32_t id = nu == 2 ? id_full : id_half;
-        const uint64_t dQs = sdesc_sw128(smem_u32(smem + L::OFF_Q + s * L::TILE), 16, 1024);
-        const uint64_t dDOs = sdesc_sw128(smem_u32(smem + L::OFF_DO + s * L::TILE), 16, 1024);
+      // Step i's products, in the order dV(i-1), S^T(i), dK(i-1), dP^T(i):
+      // S^T(i) is issued as soon as dV(i-1) has read P^T(i-1), so the
+      // softmax of step i can follow the compute warps' dS of step i-1
+      // without waiting for dK(i-1).
+      for (int i = 0; ok && i <= nsteps; ++i) {
+        const int s = i % NS, sp = (i + NS - 1) % NS;
+        const int nup = i >= 1 ? (bar.meta[sp] & 15) : 0;  // stage sp is not refilled before dK(i-1)
+        if (i >= 1) {  // dV += P^T(i-1) dO(i-1)
+          ok = mbar_wait(&bar.p_ready, (i - 1) & 1, status, 43);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t dDOmn = sdesc_sw128(smem_u32(smem + L::OFF_DO + sp * L::TILE), 128 * 128, 1024);
+          for (int ks = 0; ks < 4 * nup; ++ks)
+            mma_ts(tV, tS + pk_col(ks), dDOmn + (uint64_t)ks * 128, id_acc, (i > 1 || ks > 0) ? 1u : 0u);
+          mma_commit(&bar.dv_done);
+        }
+        uint32_t id = id_full;
+        uint64_t dDOs = 0;
+        if (i < nsteps) {  // S^T(i) = K Q(i)^T, into the columns dV(i-1) read P^T(i-1) from
+          ok = mbar_wait(&bar.q_full[s], (i / NS) & 1, status, 44);
+          if (ok && i >= 1) ok = mbar_wait(&bar.dv_done, (i - 1) & 1, status, 45);
+          if (!ok) break;
+          tc_fence_after();
+          const int nu = bar.meta[s] & 15;  // written before the stage's Q arrived
+          id = nu == 2 ? id_full : id_half;
+          const uint64_t dQs = sdesc_sw128(smem_u32(smem + L::OFF_Q + s * L::TILE), 16, 1024);
+          dDOs = sdesc_sw128(smem_u32(smem + L::OFF_DO + s * L::TILE), 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tS, dKd + kslice16(kk, 128 * 128), dQs + kslice16(kk, 128 * 128), id, kk > 0 ? 1u : 0u);
-        mma_commit(&bar.s_full);
-        if (i >= 1) ok = mbar_wait(&bar.dk_done, (i - 1) & 1, status, 46);
-        if (!ok) break;
-        tc_fence_after();
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tS, dKd + kslice16(kk, 128 * 128), dQs + kslice16(kk, 128 * 128), id, kk > 0 ? 1u : 0u);
+          mma_commit(&bar.s_full);
+        }
+        if (i >= 1) {  // dK += dS^T(i-1) Q(i-1)
+          ok = mbar_wait(&bar.ds_ready, (i - 1) & 1, status, 47);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t dQmn = sdesc_sw128(smem_u32(smem + L::OFF_Q + sp * L::TILE), 128 * 128, 1024);
+          for (int ks = 0; ks < 4 * nup; ++ks)
+            mma_ts(tK, tP + pk_col(ks), dQmn + (uint64_t)ks * 128, id_acc, (i > 1 || ks > 0) ? 1u : 0u);
+          mma_commit(&bar.dk_done);
+          mma_commit(&bar.q_empty[sp]);
+        }
+        if (i < nsteps) {  // dP^T(i) = V dO(i)^T, into the columns dK(i-1) read dS^T(i-1) from
+          if (i >= 1) ok = mbar_wait(&bar.dk_done, (i - 1) & 1, status, 46);
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tP, dVd + kslice16(kk, 128 * 128), dDOs + kslice16(kk, 128 * 128), id, kk > 0 ? 1u : 0u);
-        mma_commit(&bar.dp_full);
-        // dV += P^T dO, dK += dS^T Q
-        const uint64_t dQmn = sdesc_sw128(smem_u32(smem + L::OFF_Q + s * L::TILE), 128 * 128, 1024);
-        const uint64_t dDOmn = sdesc_sw128(smem_u32(smem + L::OFF_DO + s * L::TILE), 128 * 128, 1024);
-        ok = mbar_wait(&bar.p_ready, i & 1, status, 43);
-        if (!ok) break;
-        tc_fence_after();
-        for (int ks = 0; ks < 4 * nu; ++ks)
-          mma_ts(tV, tS + pk_col(ks), dDOmn + (uint64_t)ks * 128, id_acc, (i > 0 || ks > 0) ? 1u : 0u);
-        mma_commit(&bar.dv_done);
-        ok = mbar_wait(&bar.ds_ready, i & 1, status, 47);
-        if (!ok) break;
-        tc_fence_after();
-        for (int ks = 0; ks < 4 * nu; ++ks)
-          mma_ts(tK, tP + pk_col(ks), dQmn + (uint64_t)ks * 128, id_acc, (i > 0 || ks > 0) ? 1u : 0u);
-        mma_commit(&bar.dk_done);
-        mma_commit(&bar.q_empty[s]);
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tP, dVd + kslice16(kk, 128 * 128), dDOs + kslice16(kk, 128 * 128), id, kk > 0 ? 1u : 0u);
+          mma_commit(&bar.dp_full);
+        }
       }
       if (ok && nsteps > 0) mma_commit(&bar.fin);
       if (!ok) {

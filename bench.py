@@ -227,14 +227,21 @@ def stored_traffic(kernel):
 
 
 # ----------------------------------------------------------------------------- oracle sample
-def oracle_sample(w, inp, head=0, n_rows=2, seed=0):
-    """Time the CPU oracle on a bounded sample of the same layer: the plan and
-    the selection of one head over the full grid, and forward+backward
-    attention of `n_rows` random query blocks of that head.  The layer time
-    is extrapolated from the oracle's own numbers only: plan and selection
-    times x heads, attention time x (computed pairs of the head's full
-    selection x heads) / (pairs of the sampled blocks).  Returns (layer time,
-    layer computed pairs, description, threads, wall seconds)."""
+def oracle_sample(w, inp, head=0, n_rows=2, n_sel=512, seed=0):
+    """Time the CPU oracle on a bounded sample of the same layer: the A2V norms
+    of a row sample of a bridge output, the plan of one head over the full
+    grid, the selection of `n_sel` seeded query blocks of that head, and
+    forward+backward attention of `n_rows` of those blocks.  The layer time is
+    extrapolated from the oracle's own numbers only:
+      * norms x (N / rows normed);
+      * plan x heads;
+      * selection: its fixed part (the block means of the head, timed alone)
+        plus its per-row part x (blocks of the head / rows selected), x heads;
+      * attention x (computed pairs of the layer) / (pairs of the sampled
+        blocks), where the layer's pairs are the sampled rows' pairs x
+        (blocks / rows selected) x heads.
+    Returns (layer time, layer computed pairs, description, threads, wall
+    seconds)."""
     from threadpoolctl import threadpool_info
 
     from oracle import prism_oracle as O
@@ -244,7 +251,6 @@ def oracle_sample(w, inp, head=0, n_rows=2, seed=0):
     Kh = inp["K"][:, head:head + 1].float().cpu().numpy()
     a = inp["a"].cpu().numpy()
     dOh = inp["dO"][:, head:head + 1].float().cpu().numpy() if "dO" in inp else None
-    # the A2V norms of a row sample of a bridge output, scaled to all N rows
     n_norm = min(w.N, 16384)
     hs = make_bridge_output(inp["a"][:n_norm], w.heads * w.head_dim, seed=seed).float().cpu().numpy()
     tn = time.perf_counter()
@@ -254,32 +260,37 @@ def oracle_sample(w, inp, head=0, n_rows=2, seed=0):
     t0 = time.perf_counter()
     opl = O.plan(Vh, a, T, H, W)
     t1 = time.perf_counter()
-    osel = O.select(Qh, Kh, opl, w.topk_frac, w.topk_abs, w.top_p)
-    t2 = time.perf_counter()
     hp = opl.heads[0]
     nb = hp.blocks.shape[0]
     rng = np.random.default_rng(seed)
-    rows = sorted(rng.choice(nb, size=min(n_rows, nb), replace=False).tolist())
-    sub = [[osel[0][i] for i in rows]]
-    scale = float(np.float32(1.0 / math.sqrt(w.head_dim)))
+    sel_rows = sorted(rng.choice(nb, size=min(n_sel, nb), replace=False).tolist())
+    O.select(Qh, Kh, opl, w.topk_frac, w.topk_abs, w.top_p, rows=[])      # the fixed part: block means
+    t2 = time.perf_counter()
+    osel = O.select(Qh, Kh, opl, w.topk_frac, w.topk_abs, w.top_p, rows=sel_rows)
     t3 = time.perf_counter()
+    row_frac = nb / len(sel_rows)
+    sel_time = (t2 - t1) + max(0.0, (t3 - t2) - (t2 - t1)) * row_frac
+    picks = sorted(rng.choice(len(sel_rows), size=min(n_rows, len(sel_rows)), replace=False).tolist())
+    sub = [[osel[0][r] for r in picks]]
+    scale = float(np.float32(1.0 / math.sqrt(w.head_dim)))
+    t4 = time.perf_counter()
     O.attention_fwd(Qh, Kh, Vh, opl, sub, scale)
     if dOh is not None:
         O.attention_bwd(Qh, Kh, Vh, dOh, opl, sub, scale)
-    t4 = time.perf_counter()
-    pairs_sample = sum(int(hp.blocks[i, 4]) * int(sum(hp.blocks[j, 4] for j in ids)) for (i, ids, _) in sub[0])
-    pairs_head = sum(int(hp.blocks[i, 4]) * int(hp.blocks[ids, 4].sum()) for (i, ids, _) in osel[0])
-    P_total = pairs_head * w.heads
-    attn_time = (t4 - t3) * (P_total / max(pairs_sample, 1))
-    layer_time = norm_time + w.heads * ((t1 - t0) + (t2 - t1)) + attn_time
+    t5 = time.perf_counter()
+    pairs_sample = sum(int(hp.blocks[i, 4]) * int(hp.blocks[ids, 4].sum()) for (i, ids, _) in sub[0])
+    pairs_rows = sum(int(hp.blocks[i, 4]) * int(hp.blocks[ids, 4].sum()) for (i, ids, _) in osel[0])
+    P_total = pairs_rows * row_frac * w.heads
+    attn_time = (t5 - t4) * (P_total / max(pairs_sample, 1))
+    layer_time = norm_time + w.heads * ((t1 - t0) + sel_time) + attn_time
     threads = max([t.get("num_threads", 1) for t in threadpool_info()] + [1])
-    desc = (f"oracle A2V norms of {n_norm} bridge-output rows (x{w.N / n_norm:.1f}, {norm_time:.2f}s), "
-            f"plan+select of head {head} over the full {T}x{H}x{W} grid "
-            f"({(t1 - t0):.2f}s + {(t2 - t1):.2f}s, x{w.heads} heads) and fwd"
-            f"{'+bwd' if dOh is not None else ''} of {len(rows)} query blocks ({t4 - t3:.2f}s, "
-            f"x{P_total / max(pairs_sample, 1):.0f} by computed pairs, the head's pairs x{w.heads} heads); "
-            f"extrapolated layer time {layer_time:.1f}s")
-    return layer_time, P_total, desc, threads, (t4 - t0)
+    desc = (f"oracle A2V norms of {n_norm} bridge-output rows (x{w.N / n_norm:.1f}, {norm_time:.2f}s); "
+            f"plan of head {head} over the full {T}x{H}x{W} grid ({t1 - t0:.2f}s, x{w.heads} heads); "
+            f"selection of {len(sel_rows)} of its {nb} query blocks ({t3 - t2:.2f}s, of which block means "
+            f"{t2 - t1:.2f}s; rows x{row_frac:.1f}, x{w.heads} heads); fwd{'+bwd' if dOh is not None else ''} "
+            f"of {len(picks)} of those blocks ({t5 - t4:.2f}s, x{P_total / max(pairs_sample, 1):.0f} by computed "
+            f"pairs, estimated from the selected rows); extrapolated layer time {layer_time:.1f}s")
+    return layer_time, P_total, desc, threads, (t5 - t0)
 
 
 # ----------------------------------------------------------------------------- main arms
@@ -506,8 +517,8 @@ def run_prism(args, w, rank, world, device):
 
 def run_reference(args, w, rank, world):
     """The CPU oracle as the reference arm: each step is a bounded sample of the
-    same layer (plan + selection of one head, fwd+bwd of two query blocks),
-    extrapolated to the layer by computed pairs."""
+    same layer (the plan of one head, the selection of a seeded sample of its
+    query blocks, fwd+bwd of two of them), extrapolated to the layer."""
     if rank != 0:
         return None
     # inputs are drawn by the seeded generator (on the GPU when there is one,

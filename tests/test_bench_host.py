@@ -1,0 +1,142 @@
+"""Host arithmetic of the benchmark (no GPU).
+
+* The computed-pair count P behind every FLOP figure: bench.computed_pairs
+  reads the library's block table and CSR; here it gets the oracle's plan and
+  selection in that layout and must equal a brute-force count of the
+  (query token, key token) pairs of the dense attention mask.
+* The per-kernel roofline arithmetic (work per launch, achieved rate,
+  fraction of the peak) on hand-computed numbers.
+* The parsing of the nvidia-smi samples taken during the timed region, and
+  the rule that a stored DRAM traffic figure is dropped once its kernel's
+  source has changed."""
+import hashlib
+import json
+import types
+
+import numpy as np
+import pytest
+import torch
+
+import bench
+from dynamic_block_sparse_stats_b200.synth import WORKLOADS, make_inputs
+from oracle import prism_oracle as O
+
+
+def _library_layout(w, opl, osel):
+    """The oracle's plan and selection in the library's layout: blocks
+    [h][N/64][4] = {p0, B, n0, shape} (rows past n_blocks hold garbage), and a
+    CSR over rows h*(N/64) + i."""
+    NB = w.N // 64
+    heads = len(opl.heads)
+    blocks = torch.full((heads, NB, 4), -7, dtype=torch.int32)
+    n_blocks = torch.zeros(heads, dtype=torch.int32)
+    counts, cols = np.zeros(heads * NB, np.int64), []
+    for h, hp in enumerate(opl.heads):
+        n_blocks[h] = hp.blocks.shape[0]
+        for b, (t0, y0, x0, sid, B, p0) in enumerate(hp.blocks):
+            blocks[h, b] = torch.tensor([int(p0), int(B), int((t0 * w.H + y0) * w.W + x0), int(sid)])
+        rows = {int(i): np.asarray(ids) for (i, ids, _) in osel[h]}
+        for i in range(NB):
+            ids = rows.get(i, np.zeros(0, np.int64))
+            counts[h * NB + i] = ids.size
+            cols.append(ids)
+    row_ptr = np.concatenate([[0], np.cumsum(counts)])
+    col = np.concatenate(cols)
+    pl = types.SimpleNamespace(blocks=blocks, n_blocks=n_blocks)
+    sel = types.SimpleNamespace(row_ptr=torch.tensor(row_ptr, dtype=torch.int32),
+                                col=torch.tensor(np.concatenate([col, [-1, -1]]), dtype=torch.int32),
+                                nnz=int(col.size))
+    return pl, sel
+
+
+def _dense_mask_pairs(w, opl, osel):
+    """Pairs of the token-level mask: query token q may attend key token k
+    iff k's block is in the selection of q's block."""
+    total = 0
+    for h, hp in enumerate(opl.heads):
+        nb = hp.blocks.shape[0]
+        blk = np.empty(w.N, np.int64)
+        for b in range(nb):
+            p0, B = int(hp.blocks[b, 5]), int(hp.blocks[b, 4])
+            blk[hp.perm[p0:p0 + B]] = b
+        allowed = np.zeros((nb, nb), bool)
+        for (i, ids, _) in osel[h]:
+            allowed[i, ids] = True
+        total += int(allowed[blk[:, None], blk[None, :]].sum())
+    return total
+
+
+@pytest.mark.parametrize("name", ["tiny", "small_d64"])
+def test_computed_pairs_equals_the_dense_mask_count(name):
+    w = WORKLOADS[name]
+    inp = make_inputs(w, "cpu")
+    V, Q, K = (inp[x].float().numpy() for x in ("V", "Q", "K"))
+    opl = O.plan(V, inp["a"].numpy(), w.T, w.H, w.W)
+    osel = O.select(Q, K, opl, w.topk_frac, w.topk_abs, w.top_p)
+    pl, sel = _library_layout(w, opl, osel)
+    p = types.SimpleNamespace(T=w.T, H=w.H, W=w.W, heads=w.heads)
+    got = bench.computed_pairs(p, pl, sel)
+    assert got == _dense_mask_pairs(w, opl, osel)
+    assert 0 < got <= w.N * w.N * w.heads
+
+
+def test_kernel_roofline_arithmetic():
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops_sustained": 1000.0, "sm_max_mhz": 2000.0}
+    P, D, N, h, steps = 1.0e12, 128, 860160, 24, 2
+    nb = torch.tensor([100, 200])
+    kt = {"attn_fwd": (2, 1000.0), "attn_bwd_dq": (2, 1200.0), "block_mean": (2, 4.0),
+          "block_score": (48, 24.0), "select_row": (48, 10.0)}
+    out = bench.kernel_rooflines(kt, P, D, N, h, nb, peaks, "measured", steps)
+    fwd = out["attn_fwd"]                        # one launch per step, 500 ms each
+    assert fwd["ms_per_launch"] == 500.0
+    assert fwd["achieved"] == pytest.approx(4 * P * D / 0.5 / 1e12)
+    assert fwd["peak"] == 1000.0 and fwd["frac"] == pytest.approx(fwd["achieved"] / 1000.0)
+    assert out["attn_bwd_dq"]["achieved"] == pytest.approx(6 * P * D / 0.6 / 1e12)
+    bm = out["block_mean"]                       # one read of Q and K per launch, 2 ms
+    assert bm["achieved"] == pytest.approx(4 * N * h * D / 2e-3 / 1e9) and bm["peak"] == 6000.0
+    bs = out["block_score"]                      # 24 launches per step share 2*D*sum(nb^2)
+    per_launch = 2 * D * (100 ** 2 + 200 ** 2) * steps / 48
+    assert bs["achieved"] == pytest.approx(per_launch / 0.5e-3 / 1e12)
+    assert bs["peak"] == pytest.approx(148 * 128 * 2000e6 / 1e12)
+    assert out["select_row"]["frac"] is None and out["select_row"]["launches"] == 48
+
+
+class _FakeProc:
+    def __init__(self, out):
+        self.out = out
+
+    def terminate(self):
+        pass
+
+    def communicate(self, timeout=None):
+        return self.out, None
+
+
+def test_clock_samples_are_parsed():
+    c = bench.ClockSampler(0)
+    c.proc = _FakeProc("0, 1600, 1965, 700.5, 0x4, Not Active, Not Active, Not Active, Active\n"
+                       "0, 1700, 1965, 710.0, 0x0, Not Active, Not Active, Not Active, Not Active\n"
+                       "0, [N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active\n"
+                       "garbage line\n")
+    r = c.stop()
+    assert r == {"sm_mhz": 1650.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 2}
+    c = bench.ClockSampler(0)
+    c.proc = _FakeProc("0, 1200, 1965, 900, 0x40, Not Active, Active, Not Active, Not Active\n")
+    assert c.stop()["reasons"] == ["hw_thermal_slowdown"]
+    assert bench.ClockSampler(0).stop()["reasons"] == ["nvidia-smi unavailable"]
+
+
+def test_stored_traffic_is_dropped_when_the_kernel_source_changes(tmp_path, monkeypatch):
+    csrc = tmp_path / "dynamic_block_sparse_stats_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    src = csrc / "k.cu"
+    src.write_bytes(b"kernel v1\n")
+    digest = hashlib.sha256(b"kernel v1\n").hexdigest()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"attn_fwd": {"source": "k.cu", "source_sha256": digest, "bytes_per_launch": 123.0}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.stored_traffic("attn_fwd") == 123.0
+    assert bench.stored_traffic("attn_bwd_dq") is None
+    src.write_bytes(b"kernel v2\n")
+    assert bench.stored_traffic("attn_fwd") is None

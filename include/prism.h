@@ -24,9 +24,13 @@
  *   Memory.  Every pointer argument is DEVICE memory unless stated
  *     otherwise.  Tensor pointers (Q, K, V, O, O_res, dO, dQ, dK, dV, the
  *     bridge output of prism_a2v_norm) and the plan's block table must be
- *     16-byte aligned; a misaligned one is PRISM_ERR_INVALID_ARG.  The caller allocates and owns every buffer, including the
- *     workspaces sized by the *_workspace_size() queries; the library never
- *     allocates device memory.  Workspaces must be 256-byte aligned and may
+ *     16-byte aligned; a misaligned one is PRISM_ERR_INVALID_ARG.  The
+ *     library cannot see a buffer's size or its device: passing buffers
+ *     smaller than stated here, or on another device than the current one,
+ *     is undefined (the Python binding checks both before every call).  The
+ *     caller allocates and owns every buffer, including the workspaces sized
+ *     by the *_workspace_size() queries; the library never allocates device
+ *     memory (prism_plan_noalloc's fixed array aside).  Workspaces must be 256-byte aligned and may
  *     not be shared by calls that run concurrently.
  *   Execution.  Calls enqueue kernels on `stream` and return without waiting,
  *     except prism_select, which waits once on `stream` to read the number
@@ -240,9 +244,15 @@ size_t prism_select_workspace_size(const prism_params *p);
  * P_i = softmax_j(s_i), S_i = Top-k(P_i, k) U Top-p(P_i, top_p).
  * Precision: block means are fp32 running sums over the block's tokens in
  * raster order times 1/B; scores are fp32 running sums over channels of
- * separately rounded products, times the scale; the Top-p cumulative sum
- * is accumulated in float64.  Order: score descending, then key id
- * ascending; "passes p" is read as ">= p" with the crossing block kept.
+ * separately rounded products, times the scale.  The Top-p cumulative sum
+ * is exact: each weight exp(s_ij - max_j s_ij) is quantised to a multiple of
+ * 2^-qb, qb = 62 - ceil(log2(nb + 1)) for a head of nb blocks (2^-48 at
+ * nb = 13440, the 2K grid's maximum), and summed as 64-bit integers, so the
+ * crossing does not depend on the order of the additions and the selection
+ * is bit-reproducible; a sum moves by at most nb * 2^-(qb+1) of the row's
+ * total.  p >= 1 keeps every block.  Order:
+ * score descending, then key id ascending; "passes p" is read as ">= p"
+ * with the crossing block kept.
  *   plan   output of prism_plan for the same params.
  *   Q, K   bf16 [N][heads][head_dim].
  *   out    see prism_select_t; out->nnz is written.
@@ -323,13 +333,14 @@ uint64_t prism_kernel_launches(void);
 
 /* Optional timing of the library's main kernels, for measurement.  When
  * enabled, every launch of the zone-statistics, block-mean, block-score,
- * row-selection, forward-attention and the two backward-attention kernels is
- * bracketed by a CUDA event pair recorded on its launching stream.
+ * row-selection, forward-attention, the two backward-attention and the A2V
+ * norm kernels is bracketed by a CUDA event pair recorded on its launching
+ * stream.
  * prism_kernel_timing(1) clears the records and enables; (0) clears and
  * disables.  Returns PRISM_OK. */
 int prism_kernel_timing(int enable);
 
-/* Reads the records of kernel `id` (0 .. 6, in the order listed above): waits
+/* Reads the records of kernel `id` (0 .. 7, in the order listed above): waits
  * for its events, and returns the number of timed launches, their total
  * milliseconds and the kernel's name (library-owned string).  Returns
  * PRISM_OK, PRISM_ERR_INVALID_ARG (id out of range) or PRISM_ERR_CUDA. */
@@ -341,10 +352,12 @@ const char *prism_version(void);
 
 /*
  * prism_diag_exp2 -- diagnostics.  Evaluates, for n fp32 inputs x (device
- * memory), the two exponentials prism_attn_fwd uses for softmax weights:
- * y_poly = 2^x from the FMA-pipe polynomial (x clamped to [-125, 64];
- * relative error at most 7.5e-5, below half an fp16 ulp) and y_mufu = 2^x
- * from the MUFU instruction.  Outputs are fp32 device arrays of n entries.
+ * memory), two ways of forming softmax weights: y_poly = 2^x from the
+ * library's FMA-pipe polynomial (x clamped to [-125, 64]; relative error at
+ * most 7.5e-5, below half an fp16 ulp) and y_mufu = 2^x from the MUFU
+ * instruction.  The attention kernels can move a share of their
+ * exponentials to the polynomial; they currently use MUFU for all of them,
+ * which measured faster.  Outputs are fp32 device arrays of n entries.
  * Returns PRISM_OK, PRISM_ERR_INVALID_ARG or PRISM_ERR_CUDA.
  */
 int prism_diag_exp2(const float *x, float *y_poly, float *y_mufu, int64_t n, prism_stream_t stream);

@@ -209,10 +209,77 @@ def kernel_rooflines(ktimes, P, D, N, h, nb, peaks, peak_src, steps):
     return out
 
 
+# The source file of each timed kernel, under the package's csrc/, and the
+# ncu kernel-name fragment that identifies its launches.
+KERNEL_SOURCES = {"zone_video_stats": "plan.cu", "block_mean": "select.cu", "block_score": "select.cu",
+                  "select_row": "select.cu", "attn_fwd": "attn_fwd.cu", "attn_bwd_dkdv": "attn_bwd.cu",
+                  "attn_bwd_dq": "attn_bwd.cu", "a2v_norm": "a2v_norm.cu"}
+NCU_KERNEL_NAMES = {"a2v_norm": "a2v_norm_kernel", "zone_video_stats": "zone_video_stats_kernel",
+                    "block_mean": "block_mean_kernel", "attn_fwd": "attn_fwd_kernel",
+                    "attn_bwd_dkdv": "dkdv_kernel", "attn_bwd_dq": "dq_kernel"}
+
+
+def strip_comments(text: str) -> str:
+    """C/C++/CUDA source without its comments and formatting: // and /* */
+    comments removed, runs of spaces and tabs outside string and character
+    literals reduced to one space, lines trimmed and empty lines dropped (line
+    breaks stay: preprocessor directives depend on them)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            if not out or out[-1] != " ":
+                out.append(" ")
+            i = n if j < 0 else j + 2
+        elif c in " \t\r\f\v":
+            if not out or out[-1] != " ":
+                out.append(" ")
+            i += 1
+        else:
+            out.append(c)
+            i += 1
+    lines = (ln.strip() for ln in "".join(out).split("\n"))
+    return "\n".join(ln for ln in lines if ln) + "\n"
+
+
+def source_digest(source: str, csrc=None) -> str:
+    """sha256 of a kernel's code: its source file under csrc/ and every local
+    header it includes, transitively (quoted #include paths, resolved from the
+    including file), each with its comments and blank space removed.  A
+    comment edit leaves the digest unchanged; an edit of the code, or of a
+    header the code includes, changes it."""
+    import hashlib
+    import re
+    csrc = csrc or os.path.join(ROOT, "dynamic_block_sparse_stats_b200", "csrc")
+    todo, seen = [os.path.normpath(os.path.join(csrc, source))], {}
+    while todo:
+        path = todo.pop()
+        if path in seen:
+            continue
+        with open(path) as f:
+            seen[path] = strip_comments(f.read())
+        for inc in re.findall(r'^\s*#\s*include\s+"([^"]+)"', seen[path], flags=re.M):
+            todo.append(os.path.normpath(os.path.join(os.path.dirname(path), inc)))
+    h = hashlib.sha256()
+    for path in sorted(seen):
+        h.update(os.path.relpath(path, csrc).encode() + b"\0" + seen[path].encode() + b"\0")
+    return h.hexdigest()
+
+
 def stored_traffic(kernel):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, or None
-    when the summary is missing or the kernel's source changed since."""
-    import hashlib
+    when the summary is missing or the kernel's code (its source file or a
+    header it includes) changed since the counters were taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -220,10 +287,49 @@ def stored_traffic(kernel):
         d = json.load(f).get(kernel)
     if not d:
         return None
-    src = os.path.join(ROOT, "dynamic_block_sparse_stats_b200", "csrc", d["source"])
-    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != d["source_sha256"]:
+    try:
+        if source_digest(d["source"]) != d["code_digest"]:
+            return None
+    except (OSError, KeyError):
         return None
     return d["bytes_per_launch"]
+
+
+def write_traffic(csv_path, out_path=None):
+    """profiles/traffic.json from an ncu capture of dram__bytes_read.sum and
+    dram__bytes_write.sum (`ncu --csv --log-file`): per timed kernel, the mean
+    of read + write bytes over its captured launches, keyed to the digest of
+    the kernel's code as it is now (run it on the code that was captured)."""
+    rows, start = [], False
+    with open(csv_path) as f:
+        for line in f:
+            if line.startswith('"ID"'):
+                start = True
+            if start:
+                rows.append(line)
+    per = {}
+    for r in csv.DictReader(io.StringIO("".join(rows))):
+        if r["Metric Name"] not in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            continue
+        name = next((k for k, frag in NCU_KERNEL_NAMES.items() if frag in r["Kernel Name"]), None)
+        if name is None:
+            continue
+        scale = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "Tbyte": 1e12}[r["Metric Unit"]]
+        launch = per.setdefault(name, {}).setdefault(r["ID"], 0.0)
+        per[name][r["ID"]] = launch + float(r["Metric Value"].replace(",", "")) * scale
+    out = {"_about": "DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch, mean over the "
+                     "captured launches of each kernel (see traffic_2k_training_layer.md for the command). "
+                     "Valid while the kernel's code digest (bench.source_digest: its source file and the "
+                     "headers it includes, comments removed) equals code_digest."}
+    for name in NCU_KERNEL_NAMES:
+        if name in per:
+            vals = list(per[name].values())
+            out[name] = {"bytes_per_launch": sum(vals) / len(vals), "launches_captured": len(vals),
+                         "source": KERNEL_SOURCES[name], "code_digest": source_digest(KERNEL_SOURCES[name])}
+    with open(out_path or os.path.join(ROOT, "profiles", "traffic.json"), "w") as f:
+        json.dump(out, f, indent=1)
+        f.write("\n")
+    return out
 
 
 # ----------------------------------------------------------------------------- oracle sample
@@ -555,10 +661,15 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense SDPA comparison")
+    ap.add_argument("--write-traffic", metavar="NCU_CSV",
+                    help="write profiles/traffic.json from an ncu DRAM-bytes capture and exit (no GPU needed)")
     ap.add_argument("--shard", choices=["layers", "heads"], default="layers",
                     help="N>1: every rank its own layer (weak scaling, default) or one layer's heads split "
                          "over the ranks (strong scaling); neither exchanges data on the path")
     args = ap.parse_args()
+    if args.write_traffic:
+        print(json.dumps(write_traffic(args.write_traffic), indent=1))
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[args.workload]

@@ -17,8 +17,9 @@
 //   dkdv_kernel  one CTA per 128-key tile; walks the transpose (CSC), two
 //                query units per step: S^T = K Q^T, dP^T = V dO^T (TMEM),
 //                P^T and dS^T -> TMEM (fp16), dV += P^T dO, dK += dS^T Q (TS
-//                MMAs); the softmax of a step overlaps its dP^T product and
-//                dS^T overlaps the dV product.
+//                MMAs), issued dV(i-1), S^T(i), dK(i-1), dP^T(i): the
+//                softmax of step i overlaps dK(i-1) and dP^T(i), and S^T(i)
+//                waits only for dV(i-1) to have read P^T(i-1).
 // Operands are fp16 (exact conversions of the bf16 inputs, see the forward).
 // Roles: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer, warps 4-11
 // two compute warpgroups (one thread per TMEM lane), each taking one of the

@@ -126,17 +126,77 @@ def test_clock_samples_are_parsed():
     assert bench.ClockSampler(0).stop()["reasons"] == ["nvidia-smi unavailable"]
 
 
-def test_stored_traffic_is_dropped_when_the_kernel_source_changes(tmp_path, monkeypatch):
+def test_strip_comments_keeps_code_and_literals():
+    src = ('#include "a.h"  // trailing\n'
+           '/* block\n   comment */ int x = 1; /* inline */ int y = 2;\n'
+           '\n'
+           '\tconst  char *s = "not // a comment /* either */";\n'
+           "char c = '\\''; char d = '/'; // it's a comment\n")
+    assert bench.strip_comments(src) == ('#include "a.h"\n'
+                                         'int x = 1; int y = 2;\n'
+                                         'const char *s = "not // a comment /* either */";\n'
+                                         "char c = '\\''; char d = '/';\n")
+
+
+def _tree(tmp_path, kernel, header, shared):
     csrc = tmp_path / "dynamic_block_sparse_stats_b200" / "csrc"
-    csrc.mkdir(parents=True)
+    inc = tmp_path / "include"
+    csrc.mkdir(parents=True, exist_ok=True)
+    inc.mkdir(exist_ok=True)
+    (csrc / "k.cu").write_text('#include "k.cuh"\n' + kernel)
+    (csrc / "k.cuh").write_text('#include "../../include/api.h"\n' + header)
+    (inc / "api.h").write_text(shared)
+    return str(csrc)
+
+
+def test_code_digest_ignores_comments_and_follows_includes(tmp_path):
+    csrc = _tree(tmp_path, "int k() { return 1; }\n", "int h();\n", "int api();\n")
+    d0 = bench.source_digest("k.cu", csrc)
+    _tree(tmp_path, "// new comment\nint k() {  return 1; }  /* more */\n", "int h();  // note\n",
+          "/* doc */ int api();\n")
+    assert bench.source_digest("k.cu", csrc) == d0
+    _tree(tmp_path, "int k() { return 2; }\n", "int h();\n", "int api();\n")
+    assert bench.source_digest("k.cu", csrc) != d0          # the kernel's own code
+    _tree(tmp_path, "int k() { return 1; }\n", "int h(int);\n", "int api();\n")
+    assert bench.source_digest("k.cu", csrc) != d0          # an included header
+    _tree(tmp_path, "int k() { return 1; }\n", "int h();\n", "long api();\n")
+    assert bench.source_digest("k.cu", csrc) != d0          # a header included by a header
+
+
+_NCU_CSV = """==PROF== Connected to process 1
+"ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream","Block Size","Grid Size","Device","CC","Section Name","Metric Name","Metric Unit","Metric Value"
+"0","1","python","h","prism::fwd::attn_fwd_kernel<128>(Params)","1","7","(384, 1, 1)","(148, 1, 1)","0","10.0","m","dram__bytes_read.sum","Gbyte","2,000.5"
+"0","1","python","h","prism::fwd::attn_fwd_kernel<128>(Params)","1","7","(384, 1, 1)","(148, 1, 1)","0","10.0","m","dram__bytes_write.sum","Mbyte","500"
+"0","1","python","h","prism::fwd::attn_fwd_kernel<128>(Params)","1","7","(384, 1, 1)","(148, 1, 1)","0","10.0","m","gpu__time_duration.sum","msecond","800"
+"1","1","python","h","prism::fwd::attn_fwd_kernel<128>(Params)","1","7","(384, 1, 1)","(148, 1, 1)","0","10.0","m","dram__bytes_read.sum","Gbyte","1,000.5"
+"1","1","python","h","prism::fwd::attn_fwd_kernel<128>(Params)","1","7","(384, 1, 1)","(148, 1, 1)","0","10.0","m","dram__bytes_write.sum","Mbyte","500"
+"2","1","python","h","void at::native::elementwise_kernel<128>(int)","1","7","(128, 1, 1)","(1, 1, 1)","0","10.0","m","dram__bytes_read.sum","byte","64"
+"""
+
+
+def test_write_traffic_and_stored_traffic(tmp_path, monkeypatch):
+    _tree(tmp_path, "int k() { return 1; }\n", "int h();\n", "int api();\n")
     (tmp_path / "profiles").mkdir()
-    src = csrc / "k.cu"
-    src.write_bytes(b"kernel v1\n")
-    digest = hashlib.sha256(b"kernel v1\n").hexdigest()
-    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
-        {"attn_fwd": {"source": "k.cu", "source_sha256": digest, "bytes_per_launch": 123.0}}))
+    (tmp_path / "ncu.csv").write_text(_NCU_CSV)
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.stored_traffic("attn_fwd") == 123.0
+    monkeypatch.setitem(bench.KERNEL_SOURCES, "attn_fwd", "k.cu")
+    out = bench.write_traffic(str(tmp_path / "ncu.csv"))
+    assert set(out) == {"_about", "attn_fwd"}          # torch kernels are not ours
+    assert out["attn_fwd"]["bytes_per_launch"] == pytest.approx((2000.5e9 + 0.5e9 + 1000.5e9 + 0.5e9) / 2)
+    assert out["attn_fwd"]["launches_captured"] == 2
+    assert bench.stored_traffic("attn_fwd") == out["attn_fwd"]["bytes_per_launch"]
     assert bench.stored_traffic("attn_bwd_dq") is None
-    src.write_bytes(b"kernel v2\n")
+    (tmp_path / "dynamic_block_sparse_stats_b200" / "csrc" / "k.cu").write_text(
+        '#include "k.cuh"\n// only a comment changed\nint k() { return 1; }\n')
+    assert bench.stored_traffic("attn_fwd") is not None
+    (tmp_path / "dynamic_block_sparse_stats_b200" / "csrc" / "k.cuh").write_text(
+        '#include "../../include/api.h"\nint h(int);\n')
     assert bench.stored_traffic("attn_fwd") is None
+
+
+def test_committed_traffic_figures_cover_the_measured_kernels():
+    with open(bench.os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        d = json.load(f)
+    assert set(bench.NCU_KERNEL_NAMES) <= set(d)
+    for name in bench.NCU_KERNEL_NAMES:
+        assert d[name]["source"] == bench.KERNEL_SOURCES[name] and d[name]["bytes_per_launch"] > 0

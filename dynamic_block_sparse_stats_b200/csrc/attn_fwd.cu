@@ -7,11 +7,13 @@
 // matrix; the output goes back to the original order) and the training
 // section (the kernel walks blocks of any volume in 64-token units).
 //
-// Work unit: one CTA per 128-query tile of one head, in permuted order.  A
-// tile is two 64-token units; both belong to one block (B >= 128), or to two
-// 64-token blocks of the same zone, in which case the tile walks the union of
-// their selections and masks each key unit per row half.  Keys are streamed
-// as tiles of two 64-token units (any two units of the walk).
+// Work unit: one CTA per 256 permuted query positions of one head (grid
+// N/256 x heads): four 64-token query units, two 128-row tiles.  The CTA walks
+// the merged selections of the (up to four) distinct blocks of its units once,
+// in ascending 64-token key units; every key tile feeds both query tiles, and
+// each key unit carries a mask of the 64-row quarters whose block selected it
+// (the rows of other quarters give it weight 0).  Keys are streamed as tiles
+// of two 64-token units (any two units of the walk).
 //
 // Roles (384 threads, two 128-row query tiles t = 0, 1 per CTA):
 //   warp 0      TMA producer: Q once, then per key tile j the K tile j and

@@ -57,3 +57,27 @@ def test_reference_arm_prints_the_contract():
                            "d2h_bytes_per_step": 0}
     assert line["config"]["workload"] == "tiny" and line["metric"] == bench.METRIC
     assert bench.run_reference(args, w, rank=1, world=2) is None      # other ranks do no work
+
+
+def test_reference_arm_under_torchrun_prints_one_line_from_rank_zero():
+    """The launch the driver uses for N > 1, on the CPU: every rank exits 0,
+    rank 0 alone prints one JSON line, the other ranks do no work."""
+    import json
+    import os
+    import socket
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py", "--impl", "reference",
+           "--gpus", "2", "--steps", "1", "--warmup", "3", "--workload", "tiny"]
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="", OMP_NUM_THREADS="1")
+    r = subprocess.run(cmd, cwd=root, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0

@@ -589,7 +589,7 @@ def run_prism(args, w, rank, world, device):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        layer_time, P_or, desc, threads, wall = oracle_sample(w, inp)
+        layer_time, P_or, desc, threads, wall = oracle_sample(w, inp, n_rows=4, n_sel=2048)
         flops_or = (4.0 + (10.0 if backward else 0.0)) * P_or * D
         cpu = {"value": flops_or / layer_time / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": desc, "host_cpus": os.cpu_count(), "sample_wall_s": wall}

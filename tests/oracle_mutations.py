@@ -1,0 +1,105 @@
+"""Mutation check of the oracle's pins (not collected by pytest; run by hand).
+
+    python tests/oracle_mutations.py [mutation name ...]
+
+Each entry below plants one plausible mistake in the oracle: a dropped term,
+a wrong sign, index or axis, an off-by-one, a wrong tie-break or reading.
+For each entry the script copies the repository into a temporary directory,
+applies the mutation to the copy's oracle/prism_oracle.py and runs the CPU
+suite (-m "not gpu", stopping at the first failure) on the copy.  A mutation
+that no test catches marks a missing pin.  The repository itself is never
+modified.  A full run takes about 15 minutes on 8 cores; it exits 1 if any
+mutation survives.
+"""
+import os
+import shutil
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+M = [
+ ("r_v sample variance", "sig2[:, d] = ((prof - mu) ** 2).mean(axis=1).mean(axis=1)", "sig2[:, d] = ((prof - mu) ** 2).sum(axis=1).mean(axis=1) / (ZONE - 1)"),
+ ("H profile pools the wrong axes", "prof_H = v.mean(axis=(1, 3))", "prof_H = v.mean(axis=(1, 2))"),
+ ("spatial term around the zone mean", "spatial = ((v - prof_T[:, :, None, None, :]) ** 2)", "spatial = ((v - v.mean(axis=(1, 2, 3), keepdims=True)) ** 2)"),
+ ("temporal term over 8 not 7", "temporal = (diff ** 2).sum(axis=1).mean(axis=1) / (ZONE - 1)", "temporal = (diff ** 2).sum(axis=1).mean(axis=1) / ZONE"),
+ ("temporal term abs not square", "temporal = (diff ** 2).sum(axis=1)", "temporal = np.abs(diff).sum(axis=1)"),
+ ("a2v norm L1", "return np.sqrt((h * h).sum(axis=1))", "return np.abs(h).sum(axis=1)"),
+ ("a2v norm without sqrt", "return np.sqrt((h * h).sum(axis=1))", "return (h * h).sum(axis=1)"),
+ ("a2v profiles swapped", "for d, ax in enumerate(((2, 3), (1, 3), (1, 2))):", "for d, ax in enumerate(((1, 3), (2, 3), (1, 2))):"),
+ ("abar from zone max", "abar_raw = z.mean(axis=(1, 2, 3))", "abar_raw = z.max(axis=(1, 2, 3))"),
+ ("zero-variance shares 0", "out = np.full_like(sig2, 1.0 / 3.0)", "out = np.zeros_like(sig2)"),
+ ("eps dropped", "    return g + eps", "    return g"),
+ ("abar not applied", "g = g + abar[:, None] * vhat", "g = g + vhat"),
+ ("normalise by sum", "    return x / m\n", "    return x / x.sum()\n"),
+ ("threshold strict", "B = np.where(rho >= tau128, 64, np.where(rho >= tau256, 128, 256))", "B = np.where(rho > tau128, 64, np.where(rho > tau256, 128, 256))"),
+ ("volumes reversed", "B = np.where(rho >= tau128, 64, np.where(rho >= tau256, 128, 256))", "B = np.where(rho >= tau128, 256, np.where(rho >= tau256, 128, 64))"),
+ ("lstar sign", "return -alpha * lg + (S[..., None]", "return alpha * lg + (S[..., None]"),
+ ("lstar over 2", "alpha * lg.sum(axis=-1, keepdims=True)) / 3.0", "alpha * lg.sum(axis=-1, keepdims=True)) / 2.0"),
+ ("lstar natural log of B", "S = np.log2(B.astype(np.float64))", "S = np.log(B.astype(np.float64))"),
+ ("lstar shift ignores alpha", "(S[..., None] + alpha * lg.sum(", "(S[..., None] + 0.5 * lg.sum("),
+ ("shape tie to highest id", "            if dist < best:\n                second, best, best_id", "            if dist <= best:\n                second, best, best_id"),
+ ("shape distance L1", "dist = sum((l[d] - ls[idx][d]) ** 2 for d in range(3))", "dist = sum(abs(l[d] - ls[idx][d]) for d in range(3))"),
+ ("block tokens y fastest", "return ((t * H + y) * W + x).reshape(-1)", "return ((t * H + y) * W + x).transpose(0, 2, 1).reshape(-1)"),
+ ("zones zT fastest", "perm = (0, 2, 4, 1, 3, 5)", "perm = (4, 2, 0, 1, 3, 5)"),
+ ("candidate order reversed", "        for bT in (2, 4, 8):", "        for bT in (8, 4, 2):"),
+ ("block mean over B-1", "out[bl] = acc * np.float32(1.0 / B)", "out[bl] = acc * np.float32(1.0 / (B - 1))"),
+ ("score scale dropped", "    return acc * np.float32(scale)", "    return acc"),
+ ("top-k floor", "int(math.ceil(float(np.float32(topk_frac)) * nb))", "int(math.floor(float(np.float32(topk_frac)) * nb))"),
+ ("top-p strict", "hit = np.nonzero(csum >= target)[0]", "hit = np.nonzero(csum > target)[0]"),
+ ("top-p crossing dropped", "n_p = int(hit[0]) + 1 if hit.size else nb", "n_p = int(hit[0]) if hit.size else nb"),
+ ("ties by index descending", "order = np.lexsort((j, -s))", "order = np.lexsort((-j, -s))"),
+ ("intersection not union", "    n = max(k, n_p)", "    n = min(k, n_p)"),
+ ("p >= 1 rule dropped", "    elif p >= 1:\n        n_p = nb", "    elif p > 1:\n        n_p = nb"),
+ ("fwd scale dropped", "    s = (q @ k.T) * scale\n    m = s.max", "    s = (q @ k.T)\n    m = s.max"),
+ ("lse without the max", "lse = (m + np.log(l))[:, 0]", "lse = np.log(l)[:, 0]"),
+ ("bwd dS sign", "dS = P * (dP - Dq)", "dS = P * (Dq - dP)"),
+ ("bwd dK scale dropped", "np.add.at(dK[:, h], keys, scale * (dS.T @ q))", "np.add.at(dK[:, h], keys, dS.T @ q)"),
+ ("bwd Delta from dO.dO", "Dq = (P * dP).sum(axis=1, keepdims=True)", "Dq = (do * do).sum(axis=1, keepdims=True)"),
+ ("bwd dQ scale dropped", "dQ[qi, h] += scale * (dS @ k)", "dQ[qi, h] += dS @ k"),
+ ("guidance bits swapped", "video=not (guidance & 1), audio=not (guidance & 2)", "video=not (guidance & 2), audio=not (guidance & 1)"),
+ ("density modes swapped", "    if mode == 1:\n        return spatial", "    if mode == 1:\n        return temporal"),
+ ("vhat not normalised", "        vhat = shares(sig2a)", "        vhat = sig2a"),
+ ("rho per all heads", "        rho = normalise_by_max(density_raw(spatial, temporal, abar_raw, density))", "        rho = density_raw(spatial, temporal, abar_raw, density) / 1.0"),
+]
+
+
+def main(only):
+    tmp = tempfile.mkdtemp(prefix="oracle_mutations_")
+    dst = os.path.join(tmp, "repo")
+    try:
+        shutil.copytree(ROOT, dst, ignore=shutil.ignore_patterns(".git", "_build", "gpurun_out", "_work",
+                                                                 "__pycache__", "baseline"))
+        path = os.path.join(dst, "oracle", "prism_oracle.py")
+        with open(path) as f:
+            orig = f.read()
+        survivors = []
+        for name, old, new in M:
+            if only and name not in only:
+                continue
+            if orig.count(old) != 1:
+                print(f"SKIP     {name}: pattern found {orig.count(old)} times")
+                continue
+            with open(path, "w") as f:
+                f.write(orig.replace(old, new))
+            t = time.time()
+            r = subprocess.run([sys.executable, "-m", "pytest", "tests", "-x", "-q", "-m", "not gpu",
+                                "-p", "no:cacheprovider", "--deselect",
+                                "tests/test_bench_reference_cpu.py::"
+                                "test_reference_arm_under_torchrun_prints_one_line_from_rank_zero"],
+                               cwd=dst, capture_output=True, text=True)
+            failed = [ln for ln in r.stdout.splitlines() if ln.startswith(("FAILED", "ERROR"))][:1]
+            if r.returncode == 0:
+                survivors.append(name)
+            print(f"{'caught  ' if r.returncode else 'SURVIVED'} {name:34s} {time.time() - t:5.1f}s {failed}",
+                  flush=True)
+        print("survivors:", survivors)
+        return 1 if survivors else 0
+    finally:
+        shutil.rmtree(tmp, ignore_errors=True)
+
+
+if __name__ == "__main__":
+    sys.exit(main(sys.argv[1:]))

@@ -124,6 +124,25 @@ def test_a2v_stats_blob_and_normalisation():
     np.testing.assert_allclose(O.shares(sig2a), [[0, 0, 1], [0, 0, 1]], atol=1e-15)
 
 
+def test_a2v_direction_shares_follow_the_axis_of_variation():
+    """v_hat_{a,d}: a field that varies along one axis only puts its whole
+    share on that axis; a sum f(t) + g(y) splits it in the closed-form ratio
+    var f : var g (population variances of the 8-position profiles)."""
+    T, H, W = 8, 8, 8
+    t, y, x = np.meshgrid(np.arange(T), np.arange(H), np.arange(W), indexing="ij")
+    for d, field in enumerate((t, y, x)):
+        _, sig2a = O.zone_a2v_stats(field.astype(float).reshape(-1), T, H, W)
+        want = np.zeros(3)
+        want[d] = 1.0
+        np.testing.assert_allclose(O.shares(sig2a)[0], want, atol=1e-15)
+    f = np.array([0, 1, 0, 1, 0, 1, 0, 1], float)          # var 1/4
+    g = np.array([0, 0, 0, 0, 2, 2, 2, 2], float)          # var 1
+    a = (f[t] + g[y]).reshape(-1)
+    _, sig2a = O.zone_a2v_stats(a, T, H, W)
+    np.testing.assert_allclose(sig2a[0], [0.25, 1.0, 0.0], atol=1e-15)
+    np.testing.assert_allclose(O.shares(sig2a)[0], [0.2, 0.8, 0.0], atol=1e-15)
+
+
 def test_variation_indicator_terms_and_invariant():
     rng = np.random.default_rng(6)
     r = O.shares(rng.random((10, 3)))
@@ -274,6 +293,9 @@ def test_block_means_and_scores_on_exact_inputs():
     yb = O.block_means_fp32(Y, hp)
     s = O.block_scores_fp32(xb, yb, 1.0)
     np.testing.assert_allclose(s, xb.astype(np.float64) @ yb.astype(np.float64).T, rtol=2e-6)
+    # the attention scale multiplies the scores (a power of two scales exactly)
+    s8 = O.block_scores_fp32(xb, yb, 0.125)
+    np.testing.assert_array_equal(s8, s * np.float32(0.125))
 
 
 def _brute_select(s, k, p):
@@ -324,6 +346,28 @@ def test_select_all_and_topk_only_limits():
     assert ids.tolist() == [0]
     assert O.topk_count(100, 0.04, 0) == 4 and O.topk_count(100, 0.0, 7) == 7
     assert O.topk_count(10, 0.001, 0) == 1 and O.topk_count(10, 0.0, 50) == 10
+
+
+def test_top_p_crossing_exactly_at_p_is_kept():
+    """Reading: the Top-p prefix is the shortest whose mass is >= p.  Four
+    equal scores give P = 1/4 each, exactly, so the mass reaches p = 1/2 at
+    the second block and p = 3/4 at the third (a strict > would take one
+    more)."""
+    s = np.ones(4, np.float32)
+    ids, info = O.hybrid_select_row(s, 1, 0.5)
+    assert info["n_p"] == 2 and ids.tolist() == [0, 1]
+    ids, info = O.hybrid_select_row(s, 1, 0.75)
+    assert info["n_p"] == 3 and ids.tolist() == [0, 1, 2]
+
+
+def test_top_p_one_keeps_blocks_whose_weight_underflows():
+    """Every softmax weight is positive, so p = 1 is reached only with the
+    last block, even when float64 rounds the tail weights to 0 (exp(-800))."""
+    s = np.array([0.0, -800.0, -900.0, -800.0], np.float32)
+    ids, info = O.hybrid_select_row(s, 1, 1.0)
+    assert info["n_p"] == 4 and ids.tolist() == [0, 1, 2, 3]
+    ids, info = O.hybrid_select_row(s, 1, 0.999)
+    assert info["n_p"] == 1 and ids.tolist() == [0]
 
 
 # ---------------------------------------------------------------- attention

@@ -63,6 +63,12 @@ M = [
  ("density modes swapped", "    if mode == 1:\n        return spatial", "    if mode == 1:\n        return temporal"),
  ("vhat not normalised", "        vhat = shares(sig2a)", "        vhat = sig2a"),
  ("rho per all heads", "        rho = normalise_by_max(density_raw(spatial, temporal, abar_raw, density))", "        rho = density_raw(spatial, temporal, abar_raw, density) / 1.0"),
+ ("abar not normalised in the plan", "        abar = normalise_by_max(abar_raw)", "        abar = abar_raw"),
+ ("selection in score order", "    return np.sort(order[:n]), dict(", "    return order[:n], dict("),
+ ("temporal term over row means", "diff = prof_T[:, 1:, :] - prof_T[:, :-1, :]", "diff = prof_H[:, 1:, :] - prof_H[:, :-1, :]"),
+ ("permutation inverted", "        perm[p0:p0 + B] = block_tokens(T, H, W, t0, y0, x0, sid)", "        perm[block_tokens(T, H, W, t0, y0, x0, sid)] = np.arange(p0, p0 + B)"),
+ ("lse in log2", "lse = (m + np.log(l))[:, 0]", "lse = (m + np.log2(l))[:, 0]"),
+ ("top-k takes the lowest scores", "order = np.lexsort((j, -s))", "order = np.lexsort((j, s))"),
 ]
 
 

@@ -151,6 +151,32 @@ def computed_pairs(p, pl, sel):
     return int((Bq[row_of] * Bk).sum().item())
 
 
+def selection_stats(p, pl, sel):
+    """Realised density per query block over the live rows of all heads: the
+    number of selected key blocks, and the share of the head's tokens the
+    block's queries attend (sum of B_j over j in S_i, divided by N); each as
+    mean, median and 99th percentile (linear interpolation)."""
+    NB = p.T * p.H * p.W // 64
+    N = p.T * p.H * p.W
+    row_ptr = sel.row_ptr.long()
+    counts = row_ptr[1:] - row_ptr[:-1]
+    rows = torch.arange(p.heads * NB, device=row_ptr.device)
+    valid = (rows % NB) < pl.n_blocks.long().repeat_interleave(NB)
+    Bsz = pl.blocks[:, :, 1].reshape(-1).long()
+    row_of = torch.repeat_interleave(rows, counts)
+    col = sel.col[:sel.nnz].long()
+    keys = torch.zeros(p.heads * NB, dtype=torch.float64, device=row_ptr.device)
+    keys.index_add_(0, row_of, Bsz[(row_of // NB) * NB + col].double())
+    q = torch.tensor([0.5, 0.99], dtype=torch.float64, device=row_ptr.device)
+
+    def summary(x):
+        qs = torch.quantile(x, q)
+        return {"mean": float(x.mean()), "p50": float(qs[0]), "p99": float(qs[1])}
+
+    return {"rows": int(valid.sum()), "blocks_per_row": summary(counts[valid].double()),
+            "key_share_per_row": summary(keys[valid] / N)}
+
+
 # ----------------------------------------------------------------------------- kernel rooflines
 def read_kernel_times(lib):
     out = {}
@@ -613,7 +639,8 @@ def run_prism(args, w, rank, world, device):
                    "parallelism": (f"heads split over {world} ranks (this rank {h0}-{h1 - 1}), no collectives on the path"
                                    if heads_mode else f"weak x{world} (independent layers, no collectives)"),
                    "l2": "inputs larger than L2 (each bf16 tensor %.2f GB)" % (N * h * D * 2 / 1e9),
-                   "pairs": P, "pair_density": density, "nnz_blocks": sel.nnz},
+                   "pairs": P, "pair_density": density, "nnz_blocks": sel.nnz,
+                   "selection": selection_stats(p, pl, sel)},
         "stage_ms": stage_ms, "stage_roofline": stage_roofline, "kernels": kernels,
         "clocks": clocks, "e2e": e2e, "gpu_launches": launches, "roofline": roofline, "cpu_baseline": cpu,
         "dense_sdpa": dense,

@@ -200,3 +200,25 @@ def test_committed_traffic_figures_cover_the_measured_kernels():
     assert set(bench.NCU_KERNEL_NAMES) <= set(d)
     for name in bench.NCU_KERNEL_NAMES:
         assert d[name]["source"] == bench.KERNEL_SOURCES[name] and d[name]["bytes_per_launch"] > 0
+
+
+@pytest.mark.parametrize("name", ["tiny", "small_d64"])
+def test_selection_stats_match_the_oracle_rows(name):
+    w = WORKLOADS[name]
+    inp = make_inputs(w, "cpu")
+    V, Q, K = (inp[x].float().numpy() for x in ("V", "Q", "K"))
+    opl = O.plan(V, inp["a"].numpy(), w.T, w.H, w.W)
+    osel = O.select(Q, K, opl, w.topk_frac, w.topk_abs, w.top_p)
+    pl, sel = _library_layout(w, opl, osel)
+    p = types.SimpleNamespace(T=w.T, H=w.H, W=w.W, heads=w.heads)
+    got = bench.selection_stats(p, pl, sel)
+    nblk = np.array([len(ids) for h in range(w.heads) for (_, ids, _) in osel[h]], float)
+    share = np.array([opl.heads[h].blocks[ids, 4].sum() / w.N for h in range(w.heads) for (_, ids, _) in osel[h]])
+    assert got["rows"] == nblk.size == sum(hp.blocks.shape[0] for hp in opl.heads)
+    for key, x in (("blocks_per_row", nblk), ("key_share_per_row", share)):
+        assert got[key]["mean"] == pytest.approx(x.mean(), rel=1e-12)
+        assert got[key]["p50"] == pytest.approx(np.percentile(x, 50), rel=1e-12)
+        assert got[key]["p99"] == pytest.approx(np.percentile(x, 99), rel=1e-12)
+    # the mean key share, weighted by block size, is the pair density
+    Bq = np.array([opl.heads[h].blocks[i, 4] for h in range(w.heads) for (i, _, _) in osel[h]])
+    assert (share * Bq).sum() * w.N == pytest.approx(bench.computed_pairs(p, pl, sel), rel=1e-12)

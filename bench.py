@@ -627,6 +627,10 @@ def run_prism(args, w, rank, world, device):
             dense["speedup_of_prism_step"] = dense["ms_per_layer"] / ms
 
     density = P / (float(N) * N * h)
+    try:    # a report of the selection's shape; the measurement above does not depend on it
+        selection_report = selection_stats(p, pl, sel)
+    except (RuntimeError, ValueError) as e:
+        selection_report = {"error": str(e).splitlines()[0][:200]}
     line = {
         "metric": METRIC, "value": total_flops / (ms_max * 1e-3) / 1e12, "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
@@ -640,7 +644,7 @@ def run_prism(args, w, rank, world, device):
                                    if heads_mode else f"weak x{world} (independent layers, no collectives)"),
                    "l2": "inputs larger than L2 (each bf16 tensor %.2f GB)" % (N * h * D * 2 / 1e9),
                    "pairs": P, "pair_density": density, "nnz_blocks": sel.nnz,
-                   "selection": selection_stats(p, pl, sel)},
+                   "selection": selection_report},
         "stage_ms": stage_ms, "stage_roofline": stage_roofline, "kernels": kernels,
         "clocks": clocks, "e2e": e2e, "gpu_launches": launches, "roofline": roofline, "cpu_baseline": cpu,
         "dense_sdpa": dense,

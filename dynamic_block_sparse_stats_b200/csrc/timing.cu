@@ -31,14 +31,21 @@ cudaEvent_t take_event() {
   return e;
 }
 
+void give_event(cudaEvent_t e) {
+  if (e) g_pool.push_back(e);
+}
+
 }  // namespace
 
 KernelTimer::KernelTimer(int id, cudaStream_t st) : st_(st), idx_(-1) {
   std::lock_guard<std::mutex> lock(g_mu);
   if (!g_on) return;
   Rec r{take_event(), take_event(), id};
-  if (!r.a || !r.b) return;
-  if (cudaEventRecord(r.a, st) != cudaSuccess) return;
+  if (!r.a || !r.b || cudaEventRecord(r.a, st) != cudaSuccess) {
+    give_event(r.a);  // keep the events for the next launch
+    give_event(r.b);
+    return;
+  }
   idx_ = (int)g_recs.size();
   g_recs.push_back(r);
 }

@@ -331,7 +331,8 @@ const char *prism_last_error(void);
  * (host-side counter, incremented at every launch; never reset). */
 uint64_t prism_kernel_launches(void);
 
-/* Optional timing of the library's main kernels, for measurement.  When
+/* Optional timing of the library's main kernels, for measurement (not meant
+ * to be toggled by one thread while another launches through the library).  When
  * enabled, every launch of the zone-statistics, block-mean, block-score,
  * row-selection, forward-attention, the two backward-attention and the A2V
  * norm kernels is bracketed by a CUDA event pair recorded on its launching

@@ -20,7 +20,8 @@
 //                MMAs), issued dV(i-1), S^T(i), dK(i-1), dP^T(i): the
 //                softmax of step i overlaps dK(i-1) and dP^T(i), and S^T(i)
 //                waits only for dV(i-1) to have read P^T(i-1).
-// Operands are fp16 (exact conversions of the bf16 inputs, see the forward).
+// Operands are fp16 conversions of the bf16 inputs (exact for 2^-17 <= |x| <=
+// 65504 and for 0, see the forward).
 // Roles: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer, warps 4-11
 // two compute warpgroups (one thread per TMEM lane), each taking one of the
 // step's two 64-token units.

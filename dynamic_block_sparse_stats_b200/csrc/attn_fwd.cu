@@ -513,8 +513,10 @@ __device__ __forceinline__ uint4 to_f16x8(uint4 v, bool &bad) {
                     bf16x2_to_f16x2(v.w, bad));
 }
 
-// dst[h][p][:] = fp16(src[perm[h][p]][h][:]); a value outside the fp16 range
-// records PRISM_ERR_RANGE in *status.
+// dst[h][p][:] = fp16(src[perm[h][p]][h][:]), rounded to nearest: exact for
+// 2^-17 <= |x| <= 65504 and for 0 (bf16's 8 significant bits fit fp16's 11
+// down to its subnormal spacing 2^-24); smaller magnitudes move by at most
+// 2^-25.  A value outside the fp16 range records PRISM_ERR_RANGE in *status.
 __global__ void permute3_kernel(const int32_t *__restrict__ perm, int N, int heads, int D,
                                 const uint16_t *__restrict__ s0, const uint16_t *__restrict__ s1,
                                 const uint16_t *__restrict__ s2, uint16_t *__restrict__ d0, uint16_t *__restrict__ d1,

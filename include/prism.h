@@ -285,8 +285,9 @@ size_t prism_attn_workspace_size(const prism_params *p, int backward);
  *             with sharp attention.
  *   lse       fp32 [heads][N], natural order (natural log).
  * Runs on tcgen05 tensor cores with fp32 accumulation.  The operands are
- * fp16: Q, K, V convert exactly from bf16 for |x| <= 65504 (a larger value
- * records PRISM_ERR_RANGE in the workspace); the probabilities P (in [0, 256]
+ * fp16: Q, K, V convert from bf16 exactly for 2^-17 <= |x| <= 65504 and for
+ * 0, and within 2^-25 below that (a value above 65504 records
+ * PRISM_ERR_RANGE in the workspace); the probabilities P (in [0, 256]
  * under the lazy rescaling) are rounded to fp16, 8x finer than bf16.
  * Returns PRISM_OK, PRISM_ERR_INVALID_ARG, PRISM_ERR_UNSUPPORTED,
  * PRISM_ERR_CAPACITY or PRISM_ERR_CUDA.
@@ -319,8 +320,8 @@ int prism_attn_bwd(const prism_params *p, const prism_plan_t *plan,
 /* Waits on `stream` and returns the status a kernel recorded in
  * `workspace`: PRISM_OK, PRISM_ERR_TIMEOUT, or PRISM_ERR_RANGE (an attention
  * call met a Q/K/V/dO value with |x| > 65504, the largest fp16 value; the
- * attention tensor-core operands are fp16, to which bf16 converts exactly in
- * that range), or PRISM_ERR_CUDA. */
+ * attention tensor-core operands are fp16, to which bf16 converts exactly
+ * for 2^-17 <= |x| <= 65504), or PRISM_ERR_CUDA. */
 int prism_workspace_status(const void *workspace, prism_stream_t stream);
 
 /* Message of the calling thread's last failing call ("" if none).  The

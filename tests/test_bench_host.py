@@ -9,7 +9,6 @@
 * The parsing of the nvidia-smi samples taken during the timed region, and
   the rule that a stored DRAM traffic figure is dropped once its kernel's
   source has changed."""
-import hashlib
 import json
 import types
 

@@ -2,7 +2,6 @@
 C ABI.  Indices (volumes, shapes, block table, permutation, selected key
 blocks) must be bit-exact; a difference is excluded only where the oracle's
 decision margin is <= 1e-6, and every exclusion is reported."""
-import math
 
 import numpy as np
 import pytest

@@ -4,8 +4,6 @@ and no data-path collective are involved (the path shards without exchange)."""
 import os
 import socket
 
-import pytest
-import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 

@@ -2,7 +2,6 @@
 than itself (closed forms, hand-worked values, invariants, brute force, or an
 independent formulation), so that a dropped term, a swapped axis or a wrong
 sign in the oracle fails here.  No GPU needed."""
-import itertools
 import math
 import os
 

@@ -5,9 +5,9 @@ a2v_norm -> plan -> select -> fwd -> bwd through the C ABI on one layer.
 The oracle cannot redo the whole layer in test time, so it checks samples
 it can compute one by one, stage-wise on the library's own plan and
 selection (as everywhere else):
-  * plan: one head in full (shapes, block table, permutation bit-exact,
+  * plan: every head in full (shapes, block table, permutation bit-exact,
     statistic values within rounding);
-  * selection: 64 sampled query blocks of one head, bit-exact except at
+  * selection: 32 sampled query blocks on every head, bit-exact except at
     logged ties;
   * forward: O and LSE of 8 sampled query blocks on each of two heads;
   * backward: dQ of 3 sampled query blocks per head, and dK, dV of the key
@@ -69,32 +69,42 @@ def _csc(S, h, j):
     return S["rows"][S["col_ptr"][c]:S["col_ptr"][c + 1]]
 
 
-def test_2k_plan_one_head_in_full():
-    S = _layer()
-    w, h = S["w"], HEADS[1]
-    ref = O.plan(S["host"][h]["V"][:, None], S["a"], w.T, w.H, w.W)
-    excluded = compare_plan(w, S["pl"], ref, [h])
-    print(f"2K plan: zone decisions excluded at ties {excluded}")
+def _head(S, h, names):
+    """Host copies (fp32) of one head's tensors, [N, 1, D] for the oracle."""
+    return [S["inp"][x][:, h:h + 1].float().cpu().numpy() for x in names]
 
 
-def test_2k_selection_sampled_rows():
+def test_2k_plan_every_head_in_full():
     S = _layer()
-    w, h = S["w"], HEADS[0]
-    ref_plan = oracle_plan_from_shapes(w.T, w.H, w.W, [S["shapes"][h]])
-    rng = np.random.default_rng(1)
-    rows = sorted(rng.choice(S["nb"][h], size=64, replace=False).tolist())
-    Q, K = S["host"][h]["Q"][:, None], S["host"][h]["K"][:, None]
-    ref = O.select(Q, K, ref_plan, w.topk_frac, w.topk_abs, w.top_p, scale_of(w.head_dim), rows=rows)
+    w = S["w"]
     excluded = 0
-    for (i, ids, info) in ref[0]:
-        got = _csr(S, h, i)
-        if got.size == ids.size and (got == ids).all():
-            continue
-        if info["p_margin"] <= TIE or info["score_gap"] <= TIE * max(1.0, abs(info["score_gap"])):
-            excluded += 1
-            continue
-        raise AssertionError(f"row {i}: got {got.size} ids, want {ids.size}; info {info}")
-    print(f"2K selection: {len(rows)} rows, excluded at ties {excluded}")
+    for h in range(w.heads):
+        (V,) = _head(S, h, ("V",))
+        ref = O.plan(V, S["a"], w.T, w.H, w.W)
+        excluded += compare_plan(w, S["pl"], ref, [h])
+    print(f"2K plan: {w.heads} heads in full, zone decisions excluded at ties {excluded}")
+
+
+def test_2k_selection_sampled_rows_on_every_head():
+    S = _layer()
+    w = S["w"]
+    rng = np.random.default_rng(1)
+    excluded = checked = 0
+    for h in range(w.heads):
+        ref_plan = oracle_plan_from_shapes(w.T, w.H, w.W, [S["shapes"][h]])
+        rows = sorted(rng.choice(S["nb"][h], size=32, replace=False).tolist())
+        Q, K = _head(S, h, ("Q", "K"))
+        ref = O.select(Q, K, ref_plan, w.topk_frac, w.topk_abs, w.top_p, scale_of(w.head_dim), rows=rows)
+        for (i, ids, info) in ref[0]:
+            checked += 1
+            got = _csr(S, h, i)
+            if got.size == ids.size and (got == ids).all():
+                continue
+            if info["p_margin"] <= TIE or info["score_gap"] <= TIE * max(1.0, abs(info["score_gap"])):
+                excluded += 1
+                continue
+            raise AssertionError(f"head {h} row {i}: got {got.size} ids, want {ids.size}; info {info}")
+    print(f"2K selection: {checked} rows over {w.heads} heads, excluded at ties {excluded}")
 
 
 def test_2k_forward_sampled_blocks():

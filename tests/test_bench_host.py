@@ -221,3 +221,25 @@ def test_selection_stats_match_the_oracle_rows(name):
     # the mean key share, weighted by block size, is the pair density
     Bq = np.array([opl.heads[h].blocks[i, 4] for h in range(w.heads) for (i, _, _) in osel[h]])
     assert (share * Bq).sum() * w.N == pytest.approx(bench.computed_pairs(p, pl, sel), rel=1e-12)
+
+
+def test_every_timed_kernel_has_a_roofline_spec_and_a_source():
+    """The kernel names come from the library (no CUDA call while nothing was
+    recorded); the bench must know each one, or its line would fail."""
+    import ctypes as C
+    from dynamic_block_sparse_stats_b200 import _lib
+    lib = _lib.load()
+    names = []
+    for i in range(_lib.KERNEL_TIMING_IDS):
+        n, ms, name = C.c_int(-1), C.c_double(-1.0), C.c_char_p()
+        assert lib.prism_kernel_timing_read(i, C.byref(n), C.byref(ms), C.byref(name)) == _lib.PRISM_OK
+        assert n.value == 0 and ms.value == 0.0
+        names.append(name.value.decode())
+    assert lib.prism_kernel_timing_read(_lib.KERNEL_TIMING_IDS, C.byref(n), C.byref(ms),
+                                        C.byref(name)) == _lib.PRISM_ERR_INVALID_ARG
+    assert len(set(names)) == len(names)
+    kt = {nm: (0, 0.0) for nm in names}
+    out = bench.kernel_rooflines(kt, 1e12, 128, 860160, 24, torch.tensor([100]), {"hbm_gbs": 1.0}, "measured", 1)
+    assert set(out) == set(names)
+    assert set(names) == set(bench.KERNEL_SOURCES)
+    assert set(bench.NCU_KERNEL_NAMES) <= set(names)

@@ -134,6 +134,7 @@ class _FakeLib:
 
     def __init__(self):
         self.calls = []
+        self.selects = 0
 
     def __getattr__(self, name):
         def f(*args):
@@ -144,7 +145,8 @@ class _FakeLib:
                 return b"fake"
             if name == "prism_select":
                 sel = args[4]._obj
-                first = sum(c[0] == "prism_select" for c in self.calls) == 1
+                self.selects += 1
+                first = self.selects == 1
                 sel.nnz = sel.cap + 5 if first else sel.cap
                 return 3 if first else 0
             return 0
@@ -208,3 +210,41 @@ def test_marshalling_through_a_fake_library(monkeypatch):
     with pytest.raises(ValueError, match="dQ must be torch.bfloat16"):
         api.attn_bwd(P, pl, sel, x["Q"], x["K"], x["V"], fw.O, x["dO"], fw.lse, out=(dQ, dK, dV))
     assert api.workspace_status(fw.ws) == 0
+
+
+def test_buffer_reuse_as_the_benchmark_step_does(monkeypatch):
+    """The benchmark allocates every output once, then passes the same buffers
+    to each call of its timed step; the binding must accept them and hand the
+    library the same pointers every time."""
+    import contextlib
+
+    from dynamic_block_sparse_stats_b200 import _lib
+    fake = _FakeLib()
+    monkeypatch.setattr(_lib, "load", lambda: fake)
+    monkeypatch.setattr(api, "_check_devices", lambda named: CPU)
+    monkeypatch.setattr(torch.cuda, "device", lambda d: contextlib.nullcontext())
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda d=None: _Stream())
+    x = {k: _bf16(N, HEADS, D) for k in ("Q", "K", "V", "dO")}
+    hhat = _bf16(N, 128)
+    a = api.a2v_norm(hhat)
+    pl = api.plan(P, x["V"], a)
+    sel = api.select(P, pl, x["Q"], x["K"])               # the fake grows it once
+    sel = api.select(P, pl, x["Q"], x["K"], cap=sel.nnz + 8)
+    fw = api.attn_fwd(P, pl, sel, x["Q"], x["K"], x["V"])
+    grads = api.attn_bwd(P, pl, sel, x["Q"], x["K"], x["V"], fw.O, x["dO"], fw.lse, O_res=fw.O_res)
+    bws = torch.empty(4096, dtype=torch.uint8)
+    fake.calls.clear()
+    for _ in range(2):                                   # the timed step, twice
+        assert api.a2v_norm(hhat, out=a) is a
+        assert api.plan(P, x["V"], a, out=pl) is pl
+        assert api.select(P, pl, x["Q"], x["K"], out=sel) is sel
+        f2 = api.attn_fwd(P, pl, sel, x["Q"], x["K"], x["V"], O=fw.O, lse=fw.lse, ws=fw.ws, O_res=fw.O_res)
+        assert f2.O is fw.O and f2.lse is fw.lse and f2.ws is fw.ws and f2.O_res is fw.O_res
+        g2 = api.attn_bwd(P, pl, sel, x["Q"], x["K"], x["V"], fw.O, x["dO"], fw.lse, out=grads, ws=bws,
+                          O_res=fw.O_res)
+        assert all(u is v for u, v in zip(g2, grads))
+    names = [c[0] for c in fake.calls]
+    assert names == ["prism_a2v_norm", "prism_plan", "prism_select", "prism_attn_fwd", "prism_attn_bwd"] * 2
+    bwd = [c[1] for c in fake.calls if c[0] == "prism_attn_bwd"]
+    assert bwd[0][14].value == bws.data_ptr() and bwd[0][15] == 4096
+    assert [t.value for t in bwd[0][10:13]] == [t.data_ptr() for t in grads]

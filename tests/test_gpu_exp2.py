@@ -1,7 +1,9 @@
-"""The FMA-pipe exponential that prism_attn_fwd uses for a quarter of its
-softmax weights, checked on the device against its stated error bound
-(relative error <= 7.5e-5 against exact 2^x, from the minimax fit of the
-polynomial) and against the MUFU exponential it stands in for."""
+"""The library's FMA-pipe exponential, which the attention kernels can use
+for a share of their softmax weights (they currently take all of them from
+MUFU, which measured faster), checked on the device against its stated
+error bound (relative error <= 7.5e-5 against exact 2^x, from the minimax
+fit of the polynomial) and against the MUFU exponential it would stand in
+for."""
 import ctypes as C
 
 import numpy as np

@@ -1,7 +1,8 @@
 // Diagnostics:
-//   * the FMA-pipe exponential the attention forward uses for a share of its
-//     softmax weights, exposed so that its error can be checked against exp2
-//     on the device;
+//   * the FMA-pipe exponential the attention kernels can use for a share of
+//     their softmax weights (they take all of them from MUFU today, which
+//     measured faster), exposed so that its error can be checked against
+//     exp2 on the device;
 //   * a self-test of the failure path every kernel wait takes: a wait on an
 //     mbarrier that nothing will complete gives up after a bounded number of
 //     cycles and records PRISM_ERR_TIMEOUT in the workspace status word,

@@ -122,6 +122,13 @@ def a2v_norm(hhat: torch.Tensor, out: torch.Tensor | None = None, stream=None) -
 
 @dataclass
 class Plan:
+    """Output of prism_plan (device tensors, Z zones, NB = N/64):
+    zone_shape u8 [heads, Z] candidate id per zone; zone_g f64 [heads, Z, 3]
+    (g_T, g_H, g_W); zone_rho f64 [heads, Z] normalised density; n_blocks
+    i32 [heads]; blocks i32 [heads, NB, 4] {first permuted position, volume,
+    natural index of the block's origin token, candidate id} (rows past
+    n_blocks unspecified); perm / inv_perm i32 [heads, N]; ws the call's
+    workspace."""
     p: PrismParams
     zone_shape: torch.Tensor
     zone_g: torch.Tensor
@@ -189,6 +196,11 @@ def plan(p: PrismParams, V: torch.Tensor, a: torch.Tensor | None = None, out: Pl
 
 @dataclass
 class Selection:
+    """Output of prism_select (device tensors): a CSR over rows h*NB + i
+    (head h, query block i) with row_ptr i32 [heads*NB + 1] and col i32
+    [capacity] (selected key blocks, ascending; the first nnz entries are
+    valid), and optionally its transpose col_ptr / row (needed by the
+    backward); ws the call's workspace."""
     p: PrismParams
     row_ptr: torch.Tensor
     col: torch.Tensor
@@ -282,6 +294,10 @@ def select(p: PrismParams, pl: Plan, Q: torch.Tensor, K: torch.Tensor, out: Sele
 
 @dataclass
 class FwdResult:
+    """Output of prism_attn_fwd: O bf16 [N, heads, D] (natural order), lse
+    f32 [heads, N] (natural log), ws the call's workspace (its status word
+    says whether a kernel recorded an error), O_res the bf16 rounding
+    residual of O, or None."""
     O: torch.Tensor
     lse: torch.Tensor
     ws: torch.Tensor

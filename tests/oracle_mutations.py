@@ -1,14 +1,17 @@
-"""Mutation check of the oracle's pins (not collected by pytest; run by hand).
+"""Mutation check of the oracle's pins and of the benchmark's host
+arithmetic (not collected by pytest; run by hand).
 
     python tests/oracle_mutations.py [mutation name ...]
 
-Each entry below plants one plausible mistake in the oracle: a dropped term,
-a wrong sign, index or axis, an off-by-one, a wrong tie-break or reading.
-For each entry the script copies the repository into a temporary directory,
-applies the mutation to the copy's oracle/prism_oracle.py and runs the CPU
+Each entry below plants one plausible mistake: in the oracle (M: a dropped
+term, a wrong sign, index or axis, an off-by-one, a wrong tie-break or
+reading) or in bench.py's host logic (BENCH: the pair count, the roofline
+arithmetic, the sample extrapolation, the traffic digest, clock parsing,
+rank reductions).  For each entry the script copies the repository into a
+temporary directory, applies the mutation to the copy and runs the CPU
 suite (-m "not gpu", stopping at the first failure) on the copy.  A mutation
-that no test catches marks a missing pin.  The repository itself is never
-modified.  A full run takes about 15 minutes on 8 cores; it exits 1 if any
+that no test catches marks a missing test.  The repository itself is never
+modified.  A full run takes about 20 minutes on 8 cores; it exits 1 if any
 mutation survives.
 """
 import os
@@ -72,35 +75,58 @@ M = [
 ]
 
 
+BENCH = [
+ ("pairs: wrong head offset", "Bk = Bsz[head_of * NB + col]", "Bk = Bsz[col]"),
+ ("pairs: query size from the key", "return int((Bq[row_of] * Bk).sum().item())", "return int((Bk * Bk).sum().item())"),
+ ("roofline: work not scaled by steps", "per_launch = work * steps / n", "per_launch = work / n"),
+ ("roofline: fp32 peak counts FMA twice", "rec[\"peak\"] = 148 * 128 * peaks", "rec[\"peak\"] = 148 * 256 * peaks"),
+ ("roofline: fwd work 2PD", "\"attn_fwd\": (\"tensor\", 4.0 * P * D,", "\"attn_fwd\": (\"tensor\", 2.0 * P * D,"),
+ ("whole-job rate of one rank", "return world * units_per_rank / (ms_max * 1e-3)", "return units_per_rank / (ms_max * 1e-3)"),
+ ("head ranges ignore the remainder", "h0 = rank * base + min(rank, extra)", "h0 = rank * base"),
+ ("max over ranks sums", "torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)", "torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)"),
+ ("sample: row fraction inverted", "row_frac = nb / len(sel_rows)", "row_frac = len(sel_rows) / nb"),
+ ("sample: pairs not scaled to the heads", "P_total = pairs_rows * row_frac * w.heads", "P_total = pairs_rows * row_frac"),
+ ("selection share over 2N", "\"key_share_per_row\": summary(keys[valid] / N)}", "\"key_share_per_row\": summary(keys[valid] / (2 * N))}"),
+ ("selection counts every row", "\"blocks_per_row\": summary(counts[valid].double())", "\"blocks_per_row\": summary(counts.double())"),
+ ("digest keeps comments", "            i = n if j < 0 else j\n", "            out.append(text[i:n if j < 0 else j])\n            i = n if j < 0 else j\n"),
+ ("digest ignores includes", "            todo.append(os.path.normpath(os.path.join(os.path.dirname(path), inc)))", "            pass"),
+ ("stale traffic still reported", "        if source_digest(d[\"source\"]) != d[\"code_digest\"]:", "        if False:"),
+ ("clock median as mean", "return {\"sm_mhz\": statistics.median(sm) if sm else None", "return {\"sm_mhz\": statistics.mean(sm) if sm else None"),
+ ("throttle reasons ignored", "                if v.strip().lower() == \"active\":", "                if False:"),
+]
+
 def main(only):
     tmp = tempfile.mkdtemp(prefix="oracle_mutations_")
     dst = os.path.join(tmp, "repo")
     try:
         shutil.copytree(ROOT, dst, ignore=shutil.ignore_patterns(".git", "_build", "gpurun_out", "_work",
                                                                  "__pycache__", "baseline"))
-        path = os.path.join(dst, "oracle", "prism_oracle.py")
-        with open(path) as f:
-            orig = f.read()
         survivors = []
-        for name, old, new in M:
-            if only and name not in only:
-                continue
-            if orig.count(old) != 1:
-                print(f"SKIP     {name}: pattern found {orig.count(old)} times")
-                continue
+        for target, entries in (("oracle/prism_oracle.py", M), ("bench.py", BENCH)):
+            path = os.path.join(dst, target)
+            with open(path) as f:
+                orig = f.read()
+            for name, old, new in entries:
+                if only and name not in only:
+                    continue
+                if orig.count(old) != 1:
+                    print(f"SKIP     {name}: pattern found {orig.count(old)} times in {target}")
+                    continue
+                with open(path, "w") as f:
+                    f.write(orig.replace(old, new))
+                t = time.time()
+                r = subprocess.run([sys.executable, "-m", "pytest", "tests", "-x", "-q", "-m", "not gpu",
+                                    "-p", "no:cacheprovider", "--deselect",
+                                    "tests/test_bench_reference_cpu.py::"
+                                    "test_reference_arm_under_torchrun_prints_one_line_from_rank_zero"],
+                                   cwd=dst, capture_output=True, text=True)
+                failed = [ln for ln in r.stdout.splitlines() if ln.startswith(("FAILED", "ERROR"))][:1]
+                if r.returncode == 0:
+                    survivors.append(name)
+                print(f"{'caught  ' if r.returncode else 'SURVIVED'} {name:38s} {time.time() - t:5.1f}s {failed}",
+                      flush=True)
             with open(path, "w") as f:
-                f.write(orig.replace(old, new))
-            t = time.time()
-            r = subprocess.run([sys.executable, "-m", "pytest", "tests", "-x", "-q", "-m", "not gpu",
-                                "-p", "no:cacheprovider", "--deselect",
-                                "tests/test_bench_reference_cpu.py::"
-                                "test_reference_arm_under_torchrun_prints_one_line_from_rank_zero"],
-                               cwd=dst, capture_output=True, text=True)
-            failed = [ln for ln in r.stdout.splitlines() if ln.startswith(("FAILED", "ERROR"))][:1]
-            if r.returncode == 0:
-                survivors.append(name)
-            print(f"{'caught  ' if r.returncode else 'SURVIVED'} {name:34s} {time.time() - t:5.1f}s {failed}",
-                  flush=True)
+                f.write(orig)
         print("survivors:", survivors)
         return 1 if survivors else 0
     finally:

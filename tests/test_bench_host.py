@@ -79,6 +79,27 @@ def test_computed_pairs_equals_the_dense_mask_count(name):
     assert 0 < got <= w.N * w.N * w.heads
 
 
+def test_computed_pairs_with_a_different_block_table_per_head():
+    """Two heads with different plans (all-256 blocks vs all-64 blocks) and
+    random selections: each key's size must come from its own head's table."""
+    T, H, W = 8, 16, 16
+    w = types.SimpleNamespace(T=T, H=H, W=W, N=T * H * W, heads=2)
+    rng = np.random.default_rng(4)
+    opl = O.Plan(T, H, W)
+    osel = []
+    for sid in (13, 0):                      # (4,8,8) volume 256, then (2,4,8) volume 64
+        shapes = np.full(4, sid)
+        blocks = O.head_blocks(T, H, W, shapes)
+        opl.heads.append(O.HeadPlan(None, shapes, None, None, None, None, blocks,
+                                    O.permutation(T, H, W, blocks)))
+        nb = blocks.shape[0]
+        osel.append([(i, np.sort(rng.choice(nb, size=int(rng.integers(1, nb + 1)), replace=False)), {})
+                     for i in range(nb)])
+    pl, sel = _library_layout(w, opl, osel)
+    got = bench.computed_pairs(types.SimpleNamespace(T=T, H=H, W=W, heads=2), pl, sel)
+    assert got == _dense_mask_pairs(w, opl, osel)
+
+
 def test_kernel_roofline_arithmetic():
     peaks = {"hbm_gbs": 6000.0, "bf16_tflops_sustained": 1000.0, "sm_max_mhz": 2000.0}
     P, D, N, h, steps = 1.0e12, 128, 860160, 24, 2
@@ -115,10 +136,11 @@ def test_clock_samples_are_parsed():
     c = bench.ClockSampler(0)
     c.proc = _FakeProc("0, 1600, 1965, 700.5, 0x4, Not Active, Not Active, Not Active, Active\n"
                        "0, 1700, 1965, 710.0, 0x0, Not Active, Not Active, Not Active, Not Active\n"
+                       "0, 1000, 1965, 300.0, 0x0, Not Active, Not Active, Not Active, Not Active\n"
                        "0, [N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active\n"
                        "garbage line\n")
-    r = c.stop()
-    assert r == {"sm_mhz": 1650.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 2}
+    r = c.stop()        # the median of three samples (the mean would be 1433)
+    assert r == {"sm_mhz": 1600.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
     c = bench.ClockSampler(0)
     c.proc = _FakeProc("0, 1200, 1965, 900, 0x40, Not Active, Active, Not Active, Not Active\n")
     assert c.stop()["reasons"] == ["hw_thermal_slowdown"]

@@ -104,3 +104,18 @@ def test_heads_are_independent_in_the_oracle():
     s_part = O.select(Q[:, 2:4], K[:, 2:4], part, 0.1, 0, 0.9)
     for a_, b_ in zip(s_full, s_part):
         assert all(np.array_equal(x[1], y[1]) for x, y in zip(a_, b_))
+
+
+def test_head_ranges_tile_the_heads_with_a_remainder():
+    """Contiguous, balanced, disjoint ranges covering every head, also when
+    the ranks do not divide the heads (the first `heads % world` ranks take
+    one more)."""
+    import bench
+    for heads in (1, 5, 7, 24, 25):
+        for world in range(1, min(heads, 8) + 1):
+            ranges = [bench.head_range(r, world, heads) for r in range(world)]
+            assert ranges[0][0] == 0 and ranges[-1][1] == heads
+            assert all(ranges[r][1] == ranges[r + 1][0] for r in range(world - 1))
+            sizes = [b - a for a, b in ranges]
+            assert max(sizes) - min(sizes) <= 1 and sizes == sorted(sizes, reverse=True)
+    assert [bench.head_range(r, 3, 5) for r in range(3)] == [(0, 2), (2, 4), (4, 5)]

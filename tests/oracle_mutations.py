@@ -5,9 +5,9 @@ arithmetic (not collected by pytest; run by hand).
 
 Each entry below plants one plausible mistake: in the oracle (M: a dropped
 term, a wrong sign, index or axis, an off-by-one, a wrong tie-break or
-reading) or in bench.py's host logic (BENCH: the pair count, the roofline
+reading), in bench.py's host logic (BENCH: the pair count, the roofline
 arithmetic, the sample extrapolation, the traffic digest, clock parsing,
-rank reductions).  For each entry the script copies the repository into a
+rank reductions) or in the binding's checks (BINDING).  For each entry the script copies the repository into a
 temporary directory, applies the mutation to the copy and runs the CPU
 suite (-m "not gpu", stopping at the first failure) on the copy.  A mutation
 that no test catches marks a missing test.  The repository itself is never
@@ -95,6 +95,20 @@ BENCH = [
  ("throttle reasons ignored", "                if v.strip().lower() == \"active\":", "                if False:"),
 ]
 
+BINDING = [
+ ("binding: shape unchecked", "    if tuple(t.shape) != tuple(shape):\n        raise", "    if False:\n        raise"),
+ ("binding: dtype unchecked", "    if t.dtype != dtype:\n        raise", "    if False:\n        raise"),
+ ("binding: grid unchecked", "    if _grid(p) != _grid(q):", "    if False:"),
+ ("binding: host tensors accepted", "        if not t.is_cuda:\n            raise", "        if False:\n            raise"),
+ ("binding: capacity unchecked", "    if not 0 <= sel.nnz <= cap:", "    if False:"),
+ ("binding: transpose not required", "    elif transpose:\n        raise", "    elif False:\n        raise"),
+ ("binding: caller's stream ignored", "    s = stream if stream is not None else torch.cuda.current_stream(device)",
+  "    s = torch.cuda.current_stream(device)"),
+ ("binding: no growth on short capacity", "out.col.numel() < cs.nnz <= 0x7fffffff", "False"),
+ ("binding: residual always passed", "_ptr(O_res) if residual else None, _ptr(lse)", "_ptr(O_res), _ptr(lse)"),
+ ("binding: gradients in the wrong order", "_ptr(dQ), _ptr(dK), _ptr(dV)", "_ptr(dK), _ptr(dQ), _ptr(dV)"),
+]
+
 def main(only):
     tmp = tempfile.mkdtemp(prefix="oracle_mutations_")
     dst = os.path.join(tmp, "repo")
@@ -102,7 +116,8 @@ def main(only):
         shutil.copytree(ROOT, dst, ignore=shutil.ignore_patterns(".git", "_build", "gpurun_out", "_work",
                                                                  "__pycache__", "baseline"))
         survivors = []
-        for target, entries in (("oracle/prism_oracle.py", M), ("bench.py", BENCH)):
+        for target, entries in (("oracle/prism_oracle.py", M), ("bench.py", BENCH),
+                                 ("dynamic_block_sparse_stats_b200/api.py", BINDING)):
             path = os.path.join(dst, target)
             with open(path) as f:
                 orig = f.read()

@@ -248,3 +248,33 @@ def test_buffer_reuse_as_the_benchmark_step_does(monkeypatch):
     bwd = [c[1] for c in fake.calls if c[0] == "prism_attn_bwd"]
     assert bwd[0][14].value == bws.data_ptr() and bwd[0][15] == 4096
     assert [t.value for t in bwd[0][10:13]] == [t.data_ptr() for t in grads]
+
+
+def test_explicit_stream_and_no_residual(monkeypatch):
+    """A stream passed by the caller reaches the library (not the current
+    one), and residual=False passes a NULL O_res."""
+    import contextlib
+
+    from dynamic_block_sparse_stats_b200 import _lib
+    fake = _FakeLib()
+    monkeypatch.setattr(_lib, "load", lambda: fake)
+    monkeypatch.setattr(api, "_check_devices", lambda named: CPU)
+    monkeypatch.setattr(torch.cuda, "device", lambda d: contextlib.nullcontext())
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda d=None: _Stream())
+
+    class Mine:
+        cuda_stream = 777
+
+    x = {k: _bf16(N, HEADS, D) for k in ("Q", "K", "V")}
+    a = api.a2v_norm(_bf16(N, 64), stream=Mine())
+    assert fake.calls[-1][1][5] == 777
+    pl = api.plan(P, x["V"], a, stream=Mine())
+    assert fake.calls[-1][1][6] == 777
+    sel = api.select(P, pl, x["Q"], x["K"], cap=10 ** 4, stream=Mine())
+    assert fake.calls[-1][1][7] == 777
+    fw = api.attn_fwd(P, pl, sel, x["Q"], x["K"], x["V"], residual=False, stream=Mine())
+    name, args = fake.calls[-1]
+    assert name == "prism_attn_fwd" and args[7] is None and args[11] == 777 and fw.O_res is None
+    # a residual buffer handed over with residual=False is not written
+    fw = api.attn_fwd(P, pl, sel, x["Q"], x["K"], x["V"], O_res=_bf16(N, HEADS, D), residual=False)
+    assert fake.calls[-1][1][7] is None and fw.O_res is None

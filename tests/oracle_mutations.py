@@ -7,11 +7,12 @@ Each entry below plants one plausible mistake: in the oracle (M: a dropped
 term, a wrong sign, index or axis, an off-by-one, a wrong tie-break or
 reading), in bench.py's host logic (BENCH: the pair count, the roofline
 arithmetic, the sample extrapolation, the traffic digest, clock parsing,
-rank reductions) or in the binding's checks (BINDING).  For each entry the script copies the repository into a
+rank reductions), in the binding's checks (BINDING) or in the C ABI's
+argument validation (CABI; the copy's library is rebuilt for each).  For each entry the script copies the repository into a
 temporary directory, applies the mutation to the copy and runs the CPU
 suite (-m "not gpu", stopping at the first failure) on the copy.  A mutation
 that no test catches marks a missing test.  The repository itself is never
-modified.  A full run takes about 20 minutes on 8 cores; it exits 1 if any
+modified.  A full run takes about 30 minutes on 8 cores; it exits 1 if any
 mutation survives.
 """
 import os
@@ -109,6 +110,29 @@ BINDING = [
  ("binding: gradients in the wrong order", "_ptr(dQ), _ptr(dK), _ptr(dV)", "_ptr(dK), _ptr(dQ), _ptr(dV)"),
 ]
 
+CABI = [  # (file under the package's csrc/, name, old, new); the copy's library is rebuilt for each
+ ("api.cu", "C: zone edge unchecked", "if (p->T % 8 || p->H % 8 || p->W % 8)", "if (false)"),
+ ("api.cu", "C: head_dim 96 accepted", "if (p->head_dim != 64 && p->head_dim != 128)", "if (false)"),
+ ("api.cu", "C: grid size unchecked", "if (N * p->heads * p->head_dim >= (1LL << 40) || N >= (1LL << 30))", "if (false)"),
+ ("api.cu", "C: thresholds unchecked", "if (!(p->tau128 >= p->tau256) || !(p->tau256 >= 0.f) || !isfinite(p->tau128))", "if (false)"),
+ ("api.cu", "C: eps unchecked", "if (!(p->eps > 0.f) || !isfinite(p->eps))", "if (false)"),
+ ("api.cu", "C: top_p unchecked", "if (!(p->top_p >= 0.f) || !isfinite(p->top_p))", "if (false)"),
+ ("api.cu", "C: top-k unchecked", "if (p->topk_abs < 0 || !(p->topk_frac >= 0.f) || !isfinite(p->topk_frac))", "if (false)"),
+ ("api.cu", "C: sm_scale unchecked", "if (p->sm_scale < 0.f || !isfinite(p->sm_scale))", "if (false)"),
+ ("api.cu", "C: map_exponent unchecked", "if (!(p->map_exponent >= 0.f && p->map_exponent <= 8.f))", "if (false)"),
+ ("api.cu", "C: guidance unchecked", "if (p->guidance < 0 || p->guidance > 3)", "if (false)"),
+ ("api.cu", "C: density unchecked", "if (p->density < 0 || p->density > 3)", "if (false)"),
+ ("api.cu", "C: alignment unchecked", "if (reinterpret_cast<uintptr_t>(ptr) % 16) return fail(", "if (false) return fail("),
+ ("api.cu", "C: workspace size unchecked", "if (bytes < need) return fail(", "if (false) return fail("),
+ ("api.cu", "C: workspace alignment unchecked", "if (reinterpret_cast<uintptr_t>(ws) % 256)", "if (false)"),
+ ("api.cu", "C: density 3 without norms", "if (p->density == 3 && !a2v_norm)", "if (false)"),
+ ("api.cu", "C: backward without transpose", "if (!sel || !sel->row_ptr || !sel->col || !sel->col_ptr || !sel->row)", "if (!sel || !sel->row_ptr || !sel->col)"),
+ ("a2v_norm.cu", "C: a2v width not a multiple of 8", "if (width <= 0 || width % 8 || width > (1 << 20))", "if (width <= 0 || width > (1 << 20))"),
+ ("a2v_norm.cu", "C: a2v ld below width", "if (ld < width || ld % 8)", "if (ld % 8)"),
+ ("a2v_norm.cu", "C: a2v negative n", "if (n < 0) return", "if (false) return"),
+ ("timing.cu", "C: timing id unchecked", "if (id < 0 || id >= KT_COUNT) return", "if (false) return"),
+]
+
 def main(only):
     tmp = tempfile.mkdtemp(prefix="oracle_mutations_")
     dst = os.path.join(tmp, "repo")
@@ -142,6 +166,37 @@ def main(only):
                       flush=True)
             with open(path, "w") as f:
                 f.write(orig)
+        csrc = os.path.join(dst, "dynamic_block_sparse_stats_b200", "csrc")
+        build = [sys.executable, "-m", "dynamic_block_sparse_stats_b200.build", "--force"]
+        for fname, name, old, new in CABI:
+            if only and name not in only:
+                continue
+            path = os.path.join(csrc, fname)
+            with open(path) as f:
+                orig = f.read()
+            if orig.count(old) != 1:
+                print(f"SKIP     {name}: pattern found {orig.count(old)} times in {fname}")
+                continue
+            with open(path, "w") as f:
+                f.write(orig.replace(old, new))
+            t = time.time()
+            b = subprocess.run(build, cwd=dst, capture_output=True, text=True)
+            if b.returncode != 0:
+                print(f"NOBUILD  {name}")
+            else:
+                r = subprocess.run([sys.executable, "-m", "pytest", "tests", "-x", "-q", "-m", "not gpu",
+                                    "-p", "no:cacheprovider", "--deselect",
+                                    "tests/test_bench_reference_cpu.py::"
+                                    "test_reference_arm_under_torchrun_prints_one_line_from_rank_zero"],
+                                   cwd=dst, capture_output=True, text=True)
+                failed = [ln for ln in r.stdout.splitlines() if ln.startswith(("FAILED", "ERROR"))][:1]
+                if r.returncode == 0:
+                    survivors.append(name)
+                print(f"{'caught  ' if r.returncode else 'SURVIVED'} {name:38s} {time.time() - t:5.1f}s {failed}",
+                      flush=True)
+            with open(path, "w") as f:
+                f.write(orig)
+            subprocess.run(build, cwd=dst, capture_output=True, text=True)
         print("survivors:", survivors)
         return 1 if survivors else 0
     finally:

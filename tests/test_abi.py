@@ -45,6 +45,14 @@ def test_struct_layouts_match_header():
     (dict(map_exponent=9.0), _lib.PRISM_ERR_INVALID_ARG),
     (dict(guidance=4), _lib.PRISM_ERR_INVALID_ARG),
     (dict(density=4), _lib.PRISM_ERR_INVALID_ARG),
+    (dict(eps=0.0), _lib.PRISM_ERR_INVALID_ARG),
+    (dict(topk_abs=-1), _lib.PRISM_ERR_INVALID_ARG),
+    (dict(topk_frac=-0.1), _lib.PRISM_ERR_INVALID_ARG),
+    (dict(sm_scale=-1.0), _lib.PRISM_ERR_INVALID_ARG),
+    (dict(top_p=float("nan")), _lib.PRISM_ERR_INVALID_ARG),
+    (dict(tau128=float("nan")), _lib.PRISM_ERR_INVALID_ARG),
+    (dict(T=1024, H=1024, W=1024), _lib.PRISM_ERR_UNSUPPORTED),     # N = 2^30 tokens
+    (dict(W=0), _lib.PRISM_ERR_INVALID_ARG),
 ])
 def test_invalid_params_are_rejected_before_any_cuda_call(bad, code):
     lib = _lib.load()

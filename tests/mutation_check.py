@@ -1,7 +1,7 @@
 """Mutation check of the oracle's pins and of the benchmark's host
 arithmetic (not collected by pytest; run by hand).
 
-    python tests/oracle_mutations.py [mutation name ...]
+    python tests/mutation_check.py [mutation name ...]
 
 Each entry below plants one plausible mistake: in the oracle (M: a dropped
 term, a wrong sign, index or axis, an off-by-one, a wrong tie-break or
@@ -134,7 +134,7 @@ CABI = [  # (file under the package's csrc/, name, old, new); the copy's library
 ]
 
 def main(only):
-    tmp = tempfile.mkdtemp(prefix="oracle_mutations_")
+    tmp = tempfile.mkdtemp(prefix="mutation_check_")
     dst = os.path.join(tmp, "repo")
     try:
         shutil.copytree(ROOT, dst, ignore=shutil.ignore_patterns(".git", "_build", "gpurun_out", "_work",

@@ -27,9 +27,11 @@ Readings of points the pages leave open are marked READING where they are
 applied; each states the choice and why.
 
 Parity status: every function below is pinned by a ``-m "not gpu"`` test
-(closed forms, invariants, brute force, independent dense formulations).
-Agreement with the authors' own implementation on the READING points is
-unpinned (no implementation is available).
+(closed forms, invariants, brute force, independent dense formulations);
+tests/mutation_check.py plants plausible mistakes in a copy of this module
+and confirms that each one fails a test.  Agreement with the authors' own
+implementation on the READING points is unpinned (no implementation is
+available).
 """
 from __future__ import annotations
 

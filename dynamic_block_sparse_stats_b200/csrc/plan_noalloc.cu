@@ -6,6 +6,8 @@
 #include <stdio.h>
 
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "internal.h"
 
@@ -16,30 +18,65 @@ namespace {
 // needs about 1.8 MiB; this holds a bit more than twice that.
 constexpr size_t kNoAllocScratchBytes = 4u << 20;
 
-// Every GPU that loads the library reserves this array until the process
-// exits.  Host code may not use its name as a device address: the address is
-// fetched per device with cudaGetSymbolAddress below.
+// Every CUDA context that loads the library reserves this array until the
+// context is destroyed (for the primary context: until the process exits).
+// Host code may not use its name as a device address: the address is fetched
+// per context with cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_plan_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 256;
-std::mutex g_mu;
-void *g_scratch_addr[kMaxDevices] = {};
+// A __device__ array exists once per CUDA context that loaded the library's
+// module, not once per device: a second context on the same device
+// (cuCtxCreate) has its own copy at another address, and so has the primary
+// context that the runtime creates again after cudaDeviceReset.  The address
+// is therefore cached per context, keyed by the context's id (cuCtxGetId: an
+// id is never reused within a process, unlike a context handle).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
 
-// Device address of g_plan_scratch on the current device, looked up once per
-// device (with that device current) and cached.
+std::mutex g_mu;
+std::vector<std::pair<unsigned long long, void *>> g_scratch_addr;  // (context id, address)
+
+template <typename F>
+F driver_entry(const char *name) {
+  void *fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &fn, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<F>(fn);
+}
+
+// Id of the context current on this thread, or false when the driver cannot
+// say (no context current, or a driver without cuCtxGetId).
+bool current_context_id(unsigned long long *id) {
+  static CtxGetCurrentFn get_current = driver_entry<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static CtxGetIdFn get_id = driver_entry<CtxGetIdFn>("cuCtxGetId");
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of g_plan_scratch in the context current on this thread.
+// The first call in a context looks it up with cudaGetSymbolAddress (which
+// also sets up the runtime's context on a thread that has none yet); later
+// calls in the same context take it from the cache.
 cudaError_t scratch_address(void **out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  unsigned long long id = 0;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
-    void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_plan_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
+  if (current_context_id(&id)) {
+    for (const auto &e : g_scratch_addr)
+      if (e.first == id) {
+        *out = e.second;
+        return cudaSuccess;
+      }
   }
-  *out = g_scratch_addr[dev];
+  void *p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_plan_scratch);
+  if (e != cudaSuccess) return e;
+  // key by the context the lookup ran in (the runtime may only now have made
+  // its context current); without an id the address is simply not cached
+  if (current_context_id(&id)) g_scratch_addr.emplace_back(id, p);
+  *out = p;
   return cudaSuccess;
 }
 

@@ -194,19 +194,23 @@ int prism_plan(const prism_params *p, const uint16_t *V, const float *a2v_norm,
  * and some code may not pay the implicit device synchronisation of
  * cudaMalloc; neither can provide prism_plan's workspace.  This call needs
  * none: its scratch is a 4 MiB array in the library's device memory, which
- * every GPU that loads the library holds until the process exits.  The
+ * every CUDA context that loads the library holds until the context is
+ * destroyed (the runtime's primary context: until the process exits).  The
  * pages have no counterpart; it is an interface convenience.
  *   Inputs and outputs as prism_plan (the caller still passes V, a2v_norm and
  *   the arrays of `out`).
  *   Limit: grids whose scratch (heads*Z*44 bytes + Z*32 + 1 KiB, about
  *   1.8 MiB for the 2K grid with 24 heads) exceeds 4 MiB are rejected with
  *   PRISM_ERR_CAPACITY and a message; use prism_plan for those.
- *   The first call on a device looks up the array's device address with
- *   that device current and caches it; make that first call before any
- *   stream capture.  All calls in the process share the one array and it
- *   keeps the last call's contents (the call clears what must start at
- *   zero), so calls whose kernels overlap on the GPU race: serialise them
- *   (one stream, or events between streams).
+ *   The array exists once per CUDA context (a second context on the same
+ *   device, or the primary context created again after cudaDeviceReset,
+ *   has its own copy at another address).  The first call in a context
+ *   looks up that context's address (cudaGetSymbolAddress, with the
+ *   context current) and caches it under the context's id; make that first
+ *   call before any stream capture.  All calls in one context share its
+ *   array, which keeps the last call's contents (the call clears what must
+ *   start at zero), so calls whose kernels overlap on the GPU race:
+ *   serialise them (one stream, or events between streams).
  * Returns PRISM_OK, PRISM_ERR_INVALID_ARG, PRISM_ERR_UNSUPPORTED,
  * PRISM_ERR_CAPACITY or PRISM_ERR_CUDA.
  */

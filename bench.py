@@ -187,59 +187,124 @@ def read_kernel_times(lib):
     return out
 
 
-def kernel_rooflines(ktimes, P, D, N, h, nb, peaks, peak_src, steps):
+def kernel_rooflines(ktimes, P, D, N, h, nb, peaks, peak_src, steps, nnz=0, sm_mhz=None):
     """Per kernel: launches, ms per launch (CUDA events on the launching
     stream, timed region), algorithmic work per launch and its fraction of the
-    measured peak (sustained bf16 for tensor kernels inside this long step;
-    the STREAM copy bandwidth for HBM-bound kernels)."""
-    tensor_peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    measured peak: bf16 (sustained, for tensor kernels inside this long step;
+    the burst figure is reported beside it) or the STREAM copy bandwidth for
+    HBM-bound kernels.  `work` is per step; kernels launched several times per
+    step (once per head, or in both the forward and the backward) share it
+    evenly.  The backward's two kernels are also reported together as
+    `attn_bwd` on the FlashAttention convention, 10*P*D FLOP per layer: dK/dV
+    does 8*P*D of it (S^T, dP^T, dV, dK), dQ the remaining 2*P*D (dQ = dS K);
+    dQ's recomputed S and dP (4*P*D more) are issued work, reported as
+    `issued_TFLOPs`, not algorithmic work."""
+    sustained = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    burst = peaks.get("bf16_tflops", sustained)
     hbm = peaks["hbm_gbs"]
     sum_nb2 = float((nb.double() ** 2).sum().item())
+    sum_nb = float(nb.double().sum().item())
+    Z = N // 512
+    HBD, HN = float(N) * h * D, float(N) * h
     spec = {
-        # name: (bound, work per step, unit, description)
-        "attn_fwd": ("tensor", 4.0 * P * D, "TFLOP/s", "4*P*D FLOP (QK^T and PV on the computed pairs)"),
-        "attn_bwd_dkdv": ("tensor", 8.0 * P * D, "TFLOP/s", "8*P*D FLOP (S^T, dP^T, dV, dK on the computed pairs)"),
-        "attn_bwd_dq": ("tensor", 6.0 * P * D, "TFLOP/s", "6*P*D FLOP (S, dP, dQ on the computed pairs)"),
-        "zone_video_stats": ("hbm", 2.0 * N * h * D, "GB/s", "one read of V: 2*N*h*D bytes"),
-        "block_mean": ("hbm", 4.0 * N * h * D, "GB/s", "one read of Q and K: 4*N*h*D bytes"),
-        "block_score": ("alu", 2.0 * D * sum_nb2, "TFLOP/s", "2*D*sum_h Nb^2 fp32 FLOP (mul + add)"),
-        "select_row": ("alu", None, None, "per-row radix selection over N_b scores"),
-        "a2v_norm": ("hbm", 2.0 * N * h * D + 4.0 * N, "GB/s",
+        # name: (bound, algorithmic work per step, issued work per step or None, description)
+        "attn_fwd": ("tensor", 4.0 * P * D, None, "4*P*D FLOP (QK^T and PV on the computed pairs)"),
+        "attn_bwd_dkdv": ("tensor", 8.0 * P * D, None, "8*P*D FLOP (S^T, dP^T, dV, dK on the computed pairs)"),
+        "attn_bwd_dq": ("tensor", 2.0 * P * D, 6.0 * P * D,
+                        "2*P*D FLOP algorithmic (dQ = dS K); 6*P*D issued (S and dP recomputed)"),
+        "zone_video_stats": ("hbm", 2.0 * HBD, None, "one read of V: 2*N*h*D bytes"),
+        "zone_a2v_stats": ("hbm", 4.0 * N, None, "one read of the A2V map: 4*N bytes"),
+        "plan_finalize": ("hbm", h * Z * 77.0 + 32.0 * Z + 16.0 * sum_nb, None,
+                          "zone statistics in, plan tables out: h*Z*77 + 32*Z + 16*sum(N_b) bytes "
+                          "(one CTA per head: latency-bound)"),
+        "perm": ("hbm", 8.0 * HN + h * Z, None, "perm and inv_perm written: 8*N*h bytes"),
+        "block_mean": ("hbm", 4.0 * HBD, None, "one read of Q and K: 4*N*h*D bytes"),
+        "block_score": ("alu", 2.0 * D * sum_nb2, None, "2*D*sum_h Nb^2 fp32 FLOP (mul + add)"),
+        "select_row": ("hbm", 4.0 * sum_nb2, None, "one read of the fp32 score rows: 4*sum_h Nb^2 bytes"),
+        "select_scan": ("hbm", 8.0 * h * (N // 64), None, "row counts in, row offsets out: 8*h*NB bytes"),
+        "csr_fill": ("hbm", 4.0 * sum_nb2 + 4.0 * nnz, None, "score rows read, column ids written: "
+                                                          "4*sum_h Nb^2 + 4*nnz bytes"),
+        "csc_count": ("hbm", 8.0 * nnz, None, "column ids read, column counts incremented: 8*nnz bytes"),
+        "csc_scan": ("hbm", 8.0 * h * (N // 64), None, "column counts in, offsets out: 8*h*NB bytes"),
+        "csc_fill": ("hbm", 12.0 * nnz, None, "CSR read, transpose written: 12*nnz bytes"),
+        "csc_sort": ("hbm", 8.0 * nnz, None, "each transposed column read and written: 8*nnz bytes"),
+        "permute3": ("hbm", 2 * (12.0 * HBD + 4.0 * HN), None,
+                     "per launch three bf16 tensors read and written as fp16 (12*N*h*D bytes) + perm (4*N*h); "
+                     "launched in the forward and the backward"),
+        "unit_block": ("hbm", 2 * (16.0 * sum_nb + 4.0 * HN / 64), None,
+                       "block table read, unit->block map written (forward and backward)"),
+        "tile_units": ("hbm", 3 * 12.0 * nnz, None,
+                       "per launch the selection's ids and the block sizes they index (about 12*nnz bytes; "
+                       "one launch in the forward, two in the backward)"),
+        "bwd_prep": ("hbm", 8.0 * HBD + 16.0 * HN, None,
+                     "dO, O, O_res read, fp16 dO written (8*N*h*D bytes) + LSE, Delta (16*N*h)"),
+        "a2v_norm": ("hbm", 2.0 * HBD + 4.0 * N, None,
                      "one read of the bridge output (2*N*h*D bytes) + the fp32 norms (4*N)"),
     }
+    # nominal dense bf16 rate at the sampled SM clock: 148 SMs x 8192 FLOP per clock
+    at_clock = 148 * 8192 * sm_mhz * 1e6 / 1e12 if sm_mhz else None
     out = {}
     for name, (n, ms) in ktimes.items():
-        bound, work, unit, desc = spec[name]
+        bound, work, issued, desc = spec[name]
         rec = {"launches": n, "total_ms": ms, "ms_per_launch": ms / n if n else None, "bound": bound,
-               "algorithmic": desc, "unit": unit, "achieved": None, "peak": None, "frac": None, "peak_source": None}
-        if n and work is not None:
-            # `work` is per step; kernels launched once per head per step share
-            # it evenly
+               "algorithmic": desc, "unit": None, "achieved": None, "peak": None, "frac": None, "peak_source": None}
+        if n and work is not None and ms > 0:
             per_launch = work * steps / n
             sec = (ms / n) * 1e-3
             if bound == "tensor":
+                rec["unit"] = "TFLOP/s"
                 rec["achieved"] = per_launch / sec / 1e12
-                rec["peak"] = tensor_peak
+                rec["peak"] = sustained
                 rec["peak_source"] = f"{peak_src} bf16 sustained"
+                rec["frac_burst"] = rec["achieved"] / burst
+                if issued is not None:
+                    rec["issued_TFLOPs"] = issued * steps / n / sec / 1e12
+                if at_clock:
+                    rec["frac_nominal_at_clock"] = (issued or work) * steps / n / sec / 1e12 / at_clock
             elif bound == "hbm":
+                rec["unit"] = "GB/s"
                 rec["achieved"] = per_launch / sec / 1e9
                 rec["peak"] = hbm
                 rec["peak_source"] = f"{peak_src} HBM copy"
             else:
+                rec["unit"] = "TFLOP/s"
                 rec["achieved"] = per_launch / sec / 1e12
                 # FP32 SIMT: 148 SMs x 128 lanes x (1 op per lane per cycle) at the max SM clock
                 rec["peak"] = 148 * 128 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
                 rec["peak_source"] = "derived: 148 SMs x 128 fp32 lanes x max SM clock (one FMUL or FADD each)"
             rec["frac"] = rec["achieved"] / rec["peak"]
         out[name] = rec
+    kd, kq = out.get("attn_bwd_dkdv"), out.get("attn_bwd_dq")
+    if kd and kq and kd["launches"] and kq["launches"]:
+        ms_b = kd["ms_per_launch"] + kq["ms_per_launch"]
+        t = 10.0 * P * D / (ms_b * 1e-3) / 1e12
+        out["attn_bwd"] = {
+            "launches": kd["launches"], "ms_per_launch": ms_b, "bound": "tensor", "unit": "TFLOP/s",
+            "algorithmic": "10*P*D FLOP (FlashAttention convention) over dK/dV + dQ time",
+            "achieved": t, "peak": sustained, "frac": t / sustained, "frac_burst": t / burst,
+            "peak_source": f"{peak_src} bf16 sustained",
+            "issued_TFLOPs": 14.0 * P * D / (ms_b * 1e-3) / 1e12}
+        kf = out.get("attn_fwd")
+        if kf and kf["launches"]:
+            ms_a = ms_b + kf["ms_per_launch"]
+            t = 14.0 * P * D / (ms_a * 1e-3) / 1e12
+            out["attn_fwd_bwd"] = {
+                "launches": kd["launches"], "ms_per_launch": ms_a, "bound": "tensor", "unit": "TFLOP/s",
+                "algorithmic": "14*P*D FLOP over forward + dK/dV + dQ time",
+                "achieved": t, "peak": sustained, "frac": t / sustained, "frac_burst": t / burst,
+                "peak_source": f"{peak_src} bf16 sustained"}
     return out
 
 
 # The source file of each timed kernel, under the package's csrc/, and the
 # ncu kernel-name fragment that identifies its launches.
-KERNEL_SOURCES = {"zone_video_stats": "plan.cu", "block_mean": "select.cu", "block_score": "select.cu",
-                  "select_row": "select.cu", "attn_fwd": "attn_fwd.cu", "attn_bwd_dkdv": "attn_bwd.cu",
-                  "attn_bwd_dq": "attn_bwd.cu", "a2v_norm": "a2v_norm.cu"}
+KERNEL_SOURCES = {"zone_video_stats": "plan.cu", "zone_a2v_stats": "plan.cu", "plan_finalize": "plan.cu",
+                  "perm": "plan.cu", "block_mean": "select.cu", "block_score": "select.cu",
+                  "select_row": "select.cu", "select_scan": "select.cu", "csr_fill": "select.cu",
+                  "csc_count": "select.cu", "csc_scan": "select.cu", "csc_fill": "select.cu",
+                  "csc_sort": "select.cu", "attn_fwd": "attn_fwd.cu", "permute3": "attn_fwd.cu",
+                  "unit_block": "attn_fwd.cu", "tile_units": "attn_fwd.cu", "attn_bwd_dkdv": "attn_bwd.cu",
+                  "attn_bwd_dq": "attn_bwd.cu", "bwd_prep": "attn_bwd.cu", "a2v_norm": "a2v_norm.cu"}
 NCU_KERNEL_NAMES = {"a2v_norm": "a2v_norm_kernel", "zone_video_stats": "zone_video_stats_kernel",
                     "block_mean": "block_mean_kernel", "attn_fwd": "attn_fwd_kernel",
                     "attn_bwd_dkdv": "dkdv_kernel", "attn_bwd_dq": "dq_kernel"}
@@ -467,8 +532,27 @@ def dense_sdpa(inp, w, backward, heads=1, iters=2):
     return {"unavailable": last}
 
 
+def read_stream_gbs(device, nbytes=4 << 30, iters=5):
+    """Read-only HBM bandwidth on this GPU, for kernels that only read: a
+    sum over a buffer larger than L2 (torch's reduction; a reference figure,
+    not part of the path), timed with CUDA events."""
+    x = torch.ones(nbytes // 8, dtype=torch.int64, device=device)
+    x.sum()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        x.sum()
+    e1.record()
+    torch.cuda.synchronize(device)
+    gbs = nbytes * iters / (e0.elapsed_time(e1) * 1e-3) / 1e9
+    del x
+    return gbs
+
+
 def run_prism(args, w, rank, world, device):
     lib = _lib.load()
+    read_gbs = read_stream_gbs(device)
     heads_mode = args.shard == "heads" and world > 1
     if heads_mode and world > w.heads:
         raise SystemExit(f"--shard heads needs at most {w.heads} ranks")
@@ -596,8 +680,14 @@ def run_prism(args, w, rank, world, device):
 
     peaks, peak_src = load_peaks()
     nb = pl.n_blocks.long()
-    kernels = kernel_rooflines(ktimes, P, D, N, h, nb, peaks, peak_src, args.steps)
-    dom = max((k for k in kernels if kernels[k]["launches"]), key=lambda k: kernels[k]["total_ms"])
+    kernels = kernel_rooflines(ktimes, P, D, N, h, nb, peaks, peak_src, args.steps, nnz=sel.nnz,
+                               sm_mhz=clocks.get("sm_mhz"))
+    for name in ("a2v_norm", "zone_video_stats", "zone_a2v_stats", "block_mean", "select_row"):
+        rec = kernels.get(name)
+        if rec and rec.get("achieved") is not None:   # read-dominated: also against a read-only stream
+            rec["frac_read_stream"] = rec["achieved"] / read_gbs
+    dom = max((k for k in kernels if kernels[k]["launches"] and "total_ms" in kernels[k]),
+              key=lambda k: kernels[k]["total_ms"])
     kd = kernels[dom]
     roofline = {"kernel": dom, "bound": kd["bound"], "achieved": kd["achieved"], "peak": kd["peak"],
                 "unit": kd["unit"], "frac": kd["frac"], "peak_source": kd["peak_source"],
@@ -646,6 +736,7 @@ def run_prism(args, w, rank, world, device):
                    "pairs": P, "pair_density": density, "nnz_blocks": sel.nnz,
                    "selection": selection_report},
         "stage_ms": stage_ms, "stage_roofline": stage_roofline, "kernels": kernels,
+        "read_stream_gbs": read_gbs,
         "clocks": clocks, "e2e": e2e, "gpu_launches": launches, "roofline": roofline, "cpu_baseline": cpu,
         "dense_sdpa": dense,
     }
@@ -710,8 +801,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.gpus != world and world > 1:
-        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.gpus != world:
+        # one process per GPU: N > 1 ranks come from the launcher (torchrun), never from this process
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N > 1 GPUs with "
+                 f"`python -m torch.distributed.run --nproc-per-node {args.gpus} bench.py --gpus {args.gpus} ...`")
 
     if args.impl == "reference":
         line = run_reference(args, w, rank, world)

@@ -856,6 +856,8 @@ cudaError_t launch_attn_bwd(const prism_params &p, const prism_plan_t &plan, con
       cudaSuccess)
     return e;
   const size_t total = (size_t)p.heads * N * (D / 8);
+  {
+  KernelTimer kt_(KT_BWD_PREP, st);
   if (D == 128)
     bwd::bwd_prep_kernel<128><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(plan.perm, N, p.heads, dO, O, O_res, lse,
                                                                               w.dOp, w.lse2p, w.deltap,
@@ -864,6 +866,7 @@ cudaError_t launch_attn_bwd(const prism_params &p, const prism_plan_t &plan, con
     bwd::bwd_prep_kernel<64><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(plan.perm, N, p.heads, dO, O, O_res, lse,
                                                                              w.dOp, w.lse2p, w.deltap,
                                                                              &w.hdr->status);
+  }
   count_launches(1);
   if ((e = launch_unit_block(plan.blocks, plan.n_blocks, NB, p.heads, w.unit_block, st)) != cudaSuccess) return e;
   if ((e = launch_tile_units(sel.row_ptr, sel.col, plan.blocks, w.unit_block, N, p.heads, 2, w.tu_q, st)) !=

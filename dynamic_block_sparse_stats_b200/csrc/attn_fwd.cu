@@ -543,6 +543,7 @@ cudaError_t launch_permute3(const int32_t *perm, int N, int heads, int D, const 
                             const uint16_t *s2, uint16_t *d0, uint16_t *d1, uint16_t *d2, int *status,
                             cudaStream_t st) {
   const size_t total = (size_t)heads * N * (D / 8);
+  KernelTimer kt_(KT_PERMUTE3, st);
   fwd::permute3_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(perm, N, heads, D, s0, s1, s2, d0, d1, d2,
                                                                        status);
   count_launches(1);
@@ -551,6 +552,7 @@ cudaError_t launch_permute3(const int32_t *perm, int N, int heads, int D, const 
 
 cudaError_t launch_unit_block(const int32_t *blocks, const int32_t *n_blocks, int NB, int heads,
                               int32_t *unit_block, cudaStream_t st) {
+  KernelTimer kt_(KT_UNIT_BLOCK, st);
   fwd::unit_block_kernel<<<dim3((NB + 255) / 256, heads), 256, 0, st>>>(blocks, n_blocks, NB, unit_block);
   count_launches(1);
   return cudaGetLastError();
@@ -560,6 +562,7 @@ cudaError_t launch_tile_units(const int32_t *ptr, const int32_t *idx, const int3
                               const int32_t *unit_block, int N, int heads, int units_per_tile, int32_t *tile_units,
                               cudaStream_t st) {
   const int warps = (N / (64 * units_per_tile)) * heads;
+  KernelTimer kt_(KT_TILE_UNITS, st);
   if (units_per_tile == 4)
     fwd::tile_units_kernel<4><<<(warps * 32 + 255) / 256, 256, 0, st>>>(ptr, idx, blocks, unit_block, N, heads,
                                                                         tile_units);

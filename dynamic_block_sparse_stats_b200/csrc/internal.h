@@ -58,7 +58,7 @@ cudaError_t make_rows_map(CUtensorMap *map, const void *base, long long rows, in
 // host-side count of kernel launches (prism_kernel_launches)
 void count_launches(int n);
 
-// timing.cu: optional event timing of the main kernels (prism_kernel_timing)
+// timing.cu: optional event timing of every kernel (prism_kernel_timing)
 enum KernelTimingId {
   KT_ZONE_STATS = 0,
   KT_BLOCK_MEAN,
@@ -68,8 +68,22 @@ enum KernelTimingId {
   KT_ATTN_DKDV,
   KT_ATTN_DQ,
   KT_A2V_NORM,
+  KT_ZONE_A2V_STATS,
+  KT_PLAN_FINALIZE,
+  KT_PERM,
+  KT_SELECT_SCAN,
+  KT_CSR_FILL,
+  KT_CSC_COUNT,
+  KT_CSC_SCAN,
+  KT_CSC_FILL,
+  KT_CSC_SORT,
+  KT_PERMUTE3,
+  KT_UNIT_BLOCK,
+  KT_TILE_UNITS,
+  KT_BWD_PREP,
   KT_COUNT
 };
+static_assert(KT_COUNT == PRISM_KERNEL_TIMING_IDS, "timing ids");
 // Records an event on `st` at construction and at destruction when timing is
 // enabled; wrap exactly one kernel launch.
 class KernelTimer {

@@ -431,13 +431,22 @@ cudaError_t launch_plan(const prism_params &p, const uint16_t *V, const float *a
     zone_video_stats_kernel<64><<<g1, 256, sm, st>>>(V, p.T, p.H, p.W, p.heads, vstats);
   }
   }
-  if (a) zone_a2v_stats_kernel<<<Z, 64, 0, st>>>(a, p.T, p.H, p.W, astats);
-  plan_finalize_kernel<<<p.heads, 1024, 0, st>>>(vstats, a ? astats : nullptr, Z, p.T, p.H, p.W, p.heads, NB,
-                                                 p.tau128, p.tau256, p.eps, p.map_exponent, p.guidance,
-                                                 p.density, out.zone_shape, out.zone_g,
-                                                 out.zone_rho, out.n_blocks, out.blocks, zone_first);
+  if (a) {
+    KernelTimer kt_(KT_ZONE_A2V_STATS, st);
+    zone_a2v_stats_kernel<<<Z, 64, 0, st>>>(a, p.T, p.H, p.W, astats);
+  }
+  {
+    KernelTimer kt_(KT_PLAN_FINALIZE, st);
+    plan_finalize_kernel<<<p.heads, 1024, 0, st>>>(vstats, a ? astats : nullptr, Z, p.T, p.H, p.W, p.heads, NB,
+                                                   p.tau128, p.tau256, p.eps, p.map_exponent, p.guidance,
+                                                   p.density, out.zone_shape, out.zone_g,
+                                                   out.zone_rho, out.n_blocks, out.blocks, zone_first);
+  }
   dim3 g3((N + 255) / 256, p.heads);
-  perm_kernel<<<g3, 256, 0, st>>>(out.zone_shape, p.T, p.H, p.W, Z, out.perm, out.inv_perm);
+  {
+    KernelTimer kt_(KT_PERM, st);
+    perm_kernel<<<g3, 256, 0, st>>>(out.zone_shape, p.T, p.H, p.W, Z, out.perm, out.inv_perm);
+  }
   count_launches(a ? 4 : 3);
   return cudaGetLastError();
 }

@@ -653,10 +653,16 @@ cudaError_t launch_select(const prism_params &p, const prism_plan_t &plan, const
       select_row_kernel<<<NB, kSelThreads, sel_smem, st>>>(w.S, NB, plan.n_blocks + h, p.topk_frac, p.topk_abs,
                                                            p.top_p, w.counts + (size_t)h * NB);
     }
-    scan_kernel<<<1, 1024, 0, st>>>(w.counts + (size_t)h * NB, NB, out.row_ptr + (size_t)h * NB, &w.hdr->nnz,
-                                    h == p.heads - 1);
-    csr_fill_kernel<<<NB, 128, 0, st>>>(w.S, NB, plan.n_blocks + h, w.counts + (size_t)h * NB,
-                                        out.row_ptr + (size_t)h * NB, out.col, out.cap);
+    {
+      KernelTimer kt_(KT_SELECT_SCAN, st);
+      scan_kernel<<<1, 1024, 0, st>>>(w.counts + (size_t)h * NB, NB, out.row_ptr + (size_t)h * NB, &w.hdr->nnz,
+                                      h == p.heads - 1);
+    }
+    {
+      KernelTimer kt_(KT_CSR_FILL, st);
+      csr_fill_kernel<<<NB, 128, 0, st>>>(w.S, NB, plan.n_blocks + h, w.counts + (size_t)h * NB,
+                                          out.row_ptr + (size_t)h * NB, out.col, out.cap);
+    }
   }
   count_launches(1 + 4 * p.heads);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
@@ -670,10 +676,22 @@ cudaError_t launch_select(const prism_params &p, const prism_plan_t &plan, const
     const size_t HN = (size_t)p.heads * NB;
     if ((err = cudaMemsetAsync(w.colcnt, 0, sizeof(int32_t) * HN, st)) != cudaSuccess) return err;
     if ((err = cudaMemsetAsync(w.cursor, 0, sizeof(int32_t) * HN, st)) != cudaSuccess) return err;
-    csc_count_kernel<<<gm, 128, 0, st>>>(out.row_ptr, out.col, NB, out.cap, w.colcnt);
-    scan_kernel<<<1, 1024, 0, st>>>(w.colcnt, (int)HN, out.col_ptr, nullptr, 1);
-    csc_fill_kernel<<<gm, 128, 0, st>>>(out.row_ptr, out.col, NB, out.cap, out.col_ptr, w.cursor, out.row);
-    csc_sort_kernel<<<gm, 256, sizeof(uint32_t) * ((NB + 31) / 32), st>>>(out.col_ptr, NB, out.cap, out.row);
+    {
+      KernelTimer kt_(KT_CSC_COUNT, st);
+      csc_count_kernel<<<gm, 128, 0, st>>>(out.row_ptr, out.col, NB, out.cap, w.colcnt);
+    }
+    {
+      KernelTimer kt_(KT_CSC_SCAN, st);
+      scan_kernel<<<1, 1024, 0, st>>>(w.colcnt, (int)HN, out.col_ptr, nullptr, 1);
+    }
+    {
+      KernelTimer kt_(KT_CSC_FILL, st);
+      csc_fill_kernel<<<gm, 128, 0, st>>>(out.row_ptr, out.col, NB, out.cap, out.col_ptr, w.cursor, out.row);
+    }
+    {
+      KernelTimer kt_(KT_CSC_SORT, st);
+      csc_sort_kernel<<<gm, 256, sizeof(uint32_t) * ((NB + 31) / 32), st>>>(out.col_ptr, NB, out.cap, out.row);
+    }
     count_launches(4);
   }
   return cudaGetLastError();

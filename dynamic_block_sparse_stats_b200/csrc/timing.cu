@@ -1,5 +1,5 @@
 // Optional per-kernel timing for measurement: CUDA event pairs recorded on the
-// launching stream around the library's main kernels.
+// launching stream around every kernel launch of the library.
 #include <mutex>
 #include <vector>
 
@@ -8,8 +8,10 @@
 namespace prism {
 namespace {
 
-const char *const kNames[KT_COUNT] = {"zone_video_stats", "block_mean", "block_score", "select_row",
-                                      "attn_fwd",         "attn_bwd_dkdv", "attn_bwd_dq", "a2v_norm"};
+const char *const kNames[KT_COUNT] = {
+    "zone_video_stats", "block_mean",  "block_score", "select_row", "attn_fwd",  "attn_bwd_dkdv", "attn_bwd_dq",
+    "a2v_norm",         "zone_a2v_stats", "plan_finalize", "perm",   "select_scan", "csr_fill",    "csc_count",
+    "csc_scan",         "csc_fill",    "csc_sort",    "permute3",   "unit_block", "tile_units",    "bwd_prep"};
 
 struct Rec {
   cudaEvent_t a, b;

@@ -336,17 +336,22 @@ const char *prism_last_error(void);
  * (host-side counter, incremented at every launch; never reset). */
 uint64_t prism_kernel_launches(void);
 
-/* Optional timing of the library's main kernels, for measurement (not meant
- * to be toggled by one thread while another launches through the library).  When
- * enabled, every launch of the zone-statistics, block-mean, block-score,
- * row-selection, forward-attention, the two backward-attention and the A2V
- * norm kernels is bracketed by a CUDA event pair recorded on its launching
- * stream.
+/* Optional timing of the library's kernels, for measurement (not meant to be
+ * toggled by one thread while another launches through the library).  When
+ * enabled, every kernel launch of the path is bracketed by a CUDA event pair
+ * recorded on its launching stream.
  * prism_kernel_timing(1) clears the records and enables; (0) clears and
  * disables.  Returns PRISM_OK. */
 int prism_kernel_timing(int enable);
 
-/* Reads the records of kernel `id` (0 .. 7, in the order listed above): waits
+/* Number of kernel timing ids.  Ids, in order: 0 zone_video_stats,
+ * 1 block_mean, 2 block_score, 3 select_row, 4 attn_fwd, 5 attn_bwd_dkdv,
+ * 6 attn_bwd_dq, 7 a2v_norm, 8 zone_a2v_stats, 9 plan_finalize, 10 perm,
+ * 11 select_scan, 12 csr_fill, 13 csc_count, 14 csc_scan, 15 csc_fill,
+ * 16 csc_sort, 17 permute3, 18 unit_block, 19 tile_units, 20 bwd_prep. */
+#define PRISM_KERNEL_TIMING_IDS 21
+
+/* Reads the records of kernel `id` (0 .. PRISM_KERNEL_TIMING_IDS - 1): waits
  * for its events, and returns the number of timed launches, their total
  * milliseconds and the kernel's name (library-owned string).  Returns
  * PRISM_OK, PRISM_ERR_INVALID_ARG (id out of range) or PRISM_ERR_CUDA. */

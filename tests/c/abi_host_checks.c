@@ -78,7 +78,7 @@ int main(void) {
   int n = 0;
   double ms = 0.0;
   const char *name = NULL;
-  CHECK(prism_kernel_timing_read(8, &n, &ms, &name) == PRISM_ERR_INVALID_ARG);
+  CHECK(prism_kernel_timing_read(PRISM_KERNEL_TIMING_IDS, &n, &ms, &name) == PRISM_ERR_INVALID_ARG);
 
   if (failures) return 1;
   printf("ok\n");

@@ -137,8 +137,14 @@ def main(only):
     tmp = tempfile.mkdtemp(prefix="mutation_check_")
     dst = os.path.join(tmp, "repo")
     try:
-        shutil.copytree(ROOT, dst, ignore=shutil.ignore_patterns(".git", "_build", "gpurun_out", "_work",
-                                                                 "__pycache__", "baseline"))
+        # the copy holds the tracked files only (the committed repository)
+        tracked = subprocess.run(["git", "ls-files", "-z"], cwd=ROOT, capture_output=True, check=True).stdout
+        for rel in tracked.decode().split("\0"):
+            if rel:
+                os.makedirs(os.path.dirname(os.path.join(dst, rel)), exist_ok=True)
+                shutil.copy2(os.path.join(ROOT, rel), os.path.join(dst, rel))
+        subprocess.run([sys.executable, "-m", "dynamic_block_sparse_stats_b200.build", "--force"], cwd=dst,
+                       capture_output=True, check=True)
         survivors = []
         for target, entries in (("oracle/prism_oracle.py", M), ("bench.py", BENCH),
                                  ("dynamic_block_sparse_stats_b200/api.py", BINDING)):

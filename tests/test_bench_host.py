@@ -101,24 +101,39 @@ def test_computed_pairs_with_a_different_block_table_per_head():
 
 
 def test_kernel_roofline_arithmetic():
-    peaks = {"hbm_gbs": 6000.0, "bf16_tflops_sustained": 1000.0, "sm_max_mhz": 2000.0}
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops_sustained": 1000.0, "bf16_tflops": 1200.0, "sm_max_mhz": 2000.0}
     P, D, N, h, steps = 1.0e12, 128, 860160, 24, 2
     nb = torch.tensor([100, 200])
-    kt = {"attn_fwd": (2, 1000.0), "attn_bwd_dq": (2, 1200.0), "block_mean": (2, 4.0),
-          "block_score": (48, 24.0), "select_row": (48, 10.0)}
-    out = bench.kernel_rooflines(kt, P, D, N, h, nb, peaks, "measured", steps)
+    kt = {"attn_fwd": (2, 1000.0), "attn_bwd_dkdv": (2, 1600.0), "attn_bwd_dq": (2, 1200.0),
+          "block_mean": (2, 4.0), "block_score": (48, 24.0), "select_row": (48, 10.0)}
+    out = bench.kernel_rooflines(kt, P, D, N, h, nb, peaks, "measured", steps, nnz=1000, sm_mhz=1500.0)
     fwd = out["attn_fwd"]                        # one launch per step, 500 ms each
     assert fwd["ms_per_launch"] == 500.0
     assert fwd["achieved"] == pytest.approx(4 * P * D / 0.5 / 1e12)
     assert fwd["peak"] == 1000.0 and fwd["frac"] == pytest.approx(fwd["achieved"] / 1000.0)
-    assert out["attn_bwd_dq"]["achieved"] == pytest.approx(6 * P * D / 0.6 / 1e12)
+    assert fwd["frac_burst"] == pytest.approx(fwd["achieved"] / 1200.0)
+    assert fwd["frac_nominal_at_clock"] == pytest.approx(fwd["achieved"] / (148 * 8192 * 1500e6 / 1e12))
+    dq = out["attn_bwd_dq"]                      # algorithmic 2PD (dQ = dS K); 6PD issued
+    assert dq["achieved"] == pytest.approx(2 * P * D / 0.6 / 1e12)
+    assert dq["issued_TFLOPs"] == pytest.approx(6 * P * D / 0.6 / 1e12)
+    assert out["attn_bwd_dkdv"]["achieved"] == pytest.approx(8 * P * D / 0.8 / 1e12)
+    bwd = out["attn_bwd"]                        # the convention: 10PD over dK/dV + dQ
+    assert bwd["ms_per_launch"] == pytest.approx(1400.0)
+    assert bwd["achieved"] == pytest.approx(10 * P * D / 1.4 / 1e12)
+    assert bwd["frac"] == pytest.approx(bwd["achieved"] / 1000.0)
+    assert bwd["frac_burst"] == pytest.approx(bwd["achieved"] / 1200.0)
+    assert bwd["issued_TFLOPs"] == pytest.approx(14 * P * D / 1.4 / 1e12)
+    both = out["attn_fwd_bwd"]
+    assert both["achieved"] == pytest.approx(14 * P * D / 1.9 / 1e12)
     bm = out["block_mean"]                       # one read of Q and K per launch, 2 ms
     assert bm["achieved"] == pytest.approx(4 * N * h * D / 2e-3 / 1e9) and bm["peak"] == 6000.0
     bs = out["block_score"]                      # 24 launches per step share 2*D*sum(nb^2)
     per_launch = 2 * D * (100 ** 2 + 200 ** 2) * steps / 48
     assert bs["achieved"] == pytest.approx(per_launch / 0.5e-3 / 1e12)
     assert bs["peak"] == pytest.approx(148 * 128 * 2000e6 / 1e12)
-    assert out["select_row"]["frac"] is None and out["select_row"]["launches"] == 48
+    sr = out["select_row"]                       # one read of the score rows
+    assert sr["achieved"] == pytest.approx(4 * (100 ** 2 + 200 ** 2) * steps / 48 / (10.0 / 48 * 1e-3) / 1e9)
+    assert sr["frac"] == pytest.approx(sr["achieved"] / 6000.0)
 
 
 class _FakeProc:
@@ -262,6 +277,6 @@ def test_every_timed_kernel_has_a_roofline_spec_and_a_source():
     assert len(set(names)) == len(names)
     kt = {nm: (0, 0.0) for nm in names}
     out = bench.kernel_rooflines(kt, 1e12, 128, 860160, 24, torch.tensor([100]), {"hbm_gbs": 1.0}, "measured", 1)
-    assert set(out) == set(names)
+    assert set(out) == set(names)                 # no launches: no combined backward entries
     assert set(names) == set(bench.KERNEL_SOURCES)
     assert set(bench.NCU_KERNEL_NAMES) <= set(names)

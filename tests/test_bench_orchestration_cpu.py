@@ -20,7 +20,10 @@ from dynamic_block_sparse_stats_b200.synth import WORKLOADS
 from oracle import prism_oracle as O
 
 _KERNEL_MS = {"zone_video_stats": 0.1, "block_mean": 0.2, "block_score": 0.05, "select_row": 0.3, "attn_fwd": 8.0,
-              "attn_bwd_dkdv": 15.0, "attn_bwd_dq": 10.0, "a2v_norm": 0.05}
+              "attn_bwd_dkdv": 15.0, "attn_bwd_dq": 10.0, "a2v_norm": 0.05, "zone_a2v_stats": 0.01,
+              "plan_finalize": 0.02, "perm": 0.01, "select_scan": 0.01, "csr_fill": 0.01, "csc_count": 0.01,
+              "csc_scan": 0.01, "csc_fill": 0.01, "csc_sort": 0.01, "permute3": 0.05, "unit_block": 0.01,
+              "tile_units": 0.01, "bwd_prep": 0.03}
 
 
 class _Lib:
@@ -133,6 +136,7 @@ def test_run_prism_orchestration_on_cpu(monkeypatch):
     monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
     monkeypatch.setattr(torch.cuda, "current_stream", lambda *a, **k: _Stream())
     monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    monkeypatch.setattr(bench, "read_stream_gbs", lambda device: 7000.0)
     args = argparse.Namespace(steps=2, warmup=3, no_e2e=True, no_cpu_baseline=False, no_dense=True,
                               shard="layers", workload="tiny", backward=True)
     line = bench.run_prism(args, w, rank=0, world=1, device=torch.device("cpu"))
@@ -160,4 +164,9 @@ def test_run_prism_orchestration_on_cpu(monkeypatch):
     assert "error" not in sel and sel["rows"] == sum(hp.blocks.shape[0] for hp in state["opl"].heads)
     assert set(line["stage_ms"]) == {"plan", "select", "fwd", "bwd"}
     assert line["clocks"]["reasons"] == ["nvidia-smi unavailable"] or "sm_mhz" in line["clocks"]
-    assert set(line["kernels"]) == set(_KERNEL_MS)
+    assert set(line["kernels"]) == set(_KERNEL_MS) | {"attn_bwd", "attn_fwd_bwd"}
+    assert len(_KERNEL_MS) == _lib.KERNEL_TIMING_IDS
+    bwd = line["kernels"]["attn_bwd"]                       # the backward on the 10*P*D convention
+    assert bwd["achieved"] == pytest.approx(10.0 * P * w.head_dim / 25e-3 / 1e12, rel=1e-12)
+    assert line["kernels"]["a2v_norm"]["frac_read_stream"] == pytest.approx(
+        line["kernels"]["a2v_norm"]["achieved"] / 7000.0)

@@ -534,6 +534,43 @@ def attention_bwd(Q, K, V, dO, pl: Plan, sel, scale, heads=None):
     return dQ, dK, dV
 
 
+def attention_bwd_key_block(Qh, Kh, Vh, dOh, hp: HeadPlan, j, users, scale):
+    """dK and dV of the tokens of one key block j, from the query blocks that
+    selected it (the same textbook backward as attention_bwd, restricted to
+    the outputs of block j; [DIGEST] training section).  Each user row needs
+    its full softmax over its own selection (for P and for
+    D_q = sum_k P_qk dP_qk = dO_q . O_q), but only block j's columns of dS
+    and P enter the result:
+      dV_j = sum_i P_{i,j}^T dO_i,   dK_j = scale * sum_i dS_{i,j}^T Q_i.
+    users: (query block i, its selected key blocks) pairs, j among them.
+    Returns (natural key indices of block j, dK_j [B_j, D], dV_j [B_j, D])
+    in float64."""
+    kj = hp.perm[hp.blocks[j, 5]:hp.blocks[j, 5] + hp.blocks[j, 4]]
+    D = Qh.shape[1]
+    dK = np.zeros((kj.size, D))
+    dV = np.zeros((kj.size, D))
+    for (i, ids) in users:
+        qi = hp.perm[hp.blocks[i, 5]:hp.blocks[i, 5] + hp.blocks[i, 4]]
+        keys = np.concatenate([hp.perm[hp.blocks[b, 5]:hp.blocks[b, 5] + hp.blocks[b, 4]] for b in ids])
+        q = Qh[qi].astype(np.float64)
+        do = dOh[qi].astype(np.float64)
+        k = Kh[keys].astype(np.float64)
+        v = Vh[keys].astype(np.float64)
+        s = (q @ k.T) * scale
+        P = np.exp(s - s.max(axis=1, keepdims=True))
+        P /= P.sum(axis=1, keepdims=True)
+        o = P @ v
+        Dq = (do * o).sum(axis=1, keepdims=True)          # = sum_k P dP over the row
+        at = int(np.searchsorted(np.asarray(ids), j))     # ids ascending: block j's columns in the row
+        c0 = int(sum(hp.blocks[b, 4] for b in ids[:at]))
+        Pj = P[:, c0:c0 + kj.size]
+        dPj = do @ Vh[kj].astype(np.float64).T
+        dSj = Pj * (dPj - Dq)
+        dV += Pj.T @ do
+        dK += scale * (dSj.T @ q)
+    return kj, dK, dV
+
+
 def csr_from_selection(sel, nb_cap):
     """Flatten a per-head selection into row_ptr [heads*nb_cap+1] and col, the
     layout the library returns (row = head*nb_cap + query block)."""

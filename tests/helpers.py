@@ -42,14 +42,25 @@ def csr_rows(row_ptr, col, NB, h, i):
     return col[row_ptr[r]:row_ptr[r + 1]]
 
 
+def check_ties(excluded, total, what):
+    """Exclusions at logged ties must stay rare: at most 0.1% of the
+    decisions checked (and never more than 2 on grids too small for that
+    share to reach 1)."""
+    print(f"{what}: {excluded} of {total} excluded at ties")
+    assert excluded <= max(2.0, 1e-3 * total), f"{what}: {excluded} of {total} decisions excluded at ties"
+
+
 def compare_plan(w, pl, ref, heads):
     """Library plan vs oracle plan (heads[k] of the library = ref.heads[k]).
     Statistic values within fp32-partial-sum rounding; shapes, block table
     and permutation bit-exact except at decisions whose oracle margin is
-    <= TIE.  Returns the number of zone decisions excluded at ties."""
+    <= TIE.  A zone excluded at a tie changes only its own blocks: every zone
+    owns the permuted positions [512m, 512m + 512), so the block-table rows
+    and permutation entries of all other zones are still compared.  Returns
+    (zone decisions excluded at ties, zones checked)."""
     shapes, g, rho = to_np(pl.zone_shape), to_np(pl.zone_g), to_np(pl.zone_rho)
     nblk, blocks, perm, inv = to_np(pl.n_blocks), to_np(pl.blocks), to_np(pl.perm), to_np(pl.inv_perm)
-    excluded = 0
+    excluded = total = 0
     for k, h in enumerate(heads):
         hp = ref.heads[k]
         np.testing.assert_allclose(rho[h], hp.rho, rtol=1e-6, atol=1e-12)
@@ -58,15 +69,19 @@ def compare_plan(w, pl, ref, heads):
         tie = (hp.vol_margin <= TIE) | (hp.shape_margin <= TIE)
         assert not (diff & ~tie).any(), f"head {h}: shape differs outside ties at zones {np.nonzero(diff & ~tie)}"
         excluded += int((diff & tie).sum())
-        if diff.any():
-            continue
+        total += diff.size
+        keep = ~diff                                             # zones whose decisions agree
         nb = hp.blocks.shape[0]
-        assert nblk[h] == nb
-        got = blocks[h, :nb]
-        np.testing.assert_array_equal(got[:, 0], hp.blocks[:, 5])
-        np.testing.assert_array_equal(got[:, 1], hp.blocks[:, 4])
-        np.testing.assert_array_equal(got[:, 2], (hp.blocks[:, 0] * w.H + hp.blocks[:, 1]) * w.W + hp.blocks[:, 2])
-        np.testing.assert_array_equal(got[:, 3], hp.blocks[:, 3])
-        np.testing.assert_array_equal(perm[h], hp.perm)
+        if not diff.any():
+            assert nblk[h] == nb
+        got = blocks[h, :nblk[h]]
+        got = got[keep[got[:, 0] // 512]]
+        want = hp.blocks[keep[hp.blocks[:, 5] // 512]]
+        np.testing.assert_array_equal(got[:, 0], want[:, 5])    # p0
+        np.testing.assert_array_equal(got[:, 1], want[:, 4])    # B
+        np.testing.assert_array_equal(got[:, 2], (want[:, 0] * w.H + want[:, 1]) * w.W + want[:, 2])
+        np.testing.assert_array_equal(got[:, 3], want[:, 3])    # shape id
+        pos = np.repeat(keep, 512)
+        np.testing.assert_array_equal(perm[h][pos], hp.perm[pos])
         np.testing.assert_array_equal(inv[h][perm[h]], np.arange(w.N))
-    return excluded
+    return excluded, total

@@ -73,6 +73,10 @@ M = [
  ("permutation inverted", "        perm[p0:p0 + B] = block_tokens(T, H, W, t0, y0, x0, sid)", "        perm[block_tokens(T, H, W, t0, y0, x0, sid)] = np.arange(p0, p0 + B)"),
  ("lse in log2", "lse = (m + np.log(l))[:, 0]", "lse = (m + np.log2(l))[:, 0]"),
  ("top-k takes the lowest scores", "order = np.lexsort((j, -s))", "order = np.lexsort((j, s))"),
+ ("key-block bwd: Delta dropped", "Dq = (do * o).sum(axis=1, keepdims=True)          # = sum_k", "Dq = 0.0 * (do * o).sum(axis=1, keepdims=True)  # = sum_k"),
+ ("key-block bwd: dK without scale", "dK += scale * (dSj.T @ q)", "dK += dSj.T @ q"),
+ ("key-block bwd: wrong column offset", "at = int(np.searchsorted(np.asarray(ids), j))", "at = int(np.searchsorted(np.asarray(ids), j)) + 0 * len(ids) - (1 if j > 0 else 0)"),
+ ("key-block bwd: dV from dS", "dV += Pj.T @ do", "dV += dSj.T @ do"),
 ]
 
 

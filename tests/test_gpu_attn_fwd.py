@@ -78,6 +78,10 @@ def test_fwd_720p_sampled_rows():
     _check("720p", heads=[0, 7, 23], rows_per_head=48)
 
 
+def test_fwd_1080p_sampled_rows():
+    _check("1080p", heads=[0, 23], rows_per_head=16, seed=1)
+
+
 def test_fwd_select_all_equals_dense_sdpa():
     """Every block selected: the sparse kernel must equal dense attention."""
     w = WORKLOADS["small"]

@@ -10,10 +10,11 @@ selection (as everywhere else):
   * selection: 32 sampled query blocks on every head, bit-exact except at
     logged ties;
   * forward: O and LSE of 8 sampled query blocks on each of two heads;
-  * backward: dQ of 3 sampled query blocks per head, and dK, dV of the key
-    block with the fewest users among 256 sampled ones on each head (a key
-    block's gradients need the full rows of every query block that selected
-    it, so the sample favours short columns to keep the test to minutes).
+  * backward: dQ of 3 sampled query blocks per head, and dK, dV of three key
+    blocks per head: one drawn at random, and the ones whose columns (the
+    query blocks that selected them) have the head's median and 90th
+    percentile length (a key block's gradients need the full rows of all
+    its users, which the oracle computes block by block).
 Tolerances are the ones of the smaller grids: indices bit-exact, outputs
 within max-abs 2e-2 and mean-abs 2e-3 (fp32 gradients)."""
 import numpy as np
@@ -23,7 +24,7 @@ import torch
 from dynamic_block_sparse_stats_b200 import api
 from dynamic_block_sparse_stats_b200.synth import WORKLOADS, make_bridge_output, make_inputs
 from oracle import prism_oracle as O
-from tests.helpers import TIE, compare_plan, oracle_plan_from_shapes, scale_of, to_np
+from tests.helpers import TIE, check_ties, compare_plan, oracle_plan_from_shapes, scale_of, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -77,12 +78,13 @@ def _head(S, h, names):
 def test_2k_plan_every_head_in_full():
     S = _layer()
     w = S["w"]
-    excluded = 0
+    excluded = total = 0
     for h in range(w.heads):
         (V,) = _head(S, h, ("V",))
         ref = O.plan(V, S["a"], w.T, w.H, w.W)
-        excluded += compare_plan(w, S["pl"], ref, [h])
-    print(f"2K plan: {w.heads} heads in full, zone decisions excluded at ties {excluded}")
+        e, t = compare_plan(w, S["pl"], ref, [h])
+        excluded, total = excluded + e, total + t
+    check_ties(excluded, total, f"2K plan, {w.heads} heads in full, zone decisions")
 
 
 def test_2k_selection_sampled_rows_on_every_head():
@@ -104,7 +106,7 @@ def test_2k_selection_sampled_rows_on_every_head():
                 excluded += 1
                 continue
             raise AssertionError(f"head {h} row {i}: got {got.size} ids, want {ids.size}; info {info}")
-    print(f"2K selection: {checked} rows over {w.heads} heads, excluded at ties {excluded}")
+    check_ties(excluded, checked, f"2K selection, rows over {w.heads} heads")
 
 
 def test_2k_forward_sampled_blocks():
@@ -133,6 +135,7 @@ def test_2k_backward_sampled_blocks():
     scale = scale_of(w.head_dim)
     rng = np.random.default_rng(3)
     errs = {"dQ": [], "dK": [], "dV": []}
+    lengths = []
     for k, h in enumerate(HEADS):
         hp = oracle_plan_from_shapes(w.T, w.H, w.W, [S["shapes"][h]]).heads[0]
         sub = O.Plan(w.T, w.H, w.W, [hp])
@@ -142,14 +145,21 @@ def test_2k_backward_sampled_blocks():
             rQ, _, _ = O.attention_bwd(*X, sub, [[(int(i), _csr(S, h, int(i)), {})]], scale)
             toks = hp.perm[hp.blocks[i, 5]:hp.blocks[i, 5] + hp.blocks[i, 4]]
             errs["dQ"].append(np.abs(dQ[toks, k] - rQ[toks, 0]).reshape(-1))
-        cand = rng.choice(S["nb"][h], size=256, replace=False)
-        cand = sorted((c for c in cand if _csc(S, h, int(c)).size > 0), key=lambda c: _csc(S, h, int(c)).size)[:1]
-        for j in cand:
-            users = [(int(i), _csr(S, h, int(i)), {}) for i in _csc(S, h, int(j))]
-            _, rK, rV = O.attention_bwd(*X, sub, [users], scale)
-            toks = hp.perm[hp.blocks[j, 5]:hp.blocks[j, 5] + hp.blocks[j, 4]]
-            errs["dK"].append(np.abs(dK[toks, k] - rK[toks, 0]).reshape(-1))
-            errs["dV"].append(np.abs(dV[toks, k] - rV[toks, 0]).reshape(-1))
+        # key blocks: one drawn at random, and those whose column (number of
+        # query blocks that selected them) has the head's median and 90th
+        # percentile length, where dK/dV spends its time
+        nbh = int(S["nb"][h])
+        cl = np.array([_csc(S, h, j).size for j in range(nbh)])
+        order = np.argsort(cl, kind="stable")
+        live = order[cl[order] > 0]
+        picks = [int(rng.choice(live)), int(live[len(live) // 2]), int(live[(9 * len(live)) // 10])]
+        for j in picks:
+            users = [(int(i), _csr(S, h, int(i))) for i in _csc(S, h, j)]
+            kj, rK, rV = O.attention_bwd_key_block(H_["Q"], H_["K"], H_["V"], H_["dO"], hp, j, users, scale)
+            errs["dK"].append(np.abs(dK[kj, k] - rK).reshape(-1))
+            errs["dV"].append(np.abs(dV[kj, k] - rV).reshape(-1))
+            lengths.append(len(users))
+    print(f"2K dK/dV columns checked (users per key block): {lengths}")
     for nm, e in errs.items():
         e = np.concatenate(e)
         print(f"2K {nm}: max-abs {e.max():.3e} mean-abs {e.mean():.3e} over {e.size}")

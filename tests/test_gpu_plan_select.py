@@ -10,7 +10,7 @@ import torch
 from dynamic_block_sparse_stats_b200 import api
 from dynamic_block_sparse_stats_b200.synth import WORKLOADS, make_inputs
 from oracle import prism_oracle as O
-from tests.helpers import TIE, oracle_plan_from_shapes, scale_of, to_np
+from tests.helpers import TIE, check_ties, compare_plan, oracle_plan_from_shapes, scale_of, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -35,56 +35,23 @@ def test_plan_matches_oracle(name):
     w, inp, p, pl, sel = _run(name)
     V = inp["V"].float().cpu().numpy()
     a = inp["a"].cpu().numpy()
-    heads = range(w.heads) if w.heads <= 3 else [0, 5, 23]
-    ref = O.plan(V[:, list(heads)], a, w.T, w.H, w.W)
-    shapes = to_np(pl.zone_shape)
-    g = to_np(pl.zone_g)
-    rho = to_np(pl.zone_rho)
-    nblk = to_np(pl.n_blocks)
-    blocks = to_np(pl.blocks)
-    perm = to_np(pl.perm)
-    inv = to_np(pl.inv_perm)
-    excluded = 0
-    for k, h in enumerate(heads):
-        hp = ref.heads[k]
-        # statistic values: fp32 partial sums of <= 8 terms combined in float64
-        # (<= 8 fp32 ulps relative); the decisions below are compared exactly
-        np.testing.assert_allclose(rho[h], hp.rho, rtol=1e-6, atol=1e-12)
-        np.testing.assert_allclose(g[h], hp.g, rtol=1e-6, atol=1e-12)
-        diff = shapes[h] != hp.shape
-        tie = (hp.vol_margin <= TIE) | (hp.shape_margin <= TIE)
-        assert not (diff & ~tie).any(), f"head {h}: shape differs outside ties at zones {np.nonzero(diff & ~tie)}"
-        excluded += int((diff & tie).sum())
-        if diff.any():
-            continue
-        nb = hp.blocks.shape[0]
-        assert nblk[h] == nb
-        got = blocks[h, :nb]
-        np.testing.assert_array_equal(got[:, 0], hp.blocks[:, 5])      # p0
-        np.testing.assert_array_equal(got[:, 1], hp.blocks[:, 4])      # B
-        np.testing.assert_array_equal(got[:, 2], (hp.blocks[:, 0] * w.H + hp.blocks[:, 1]) * w.W + hp.blocks[:, 2])
-        np.testing.assert_array_equal(got[:, 3], hp.blocks[:, 3])      # shape id
-        np.testing.assert_array_equal(perm[h], hp.perm)
-        np.testing.assert_array_equal(inv[h][perm[h]], np.arange(w.N))
-    print(f"{name}: shape decisions excluded at ties: {excluded}")
+    heads = list(range(w.heads)) if w.heads <= 3 else [0, 5, 23]
+    ref = O.plan(V[:, heads], a, w.T, w.H, w.W)
+    # statistic values: fp32 partial sums of <= 8 terms combined in float64
+    # (<= 8 fp32 ulps relative); the decisions are compared exactly, zone by
+    # zone, except at logged ties
+    excluded, total = compare_plan(w, pl, ref, heads)
+    check_ties(excluded, total, f"{name} plan zones")
 
 
-@pytest.mark.parametrize("name", ["tiny", "small", "small_d64", "720p"])
-def test_select_matches_oracle_on_gpu_plan(name):
-    w, inp, p, pl, sel = _run(name)
-    shapes = to_np(pl.zone_shape)
+def _check_rows(name, w, sel, ref, heads, ref_plan):
     NB = w.N // 64
-    Q = inp["Q"].float().cpu().numpy()
-    K = inp["K"].float().cpu().numpy()
     row_ptr = to_np(sel.row_ptr).astype(np.int64)
     col = to_np(sel.col)[:sel.nnz]
-    heads = range(w.heads) if w.heads <= 3 else [0, 11, 23]
-    ref_plan = oracle_plan_from_shapes(w.T, w.H, w.W, [shapes[h] for h in heads])
-    ref = O.select(Q[:, list(heads)], K[:, list(heads)], ref_plan, w.topk_frac, w.topk_abs, w.top_p,
-                   scale_of(w.head_dim))
-    excluded = 0
+    excluded = checked = 0
     for k, h in enumerate(heads):
         for (i, ids, info) in ref[k]:
+            checked += 1
             got = col[row_ptr[h * NB + i]:row_ptr[h * NB + i + 1]]
             if got.size == ids.size and (got == ids).all():
                 continue
@@ -94,7 +61,39 @@ def test_select_matches_oracle_on_gpu_plan(name):
             raise AssertionError(f"head {h} row {i}: got {got.tolist()} want {ids.tolist()} info {info}")
         nb = ref_plan.heads[k].blocks.shape[0]
         assert row_ptr[h * NB + nb] == row_ptr[(h + 1) * NB]  # rows past n_blocks are empty
-    print(f"{name}: selection rows excluded at ties: {excluded}")
+    check_ties(excluded, checked, f"{name} selection rows")
+
+
+@pytest.mark.parametrize("name", ["tiny", "small", "small_d64", "720p"])
+def test_select_matches_oracle_on_gpu_plan(name):
+    w, inp, p, pl, sel = _run(name)
+    shapes = to_np(pl.zone_shape)
+    Q = inp["Q"].float().cpu().numpy()
+    K = inp["K"].float().cpu().numpy()
+    heads = list(range(w.heads)) if w.heads <= 3 else [0, 11, 23]
+    ref_plan = oracle_plan_from_shapes(w.T, w.H, w.W, [shapes[h] for h in heads])
+    ref = O.select(Q[:, heads], K[:, heads], ref_plan, w.topk_frac, w.topk_abs, w.top_p, scale_of(w.head_dim))
+    _check_rows(name, w, sel, ref, heads, ref_plan)
+
+
+def test_select_1080p_sampled_rows_on_every_head():
+    """The 1080p grid has exactly static zones (s_q = 0.5 there), whose flat
+    score rows make Top-p expand ([DIGEST] hybrid selection section): 48
+    seeded rows on each of the 24 heads, bit-exact except logged ties."""
+    w, inp, p, pl, sel = _run("1080p")
+    shapes = to_np(pl.zone_shape)
+    nb = to_np(pl.n_blocks)
+    rng = np.random.default_rng(7)
+    heads = list(range(w.heads))
+    ref_plan = oracle_plan_from_shapes(w.T, w.H, w.W, [shapes[h] for h in heads])
+    refs = []
+    for h in heads:
+        rows = sorted(rng.choice(nb[h], size=48, replace=False).tolist())
+        Q = inp["Q"][:, h:h + 1].float().cpu().numpy()
+        K = inp["K"][:, h:h + 1].float().cpu().numpy()
+        sub = O.Plan(w.T, w.H, w.W, [ref_plan.heads[h]])
+        refs.append(O.select(Q, K, sub, w.topk_frac, w.topk_abs, w.top_p, scale_of(w.head_dim), rows=rows)[0])
+    _check_rows("1080p", w, sel, refs, heads, ref_plan)
 
 
 @pytest.mark.parametrize("name", ["small", "720p"])

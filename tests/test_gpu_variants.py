@@ -9,7 +9,7 @@ import torch
 from dynamic_block_sparse_stats_b200 import api
 from dynamic_block_sparse_stats_b200.synth import WORKLOADS, make_inputs
 from oracle import prism_oracle as O
-from tests.helpers import TIE, compare_plan, oracle_plan_from_shapes, scale_of, to_np
+from tests.helpers import TIE, check_ties, compare_plan, oracle_plan_from_shapes, scale_of, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -45,13 +45,13 @@ def test_plan_variant_matches_oracle(name, var):
     kw = dict(var)
     kw["map_exponent"] = kw.get("map_exponent", 0.5)
     ref = O.plan(inp["V"][:, heads].float().cpu().numpy(), inp["a"].cpu().numpy(), w.T, w.H, w.W, **kw)
-    excluded = compare_plan(w, pl, ref, heads)
+    excluded, total = compare_plan(w, pl, ref, heads)
+    check_ties(excluded, total, f"{name} {var} plan zones")
     B = to_np(pl.zone_shape)
     if var.get("tau128") == 0.0:
         assert (B[heads] <= 6).all()                       # ids 0..6 are the 64-token shapes
     if var.get("tau128") == 2.0:
         assert (B[heads] >= 13).all()                      # ids 13..15 are the 256-token shapes
-    print(f"{name} {var}: excluded at ties {excluded}")
 
 
 def test_plan_from_keys_matches_oracle():
@@ -98,10 +98,11 @@ def test_selection_variant_matches_oracle(name, var):
     ref = O.select(Q, K, ref_plan, kw["topk_frac"], kw["topk_abs"], kw["top_p"], scale_of(w.head_dim))
     row_ptr = to_np(sel.row_ptr).astype(np.int64)
     col = to_np(sel.col)[:sel.nnz]
-    excluded = 0
+    excluded = checked = 0
     for k, h in enumerate(heads):
         nb = ref_plan.heads[k].blocks.shape[0]
         for (i, ids, info) in ref[k]:
+            checked += 1
             got = col[row_ptr[h * NB + i]:row_ptr[h * NB + i + 1]]
             if got.size == ids.size and (got == ids).all():
                 continue
@@ -113,4 +114,4 @@ def test_selection_variant_matches_oracle(name, var):
         assert (counts >= 1).all() and (counts <= nb).all()
         if kw["top_p"] >= 1.0:
             assert (counts == nb).all()                    # p = 1 keeps every block
-    print(f"{name} {var}: rows excluded at ties {excluded}")
+    check_ties(excluded, checked, f"{name} {var} selection rows")

@@ -468,3 +468,44 @@ def test_backward_select_all_equals_torch_autograd():
     np.testing.assert_allclose(dQ[:, 0], q.grad.numpy(), atol=1e-11)
     np.testing.assert_allclose(dK[:, 0], k.grad.numpy(), atol=1e-11)
     np.testing.assert_allclose(dV[:, 0], v.grad.numpy(), atol=1e-11)
+
+
+def test_key_block_backward_matches_central_differences_and_the_full_backward():
+    """attention_bwd_key_block (one key block's dK, dV from the rows that
+    selected it) against float64 central differences of <O, dO> with respect
+    to that block's keys and values, and against attention_bwd's rows of the
+    same block, on every key block of a small grid."""
+    Q, K, V, pl = _small_problem(18, D=8)
+    sel = O.select(Q, K, pl, topk_abs=2, top_p=0.4)
+    rng = np.random.default_rng(19)
+    dO = rng.normal(size=Q.shape)
+    scale = 0.35
+    hp = pl.heads[0]
+    _, gK, gV = O.attention_bwd(Q, K, V, dO, pl, sel, scale)
+    rows = {i: ids for (i, ids, _info) in sel[0]}
+    nb = hp.blocks.shape[0]
+    for j in range(nb):
+        users = [(i, ids) for i, ids in rows.items() if j in ids]
+        kj, dK, dV = O.attention_bwd_key_block(Q[:, 0], K[:, 0], V[:, 0], dO[:, 0], hp, j, users, scale)
+        np.testing.assert_allclose(dK, gK[kj, 0], atol=1e-12)
+        np.testing.assert_allclose(dV, gV[kj, 0], atol=1e-12)
+
+    def f(Kx, Vx):
+        Ox, _ = O.attention_fwd(Q, Kx, Vx, pl, sel, scale)
+        return float((Ox * dO).sum())
+
+    j = max(range(nb), key=lambda b: sum(b in ids for ids in rows.values()))   # the most-used key block
+    users = [(i, ids) for i, ids in rows.items() if j in ids]
+    kj, dK, dV = O.attention_bwd_key_block(Q[:, 0], K[:, 0], V[:, 0], dO[:, 0], hp, j, users, scale)
+    eps = 1e-6
+    for t in (0, kj.size // 2, kj.size - 1):
+        for c in (0, 5):
+            for X, G in ((K, dK), (V, dV)):
+                Xp, Xm = X.copy(), X.copy()
+                Xp[kj[t], 0, c] += eps
+                Xm[kj[t], 0, c] -= eps
+                if X is K:
+                    num = (f(Xp, V) - f(Xm, V)) / (2 * eps)
+                else:
+                    num = (f(K, Xp) - f(K, Xm)) / (2 * eps)
+                assert abs(num - G[t, c]) < 1e-6 * max(1.0, abs(num)), (t, c, num, G[t, c])

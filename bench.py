@@ -37,7 +37,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from dynamic_block_sparse_stats_b200 import _lib, api  # noqa: E402
-from dynamic_block_sparse_stats_b200.synth import WORKLOADS, make_bridge_output, make_inputs  # noqa: E402
+from dynamic_block_sparse_stats_b200.synth import (WORKLOADS, make_bridge_output, make_inputs,  # noqa: E402
+                                                   make_projection)
 
 METRIC = "Prism sparse-attn fwd+bwd ms/layer & effective TFLOP/s at ~860K tokens"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -187,7 +188,7 @@ def read_kernel_times(lib):
     return out
 
 
-def kernel_rooflines(ktimes, P, D, N, h, nb, peaks, peak_src, steps, nnz=0, sm_mhz=None):
+def kernel_rooflines(ktimes, P, D, N, h, nb, peaks, peak_src, steps, nnz=0, sm_mhz=None, proj_c=None):
     """Per kernel: launches, ms per launch (CUDA events on the launching
     stream, timed region), algorithmic work per launch and its fraction of the
     measured peak: bf16 (sustained, for tensor kernels inside this long step;
@@ -240,6 +241,8 @@ def kernel_rooflines(ktimes, P, D, N, h, nb, peaks, peak_src, steps, nnz=0, sm_m
                      "dO, O, O_res read, fp16 dO written (8*N*h*D bytes) + LSE, Delta (16*N*h)"),
         "a2v_norm": ("hbm", 2.0 * HBD + 4.0 * N, None,
                      "one read of the bridge output (2*N*h*D bytes) + the fp32 norms (4*N)"),
+        "project_v": ("tensor", 2.0 * N * proj_c * h * D if proj_c else None, None,
+                      "2*N*C*h*D FLOP (V = X Wv^T; the zone statistics ride in its epilogue)"),
     }
     # nominal dense bf16 rate at the sampled SM clock: 148 SMs x 8192 FLOP per clock
     at_clock = 148 * 8192 * sm_mhz * 1e6 / 1e12 if sm_mhz else None
@@ -298,7 +301,7 @@ def kernel_rooflines(ktimes, P, D, N, h, nb, peaks, peak_src, steps, nnz=0, sm_m
 
 # The source file of each timed kernel, under the package's csrc/, and the
 # ncu kernel-name fragment that identifies its launches.
-KERNEL_SOURCES = {"zone_video_stats": "plan.cu", "zone_a2v_stats": "plan.cu", "plan_finalize": "plan.cu",
+KERNEL_SOURCES = {"project_v": "project.cu", "zone_video_stats": "plan.cu", "zone_a2v_stats": "plan.cu", "plan_finalize": "plan.cu",
                   "perm": "plan.cu", "block_mean": "select.cu", "block_score": "select.cu",
                   "select_row": "select.cu", "select_scan": "select.cu", "csr_fill": "select.cu",
                   "csc_count": "select.cu", "csc_scan": "select.cu", "csc_fill": "select.cu",
@@ -454,6 +457,16 @@ def oracle_sample(w, inp, head=0, n_rows=2, n_sel=512, seed=0):
     O.a2v_norm(hs)
     norm_time = (time.perf_counter() - tn) * (w.N / n_norm)
     del hs
+    proj_time, proj_desc = 0.0, ""
+    if "X" in inp and "Wv" in inp:    # the value projection of a row sample, all heads
+        n_pr = min(w.N, 2048)
+        Xs = inp["X"][:n_pr].float().cpu().numpy()
+        Ws = inp["Wv"].float().cpu().numpy()
+        tp = time.perf_counter()
+        O.project_v(Xs, Ws)
+        proj_time = (time.perf_counter() - tp) * (w.N / n_pr)
+        proj_desc = f"value projection of {n_pr} token rows (x{w.N / n_pr:.0f}, {proj_time:.2f}s); "
+        del Xs, Ws
     t0 = time.perf_counter()
     opl = O.plan(Vh, a, T, H, W)
     t1 = time.perf_counter()
@@ -479,9 +492,9 @@ def oracle_sample(w, inp, head=0, n_rows=2, n_sel=512, seed=0):
     pairs_rows = sum(int(hp.blocks[i, 4]) * int(hp.blocks[ids, 4].sum()) for (i, ids, _) in osel[0])
     P_total = pairs_rows * row_frac * w.heads
     attn_time = (t5 - t4) * (P_total / max(pairs_sample, 1))
-    layer_time = norm_time + w.heads * ((t1 - t0) + sel_time) + attn_time
+    layer_time = norm_time + proj_time + w.heads * ((t1 - t0) + sel_time) + attn_time
     threads = max([t.get("num_threads", 1) for t in threadpool_info()] + [1])
-    desc = (f"oracle A2V norms of {n_norm} bridge-output rows (x{w.N / n_norm:.1f}, {norm_time:.2f}s); "
+    desc = (f"oracle A2V norms of {n_norm} bridge-output rows (x{w.N / n_norm:.1f}, {norm_time:.2f}s); {proj_desc}"
             f"plan of head {head} over the full {T}x{H}x{W} grid ({t1 - t0:.2f}s, x{w.heads} heads); "
             f"selection of {len(sel_rows)} of its {nb} query blocks ({t3 - t2:.2f}s, of which block means "
             f"{t2 - t1:.2f}s; rows x{row_frac:.1f}, x{w.heads} heads); fwd{'+bwd' if dOh is not None else ''} "
@@ -569,6 +582,12 @@ def run_prism(args, w, rank, world, device):
         h = h1 - h0
     p = api.params_for(w)
     Q, K, V = inp["Q"], inp["K"], inp["V"]
+    # the layer's value projection, with the plan's zone statistics in its
+    # epilogue (the synthetic V becomes the projection's input features)
+    proj = not args.no_projection
+    if proj:
+        X, Wv = make_projection(V, seed=0 if heads_mode else rank_seed(rank))
+        inp["X"], inp["Wv"] = X, Wv
     # the previous layer's bridge output, whose row norms are this layer's A2V map
     hhat = make_bridge_output(inp["a"], (w.heads if not heads_mode else WORKLOADS[args.workload].heads) * D,
                               seed=0 if heads_mode else rank_seed(rank))
@@ -577,7 +596,10 @@ def run_prism(args, w, rank, world, device):
     backward = dO is not None
     # buffers reused by every step
     a = api.a2v_norm(hhat)
-    pl = api.plan(p, V, a)
+    if proj:
+        V, pl = api.project_v_plan(p, X, Wv, a)
+    else:
+        pl = api.plan(p, V, a)
     sel = api.select(p, pl, Q, K)
     sel = api.select(p, pl, Q, K, cap=int(sel.nnz * 1.1) + 1024)
     fw = api.attn_fwd(p, pl, sel, Q, K, V)
@@ -594,7 +616,10 @@ def run_prism(args, w, rank, world, device):
         if ev is not None:
             ev[0].record(stream)
         api.a2v_norm(hhat, out=a)
-        api.plan(p, V, a, out=pl)
+        if proj:
+            api.project_v_plan(p, X, Wv, a, V=V, out=pl)
+        else:
+            api.plan(p, V, a, out=pl)
         if ev is not None:
             ev[1].record(stream)
         api.select(p, pl, Q, K, out=sel)
@@ -646,10 +671,11 @@ def run_prism(args, w, rank, world, device):
     # end to end through host buffers
     e2e = None
     if not args.no_e2e:
-        hin = {k: inp[k].cpu().pin_memory() for k in (["Q", "K", "V", "hhat"] + (["dO"] if backward else []))}
+        names = ["Q", "K", "X" if proj else "V", "hhat"] + (["dO"] if backward else [])
+        hin = {k: inp[k].cpu().pin_memory() for k in names}
         outs = [O_] + (list(grads) if backward else [])
         hout = [torch.empty_like(t, device="cpu").pin_memory() for t in outs]
-        dev = {"Q": Q, "K": K, "V": V, "hhat": hhat, "dO": dO}
+        dev = {"Q": Q, "K": K, "V": V, "hhat": hhat, "dO": dO, "X": inp.get("X")}
         h2d = sum(t.numel() * t.element_size() for t in hin.values())
         d2h = sum(t.numel() * t.element_size() for t in hout)
 
@@ -681,7 +707,7 @@ def run_prism(args, w, rank, world, device):
     peaks, peak_src = load_peaks()
     nb = pl.n_blocks.long()
     kernels = kernel_rooflines(ktimes, P, D, N, h, nb, peaks, peak_src, args.steps, nnz=sel.nnz,
-                               sm_mhz=clocks.get("sm_mhz"))
+                               sm_mhz=clocks.get("sm_mhz"), proj_c=X.shape[1] if proj else None)
     for name in ("a2v_norm", "zone_video_stats", "zone_a2v_stats", "block_mean", "select_row"):
         rec = kernels.get(name)
         if rec and rec.get("achieved") is not None:   # read-dominated: also against a read-only stream
@@ -694,8 +720,10 @@ def run_prism(args, w, rank, world, device):
                 "traffic": stored_traffic(dom), "algorithmic": kd["algorithmic"],
                 "ms_per_launch": kd["ms_per_launch"]}
     peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
-    plan_bytes = N * h * D * 2 + N * 4        # the plan stage reads V and a; a2v_norm is in it too
-    plan_bytes += N * h * D * 2 + N * 4
+    # the plan stage: a2v_norm reads the bridge output, and the plan reads V
+    # (with the fused projection V is written instead, and X read)
+    plan_bytes = N * h * D * 2 + N * 4
+    plan_bytes += N * h * D * 2 + N * 4 if not proj else N * X.shape[1] * 2 + N * h * D * 2
     stage_roofline = {
         "plan_GBps": plan_bytes / (stage_ms["plan"] * 1e-3) / 1e9,
         "plan_frac_hbm": plan_bytes / (stage_ms["plan"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
@@ -730,6 +758,8 @@ def run_prism(args, w, rank, world, device):
         "config": {"workload": w.name, "T": w.T, "H": w.H, "W": w.W, "tokens": N,
                    "heads": WORKLOADS[args.workload].heads, "heads_per_rank": h, "head_dim": D,
                    "topk_frac": w.topk_frac, "top_p": w.top_p, "backward": backward,
+                   "plan_from": ("prism_project_v_plan: V = X Wv^T (C = %d) with the zone statistics in the "
+                                 "GEMM epilogue" % X.shape[1]) if proj else "prism_plan of a given V",
                    "parallelism": (f"heads split over {world} ranks (this rank {h0}-{h1 - 1}), no collectives on the path"
                                    if heads_mode else f"weak x{world} (independent layers, no collectives)"),
                    "l2": "inputs larger than L2 (each bf16 tensor %.2f GB)" % (N * h * D * 2 / 1e9),
@@ -753,6 +783,8 @@ def run_reference(args, w, rank, world):
     # only for speed); every computation below is the CPU oracle's
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = make_inputs(w, dev, seed=0)  # oracle_sample moves one head at a time to the host
+    if not args.no_projection:         # the same step as the library arm: plan from the value projection
+        inp["X"], inp["Wv"] = make_projection(inp["V"], seed=0)
     times, rates, desc, threads = [], [], "", 1
     for k in range(args.warmup + args.steps):
         lt, P, desc, threads, _wall = oracle_sample(w, inp, head=k % w.heads, seed=k)
@@ -783,6 +815,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense SDPA comparison")
+    ap.add_argument("--no-projection", action="store_true",
+                    help="plan from a given V (prism_plan) instead of the fused value projection "
+                         "(prism_project_v_plan) in the step")
     ap.add_argument("--write-traffic", metavar="NCU_CSV",
                     help="write profiles/traffic.json from an ncu DRAM-bytes capture and exit (no GPU needed)")
     ap.add_argument("--shard", choices=["layers", "heads"], default="layers",

@@ -28,9 +28,9 @@ EXPORTS = (
     "prism_attn_workspace_size", "prism_attn_fwd", "prism_attn_bwd", "prism_workspace_status",
     "prism_last_error", "prism_version", "prism_kernel_launches", "prism_plan_noalloc",
     "prism_kernel_timing", "prism_kernel_timing_read", "prism_a2v_norm", "prism_diag_exp2",
-    "prism_diag_wait_timeout",
+    "prism_diag_wait_timeout", "prism_project_v_plan",
 )
-KERNEL_TIMING_IDS = 21  # PRISM_KERNEL_TIMING_IDS in include/prism.h
+KERNEL_TIMING_IDS = 22  # PRISM_KERNEL_TIMING_IDS in include/prism.h
 
 
 class PrismParams(C.Structure):
@@ -90,6 +90,7 @@ def load() -> C.CDLL:
         "prism_a2v_norm": (C.c_int, [vp, C.c_int64, C.c_int32, C.c_int64, vp, st]),
         "prism_diag_exp2": (C.c_int, [vp, vp, vp, C.c_int64, st]),
         "prism_diag_wait_timeout": (C.c_int, [vp, sz, C.c_int64, st]),
+        "prism_project_v_plan": (C.c_int, [P(PrismParams), vp, C.c_int32, vp, vp, vp, P(PrismPlan), vp, sz, st]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)

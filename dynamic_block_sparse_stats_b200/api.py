@@ -194,6 +194,32 @@ def plan(p: PrismParams, V: torch.Tensor, a: torch.Tensor | None = None, out: Pl
     return out
 
 
+def project_v_plan(p: PrismParams, X: torch.Tensor, Wv: torch.Tensor, a: torch.Tensor | None = None,
+                   V: torch.Tensor | None = None, out: Plan | None = None, stream=None):
+    """prism_project_v_plan: V = X Wv^T (bf16 [N, heads, head_dim]) with the
+    plan computed from the zone statistics of the projection's own tiles.
+    X bf16 [N, C], Wv bf16 [heads*head_dim, C].  Returns (V, plan)."""
+    N = p.T * p.H * p.W
+    if not isinstance(X, torch.Tensor) or X.dim() != 2:
+        raise ValueError("X must be a 2-D tensor [N, C]")
+    Cin = X.shape[1]
+    _check_tensor(X, "X", torch.bfloat16, (N, Cin))
+    _check_tensor(Wv, "Wv", torch.bfloat16, (p.heads * p.head_dim, Cin))
+    if V is not None:
+        _check_tensor(V, "V", torch.bfloat16, (N, p.heads, p.head_dim))
+    if a is not None:
+        _check_tensor(a, "a2v_norm", torch.float32, (N,))
+    named = [("X", X), ("Wv", Wv), ("V", V), ("a2v_norm", a)] + (_check_plan(p, out) if out is not None else [])
+    dev = _check_devices(named)
+    with torch.cuda.device(dev):
+        V = V if V is not None else torch.empty((N, p.heads, p.head_dim), dtype=torch.bfloat16, device=dev)
+        out = out if out is not None else alloc_plan(p, dev)
+        cs = out.c_struct()
+        check(_lib.load().prism_project_v_plan(C.byref(p), _ptr(X), Cin, _ptr(Wv), _ptr(V), _ptr(a), C.byref(cs),
+                                               _ptr(out.ws), out.ws.numel(), _stream(stream, dev)))
+    return V, out
+
+
 @dataclass
 class Selection:
     """Output of prism_select (device tensors): a CSR over rows h*NB + i

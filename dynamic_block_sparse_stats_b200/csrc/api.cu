@@ -128,6 +128,26 @@ int prism_plan(const prism_params *p, const uint16_t *V, const float *a2v_norm, 
   return PRISM_OK;
 }
 
+int prism_project_v_plan(const prism_params *p, const uint16_t *X, int32_t C, const uint16_t *Wv, uint16_t *V,
+                         const float *a2v_norm, const prism_plan_t *out, void *workspace, size_t ws_bytes,
+                         prism_stream_t stream) {
+  int rc;
+  if ((rc = check_plan_call(p, V, a2v_norm, out)) != PRISM_OK) return rc;
+  if (!X || !Wv) return fail(PRISM_ERR_INVALID_ARG, "X or Wv is NULL");
+  if ((rc = check_aligned16(X, "X")) != PRISM_OK || (rc = check_aligned16(Wv, "Wv")) != PRISM_OK) return rc;
+  if (C <= 0 || C % 64 || C > (1 << 16))
+    return fail(PRISM_ERR_INVALID_ARG, "C must be a positive multiple of 64, at most 65536 (got %d)", C);
+  if ((rc = check_ws(workspace, ws_bytes, plan_ws_bytes(*p))) != PRISM_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, kWsHeader, st);
+  if (e == cudaSuccess)
+    e = launch_project_v(*p, X, C, Wv, V, plan_vstats(workspace), &static_cast<WsHeader *>(workspace)->status, st);
+  if (e == cudaSuccess) e = launch_plan_tail(*p, a2v_norm, *out, workspace, st);
+  if (e != cudaSuccess) return cuda_fail(e, "prism_project_v_plan");
+  g_last_error.clear();
+  return PRISM_OK;
+}
+
 size_t prism_select_workspace_size(const prism_params *p) {
   if (check_params(p) != PRISM_OK) return 0;
   return select_ws_bytes(*p);

@@ -13,6 +13,16 @@ namespace prism {
 size_t plan_ws_bytes(const prism_params &p);
 cudaError_t launch_plan(const prism_params &p, const uint16_t *V, const float *a, const prism_plan_t &out, void *ws,
                         cudaStream_t st);
+// the plan after the zone statistics of V (K1a, K2, K3), from the statistics
+// already in the workspace (plan_vstats)
+cudaError_t launch_plan_tail(const prism_params &p, const float *a, const prism_plan_t &out, void *ws,
+                             cudaStream_t st);
+// where the workspace holds the per-(head, zone) statistics of V: double [heads][Z][5]
+double *plan_vstats(void *ws);
+
+// project.cu
+cudaError_t launch_project_v(const prism_params &p, const uint16_t *X, int C, const uint16_t *Wv, uint16_t *V,
+                             double *vstats, int *status, cudaStream_t st);
 
 // select.cu
 size_t select_ws_bytes(const prism_params &p);
@@ -54,6 +64,10 @@ cudaError_t launch_tile_units(const int32_t *ptr, const int32_t *idx, const int3
                               cudaStream_t st);
 // 2-D fp16 tensor map over rows of D elements, box 64 x box_rows, 128B swizzle.
 cudaError_t make_rows_map(CUtensorMap *map, const void *base, long long rows, int D, int box_rows);
+// bf16 tensor map of rank 2..5, 128B swizzle (dims, box innermost first;
+// strides in bytes for dims 1..rank-1).
+cudaError_t make_bf16_map(CUtensorMap *map, const void *base, int rank, const unsigned long long *dims,
+                          const unsigned long long *strides, const unsigned *box);
 
 // host-side count of kernel launches (prism_kernel_launches)
 void count_launches(int n);
@@ -81,6 +95,7 @@ enum KernelTimingId {
   KT_UNIT_BLOCK,
   KT_TILE_UNITS,
   KT_BWD_PREP,
+  KT_PROJECT_V,
   KT_COUNT
 };
 static_assert(KT_COUNT == PRISM_KERNEL_TIMING_IDS, "timing ids");

@@ -9,6 +9,7 @@
 // sections 1 and 2 (sigma^2_{v,d}, r_{v,d}, g_d, B(m), l*_d, nearest
 // candidate in log2 space).
 #include "internal.h"
+#include "zone_stats.cuh"
 
 namespace prism {
 
@@ -37,154 +38,25 @@ __host__ __device__ constexpr ShapeTable make_shape_table() {
 __constant__ ShapeTable c_shapes = make_shape_table();
 
 // ---------------------------------------------------------------------------
-// K1: per (zone, head) statistics of V.
-// 8 warps; warp t owns frame t of the zone.  Lane = (channel vector cv of 8
-// channels, token group xg).  For every row y the warp forms the fp32 row
-// sum over x (fixed shuffle tree, identical for every frame so that equal
-// frames give bit-equal frame sums), keeps fp32 column sums over y, and a
-// sum of squares.  The 8-term partial sums are combined in float64.
-//   out[h][z][0..4] = sigma2_T, sigma2_H, sigma2_W, spatial, temporal
+// K1: per (zone, head) statistics of V (arithmetic in zone_stats.cuh, shared
+// with the value projection's epilogue).  One 256-thread CTA per (zone, head).
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) zone_video_stats_kernel(const uint16_t *__restrict__ V, int T, int H, int W,
                                                                int heads, double *__restrict__ out) {
-  constexpr int CV = D / 8;     // 16-byte channel vectors per token
-  constexpr int GPL = 32 / CV;  // token groups per warp row
-  constexpr int TPL = 8 / GPL;  // tokens per lane
   extern __shared__ __align__(16) float zs_smem[];
-  float(*rowsum)[8][D] = reinterpret_cast<float(*)[8][D]>(zs_smem);                // [t][y][c]
-  float(*colsum)[8][D] = reinterpret_cast<float(*)[8][D]>(zs_smem + 8 * 8 * D);    // [t][x][c]
   __shared__ double red[8][8];
-
   const int z = blockIdx.x, h = blockIdx.y;
   const int ZH = H / 8, ZW = W / 8;
   const int zt = z / (ZH * ZW), zh = (z / ZW) % ZH, zw = z % ZW;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = warp;
-  const int cv = lane % CV, xg = lane / CV;
-
-  float colacc[TPL][8];
-#pragma unroll
-  for (int i = 0; i < TPL; ++i)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) colacc[i][c] = 0.f;
-  double sq = 0.0;
-
   const size_t tok_stride = (size_t)heads * D;  // elements between tokens
-  const uint16_t *base = V + (size_t)h * D + cv * 8;
-#pragma unroll 2
-  for (int y = 0; y < 8; ++y) {
-    const size_t n0 = ((size_t)(zt * 8 + t) * H + (zh * 8 + y)) * W + zw * 8 + xg * TPL;
-    uint4 raw[TPL];
-#pragma unroll
-    for (int i = 0; i < TPL; ++i) raw[i] = __ldg(reinterpret_cast<const uint4 *>(base + (n0 + i) * tok_stride));
-    float r[8];
-    float s2 = 0.f;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) r[c] = 0.f;
-#pragma unroll
-    for (int i = 0; i < TPL; ++i) {
-      const uint32_t w4[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float a = bf16lo(w4[q]), b = bf16hi(w4[q]);
-        r[2 * q] += a;
-        r[2 * q + 1] += b;
-        colacc[i][2 * q] += a;
-        colacc[i][2 * q + 1] += b;
-        s2 = fmaf(a, a, s2);
-        s2 = fmaf(b, b, s2);
-      }
-    }
-    sq += (double)s2;
-    // combine the token groups of this row: fixed tree
-#pragma unroll
-    for (int o = CV; o < 32; o <<= 1)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) r[c] += __shfl_xor_sync(0xffffffffu, r[c], o);
-    if (xg == 0) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) rowsum[t][y][cv * 8 + c] = r[c];
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < TPL; ++i)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) colsum[t][xg * TPL + i][cv * 8 + c] = colacc[i][c];
-  sq = warp_sum(sq);
-  if (lane == 0) red[warp][5] = sq;
-  __syncthreads();
-
-  // Per channel (first D threads): profiles along T, H, W in float64.
-  double acc[5] = {0, 0, 0, 0, 0};  // var_T, var_H, var_W, temporal, sum_t mu_t^2
-  if (threadIdx.x < D) {
-    const int c = threadIdx.x;
-    double pT[8], pH[8], pW[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      pT[i] = 0.0;
-      pH[i] = 0.0;
-      pW[i] = 0.0;
-    }
-#pragma unroll
-    for (int a = 0; a < 8; ++a)
-#pragma unroll
-      for (int b = 0; b < 8; ++b) {
-        const double rv = (double)rowsum[a][b][c];
-        pT[a] += rv;
-        pH[b] += rv;
-        pW[b] += (double)colsum[a][b][c];
-      }
-    const double inv64 = 1.0 / 64.0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      pT[i] *= inv64;
-      pH[i] *= inv64;
-      pW[i] *= inv64;
-    }
-    double mT = 0, mH = 0, mW = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      mT += pT[i];
-      mH += pH[i];
-      mW += pW[i];
-    }
-    mT *= 0.125;
-    mH *= 0.125;
-    mW *= 0.125;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      acc[0] += (pT[i] - mT) * (pT[i] - mT);
-      acc[1] += (pH[i] - mH) * (pH[i] - mH);
-      acc[2] += (pW[i] - mW) * (pW[i] - mW);
-      acc[4] += pT[i] * pT[i];
-    }
-    acc[0] *= 0.125;
-    acc[1] *= 0.125;
-    acc[2] *= 0.125;
-#pragma unroll
-    for (int i = 0; i < 7; ++i) acc[3] += (pT[i + 1] - pT[i]) * (pT[i + 1] - pT[i]);
-    acc[3] *= (1.0 / 7.0);
-  }
-#pragma unroll
-  for (int k = 0; k < 5; ++k) acc[k] = warp_sum(acc[k]);
-  if (lane == 0)
-#pragma unroll
-    for (int k = 0; k < 5; ++k) red[warp][k] = acc[k];
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double tot[6] = {0, 0, 0, 0, 0, 0};
-    for (int w = 0; w < 8; ++w)
-      for (int k = 0; k < 6; ++k) tot[k] += red[w][k];
-    double *o = out + ((size_t)h * gridDim.x + z) * 5;
-    o[0] = tot[0] / D;
-    o[1] = tot[1] / D;
-    o[2] = tot[2] / D;
-    // sum over t,y,x,c of (V - frame mean)^2 = sum V^2 - 64 sum_{t,c} mu_t,c^2
-    double sp = (tot[5] - 64.0 * tot[4]) / (512.0 * D);
-    o[3] = sp > 0.0 ? sp : 0.0;
-    o[4] = tot[3] / D;
-  }
+  const uint16_t *base = V + (size_t)h * D;
+  const auto load = [&](int t, int y, int x, int cv) {
+    const size_t n = ((size_t)(zt * 8 + t) * H + (zh * 8 + y)) * W + zw * 8 + x;
+    return __ldg(reinterpret_cast<const uint4 *>(base + n * tok_stride + cv * 8));
+  };
+  zone_stats_core<D>(load, threadIdx.x, zs_smem, red, out + ((size_t)h * gridDim.x + z) * 5,
+                     [] { __syncthreads(); });
 }
 
 // ---------------------------------------------------------------------------
@@ -407,8 +279,10 @@ size_t plan_ws_bytes(const prism_params &p) {
   return s;
 }
 
-cudaError_t launch_plan(const prism_params &p, const uint16_t *V, const float *a, const prism_plan_t &out, void *ws,
-                        cudaStream_t st) {
+double *plan_vstats(void *ws) { return reinterpret_cast<double *>(static_cast<char *>(ws) + kWsHeader); }
+
+cudaError_t launch_plan_tail(const prism_params &p, const float *a, const prism_plan_t &out, void *ws,
+                             cudaStream_t st) {
   const int Z = (p.T / 8) * (p.H / 8) * (p.W / 8);
   const int N = p.T * p.H * p.W;
   const int NB = N / 64;
@@ -418,19 +292,6 @@ cudaError_t launch_plan(const prism_params &p, const uint16_t *V, const float *a
   double *astats = reinterpret_cast<double *>(w);
   w += align_up(sizeof(double) * Z * 4, 256);
   int32_t *zone_first = reinterpret_cast<int32_t *>(w);
-
-  dim3 g1(Z, p.heads);
-  {
-  KernelTimer kt_(KT_ZONE_STATS, st);
-  if (p.head_dim == 128) {
-    const int sm = 2 * 8 * 8 * 128 * sizeof(float);
-    cudaFuncSetAttribute(zone_video_stats_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-    zone_video_stats_kernel<128><<<g1, 256, sm, st>>>(V, p.T, p.H, p.W, p.heads, vstats);
-  } else {
-    const int sm = 2 * 8 * 8 * 64 * sizeof(float);
-    zone_video_stats_kernel<64><<<g1, 256, sm, st>>>(V, p.T, p.H, p.W, p.heads, vstats);
-  }
-  }
   if (a) {
     KernelTimer kt_(KT_ZONE_A2V_STATS, st);
     zone_a2v_stats_kernel<<<Z, 64, 0, st>>>(a, p.T, p.H, p.W, astats);
@@ -447,8 +308,30 @@ cudaError_t launch_plan(const prism_params &p, const uint16_t *V, const float *a
     KernelTimer kt_(KT_PERM, st);
     perm_kernel<<<g3, 256, 0, st>>>(out.zone_shape, p.T, p.H, p.W, Z, out.perm, out.inv_perm);
   }
-  count_launches(a ? 4 : 3);
+  count_launches(a ? 3 : 2);
   return cudaGetLastError();
+}
+
+cudaError_t launch_plan(const prism_params &p, const uint16_t *V, const float *a, const prism_plan_t &out, void *ws,
+                        cudaStream_t st) {
+  const int Z = (p.T / 8) * (p.H / 8) * (p.W / 8);
+  double *vstats = plan_vstats(ws);
+  dim3 g1(Z, p.heads);
+  {
+  KernelTimer kt_(KT_ZONE_STATS, st);
+  if (p.head_dim == 128) {
+    const int sm = 2 * 8 * 8 * 128 * sizeof(float);
+    cudaFuncSetAttribute(zone_video_stats_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    zone_video_stats_kernel<128><<<g1, 256, sm, st>>>(V, p.T, p.H, p.W, p.heads, vstats);
+  } else {
+    const int sm = 2 * 8 * 8 * 64 * sizeof(float);
+    zone_video_stats_kernel<64><<<g1, 256, sm, st>>>(V, p.T, p.H, p.W, p.heads, vstats);
+  }
+  }
+  count_launches(1);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_plan_tail(p, a, out, ws, st);
 }
 
 }  // namespace prism

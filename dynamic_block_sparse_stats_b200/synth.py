@@ -87,7 +87,7 @@ WORKLOADS = {
 }
 
 # tensor ids used as generator streams
-_ID_VBG, _ID_VREG, _ID_F, _ID_N1, _ID_N2, _ID_ANOISE, _ID_DO, _ID_LAYOUT, _ID_HHAT = range(1, 10)
+_ID_VBG, _ID_VREG, _ID_F, _ID_N1, _ID_N2, _ID_ANOISE, _ID_DO, _ID_LAYOUT, _ID_HHAT, _ID_WV = range(1, 11)
 _CHUNK = 256  # channels per generation chunk (fixed, so bits do not depend on memory)
 
 
@@ -318,3 +318,22 @@ def make_bridge_output(a: torch.Tensor, width: int, seed: int = 0) -> torch.Tens
         out[:, c0:c1] = (scale * z).to(torch.bfloat16)
         del z
     return out
+
+
+def make_projection(V: torch.Tensor, seed: int = 0):
+    """Inputs of a value projection whose output has the workload's value
+    structure: X = the workload's V viewed as token features [N, heads*D]
+    (bf16), and Wv [heads*D, heads*D] (bf16) block-diagonal with one seeded
+    random orthogonal D x D block per head (the Q factor of a Gaussian
+    matrix).  An orthogonal mix of a head's channels keeps every sum of
+    squares over its channels, so X Wv^T carries the workload's zone
+    structure; the projection still multiplies the full dense matrix."""
+    N, h, D = V.shape
+    X = V.reshape(N, h * D).contiguous()
+    W = torch.zeros((h * D, h * D), dtype=torch.float32)
+    for k in range(h):
+        g = torch.randn((D, D), generator=_gen("cpu", seed, _ID_WV, k), dtype=torch.float64)
+        q, r = torch.linalg.qr(g)
+        q = q * torch.sign(torch.diagonal(r)).view(1, D)
+        W[k * D:(k + 1) * D, k * D:(k + 1) * D] = q.float()
+    return X, W.to(torch.bfloat16).to(V.device)

@@ -188,6 +188,34 @@ int prism_plan(const prism_params *p, const uint16_t *V, const float *a2v_norm,
                prism_stream_t stream);
 
 /*
+ * prism_project_v_plan -- the layer's value projection with the plan fused
+ * into it: V = X Wv^T for every video token, on tcgen05 tensor cores, with
+ * prism_plan's zone statistics of V computed in the GEMM's epilogue from the
+ * tile just produced (the statistics come from the value features the
+ * attention computes anyway: digest, section on zone guidance and Figure 4),
+ * then the rest of prism_plan.  The plan never reads V back from memory; its
+ * outputs are bit-identical to prism_plan(p, V, a2v_norm) on the V written
+ * here (the statistics use the same arithmetic, in the same order).
+ *   X         bf16 [N][C] token features, natural token order.
+ *   C         channels of X: a positive multiple of 64, at most 65536.
+ *   Wv        bf16 [heads*head_dim][C] projection weight (output x input, the
+ *             layout of a linear layer's weight); output channel h*head_dim+d
+ *             is channel d of head h.
+ *   V         bf16 [N][heads][head_dim] output: X Wv^T, accumulated in fp32 and
+ *             rounded to bf16.
+ *   a2v_norm, out, workspace, ws_bytes  as prism_plan (the workspace size is
+ *             prism_plan_workspace_size(p)).
+ * X, Wv and V must be 16-byte aligned.  Returns PRISM_OK,
+ * PRISM_ERR_INVALID_ARG, PRISM_ERR_UNSUPPORTED, PRISM_ERR_CAPACITY or
+ * PRISM_ERR_CUDA; a kernel that gives up on an internal wait records
+ * PRISM_ERR_TIMEOUT in the workspace (prism_workspace_status).
+ */
+int prism_project_v_plan(const prism_params *p, const uint16_t *X, int32_t C,
+                         const uint16_t *Wv, uint16_t *V, const float *a2v_norm,
+                         const prism_plan_t *out, void *workspace,
+                         size_t ws_bytes, prism_stream_t stream);
+
+/*
  * prism_plan_noalloc -- the same computation and outputs as prism_plan, for
  * callers that cannot allocate device memory.  Some hosts own every device
  * allocation themselves (a plugin inside another program's memory manager),
@@ -348,8 +376,9 @@ int prism_kernel_timing(int enable);
  * 1 block_mean, 2 block_score, 3 select_row, 4 attn_fwd, 5 attn_bwd_dkdv,
  * 6 attn_bwd_dq, 7 a2v_norm, 8 zone_a2v_stats, 9 plan_finalize, 10 perm,
  * 11 select_scan, 12 csr_fill, 13 csc_count, 14 csc_scan, 15 csc_fill,
- * 16 csc_sort, 17 permute3, 18 unit_block, 19 tile_units, 20 bwd_prep. */
-#define PRISM_KERNEL_TIMING_IDS 21
+ * 16 csc_sort, 17 permute3, 18 unit_block, 19 tile_units, 20 bwd_prep,
+ * 21 project_v. */
+#define PRISM_KERNEL_TIMING_IDS 22
 
 /* Reads the records of kernel `id` (0 .. PRISM_KERNEL_TIMING_IDS - 1): waits
  * for its events, and returns the number of timed launches, their total

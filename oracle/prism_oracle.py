@@ -290,6 +290,15 @@ def permutation(T, H, W, blocks):
     return perm
 
 
+def project_v(X, Wv):
+    """The layer's value features V = X Wv^T ([DIGEST] zone-guidance section
+    and Figure 4: the zone statistics are taken from the value features that
+    the video self-attention computes from the tokens).  X [N, C], Wv
+    [heads*D, C] (linear-layer weight layout); float64, from the given
+    (bf16-rounded) values.  Returns [N, heads*D]."""
+    return np.asarray(X, dtype=np.float64) @ np.asarray(Wv, dtype=np.float64).T
+
+
 def density_raw(spatial, temporal, abar_raw, mode=0):
     """rho_raw(m) ([DIGEST] density section: the intra-zone spatial variance
     plus the temporal frame-difference variance).  The density ablation of

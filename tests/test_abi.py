@@ -139,3 +139,24 @@ def test_misaligned_tensor_pointers_are_rejected_before_any_cuda_call():
     rc = lib.prism_attn_bwd(C.byref(p), C.byref(plan), C.byref(sel), *[C.c_void_p(256)] * 5, C.c_void_p(256),
                             C.c_void_p(256), C.c_void_p(256), C.c_void_p(260), C.c_void_p(256), 1, ws, 1 << 40, None)
     assert rc == _lib.PRISM_ERR_INVALID_ARG and "dK" in lib.prism_last_error().decode()
+
+
+@pytest.mark.parametrize("C_", [0, 32, 100, 70000])
+def test_project_v_plan_rejects_bad_channel_counts(C_):
+    lib = _lib.load()
+    p = api.params(8, 16, 16, 1, 64, topk_abs=2)
+    dummy = _lib.PrismPlan(256, 256, 256, 256, 256, 256, 256)
+    rc = lib.prism_project_v_plan(C.byref(p), C.c_void_p(256), C_, C.c_void_p(256), C.c_void_p(256), None,
+                                  C.byref(dummy), C.c_void_p(256), 1 << 20, None)
+    assert rc == _lib.PRISM_ERR_INVALID_ARG
+    assert "multiple of 64" in lib.prism_last_error().decode()
+
+
+def test_project_v_plan_rejects_null_and_misaligned_inputs():
+    lib = _lib.load()
+    p = api.params(8, 16, 16, 1, 64, topk_abs=2)
+    dummy = _lib.PrismPlan(256, 256, 256, 256, 256, 256, 256)
+    for X, Wv in ((None, 256), (256, None), (264, 256), (256, 260)):
+        rc = lib.prism_project_v_plan(C.byref(p), C.c_void_p(X) if X else None, 64, C.c_void_p(Wv) if Wv else None,
+                                      C.c_void_p(256), None, C.byref(dummy), C.c_void_p(256), 1 << 20, None)
+        assert rc == _lib.PRISM_ERR_INVALID_ARG, (X, Wv)

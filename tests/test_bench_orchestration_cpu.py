@@ -23,7 +23,7 @@ _KERNEL_MS = {"zone_video_stats": 0.1, "block_mean": 0.2, "block_score": 0.05, "
               "attn_bwd_dkdv": 15.0, "attn_bwd_dq": 10.0, "a2v_norm": 0.05, "zone_a2v_stats": 0.01,
               "plan_finalize": 0.02, "perm": 0.01, "select_scan": 0.01, "csr_fill": 0.01, "csc_count": 0.01,
               "csc_scan": 0.01, "csc_fill": 0.01, "csc_sort": 0.01, "permute3": 0.05, "unit_block": 0.01,
-              "tile_units": 0.01, "bwd_prep": 0.03}
+              "tile_units": 0.01, "bwd_prep": 0.03, "project_v": 0.5}
 
 
 class _Lib:
@@ -121,8 +121,13 @@ def _oracle_api(monkeypatch, w):
         calls.append("attn_bwd")
         return out if out is not None else tuple(torch.zeros_like(Q) for _ in range(3))
 
+    def project_v_plan(p, X, Wv, a, V=None, out=None, stream=None):
+        calls.append("project_v_plan")
+        Vx = (X.float() @ Wv.float().T).to(torch.bfloat16).view(w.N, w.heads, w.head_dim)
+        return Vx, plan(p, Vx, a, out=out)
+
     for name, fn in (("a2v_norm", a2v_norm), ("plan", plan), ("select", select), ("attn_fwd", attn_fwd),
-                     ("attn_bwd", attn_bwd)):
+                     ("attn_bwd", attn_bwd), ("project_v_plan", project_v_plan)):
         monkeypatch.setattr(api, name, fn)
     return calls, state
 
@@ -138,7 +143,7 @@ def test_run_prism_orchestration_on_cpu(monkeypatch):
     monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
     monkeypatch.setattr(bench, "read_stream_gbs", lambda device: 7000.0)
     args = argparse.Namespace(steps=2, warmup=3, no_e2e=True, no_cpu_baseline=False, no_dense=True,
-                              shard="layers", workload="tiny", backward=True)
+                              shard="layers", workload="tiny", backward=True, no_projection=False)
     line = bench.run_prism(args, w, rank=0, world=1, device=torch.device("cpu"))
     json.dumps(line)                                        # serialisable as one JSON line
 
@@ -165,6 +170,10 @@ def test_run_prism_orchestration_on_cpu(monkeypatch):
     assert set(line["stage_ms"]) == {"plan", "select", "fwd", "bwd"}
     assert line["clocks"]["reasons"] == ["nvidia-smi unavailable"] or "sm_mhz" in line["clocks"]
     assert set(line["kernels"]) == set(_KERNEL_MS) | {"attn_bwd", "attn_fwd_bwd"}
+    # every step plans through the fused projection (whose stand-in plans with the oracle)
+    assert calls.count("project_v_plan") == 1 + 3 + 2 == calls.count("plan")
+    pv = line["kernels"]["project_v"]                     # 2*N*C*h*D FLOP per launch, C = h*D here
+    assert pv["achieved"] == pytest.approx(2.0 * w.N * (w.heads * w.head_dim) ** 2 / 0.5e-3 / 1e12)
     assert len(_KERNEL_MS) == _lib.KERNEL_TIMING_IDS
     bwd = line["kernels"]["attn_bwd"]                       # the backward on the 10*P*D convention
     assert bwd["achieved"] == pytest.approx(10.0 * P * w.head_dim / 25e-3 / 1e12, rel=1e-12)

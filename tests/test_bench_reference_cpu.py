@@ -48,7 +48,7 @@ def test_sampler_extrapolates_a_row_sample_by_its_fraction():
 
 def test_reference_arm_prints_the_contract():
     w = WORKLOADS["tiny"]
-    args = argparse.Namespace(warmup=3, steps=2)
+    args = argparse.Namespace(warmup=3, steps=2, no_projection=False)
     line = bench.run_reference(args, w, rank=0, world=1)
     assert line["impl"] == "reference" and line["steps"] == 2 and line["warmup"] == 3
     assert line["unit"] == "TFLOP/s" and line["higher_is_better"] is True and line["value"] > 0

@@ -199,3 +199,40 @@ def test_topk_only_and_topp_only_rows():
         assert sorted(kept) == sorted(order[:n])
         kept, _ = O.hybrid_select_row(s, 1, 1.0)                 # p = 1 keeps every block
         assert sorted(kept) == list(range(nb))
+
+
+def test_value_projection_closed_forms():
+    """project_v: the identity weight returns X; a permutation weight permutes
+    X's channels; a loop over the definition on a tiny case; linearity in
+    Wv."""
+    rng = np.random.default_rng(31)
+    X = rng.normal(size=(6, 8))
+    np.testing.assert_array_equal(O.project_v(X, np.eye(8)), X)
+    perm = rng.permutation(8)
+    Wp = np.eye(8)[perm]                       # output channel o reads input channel perm[o]
+    np.testing.assert_array_equal(O.project_v(X, Wp), X[:, perm])
+    W = rng.normal(size=(4, 8))
+    loop = np.array([[sum(X[n, c] * W[o, c] for c in range(8)) for o in range(4)] for n in range(6)])
+    np.testing.assert_allclose(O.project_v(X, W), loop, rtol=1e-14, atol=1e-14)
+    W2 = rng.normal(size=(4, 8))
+    np.testing.assert_allclose(O.project_v(X, W + 2.0 * W2), O.project_v(X, W) + 2.0 * O.project_v(X, W2),
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_plan_from_orthogonally_mixed_values_equals_plan_from_values():
+    """The projection inputs the benchmark uses (synth.make_projection): a
+    per-head orthogonal mix of the channels keeps the zone statistics, so the
+    oracle's plan of X Wv^T equals its plan of V (up to float64 rounding in
+    the statistics, far from any decision on this grid)."""
+    import torch
+    from dynamic_block_sparse_stats_b200.synth import WORKLOADS, make_inputs, make_projection
+    w = WORKLOADS["small"]
+    inp = make_inputs(w, "cpu")
+    X, Wv = make_projection(inp["V"])
+    Vp = O.project_v(X.float().numpy(), Wv.float().numpy()).reshape(w.N, w.heads, w.head_dim)
+    a = inp["a"].numpy()
+    ref = O.plan(inp["V"].float().numpy(), a, w.T, w.H, w.W)
+    got = O.plan(Vp, a, w.T, w.H, w.W)
+    for hr, hg in zip(ref.heads, got.heads):
+        np.testing.assert_allclose(hg.rho, hr.rho, rtol=1e-2, atol=1e-3)
+        assert (hg.shape == hr.shape).mean() > 0.97

@@ -148,7 +148,8 @@ __global__ void __launch_bounds__(256) block_score_kernel(const float *__restric
 // does not depend on the order of the atomic additions: the selection is
 // deterministic.  With p >= 1 every block is kept (in exact arithmetic the
 // cumulative probability reaches 1 only at the last block).  A
-// most-significant-byte radix descent over the keys finds the Top-p crossing
+// most-significant-digit radix descent over the keys (8-bit digits, from the
+// highest bit in which the row's keys differ) finds the Top-p crossing
 // key and the Top-k threshold without sorting; the kept ids are emitted in
 // ascending order into the row's own scratch, and the count into counts[i].
 // ---------------------------------------------------------------------------
@@ -182,6 +183,7 @@ struct SelShared {
   int wtot2[kSelThreads / 32];
   unsigned long long zred[kSelThreads / 32];
   uint32_t ured[kSelThreads / 32];
+  uint32_t ured2[kSelThreads / 32];
   // descent state broadcast
   uint32_t prefix;
   int found;
@@ -298,19 +300,35 @@ __global__ void __launch_bounds__(kSelThreads) select_row_kernel(float *__restri
   float *ev = reinterpret_cast<float *>(sel_smem + ((NB + 3) & ~3));
   float *row = S + (size_t)i * NB;
 
-  // 1. keys and the maximum
-  uint32_t kmax = 0;
+  // 1. keys, their maximum and minimum
+  uint32_t kmax = 0, kmin = 0xffffffffu;
   for (int j = tid; j < nb; j += kSelThreads) {
     const uint32_t u = score_key(row[j]);
     key[j] = u;
     kmax = max(kmax, u);
+    kmin = min(kmin, u);
   }
   kmax = warp_max(kmax);
-  if (lane == 0) sh.ured[warp] = kmax;
+  kmin = ~warp_max(~kmin);
+  if (lane == 0) {
+    sh.ured[warp] = kmax;
+    sh.ured2[warp] = kmin;
+  }
   __syncthreads();
   kmax = 0;
-  for (int w = 0; w < kSelThreads / 32; ++w) kmax = max(kmax, sh.ured[w]);
+  kmin = 0xffffffffu;
+  for (int w = 0; w < kSelThreads / 32; ++w) {
+    kmax = max(kmax, sh.ured[w]);
+    kmin = min(kmin, sh.ured2[w]);
+  }
   const double m = (double)key_score(kmax);
+  // The radix descent below only resolves the bits in which the row's keys
+  // differ: the bits above the highest differing bit hb are common to every
+  // key, so the first 8-bit digit is taken just below them, where the keys
+  // spread over all 256 buckets (starting at the top byte would put nearly
+  // every key of a row into one or two buckets).  At least one full digit.
+  const int hb = max(31 - __clz((int)(kmax ^ kmin)), 7);  // clz(0) = 32 gives -1
+  const uint32_t common = hb >= 31 ? 0u : ~((2u << hb) - 1u);
 
   // 2. weights, quantised to multiples of 2^-qb, and their exact total
   const int qb = 62 - (32 - __clz(nb));  // nb < 2^(32 - clz(nb)), so the total stays below 2^62
@@ -355,16 +373,18 @@ __global__ void __launch_bounds__(kSelThreads) select_row_kernel(float *__restri
     n_p = nb;
   } else if (top_p > 0.0f) {
     if (tid == 0) {
-      sh.prefix = 0;
+      sh.prefix = kmax & common;
       sh.cabove = 0;
       sh.sabove = 0;
       sh.found = 1;
     }
     __syncthreads();
-    uint32_t pmask = 0;
+    uint32_t pmask = common, last_mask = 255u;
     bool ok = true;
-    for (int level = 0; level < 4; ++level) {
-      const int shift = 24 - 8 * level;
+    for (int hi = hb + 1; hi > 0; hi -= 8) {  // digit = key bits [lo, hi)
+      const int shift = max(hi - 8, 0);
+      const uint32_t dmask = (1u << (hi - shift)) - 1u;
+      last_mask = dmask;
       for (int b = tid; b < 256; b += kSelThreads) {
         sh.hcnt[b] = 0;
         sh.hsum[b] = 0;
@@ -374,7 +394,7 @@ __global__ void __launch_bounds__(kSelThreads) select_row_kernel(float *__restri
       for (int j = tid; j < nb; j += kSelThreads) {
         const uint32_t u = key[j];
         if ((u & pmask) == prefix) {
-          const int b = (u >> shift) & 255;
+          const int b = (u >> shift) & dmask;
           atomicAdd(&sh.hcnt[b], 1);
           atomicAdd(&sh.hsum[b], quant_weight(ev[j], qscale));
         }
@@ -386,14 +406,14 @@ __global__ void __launch_bounds__(kSelThreads) select_row_kernel(float *__restri
         ok = false;
         break;
       }
-      pmask |= 0xffu << shift;
+      pmask |= dmask << shift;
     }
     if (!ok) {
       n_p = nb;  // cannot happen for p < 1 (target <= Z); kept as a safe bound
     } else {
       // every key of the final bucket is the same score, hence the same weight
       const uint32_t ustar = sh.prefix;
-      const int cstar = sh.hcnt[ustar & 255];
+      const int cstar = sh.hcnt[ustar & last_mask];  // the last digit is bits [0, width)
       const unsigned long long estar = quant_weight(score_weight(key_score(ustar), m), qscale);
       const unsigned long long sab = sh.sabove;
       int q = 1;
@@ -410,15 +430,16 @@ __global__ void __launch_bounds__(kSelThreads) select_row_kernel(float *__restri
   if (!(have_thr && n == n_p)) {
     // count-based radix select of the n-th largest key
     if (tid == 0) {
-      sh.prefix = 0;
+      sh.prefix = kmax & common;
       sh.cabove = 0;
       sh.sabove = 0;
       sh.found = 1;
     }
     __syncthreads();
-    uint32_t pmask = 0;
-    for (int level = 0; level < 4; ++level) {
-      const int shift = 24 - 8 * level;
+    uint32_t pmask = common;
+    for (int hi = hb + 1; hi > 0; hi -= 8) {  // digit = key bits [lo, hi)
+      const int shift = max(hi - 8, 0);
+      const uint32_t dmask = (1u << (hi - shift)) - 1u;
       for (int b = tid; b < 256; b += kSelThreads) {
         sh.hcnt[b] = 0;
         sh.hsum[b] = 0;
@@ -427,12 +448,12 @@ __global__ void __launch_bounds__(kSelThreads) select_row_kernel(float *__restri
       const uint32_t prefix = sh.prefix;
       for (int j = tid; j < nb; j += kSelThreads) {
         const uint32_t u = key[j];
-        if ((u & pmask) == prefix) atomicAdd(&sh.hcnt[(u >> shift) & 255], 1);
+        if ((u & pmask) == prefix) atomicAdd(&sh.hcnt[(u >> shift) & dmask], 1);
       }
       __syncthreads();
       if (warp == 0) bucket_descent(sh, false, 0ull, n, shift);
       __syncthreads();
-      pmask |= 0xffu << shift;
+      pmask |= dmask << shift;
     }
     thr = sh.prefix;
     need = n - sh.cabove;

@@ -2,8 +2,9 @@
 statistics in its epilogue) through the C ABI.
 
   * V = X Wv^T against the oracle's float64 product: within the bf16
-    rounding of the output (half an ulp, 2^-9 relative) plus the fp32
-    accumulation error (C * 2^-24 * sum_c |x_c w_c|, taken four times);
+    rounding of the output (half an ulp: at most 2^-8 of the value, bf16
+    having 8 significant bits) plus the fp32 accumulation error
+    (C * 2^-24 * sum_c |x_c w_c|, taken four times);
   * the plan from the epilogue's statistics is bit-identical to prism_plan's
     plan of the V just written (both run the same statistics arithmetic);
   * stage-wise, that plan equals the oracle's plan of the same V except at
@@ -42,7 +43,7 @@ def _check_v(X, Wv, V, rows):
     ref = O.project_v(Xh, Wh)
     mag = np.abs(Xh) @ np.abs(Wh).T
     got = V.reshape(V.shape[0], -1)[idx].float().cpu().numpy()
-    bound = 2.0 ** -9 * np.abs(ref) + 4.0 * Xh.shape[1] * 2.0 ** -24 * mag + 1e-30
+    bound = 2.0 ** -8 * np.abs(ref) + 4.0 * Xh.shape[1] * 2.0 ** -24 * mag + 1e-30
     err = np.abs(got - ref)
     print(f"V: max |err| / bound = {(err / bound).max():.3f} over {err.size} values")
     assert (err <= bound).all()

@@ -460,26 +460,34 @@ __global__ void __launch_bounds__(kSelThreads) select_row_kernel(float *__restri
     __syncthreads();
   }
 
-  // 4. emit kept ids in ascending order into the row's scratch
+  // 4. emit kept ids in ascending order into the row's scratch.  Thread t
+  // owns the contiguous keys [t*Lp, t*Lp + Lp) (Lp odd, so that the threads'
+  // shared-memory reads fall in different banks); the keys above thr are
+  // kept, and of the keys equal to thr the first `need` in id order.  Two
+  // block scans give each thread its tie rank and its output offset.
   int32_t *out = reinterpret_cast<int32_t *>(row);
-  int carry_tie = 0, carry_sel = 0;
-  for (int j0 = 0; j0 < nb; j0 += kSelThreads) {
-    const int j = j0 + tid;
-    uint32_t u = 0;
-    if (j < nb) u = key[j];
-    const int tie = (j < nb && u == thr) ? 1 : 0;
-    const int gt = (j < nb && u > thr) ? 1 : 0;
-    // tie rank needs the tie scan first; selection depends on it
-    int etie, dummy, ttie, tdummy;
-    block_excl_scan2(tie, 0, etie, dummy, ttie, tdummy, sh);
-    const int sel = gt || (tie && carry_tie + etie < need);
-    int esel, d2, tsel, t2;
-    block_excl_scan2(sel, 0, esel, d2, tsel, t2, sh);
-    if (sel) out[carry_sel + esel] = j;
-    carry_tie += ttie;
-    carry_sel += tsel;
+  const int Lp = ((nb + kSelThreads - 1) / kSelThreads) | 1;
+  const int jb = min(nb, tid * Lp), je = min(nb, jb + Lp);
+  int n_gt = 0, n_tie = 0;
+  for (int j = jb; j < je; ++j) {
+    const uint32_t u = key[j];
+    n_gt += u > thr;
+    n_tie += u == thr;
   }
-  if (tid == 0) counts[i] = carry_sel;
+  int e_tie, e0, t_tie, t0;
+  block_excl_scan2(n_tie, 0, e_tie, e0, t_tie, t0, sh);
+  const int keep_tie = min(n_tie, max(0, need - e_tie));
+  int e_sel, e1, t_sel, t1;
+  block_excl_scan2(n_gt + keep_tie, 0, e_sel, e1, t_sel, t1, sh);
+  int o = e_sel, ties_left = keep_tie;
+  for (int j = jb; j < je; ++j) {
+    const uint32_t u = key[j];
+    if (u > thr || (u == thr && ties_left > 0)) {
+      out[o++] = j;
+      ties_left -= (u == thr);
+    }
+  }
+  if (tid == 0) counts[i] = t_sel;
 }
 
 // ---------------------------------------------------------------------------

@@ -241,6 +241,8 @@ def kernel_rooflines(ktimes, P, D, N, h, nb, peaks, peak_src, steps, nnz=0, sm_m
                      "dO, O, O_res read, fp16 dO written (8*N*h*D bytes) + LSE, Delta (16*N*h)"),
         "a2v_norm": ("hbm", 2.0 * HBD + 4.0 * N, None,
                      "one read of the bridge output (2*N*h*D bytes) + the fp32 norms (4*N)"),
+        "range_fix": ("hbm", None, None, "pre-scale fix-up of operands above the fp16 range: every block "
+                                         "returns at once when no value is"),
         "project_v": ("tensor", 2.0 * N * proj_c * h * D if proj_c else None, None,
                       "2*N*C*h*D FLOP (V = X Wv^T; the zone statistics ride in its epilogue)"),
     }
@@ -307,7 +309,8 @@ KERNEL_SOURCES = {"project_v": "project.cu", "zone_video_stats": "plan.cu", "zon
                   "csc_count": "select.cu", "csc_scan": "select.cu", "csc_fill": "select.cu",
                   "csc_sort": "select.cu", "attn_fwd": "attn_fwd.cu", "permute3": "attn_fwd.cu",
                   "unit_block": "attn_fwd.cu", "tile_units": "attn_fwd.cu", "attn_bwd_dkdv": "attn_bwd.cu",
-                  "attn_bwd_dq": "attn_bwd.cu", "bwd_prep": "attn_bwd.cu", "a2v_norm": "a2v_norm.cu"}
+                  "attn_bwd_dq": "attn_bwd.cu", "bwd_prep": "attn_bwd.cu", "a2v_norm": "a2v_norm.cu",
+                  "range_fix": "range.cu"}
 NCU_KERNEL_NAMES = {"a2v_norm": "a2v_norm_kernel", "zone_video_stats": "zone_video_stats_kernel",
                     "block_mean": "block_mean_kernel", "attn_fwd": "attn_fwd_kernel",
                     "attn_bwd_dkdv": "dkdv_kernel", "attn_bwd_dq": "dq_kernel"}

@@ -30,7 +30,7 @@ EXPORTS = (
     "prism_kernel_timing", "prism_kernel_timing_read", "prism_a2v_norm", "prism_diag_exp2",
     "prism_diag_wait_timeout", "prism_project_v_plan",
 )
-KERNEL_TIMING_IDS = 22  # PRISM_KERNEL_TIMING_IDS in include/prism.h
+KERNEL_TIMING_IDS = 23  # PRISM_KERNEL_TIMING_IDS in include/prism.h
 
 
 class PrismParams(C.Structure):

@@ -37,7 +37,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 // ---------------------------------------------------------------------------
 // prep: dOp[h][p] = fp16(dO[perm][h]), delta[h][p] = sum_c dO*(O + O_res)
-// (O_res, the forward's bf16 rounding residual, may be NULL), lse2 = lse*log2e
+// (O_res, the forward's bf16 rounding residual, may be NULL), lse2 = lse*log2e;
+// a dO value outside the fp16 range flags its head in range_flag_do
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const int32_t *__restrict__ perm, int N, int heads,
@@ -46,7 +47,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const int32_t *__restrict
                                                        const uint16_t *__restrict__ O_res,
                                                        const float *__restrict__ lse, uint16_t *__restrict__ dOp,
                                                        float *__restrict__ lse2p, float *__restrict__ deltap,
-                                                       int *status) {
+                                                       int32_t *__restrict__ range_flag_do) {
   constexpr int G = D / 8;  // lanes per row
   const size_t g = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const size_t r = g / G;
@@ -64,7 +65,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const int32_t *__restrict
     *reinterpret_cast<uint4 *>(dOp + r * D + v * 8) =
         make_uint4(bf16x2_to_f16x2(a.x, bad), bf16x2_to_f16x2(a.y, bad), bf16x2_to_f16x2(a.z, bad),
                    bf16x2_to_f16x2(a.w, bad));
-    if (bad) record_status(status, PRISM_ERR_RANGE, 101);
+    if (bad) atomicOr(&range_flag_do[h], 1);  // range.cu converts this head again, pre-scaled
     const uint4 c = O_res ? __ldg(reinterpret_cast<const uint4 *>(O_res + src)) : make_uint4(0, 0, 0, 0);
     const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w}, cw[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
@@ -170,8 +171,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int32_t *__restrict__ row_ptr, const int32_t *__restrict__ col, const int32_t *__restrict__ blocks,
               const int32_t *__restrict__ unit_block, const int32_t *__restrict__ tile_units,
               const int32_t *__restrict__ perm, const float *__restrict__ lse2p, const float *__restrict__ deltap,
-              void *__restrict__ dQ, int grad_fp32, int N, int heads, float scale_log2, float sm_scale,
-              int *status) {
+              void *__restrict__ dQ, int grad_fp32, int N, int heads, float scale_log2_in, float sm_scale_in,
+              const unsigned *__restrict__ range_max, int *status) {
   using L = DqSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -180,6 +181,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tile = blockIdx.x, h = blockIdx.y;
   const int NB = N / 64;
   const int32_t *blocks_h = blocks + (size_t)h * NB * 4;
+  // operands pre-scaled by 2^-e (range.cu; e = 0, no change, for in-range
+  // heads): S = scale Q K^T takes 2^(eQ + eK) back, Delta already carries
+  // 2^-(edO + eV) like dP, and dQ = scale dS K takes 2^(edO + eV + eK)
+  const int eQ = range_exp(range_max[h]), eK = range_exp(range_max[heads + h]);
+  const int eV = range_exp(range_max[2 * heads + h]), eO = range_exp(range_max[3 * heads + h]);
+  const float scale_log2 = ldexpf(scale_log2_in, eQ + eK);
+  const float sm_scale = ldexpf(sm_scale_in, eO + eV + eK);
 
   if (threadIdx.x == 0) bar.abort = *reinterpret_cast<volatile int *>(status);
   __syncthreads();
@@ -478,8 +486,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int32_t *__restrict__ blocks, const int32_t *__restrict__ unit_block,
                 const int32_t *__restrict__ tile_units, const int32_t *__restrict__ perm,
                 const float *__restrict__ lse2p, const float *__restrict__ deltap, void *__restrict__ dK,
-                void *__restrict__ dV, int grad_fp32, int N, int heads, float scale_log2, float sm_scale,
-                int *status) {
+                void *__restrict__ dV, int grad_fp32, int N, int heads, float scale_log2_in, float sm_scale_in,
+                const unsigned *__restrict__ range_max, int *status) {
   using L = KvSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -489,6 +497,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tile = blockIdx.x, h = blockIdx.y;
   const int NB = N / 64;
   const int32_t *blocks_h = blocks + (size_t)h * NB * 4;
+  // operands pre-scaled by 2^-e (range.cu; e = 0, no change, for in-range
+  // heads): S^T takes 2^(eQ + eK) back, dV = P^T dO takes 2^edO, and
+  // dK = scale dS^T Q takes 2^(edO + eV + eQ) (Delta carries 2^-(edO + eV))
+  const int eQ = range_exp(range_max[h]), eK = range_exp(range_max[heads + h]);
+  const int eV = range_exp(range_max[2 * heads + h]), eO = range_exp(range_max[3 * heads + h]);
+  const float scale_log2 = ldexpf(scale_log2_in, eQ + eK);
+  const float sm_scale = ldexpf(sm_scale_in, eO + eV + eQ);
+  const float dv_scale = ldexpf(1.0f, eO);
 
   if (threadIdx.x == 0) bar.abort = *reinterpret_cast<volatile int *>(status);
   __syncthreads();
@@ -751,7 +767,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < 32; ++k) o[k] = 0u;
         }
-        store_row<D>(g == 0 ? dV : dK, grad_fp32 != 0, off + c, o, g == 0 ? 1.0f : sm_scale);
+        store_row<D>(g == 0 ? dV : dK, grad_fp32 != 0, off + c, o, g == 0 ? dv_scale : sm_scale);
       }
     } else {
       bar.abort = 1;
@@ -775,6 +791,8 @@ struct BwdWs {
   uint16_t *Qp, *Kp, *Vp, *dOp;
   float *lse2p, *deltap;
   int32_t *unit_block, *tu_q, *tu_k;
+  int32_t *range_flag;   // [4][heads]
+  unsigned *range_max;   // [4][heads]
 };
 static BwdWs carve_bwd(const prism_params &p, void *ws) {
   const size_t N = (size_t)p.T * p.H * p.W, h = p.heads, D = p.head_dim;
@@ -800,13 +818,17 @@ static BwdWs carve_bwd(const prism_params &p, void *ws) {
   b.tu_q = reinterpret_cast<int32_t *>(w);
   w += align_up(sizeof(int32_t) * h * (N / 128), 256);
   b.tu_k = reinterpret_cast<int32_t *>(w);
+  w += align_up(sizeof(int32_t) * h * (N / 128), 256);
+  b.range_flag = reinterpret_cast<int32_t *>(w);
+  b.range_max = reinterpret_cast<unsigned *>(w + sizeof(int32_t) * 4 * h);
   return b;
 }
 
 size_t attn_bwd_ws_bytes(const prism_params &p) {
   const size_t N = (size_t)p.T * p.H * p.W, h = p.heads, D = p.head_dim;
   return kWsHeader + 4 * align_up(sizeof(uint16_t) * h * N * D, 256) + 2 * align_up(sizeof(float) * h * N, 256) +
-         align_up(sizeof(int32_t) * h * (N / 64), 256) + 2 * align_up(sizeof(int32_t) * h * (N / 128), 256);
+         align_up(sizeof(int32_t) * h * (N / 64), 256) + 2 * align_up(sizeof(int32_t) * h * (N / 128), 256) +
+         align_up(sizeof(int32_t) * 8 * h, 256);
 }
 
 template <int D>
@@ -831,7 +853,8 @@ static cudaError_t run_bwd(const prism_params &p, const prism_plan_t &plan, cons
   KernelTimer kt_(KT_ATTN_DKDV, st);
   bwd::dkdv_kernel<D><<<grid, bwd::kThreads, s1, st>>>(mQ64, mDO64, mK128, mV128, sel.col_ptr, sel.row, plan.blocks,
                                                        w.unit_block, w.tu_k, plan.perm, w.lse2p, w.deltap, dK, dV,
-                                                       grad_fp32, N, p.heads, scale_log2, scale, &w.hdr->status);
+                                                       grad_fp32, N, p.heads, scale_log2, scale, w.range_max,
+                                                       &w.hdr->status);
   }
   const int s2 = bwd::DqSmem<D>::BYTES + 1024;
   cudaFuncSetAttribute(bwd::dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, s2);
@@ -839,7 +862,8 @@ static cudaError_t run_bwd(const prism_params &p, const prism_plan_t &plan, cons
   KernelTimer kt_(KT_ATTN_DQ, st);
   bwd::dq_kernel<D><<<grid, bwd::kThreads, s2, st>>>(mK64, mV64, w.Qp, w.dOp, sel.row_ptr, sel.col, plan.blocks,
                                                      w.unit_block, w.tu_q, plan.perm, w.lse2p, w.deltap, dQ,
-                                                     grad_fp32, N, p.heads, scale_log2, scale, &w.hdr->status);
+                                                     grad_fp32, N, p.heads, scale_log2, scale, w.range_max,
+                                                     &w.hdr->status);
   }
   count_launches(2);
   return cudaGetLastError();
@@ -852,8 +876,8 @@ cudaError_t launch_attn_bwd(const prism_params &p, const prism_plan_t &plan, con
   const int N = p.T * p.H * p.W, NB = N / 64, D = p.head_dim;
   BwdWs w = carve_bwd(p, ws);
   cudaError_t e;
-  if ((e = launch_permute3(plan.perm, N, p.heads, D, Q, K, V, w.Qp, w.Kp, w.Vp, &w.hdr->status, st)) !=
-      cudaSuccess)
+  if ((e = cudaMemsetAsync(w.range_flag, 0, sizeof(int32_t) * 8 * p.heads, st)) != cudaSuccess) return e;
+  if ((e = launch_permute3(plan.perm, N, p.heads, D, Q, K, V, w.Qp, w.Kp, w.Vp, w.range_flag, st)) != cudaSuccess)
     return e;
   const size_t total = (size_t)p.heads * N * (D / 8);
   {
@@ -861,13 +885,16 @@ cudaError_t launch_attn_bwd(const prism_params &p, const prism_plan_t &plan, con
   if (D == 128)
     bwd::bwd_prep_kernel<128><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(plan.perm, N, p.heads, dO, O, O_res, lse,
                                                                               w.dOp, w.lse2p, w.deltap,
-                                                                              &w.hdr->status);
+                                                                              w.range_flag + 3 * p.heads);
   else
     bwd::bwd_prep_kernel<64><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(plan.perm, N, p.heads, dO, O, O_res, lse,
                                                                              w.dOp, w.lse2p, w.deltap,
-                                                                             &w.hdr->status);
+                                                                             w.range_flag + 3 * p.heads);
   }
   count_launches(1);
+  if ((e = launch_range_fix(plan.perm, N, p.heads, D, RangeSrc{{Q, K, V, dO}}, RangeDst{{w.Qp, w.Kp, w.Vp, w.dOp}},
+                            w.range_flag, w.range_max, w.deltap, &w.hdr->status, st)) != cudaSuccess)
+    return e;
   if ((e = launch_unit_block(plan.blocks, plan.n_blocks, NB, p.heads, w.unit_block, st)) != cudaSuccess) return e;
   if ((e = launch_tile_units(sel.row_ptr, sel.col, plan.blocks, w.unit_block, N, p.heads, 2, w.tu_q, st)) !=
       cudaSuccess)

@@ -81,7 +81,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int32_t *__restrict__ col, const int32_t *__restrict__ blocks,
                     const int32_t *__restrict__ unit_block, const int32_t *__restrict__ tile_units,
                     const int32_t *__restrict__ perm, uint16_t *__restrict__ O, uint16_t *__restrict__ O_res,
-                    float *__restrict__ lse, int N, int heads, float scale_log2, int *status) {
+                    float *__restrict__ lse, int N, int heads, float scale_log2_in,
+                    const unsigned *__restrict__ range_max, int *status) {
   using L = Smem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -90,6 +91,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int quad = blockIdx.x, h = blockIdx.y;
   const int NB = N / 64;
   const int32_t *blocks_h = blocks + (size_t)h * NB * 4;
+  // operands pre-scaled by 2^-e (range.cu): Q and K fold into the score
+  // scale, V into the output; e = 0 (no change at all) for in-range heads
+  const float scale_log2 = ldexpf(scale_log2_in, range_exp(range_max[h]) + range_exp(range_max[heads + h]));
+  const float out_scale = ldexpf(1.0f, range_exp(range_max[2 * heads + h]));
 
   // a CTA that starts after another one gave up does no work
   if (threadIdx.x == 0) bar.abort = *reinterpret_cast<volatile int *>(status);
@@ -401,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int p = quad * BQ + t * 128 + row;
       const int n = perm[(size_t)h * N + p];
-      const float inv = (l > 0.f) ? 1.0f / l : 0.f;
+      const float inv = (l > 0.f) ? (1.0f / l) * out_scale : 0.f;
       uint16_t *dst = O + ((size_t)n * heads + h) * D;
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
@@ -516,11 +521,13 @@ __device__ __forceinline__ uint4 to_f16x8(uint4 v, bool &bad) {
 // dst[h][p][:] = fp16(src[perm[h][p]][h][:]), rounded to nearest: exact for
 // 2^-17 <= |x| <= 65504 and for 0 (bf16's 8 significant bits fit fp16's 11
 // down to its subnormal spacing 2^-24); smaller magnitudes move by at most
-// 2^-25.  A value outside the fp16 range records PRISM_ERR_RANGE in *status.
+// 2^-25.  A value outside the fp16 range flags its (operand, head) in
+// range_flag [3][heads] (operands s0, s1, s2); range.cu converts those heads
+// again with a pre-scale.
 __global__ void permute3_kernel(const int32_t *__restrict__ perm, int N, int heads, int D,
                                 const uint16_t *__restrict__ s0, const uint16_t *__restrict__ s1,
                                 const uint16_t *__restrict__ s2, uint16_t *__restrict__ d0, uint16_t *__restrict__ d1,
-                                uint16_t *__restrict__ d2, int *status) {
+                                uint16_t *__restrict__ d2, int32_t *__restrict__ range_flag) {
   const int vpr = D / 8;  // 16-byte vectors per row
   const size_t g = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const size_t rows = (size_t)heads * N;
@@ -530,22 +537,24 @@ __global__ void permute3_kernel(const int32_t *__restrict__ perm, int N, int hea
   const int h = (int)(r / N);
   const int n = perm[r];
   const size_t src = ((size_t)n * heads + h) * D + v * 8, dst = r * D + v * 8;
-  bool bad = false;
-  *reinterpret_cast<uint4 *>(d0 + dst) = to_f16x8(__ldg(reinterpret_cast<const uint4 *>(s0 + src)), bad);
-  if (s1) *reinterpret_cast<uint4 *>(d1 + dst) = to_f16x8(__ldg(reinterpret_cast<const uint4 *>(s1 + src)), bad);
-  if (s2) *reinterpret_cast<uint4 *>(d2 + dst) = to_f16x8(__ldg(reinterpret_cast<const uint4 *>(s2 + src)), bad);
-  if (bad) record_status(status, PRISM_ERR_RANGE, 100);
+  bool bad0 = false, bad1 = false, bad2 = false;
+  *reinterpret_cast<uint4 *>(d0 + dst) = to_f16x8(__ldg(reinterpret_cast<const uint4 *>(s0 + src)), bad0);
+  if (s1) *reinterpret_cast<uint4 *>(d1 + dst) = to_f16x8(__ldg(reinterpret_cast<const uint4 *>(s1 + src)), bad1);
+  if (s2) *reinterpret_cast<uint4 *>(d2 + dst) = to_f16x8(__ldg(reinterpret_cast<const uint4 *>(s2 + src)), bad2);
+  if (bad0) atomicOr(&range_flag[h], 1);
+  if (bad1) atomicOr(&range_flag[heads + h], 1);
+  if (bad2) atomicOr(&range_flag[2 * heads + h], 1);
 }
 
 }  // namespace fwd
 
 cudaError_t launch_permute3(const int32_t *perm, int N, int heads, int D, const uint16_t *s0, const uint16_t *s1,
-                            const uint16_t *s2, uint16_t *d0, uint16_t *d1, uint16_t *d2, int *status,
+                            const uint16_t *s2, uint16_t *d0, uint16_t *d1, uint16_t *d2, int32_t *range_flag,
                             cudaStream_t st) {
   const size_t total = (size_t)heads * N * (D / 8);
   KernelTimer kt_(KT_PERMUTE3, st);
   fwd::permute3_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(perm, N, heads, D, s0, s1, s2, d0, d1, d2,
-                                                                       status);
+                                                                       range_flag);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -633,6 +642,8 @@ struct FwdWs {
   WsHeader *hdr;
   uint16_t *Qp, *Kp, *Vp;
   int32_t *unit_block, *tile_units;
+  int32_t *range_flag;   // [4][heads]
+  unsigned *range_max;   // [4][heads]
 };
 static FwdWs carve_fwd(const prism_params &p, void *ws) {
   const size_t N = (size_t)p.T * p.H * p.W, h = p.heads, D = p.head_dim;
@@ -650,13 +661,16 @@ static FwdWs carve_fwd(const prism_params &p, void *ws) {
   f.unit_block = reinterpret_cast<int32_t *>(w);
   w += align_up(sizeof(int32_t) * h * (N / 64), 256);
   f.tile_units = reinterpret_cast<int32_t *>(w);
+  w += align_up(sizeof(int32_t) * h * (N / 256), 256);
+  f.range_flag = reinterpret_cast<int32_t *>(w);
+  f.range_max = reinterpret_cast<unsigned *>(w + sizeof(int32_t) * 4 * h);
   return f;
 }
 
 size_t attn_fwd_ws_bytes(const prism_params &p) {
   const size_t N = (size_t)p.T * p.H * p.W, h = p.heads, D = p.head_dim;
   return kWsHeader + 3 * align_up(sizeof(uint16_t) * h * N * D, 256) + align_up(sizeof(int32_t) * h * (N / 64), 256) +
-         align_up(sizeof(int32_t) * h * (N / 256), 256);
+         align_up(sizeof(int32_t) * h * (N / 256), 256) + align_up(sizeof(int32_t) * 8 * h, 256);
 }
 
 template <int D>
@@ -675,7 +689,7 @@ static cudaError_t run_fwd(const prism_params &p, const prism_plan_t &plan, cons
   KernelTimer kt_(KT_ATTN_FWD, st);
   fwd::attn_fwd_kernel<D><<<grid, fwd::kThreads, smem, st>>>(mQ, mK, mV, sel.row_ptr, sel.col, plan.blocks,
                                                              w.unit_block, w.tile_units, plan.perm, O, O_res, lse,
-                                                             N, p.heads, scale_log2, &w.hdr->status);
+                                                             N, p.heads, scale_log2, w.range_max, &w.hdr->status);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -686,8 +700,12 @@ cudaError_t launch_attn_fwd(const prism_params &p, const prism_plan_t &plan, con
   const int N = p.T * p.H * p.W, NB = N / 64, D = p.head_dim;
   FwdWs w = carve_fwd(p, ws);
   cudaError_t e;
-  if ((e = launch_permute3(plan.perm, N, p.heads, D, Q, K, V, w.Qp, w.Kp, w.Vp, &w.hdr->status, st)) !=
-      cudaSuccess)
+  if ((e = cudaMemsetAsync(w.range_flag, 0, sizeof(int32_t) * 8 * p.heads, st)) != cudaSuccess) return e;
+  if ((e = launch_permute3(plan.perm, N, p.heads, D, Q, K, V, w.Qp, w.Kp, w.Vp, w.range_flag, st)) != cudaSuccess)
+    return e;
+  if ((e = launch_range_fix(plan.perm, N, p.heads, D, RangeSrc{{Q, K, V, nullptr}},
+                            RangeDst{{w.Qp, w.Kp, w.Vp, nullptr}}, w.range_flag, w.range_max, nullptr,
+                            &w.hdr->status, st)) != cudaSuccess)
     return e;
   if ((e = launch_unit_block(plan.blocks, plan.n_blocks, NB, p.heads, w.unit_block, st)) != cudaSuccess) return e;
   if ((e = launch_tile_units(sel.row_ptr, sel.col, plan.blocks, w.unit_block, N, p.heads, 4, w.tile_units, st)) !=

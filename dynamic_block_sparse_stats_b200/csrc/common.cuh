@@ -64,12 +64,25 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
-// bf16 pair -> fp16 pair (exact for |x| <= 65504 and |x| >= 2^-14); sets
-// *bad when a value lies outside the fp16 range.
+// bf16 pair -> fp16 pair, rounded to nearest: exact for 2^-17 <= |x| <= 65504
+// and for 0 (bf16's 8 significant bits fit fp16's grid down to its subnormal
+// spacing 2^-24); sets *bad when a value lies outside the fp16 range.
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v, bool &bad) {
   const float lo = bf16lo(v), hi = bf16hi(v);
   bad |= !(fabsf(lo) <= 65504.f) || !(fabsf(hi) <= 65504.f);
   return pack_f16(lo, hi);
+}
+
+// Power-of-two pre-scale exponent of an attention operand (tensor, head) from
+// its largest magnitude (float bits; 0 when the head was never scanned): the
+// smallest e with max * 2^-e <= 65504, the largest fp16 value; 0 when the
+// maximum fits already or is not finite.
+__device__ __forceinline__ int range_exp(unsigned bits) {
+  const float m = __uint_as_float(bits);
+  if (!(m > 65504.f) || !(m < INFINITY)) return 0;
+  int e = 1;
+  while (ldexpf(m, -e) > 65504.f) ++e;
+  return e;
 }
 
 // ---------------------------------------------------------------------------
@@ -180,7 +193,8 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-// D[tmem] (+)= A[smem] * B[smem]^T-ish per the descriptors; kind::f16, bf16 in, fp32 acc.
+// D[tmem] (+)= A[smem] * B[smem] per the descriptors; kind::f16 (fp16 or bf16
+// operands, as the instruction descriptor says), fp32 accumulation.
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accumulate) {
   asm volatile(

@@ -45,11 +45,27 @@ cudaError_t launch_attn_bwd(const prism_params &p, const prism_plan_t &plan, con
 
 // shared launch helper: token gather into permuted head-major order with the
 // bf16 -> fp16 conversion of the attention operands:
-// dst[h][p][:] = fp16(src[perm[h][p]][h][:]) for up to three tensors at once;
-// out-of-range values record PRISM_ERR_RANGE in *status.
+// dst[h][p][:] = fp16(src[perm[h][p]][h][:]) for up to three tensors at once
+// (operand ids 0, 1, 2 = Q, K, V); a value outside the fp16 range sets
+// range_flag[id][h] (range.cu then converts that head again, pre-scaled).
 cudaError_t launch_permute3(const int32_t *perm, int N, int heads, int D, const uint16_t *s0, const uint16_t *s1,
-                            const uint16_t *s2, uint16_t *d0, uint16_t *d1, uint16_t *d2, int *status,
+                            const uint16_t *s2, uint16_t *d0, uint16_t *d1, uint16_t *d2, int32_t *range_flag,
                             cudaStream_t st);
+
+// range.cu: full bf16 range of the attention operands (ids 0..3 = Q, K, V,
+// dO).  For every (operand, head) flagged by the gather: its largest
+// magnitude into range_max[id][h] (float bits), then the gather again with the
+// pre-scale 2^-range_exp(range_max[id][h]); Delta (when given) divided by
+// 2^(e_dO + e_V).  range_flag and range_max are [4][heads], zeroed by the
+// caller before the gather.
+struct RangeSrc {
+  const uint16_t *p[4];
+};
+struct RangeDst {
+  uint16_t *p[4];
+};
+cudaError_t launch_range_fix(const int32_t *perm, int N, int heads, int D, RangeSrc src, RangeDst dst,
+                             int32_t *range_flag, unsigned *range_max, float *delta, int *status, cudaStream_t st);
 
 float effective_scale(const prism_params &p);
 
@@ -96,6 +112,7 @@ enum KernelTimingId {
   KT_TILE_UNITS,
   KT_BWD_PREP,
   KT_PROJECT_V,
+  KT_RANGE_FIX,
   KT_COUNT
 };
 static_assert(KT_COUNT == PRISM_KERNEL_TIMING_IDS, "timing ids");

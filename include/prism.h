@@ -59,7 +59,7 @@ typedef enum prism_status {
   PRISM_ERR_CAPACITY = 3,     /* an output or workspace is too small          */
   PRISM_ERR_CUDA = 4,         /* a CUDA runtime call failed                   */
   PRISM_ERR_TIMEOUT = 5,      /* a kernel gave up on an internal wait         */
-  PRISM_ERR_RANGE = 6         /* an attention input is outside the fp16 range */
+  PRISM_ERR_RANGE = 6         /* an attention input is infinite or NaN       */
 } prism_status;
 
 /*
@@ -318,9 +318,13 @@ size_t prism_attn_workspace_size(const prism_params *p, int backward);
  *   lse       fp32 [heads][N], natural order (natural log).
  * Runs on tcgen05 tensor cores with fp32 accumulation.  The operands are
  * fp16: Q, K, V convert from bf16 exactly for 2^-17 <= |x| <= 65504 and for
- * 0, and within 2^-25 below that (a value above 65504 records
- * PRISM_ERR_RANGE in the workspace); the probabilities P (in [0, 256]
- * under the lazy rescaling) are rounded to fp16, 8x finer than bf16.
+ * 0, and within 2^-25 below that.  A head whose Q, K or V holds a value
+ * above 65504 (any finite bf16 value is accepted) is converted with a
+ * power-of-two pre-scale that the kernels fold back exactly into the score
+ * scale and the output; heads within the fp16 range are unaffected.  An
+ * infinite or NaN input records PRISM_ERR_RANGE in the workspace.  The
+ * probabilities P (in [0, 256] under the lazy rescaling) are rounded to fp16,
+ * 8x finer than bf16.
  * Returns PRISM_OK, PRISM_ERR_INVALID_ARG, PRISM_ERR_UNSUPPORTED,
  * PRISM_ERR_CAPACITY or PRISM_ERR_CUDA.
  */
@@ -351,9 +355,7 @@ int prism_attn_bwd(const prism_params *p, const prism_plan_t *plan,
 
 /* Waits on `stream` and returns the status a kernel recorded in
  * `workspace`: PRISM_OK, PRISM_ERR_TIMEOUT, or PRISM_ERR_RANGE (an attention
- * call met a Q/K/V/dO value with |x| > 65504, the largest fp16 value; the
- * attention tensor-core operands are fp16, to which bf16 converts exactly
- * for 2^-17 <= |x| <= 65504), or PRISM_ERR_CUDA. */
+ * call met an infinite or NaN Q/K/V/dO value), or PRISM_ERR_CUDA. */
 int prism_workspace_status(const void *workspace, prism_stream_t stream);
 
 /* Message of the calling thread's last failing call ("" if none).  The
@@ -377,8 +379,10 @@ int prism_kernel_timing(int enable);
  * 6 attn_bwd_dq, 7 a2v_norm, 8 zone_a2v_stats, 9 plan_finalize, 10 perm,
  * 11 select_scan, 12 csr_fill, 13 csc_count, 14 csc_scan, 15 csc_fill,
  * 16 csc_sort, 17 permute3, 18 unit_block, 19 tile_units, 20 bwd_prep,
- * 21 project_v. */
-#define PRISM_KERNEL_TIMING_IDS 22
+ * 21 project_v, 22 range_fix (both launches of the pre-scale fix-up of
+ * operands above the fp16 range; their blocks return at once when no value
+ * is). */
+#define PRISM_KERNEL_TIMING_IDS 23
 
 /* Reads the records of kernel `id` (0 .. PRISM_KERNEL_TIMING_IDS - 1): waits
  * for its events, and returns the number of timed launches, their total

@@ -23,7 +23,8 @@ _KERNEL_MS = {"zone_video_stats": 0.1, "block_mean": 0.2, "block_score": 0.05, "
               "attn_bwd_dkdv": 15.0, "attn_bwd_dq": 10.0, "a2v_norm": 0.05, "zone_a2v_stats": 0.01,
               "plan_finalize": 0.02, "perm": 0.01, "select_scan": 0.01, "csr_fill": 0.01, "csc_count": 0.01,
               "csc_scan": 0.01, "csc_fill": 0.01, "csc_sort": 0.01, "permute3": 0.05, "unit_block": 0.01,
-              "tile_units": 0.01, "bwd_prep": 0.03, "project_v": 0.5}
+              "tile_units": 0.01, "bwd_prep": 0.03, "project_v": 0.5,
+              "range_fix": 0.01}
 
 
 class _Lib:

@@ -10,7 +10,8 @@ import ctypes as C
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libprism.so")
+# PRISM_LIB=debug selects the build with device-side bounds checks
+LIB_PATH = os.path.join(_HERE, "libprism_debug.so" if os.environ.get("PRISM_LIB") == "debug" else "libprism.so")
 
 PRISM_OK = 0
 PRISM_ERR_INVALID_ARG = 1
@@ -65,8 +66,9 @@ def load() -> C.CDLL:
     if _lib is not None:
         return _lib
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libprism.so not found at {LIB_PATH}; build it with "
-                          "`python -m dynamic_block_sparse_stats_b200.build`")
+        raise ImportError(f"{os.path.basename(LIB_PATH)} not found at {LIB_PATH}; build it with "
+                          "`python -m dynamic_block_sparse_stats_b200.build`"
+                          + (" --debug" if LIB_PATH.endswith("_debug.so") else ""))
     lib = C.CDLL(LIB_PATH)
     P = C.POINTER
     vp, sz, st = C.c_void_p, C.c_size_t, C.c_void_p

@@ -79,6 +79,7 @@ using namespace prism;
 
 extern "C" int prism_a2v_norm(const uint16_t *hhat, int64_t n, int32_t width, int64_t ld, float *a2v_norm,
                               prism_stream_t stream) {
+  NvtxRange nvtx_("prism_a2v_norm");
   if (n < 0) return report_error(PRISM_ERR_INVALID_ARG, "prism_a2v_norm: n must be >= 0");
   if (width <= 0 || width % 8 || width > (1 << 20))
     return report_error(PRISM_ERR_INVALID_ARG, "prism_a2v_norm: width must be a positive multiple of 8, <= 2^20");

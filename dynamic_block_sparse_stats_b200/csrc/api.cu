@@ -117,6 +117,7 @@ size_t prism_plan_workspace_size(const prism_params *p) {
 
 int prism_plan(const prism_params *p, const uint16_t *V, const float *a2v_norm, const prism_plan_t *out,
                void *workspace, size_t ws_bytes, prism_stream_t stream) {
+  NvtxRange nvtx_("prism_plan");
   int rc;
   if ((rc = check_plan_call(p, V, a2v_norm, out)) != PRISM_OK) return rc;
   if ((rc = check_ws(workspace, ws_bytes, plan_ws_bytes(*p))) != PRISM_OK) return rc;
@@ -131,6 +132,7 @@ int prism_plan(const prism_params *p, const uint16_t *V, const float *a2v_norm, 
 int prism_project_v_plan(const prism_params *p, const uint16_t *X, int32_t C, const uint16_t *Wv, uint16_t *V,
                          const float *a2v_norm, const prism_plan_t *out, void *workspace, size_t ws_bytes,
                          prism_stream_t stream) {
+  NvtxRange nvtx_("prism_project_v_plan");
   int rc;
   if ((rc = check_plan_call(p, V, a2v_norm, out)) != PRISM_OK) return rc;
   if (!X || !Wv) return fail(PRISM_ERR_INVALID_ARG, "X or Wv is NULL");
@@ -155,6 +157,7 @@ size_t prism_select_workspace_size(const prism_params *p) {
 
 int prism_select(const prism_params *p, const prism_plan_t *plan, const uint16_t *Q, const uint16_t *K,
                  prism_select_t *out, void *workspace, size_t ws_bytes, prism_stream_t stream) {
+  NvtxRange nvtx_("prism_select");
   int rc;
   if ((rc = check_params(p)) != PRISM_OK) return rc;
   if (!Q || !K) return fail(PRISM_ERR_INVALID_ARG, "Q or K is NULL");
@@ -189,6 +192,7 @@ size_t prism_attn_workspace_size(const prism_params *p, int backward) {
 int prism_attn_fwd(const prism_params *p, const prism_plan_t *plan, const prism_select_t *sel, const uint16_t *Q,
                    const uint16_t *K, const uint16_t *V, uint16_t *O, uint16_t *O_res, float *lse, void *workspace,
                    size_t ws_bytes, prism_stream_t stream) {
+  NvtxRange nvtx_("prism_attn_fwd");
   int rc;
   if ((rc = check_params(p)) != PRISM_OK) return rc;
   if (!Q || !K || !V || !O || !lse) return fail(PRISM_ERR_INVALID_ARG, "Q, K, V, O or lse is NULL");
@@ -213,6 +217,7 @@ int prism_attn_bwd(const prism_params *p, const prism_plan_t *plan, const prism_
                    const uint16_t *K, const uint16_t *V, const uint16_t *O, const uint16_t *O_res, const uint16_t *dO,
                    const float *lse, void *dQ, void *dK, void *dV, int grad_fp32, void *workspace, size_t ws_bytes,
                    prism_stream_t stream) {
+  NvtxRange nvtx_("prism_attn_bwd");
   int rc;
   if ((rc = check_params(p)) != PRISM_OK) return rc;
   if (!Q || !K || !V || !O || !dO || !lse || !dQ || !dK || !dV)

@@ -237,6 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         walk_next<2>(w, col, blocks_h, ub, mb);
         nu = 2;
       }
+      PRISM_CHECK(ua < (uint32_t)NB && ub < (uint32_t)NB, status, 125);
       ua = min(ua, (uint32_t)(NB - 1));  // a well-formed walk never clamps
       ub = min(ub, (uint32_t)(NB - 1));
       if (lane == 0) {
@@ -422,7 +423,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && nsteps > 0) ok = mbar_wait_warp(&bar.fin, 0, status, 30);
     if (ok) {
       tc_fence_after();
-      const int n = perm[prow];
+      int n = perm[prow];
+      if (!PRISM_CHECK((unsigned)n < (unsigned)N, status, 127)) n = 0;
       const size_t off = ((size_t)n * heads + h) * D;
 #pragma unroll 1
       for (int c = g * (D / 2); c < (g + 1) * (D / 2); c += 32) {
@@ -561,6 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         walk_next<2>(w, rowidx, blocks_h, ub, mb);
         nu = 2;
       }
+      PRISM_CHECK(ua < (uint32_t)NB && ub < (uint32_t)NB, status, 126);
       ua = min(ua, (uint32_t)(NB - 1));
       ub = min(ub, (uint32_t)(NB - 1));
       if (lane == 0) {
@@ -753,7 +756,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       tc_fence_after();
       const size_t prow = (size_t)h * N + (size_t)tile * 128 + row;
-      const int n = perm[prow];
+      int n = perm[prow];
+      if (!PRISM_CHECK((unsigned)n < (unsigned)N, status, 128)) n = 0;
       const size_t off = ((size_t)n * heads + h) * D;
       // warpgroup 0 writes dV, warpgroup 1 writes dK
       const uint32_t src = g == 0 ? tV : tK;
@@ -877,7 +881,8 @@ cudaError_t launch_attn_bwd(const prism_params &p, const prism_plan_t &plan, con
   BwdWs w = carve_bwd(p, ws);
   cudaError_t e;
   if ((e = cudaMemsetAsync(w.range_flag, 0, sizeof(int32_t) * 8 * p.heads, st)) != cudaSuccess) return e;
-  if ((e = launch_permute3(plan.perm, N, p.heads, D, Q, K, V, w.Qp, w.Kp, w.Vp, w.range_flag, st)) != cudaSuccess)
+  if ((e = launch_permute3(plan.perm, N, p.heads, D, Q, K, V, w.Qp, w.Kp, w.Vp, w.range_flag, &w.hdr->status,
+                           st)) != cudaSuccess)
     return e;
   const size_t total = (size_t)p.heads * N * (D / 8);
   {

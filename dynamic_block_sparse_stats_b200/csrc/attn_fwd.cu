@@ -164,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           walk_next<4>(w, col, blocks_h, ub, mb);
           nu = 2;
         }
+        PRISM_CHECK(ua < (uint32_t)NB && ub < (uint32_t)NB, status, 123);
         ua = min(ua, (uint32_t)(NB - 1));  // a well-formed walk never clamps
         ub = min(ub, (uint32_t)(NB - 1));
       }
@@ -405,7 +406,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       tc_fence_after();
       const int p = quad * BQ + t * 128 + row;
-      const int n = perm[(size_t)h * N + p];
+      int n = perm[(size_t)h * N + p];
+      if (!PRISM_CHECK((unsigned)n < (unsigned)N, status, 124)) n = 0;
       const float inv = (l > 0.f) ? (1.0f / l) * out_scale : 0.f;
       uint16_t *dst = O + ((size_t)n * heads + h) * D;
 #pragma unroll 1
@@ -527,7 +529,7 @@ __device__ __forceinline__ uint4 to_f16x8(uint4 v, bool &bad) {
 __global__ void permute3_kernel(const int32_t *__restrict__ perm, int N, int heads, int D,
                                 const uint16_t *__restrict__ s0, const uint16_t *__restrict__ s1,
                                 const uint16_t *__restrict__ s2, uint16_t *__restrict__ d0, uint16_t *__restrict__ d1,
-                                uint16_t *__restrict__ d2, int32_t *__restrict__ range_flag) {
+                                uint16_t *__restrict__ d2, int32_t *__restrict__ range_flag, int *status) {
   const int vpr = D / 8;  // 16-byte vectors per row
   const size_t g = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const size_t rows = (size_t)heads * N;
@@ -536,6 +538,7 @@ __global__ void permute3_kernel(const int32_t *__restrict__ perm, int N, int hea
   const int v = (int)(g % vpr);
   const int h = (int)(r / N);
   const int n = perm[r];
+  if (!PRISM_CHECK((unsigned)n < (unsigned)N, status, 122)) return;
   const size_t src = ((size_t)n * heads + h) * D + v * 8, dst = r * D + v * 8;
   bool bad0 = false, bad1 = false, bad2 = false;
   *reinterpret_cast<uint4 *>(d0 + dst) = to_f16x8(__ldg(reinterpret_cast<const uint4 *>(s0 + src)), bad0);
@@ -550,11 +553,11 @@ __global__ void permute3_kernel(const int32_t *__restrict__ perm, int N, int hea
 
 cudaError_t launch_permute3(const int32_t *perm, int N, int heads, int D, const uint16_t *s0, const uint16_t *s1,
                             const uint16_t *s2, uint16_t *d0, uint16_t *d1, uint16_t *d2, int32_t *range_flag,
-                            cudaStream_t st) {
+                            int *status, cudaStream_t st) {
   const size_t total = (size_t)heads * N * (D / 8);
   KernelTimer kt_(KT_PERMUTE3, st);
   fwd::permute3_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(perm, N, heads, D, s0, s1, s2, d0, d1, d2,
-                                                                       range_flag);
+                                                                       range_flag, status);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -701,7 +704,8 @@ cudaError_t launch_attn_fwd(const prism_params &p, const prism_plan_t &plan, con
   FwdWs w = carve_fwd(p, ws);
   cudaError_t e;
   if ((e = cudaMemsetAsync(w.range_flag, 0, sizeof(int32_t) * 8 * p.heads, st)) != cudaSuccess) return e;
-  if ((e = launch_permute3(plan.perm, N, p.heads, D, Q, K, V, w.Qp, w.Kp, w.Vp, w.range_flag, st)) != cudaSuccess)
+  if ((e = launch_permute3(plan.perm, N, p.heads, D, Q, K, V, w.Qp, w.Kp, w.Vp, w.range_flag, &w.hdr->status,
+                           st)) != cudaSuccess)
     return e;
   if ((e = launch_range_fix(plan.perm, N, p.heads, D, RangeSrc{{Q, K, V, nullptr}},
                             RangeDst{{w.Qp, w.Kp, w.Vp, nullptr}}, w.range_flag, w.range_max, nullptr,

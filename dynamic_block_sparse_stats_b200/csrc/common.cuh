@@ -35,6 +35,17 @@ __device__ __forceinline__ void record_status(int *status, int code, int where) 
     atomicExch(status + 1, where);
   }
 }
+// Debug builds (-DPRISM_DEBUG, `build --debug`): device-side bounds checks
+// that record PRISM_ERR_INVALID_ARG and the check's site in the status word,
+// and let the caller skip the access, instead of trapping; release builds
+// compile every check to `true`.
+#ifdef PRISM_DEBUG
+#define PRISM_CHECK(cond, status, where) \
+  ((cond) ? true : (record_status((status), (int)PRISM_ERR_INVALID_ARG, (where)), false))
+#else
+#define PRISM_CHECK(cond, status, where) true
+#endif
+
 __device__ __forceinline__ void record_timeout(int *status, int where) {
   if (status) {
     atomicExch(status, (int)PRISM_ERR_TIMEOUT);

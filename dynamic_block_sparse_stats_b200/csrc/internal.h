@@ -5,9 +5,19 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 
 namespace prism {
+
+// NVTX range around a C-ABI call (a no-op unless a profiler is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange &) = delete;
+  NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 // plan.cu
 size_t plan_ws_bytes(const prism_params &p);
@@ -50,7 +60,7 @@ cudaError_t launch_attn_bwd(const prism_params &p, const prism_plan_t &plan, con
 // range_flag[id][h] (range.cu then converts that head again, pre-scaled).
 cudaError_t launch_permute3(const int32_t *perm, int N, int heads, int D, const uint16_t *s0, const uint16_t *s1,
                             const uint16_t *s2, uint16_t *d0, uint16_t *d1, uint16_t *d2, int32_t *range_flag,
-                            cudaStream_t st);
+                            int *status, cudaStream_t st);
 
 // range.cu: full bf16 range of the attention operands (ids 0..3 = Q, K, V,
 // dO).  For every (operand, head) flagged by the gather: its largest

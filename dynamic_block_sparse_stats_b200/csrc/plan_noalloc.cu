@@ -87,6 +87,7 @@ using namespace prism;
 
 extern "C" int prism_plan_noalloc(const prism_params *p, const uint16_t *V, const float *a2v_norm,
                                   const prism_plan_t *out, prism_stream_t stream) {
+  NvtxRange nvtx_("prism_plan_noalloc");
   int rc = check_plan_call(p, V, a2v_norm, out);
   if (rc != PRISM_OK) return rc;
   const size_t need = plan_ws_bytes(*p);

@@ -160,3 +160,19 @@ def test_project_v_plan_rejects_null_and_misaligned_inputs():
         rc = lib.prism_project_v_plan(C.byref(p), C.c_void_p(X) if X else None, 64, C.c_void_p(Wv) if Wv else None,
                                       C.c_void_p(256), None, C.byref(dummy), C.c_void_p(256), 1 << 20, None)
         assert rc == _lib.PRISM_ERR_INVALID_ARG, (X, Wv)
+
+
+def test_debug_build_exports_the_same_functions():
+    """The PRISM_DEBUG build (device-side bounds checks) is the same ABI."""
+    import subprocess
+    import sys
+    from dynamic_block_sparse_stats_b200 import build
+    lib = build.build(debug=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", lib], capture_output=True, text=True, check=True).stdout
+    names = {ln.split()[-1] for ln in out.splitlines() if " T prism_" in ln}
+    assert names == set(declared_functions())
+    code = ("import os; os.environ['PRISM_LIB'] = 'debug'; import sys; sys.path.insert(0, %r); "
+            "from dynamic_block_sparse_stats_b200 import _lib; l = _lib.load(); "
+            "assert _lib.LIB_PATH.endswith('libprism_debug.so'); print(l.prism_version().decode())" % ROOT)
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.count(".") == 2, r.stderr

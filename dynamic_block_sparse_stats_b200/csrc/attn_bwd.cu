@@ -184,8 +184,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // operands pre-scaled by 2^-e (range.cu; e = 0, no change, for in-range
   // heads): S = scale Q K^T takes 2^(eQ + eK) back, Delta already carries
   // 2^-(edO + eV) like dP, and dQ = scale dS K takes 2^(edO + eV + eK)
-  const int eQ = range_exp(range_max[h]), eK = range_exp(range_max[heads + h]);
-  const int eV = range_exp(range_max[2 * heads + h]), eO = range_exp(range_max[3 * heads + h]);
+  const int eQ = range_exp(range_max[h], 0), eK = range_exp(range_max[heads + h], 1);
+  const int eV = range_exp(range_max[2 * heads + h], 2), eO = range_exp(range_max[3 * heads + h], 3);
   const float scale_log2 = ldexpf(scale_log2_in, eQ + eK);
   const float sm_scale = ldexpf(sm_scale_in, eO + eV + eK);
 
@@ -502,8 +502,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // operands pre-scaled by 2^-e (range.cu; e = 0, no change, for in-range
   // heads): S^T takes 2^(eQ + eK) back, dV = P^T dO takes 2^edO, and
   // dK = scale dS^T Q takes 2^(edO + eV + eQ) (Delta carries 2^-(edO + eV))
-  const int eQ = range_exp(range_max[h]), eK = range_exp(range_max[heads + h]);
-  const int eV = range_exp(range_max[2 * heads + h]), eO = range_exp(range_max[3 * heads + h]);
+  const int eQ = range_exp(range_max[h], 0), eK = range_exp(range_max[heads + h], 1);
+  const int eV = range_exp(range_max[2 * heads + h], 2), eO = range_exp(range_max[3 * heads + h], 3);
   const float scale_log2 = ldexpf(scale_log2_in, eQ + eK);
   const float sm_scale = ldexpf(sm_scale_in, eO + eV + eQ);
   const float dv_scale = ldexpf(1.0f, eO);

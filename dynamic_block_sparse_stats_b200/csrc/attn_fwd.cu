@@ -93,8 +93,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int32_t *blocks_h = blocks + (size_t)h * NB * 4;
   // operands pre-scaled by 2^-e (range.cu): Q and K fold into the score
   // scale, V into the output; e = 0 (no change at all) for in-range heads
-  const float scale_log2 = ldexpf(scale_log2_in, range_exp(range_max[h]) + range_exp(range_max[heads + h]));
-  const float out_scale = ldexpf(1.0f, range_exp(range_max[2 * heads + h]));
+  const float scale_log2 = ldexpf(scale_log2_in, range_exp(range_max[h], 0) + range_exp(range_max[heads + h], 1));
+  const float out_scale = ldexpf(1.0f, range_exp(range_max[2 * heads + h], 2));
 
   // a CTA that starts after another one gave up does no work
   if (threadIdx.x == 0) bar.abort = *reinterpret_cast<volatile int *>(status);

@@ -84,15 +84,19 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v, bool &bad) {
   return pack_f16(lo, hi);
 }
 
-// Power-of-two pre-scale exponent of an attention operand (tensor, head) from
-// its largest magnitude (float bits; 0 when the head was never scanned): the
-// smallest e with max * 2^-e <= 65504, the largest fp16 value; 0 when the
-// maximum fits already or is not finite.
-__device__ __forceinline__ int range_exp(unsigned bits) {
+// Power-of-two pre-scale exponent of attention operand `id` (0..3 = Q, K, V,
+// dO) of a head from its largest magnitude (float bits; 0 when the head was
+// never scanned, i.e. every value fits fp16).  Q and K: the smallest e with
+// max * 2^-e <= 65504, the largest fp16 value.  V and dO: the smallest e with
+// max * 2^-e <= 16, because they meet in dP = dO V^T, whose D-term sums must
+// keep dS = P (dP - Delta) within fp16 (|dP| <= D * 16 * 16).  0 when the
+// maximum fits fp16 or is not finite.
+__device__ __forceinline__ int range_exp(unsigned bits, int id) {
   const float m = __uint_as_float(bits);
   if (!(m > 65504.f) || !(m < INFINITY)) return 0;
+  const float limit = id < 2 ? 65504.f : 16.f;
   int e = 1;
-  while (ldexpf(m, -e) > 65504.f) ++e;
+  while (ldexpf(m, -e) > limit) ++e;
   return e;
 }
 

@@ -4,7 +4,8 @@
 // and flags every (tensor, head) that holds a value above 65504.  For those
 // only, these kernels find the head's largest magnitude and convert it again
 // with a power-of-two pre-scale 2^-e (the smallest e that brings the maximum
-// to 65504 or below).  The attention kernels fold the scales back exactly:
+// to 65504 or below for Q and K, to 16 or below for V and dO, whose products
+// dP = dO V^T feed dS, which must stay within fp16 too).  The attention kernels fold the scales back exactly:
 // Q and K into the score scale, V and dO into the output stores and into
 // Delta, which the fix-up divides by 2^(e_dO + e_V) for the heads concerned.
 // A head with no flag keeps e = 0 and its results are bit-identical to the
@@ -60,8 +61,8 @@ __global__ void __launch_bounds__(256) range_fix_kernel(const int32_t *__restric
                                                         const unsigned *__restrict__ maxbits,
                                                         float *__restrict__ delta) {
   const int t = blockIdx.z, h = blockIdx.y;
-  const int es = (t == 3 && delta) ? range_exp(maxbits[3 * heads + h]) + range_exp(maxbits[2 * heads + h]) : 0;
-  const int e = (src.p[t] && flag[t * heads + h]) ? range_exp(maxbits[t * heads + h]) : 0;
+  const int es = (t == 3 && delta) ? range_exp(maxbits[3 * heads + h], 3) + range_exp(maxbits[2 * heads + h], 2) : 0;
+  const int e = (src.p[t] && flag[t * heads + h]) ? range_exp(maxbits[t * heads + h], t) : 0;
   if (es == 0 && e == 0) return;  // uniform over the block; e = 0 also for a non-finite maximum
   const int G = D / 8;
   const size_t stride = (size_t)gridDim.x * blockDim.x;

@@ -199,7 +199,9 @@ def kernel_rooflines(ktimes, P, D, N, h, nb, peaks, peak_src, steps, nnz=0, sm_m
     `attn_bwd` on the FlashAttention convention, 10*P*D FLOP per layer: dK/dV
     does 8*P*D of it (S^T, dP^T, dV, dK), dQ the remaining 2*P*D (dQ = dS K);
     dQ's recomputed S and dP (4*P*D more) are issued work, reported as
-    `issued_TFLOPs`, not algorithmic work."""
+    `issued_TFLOPs`, not algorithmic work.  On the fused path (one kernel
+    for dK, dV and dQ, then the accumulator's conversion) `attn_bwd` is
+    10*P*D over those two kernels' time, issued and algorithmic alike."""
     sustained = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     burst = peaks.get("bf16_tflops", sustained)
     hbm = peaks["hbm_gbs"]
@@ -213,6 +215,11 @@ def kernel_rooflines(ktimes, P, D, N, h, nb, peaks, peak_src, steps, nnz=0, sm_m
         "attn_bwd_dkdv": ("tensor", 8.0 * P * D, None, "8*P*D FLOP (S^T, dP^T, dV, dK on the computed pairs)"),
         "attn_bwd_dq": ("tensor", 2.0 * P * D, 6.0 * P * D,
                         "2*P*D FLOP algorithmic (dQ = dS K); 6*P*D issued (S and dP recomputed)"),
+        "attn_bwd_fused": ("tensor", 10.0 * P * D, None,
+                           "10*P*D FLOP (S^T, dP^T, dV, dK, dQ^T on the computed pairs; dQ added by fp32 "
+                           "reductions)"),
+        "dq_convert": ("hbm", 6.0 * HBD + 4.0 * HN, None,
+                       "fp32 dQ accumulator read, bf16 dQ written (6*N*h*D bytes) + perm (4*N*h)"),
         "zone_video_stats": ("hbm", 2.0 * HBD, None, "one read of V: 2*N*h*D bytes"),
         "zone_a2v_stats": ("hbm", 4.0 * N, None, "one read of the A2V map: 4*N bytes"),
         "plan_finalize": ("hbm", h * Z * 77.0 + 32.0 * Z + 16.0 * sum_nb, None,
@@ -279,23 +286,31 @@ def kernel_rooflines(ktimes, P, D, N, h, nb, peaks, peak_src, steps, nnz=0, sm_m
                 rec["peak_source"] = "derived: 148 SMs x 128 fp32 lanes x max SM clock (one FMUL or FADD each)"
             rec["frac"] = rec["achieved"] / rec["peak"]
         out[name] = rec
-    kd, kq = out.get("attn_bwd_dkdv"), out.get("attn_bwd_dq")
-    if kd and kq and kd["launches"] and kq["launches"]:
+    def launched(*names):
+        recs = [out.get(n) for n in names]
+        return recs if all(r and r["launches"] and r["total_ms"] > 0 for r in recs) else None
+
+    two = launched("attn_bwd_dkdv", "attn_bwd_dq")
+    one = launched("attn_bwd_fused", "dq_convert")
+    if two or one:
+        kd, kq = one or two
         ms_b = kd["ms_per_launch"] + kq["ms_per_launch"]
         t = 10.0 * P * D / (ms_b * 1e-3) / 1e12
         out["attn_bwd"] = {
             "launches": kd["launches"], "ms_per_launch": ms_b, "bound": "tensor", "unit": "TFLOP/s",
-            "algorithmic": "10*P*D FLOP (FlashAttention convention) over dK/dV + dQ time",
+            "algorithmic": ("10*P*D FLOP (FlashAttention convention) over the fused kernel + dQ conversion time"
+                            if one else "10*P*D FLOP (FlashAttention convention) over dK/dV + dQ time"),
+            "path": "fused" if one else "two-kernel deterministic",
             "achieved": t, "peak": sustained, "frac": t / sustained, "frac_burst": t / burst,
             "peak_source": f"{peak_src} bf16 sustained",
-            "issued_TFLOPs": 14.0 * P * D / (ms_b * 1e-3) / 1e12}
+            "issued_TFLOPs": (10.0 if one else 14.0) * P * D / (ms_b * 1e-3) / 1e12}
         kf = out.get("attn_fwd")
         if kf and kf["launches"]:
             ms_a = ms_b + kf["ms_per_launch"]
             t = 14.0 * P * D / (ms_a * 1e-3) / 1e12
             out["attn_fwd_bwd"] = {
                 "launches": kd["launches"], "ms_per_launch": ms_a, "bound": "tensor", "unit": "TFLOP/s",
-                "algorithmic": "14*P*D FLOP over forward + dK/dV + dQ time",
+                "algorithmic": "14*P*D FLOP over forward + backward time",
                 "achieved": t, "peak": sustained, "frac": t / sustained, "frac_burst": t / burst,
                 "peak_source": f"{peak_src} bf16 sustained"}
     return out
@@ -310,6 +325,7 @@ KERNEL_SOURCES = {"project_v": "project.cu", "zone_video_stats": "plan.cu", "zon
                   "csc_sort": "select.cu", "attn_fwd": "attn_fwd.cu", "permute3": "attn_fwd.cu",
                   "unit_block": "attn_fwd.cu", "tile_units": "attn_fwd.cu", "attn_bwd_dkdv": "attn_bwd.cu",
                   "attn_bwd_dq": "attn_bwd.cu", "bwd_prep": "attn_bwd.cu", "a2v_norm": "a2v_norm.cu",
+                  "attn_bwd_fused": "attn_bwd.cu", "dq_convert": "attn_bwd.cu",
                   "range_fix": "range.cu"}
 NCU_KERNEL_NAMES = {"a2v_norm": "a2v_norm_kernel", "zone_video_stats": "zone_video_stats_kernel",
                     "block_mean": "block_mean_kernel", "attn_fwd": "attn_fwd_kernel",
@@ -610,7 +626,7 @@ def run_prism(args, w, rank, world, device):
     grads = None
     bws = None
     if backward:
-        grads = api.attn_bwd(p, pl, sel, Q, K, V, O_, dO, lse, O_res=O_res)
+        grads = api.attn_bwd(p, pl, sel, Q, K, V, O_, dO, lse, O_res=O_res, deterministic=args.deterministic)
         bws = torch.empty(lib.prism_attn_workspace_size(api.C.byref(p), 1), dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
     stages = ["plan", "select", "fwd", "bwd"] if backward else ["plan", "select", "fwd"]
@@ -632,7 +648,8 @@ def run_prism(args, w, rank, world, device):
         if ev is not None:
             ev[3].record(stream)
         if backward:
-            api.attn_bwd(p, pl, sel, Q, K, V, O_, dO, lse, out=grads, ws=bws, O_res=O_res)
+            api.attn_bwd(p, pl, sel, Q, K, V, O_, dO, lse, out=grads, ws=bws, O_res=O_res,
+                         deterministic=args.deterministic)
             if ev is not None:
                 ev[4].record(stream)
 
@@ -761,6 +778,9 @@ def run_prism(args, w, rank, world, device):
         "config": {"workload": w.name, "T": w.T, "H": w.H, "W": w.W, "tokens": N,
                    "heads": WORKLOADS[args.workload].heads, "heads_per_rank": h, "head_dim": D,
                    "topk_frac": w.topk_frac, "top_p": w.top_p, "backward": backward,
+                   "bwd_path": (None if not backward else
+                                "two-kernel, deterministic" if args.deterministic or D != 128 else
+                                "fused dK/dV/dQ, dQ by fp32 atomic adds"),
                    "plan_from": ("prism_project_v_plan: V = X Wv^T (C = %d) with the zone statistics in the "
                                  "GEMM epilogue" % X.shape[1]) if proj else "prism_plan of a given V",
                    "parallelism": (f"heads split over {world} ranks (this rank {h0}-{h1 - 1}), no collectives on the path"
@@ -815,6 +835,8 @@ def main():
     ap.add_argument("--impl", choices=["prism", "reference"], default="prism")
     ap.add_argument("--workload", default="2k_train", choices=sorted(WORKLOADS))
     ap.add_argument("--backward", action="store_true", help="time the backward on any workload")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="backward on the two-kernel, bitwise reproducible path (default: the fused kernel)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense SDPA comparison")

@@ -31,7 +31,7 @@ EXPORTS = (
     "prism_kernel_timing", "prism_kernel_timing_read", "prism_a2v_norm", "prism_diag_exp2",
     "prism_diag_wait_timeout", "prism_project_v_plan",
 )
-KERNEL_TIMING_IDS = 23  # PRISM_KERNEL_TIMING_IDS in include/prism.h
+KERNEL_TIMING_IDS = 25  # PRISM_KERNEL_TIMING_IDS in include/prism.h
 
 
 class PrismParams(C.Structure):
@@ -81,7 +81,7 @@ def load() -> C.CDLL:
         "prism_attn_fwd": (C.c_int, [P(PrismParams), P(PrismPlan), P(PrismSelect), vp, vp, vp, vp, vp, vp, vp, sz,
                                      st]),
         "prism_attn_bwd": (C.c_int, [P(PrismParams), P(PrismPlan), P(PrismSelect), vp, vp, vp, vp, vp, vp, vp, vp,
-                                     vp, vp, C.c_int, vp, sz, st]),
+                                     vp, vp, C.c_int, C.c_int, vp, sz, st]),
         "prism_workspace_status": (C.c_int, [vp, st]),
         "prism_last_error": (C.c_char_p, []),
         "prism_version": (C.c_char_p, []),

@@ -365,9 +365,12 @@ def attn_fwd(p: PrismParams, pl: Plan, sel: Selection, Q, K, V, O=None, lse=None
 
 
 def attn_bwd(p: PrismParams, pl: Plan, sel: Selection, Q, K, V, O, dO, lse, grad_fp32=False, out=None, ws=None,
-             O_res=None, stream=None):
+             O_res=None, stream=None, deterministic=False):
     """prism_attn_bwd: dQ, dK, dV through the selected blocks (natural order).
-    Pass the forward's O_res for an fp32-accurate Delta."""
+    Pass the forward's O_res for an fp32-accurate Delta.  deterministic=False
+    (head_dim 128) takes the fused kernel, whose dQ is summed by fp32 atomic
+    adds in no fixed order; True takes the two-kernel path, bitwise
+    reproducible."""
     N = p.T * p.H * p.W
     shape = (N, p.heads, p.head_dim)
     for name, t in (("Q", Q), ("K", K), ("V", V), ("O", O), ("dO", dO)):
@@ -397,7 +400,8 @@ def attn_bwd(p: PrismParams, pl: Plan, sel: Selection, Q, K, V, O, dO, lse, grad
         dQ, dK, dV = out
         check(lib.prism_attn_bwd(C.byref(p), C.byref(cpl), C.byref(cs), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
                                  _ptr(O_res), _ptr(dO), _ptr(lse), _ptr(dQ), _ptr(dK), _ptr(dV),
-                                 int(bool(grad_fp32)), _ptr(ws), ws.numel(), _stream(stream, dev)))
+                                 int(bool(grad_fp32)), int(bool(deterministic)), _ptr(ws), ws.numel(),
+                                 _stream(stream, dev)))
     return dQ, dK, dV
 
 

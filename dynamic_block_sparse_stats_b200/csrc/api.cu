@@ -215,11 +215,12 @@ int prism_attn_fwd(const prism_params *p, const prism_plan_t *plan, const prism_
 
 int prism_attn_bwd(const prism_params *p, const prism_plan_t *plan, const prism_select_t *sel, const uint16_t *Q,
                    const uint16_t *K, const uint16_t *V, const uint16_t *O, const uint16_t *O_res, const uint16_t *dO,
-                   const float *lse, void *dQ, void *dK, void *dV, int grad_fp32, void *workspace, size_t ws_bytes,
-                   prism_stream_t stream) {
+                   const float *lse, void *dQ, void *dK, void *dV, int grad_fp32, int deterministic,
+                   void *workspace, size_t ws_bytes, prism_stream_t stream) {
   NvtxRange nvtx_("prism_attn_bwd");
   int rc;
   if ((rc = check_params(p)) != PRISM_OK) return rc;
+  if (deterministic != 0 && deterministic != 1) return fail(PRISM_ERR_INVALID_ARG, "deterministic must be 0 or 1");
   if (!Q || !K || !V || !O || !dO || !lse || !dQ || !dK || !dV)
     return fail(PRISM_ERR_INVALID_ARG, "a tensor argument is NULL");
   {
@@ -235,7 +236,8 @@ int prism_attn_bwd(const prism_params *p, const prism_plan_t *plan, const prism_
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(workspace, 0, kWsHeader, st);
   if (e == cudaSuccess)
-    e = launch_attn_bwd(*p, *plan, *sel, Q, K, V, O, O_res, dO, lse, dQ, dK, dV, grad_fp32, workspace, st);
+    e = launch_attn_bwd(*p, *plan, *sel, Q, K, V, O, O_res, dO, lse, dQ, dK, dV, grad_fp32, deterministic,
+                        workspace, st);
   if (e != cudaSuccess) return cuda_fail(e, "prism_attn_bwd");
   g_last_error.clear();
   return PRISM_OK;

@@ -37,7 +37,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 // ---------------------------------------------------------------------------
 // prep: dOp[h][p] = fp16(dO[perm][h]), delta[h][p] = sum_c dO*(O + O_res)
-// (O_res, the forward's bf16 rounding residual, may be NULL), lse2 = lse*log2e;
+// (O_res, the forward's bf16 rounding residual, may be NULL), lse2 = lse*log2e,
+// and, for the fused kernel, the fp32 dQ accumulator's row p zeroed;
 // a dO value outside the fp16 range flags its head in range_flag_do
 // ---------------------------------------------------------------------------
 template <int D>
@@ -47,7 +48,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const int32_t *__restrict
                                                        const uint16_t *__restrict__ O_res,
                                                        const float *__restrict__ lse, uint16_t *__restrict__ dOp,
                                                        float *__restrict__ lse2p, float *__restrict__ deltap,
-                                                       int32_t *__restrict__ range_flag_do) {
+                                                       int32_t *__restrict__ range_flag_do,
+                                                       float *__restrict__ dq_acc) {
   constexpr int G = D / 8;  // lanes per row
   const size_t g = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const size_t r = g / G;
@@ -74,6 +76,11 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const int32_t *__restrict
       acc = fmaf(bf16hi(aw[q]), bf16hi(bw[q]) + bf16hi(cw[q]), acc);
     }
     if (v == 0) lse2p[r] = lse[(size_t)h * N + n] * kLog2e;
+    if (dq_acc) {  // the fused kernel adds into it
+      float4 *z = reinterpret_cast<float4 *>(dq_acc + r * D + v * 8);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
 #pragma unroll
   for (int o = 1; o < G; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -785,6 +792,405 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Fused dK/dV/dQ kernel (head_dim 128): the dK/dV kernel's walk over a
+// 128-key tile's query units, plus dQ^T(i) = K^T dS^T(i) per step, added
+// into an fp32 [heads][N][128] accumulator in permuted order by fp32
+// reductions at L2 (red.global.add).  No S or dP is recomputed for dQ, so
+// the backward issues 10 P D flops instead of the two-kernel path's 14 P D.
+// The reduction order is not fixed: dQ is not bitwise reproducible from run
+// to run (dK and dV are; each CTA owns its key rows).
+//   TMEM: dV [0, 128), dK [128, 256), S^T [256, 384) (P^T packed into it,
+//   read by dV as a TS product), dP^T [384, 512), and dQ^T of the same step
+//   in those columns once the compute warps have read dP^T.
+//   Shared memory: dS^T (fp16, 128 keys x 128 queries, 128-byte swizzle)
+//   is written over the step's dO in its ring stage once dV has read dO.  It
+//   is the K-major A operand of dK += dS^T Q and the MN-major B operand of
+//   dQ^T = K^T dS^T, whose A is the resident K tile read MN-major.
+//   MMA issue order of iteration i: dV(i-1), S^T(i), dQ^T(i-1), dK(i-1),
+//   dP^T(i) (the last once the compute warps have drained dQ^T(i-1)).
+// ---------------------------------------------------------------------------
+struct FusedBars {
+  uint64_t kv_full;
+  uint64_t q_full[NS], q_empty[NS];
+  uint64_t s_full, dp_full, p_ready, ds_ready, dv_done, dq_full, dq_free;
+  uint64_t fin;    // single use: every MMA of the tile has completed
+  uint64_t drain;  // single use: the MMA thread's in-flight products after an abort
+  int meta[NS];    // units | mask_a << 4 | mask_b << 8 (bit = 64-row half of the key tile)
+  int unit[NS][2];  // the stage's query units
+  uint32_t tmem_base;
+  int nsteps, nunits, abort;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    dkdvq_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapDO,
+                 const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
+                 const int32_t *__restrict__ col_ptr, const int32_t *__restrict__ rowidx,
+                 const int32_t *__restrict__ blocks, const int32_t *__restrict__ unit_block,
+                 const int32_t *__restrict__ tile_units, const int32_t *__restrict__ perm,
+                 const float *__restrict__ lse2p, const float *__restrict__ deltap, float *__restrict__ dq_acc,
+                 void *__restrict__ dK, void *__restrict__ dV, int grad_fp32, int N, int heads,
+                 float scale_log2_in, float sm_scale_in, const unsigned *__restrict__ range_max, int *status) {
+  constexpr int D = 128;
+  using L = KvSmem<D>;
+  static_assert(sizeof(FusedBars) <= L::BYTES - L::OFF_BAR, "barrier block");
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  FusedBars &bar = *reinterpret_cast<FusedBars *>(smem + L::OFF_BAR);
+  float *stat = reinterpret_cast<float *>(smem + L::OFF_STAT);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, h = blockIdx.y;
+  const int NB = N / 64;
+  const int32_t *blocks_h = blocks + (size_t)h * NB * 4;
+  // operand pre-scales as in dkdv_kernel; dQ's 2^(edO + eV + eK) is applied
+  // by the conversion pass
+  const int eQ = range_exp(range_max[h], 0), eK = range_exp(range_max[heads + h], 1);
+  const int eV = range_exp(range_max[2 * heads + h], 2), eO = range_exp(range_max[3 * heads + h], 3);
+  const float scale_log2 = ldexpf(scale_log2_in, eQ + eK);
+  const float sm_scale = ldexpf(sm_scale_in, eO + eV + eQ);
+  const float dv_scale = ldexpf(1.0f, eO);
+
+  if (threadIdx.x == 0) bar.abort = *reinterpret_cast<volatile int *>(status);
+  __syncthreads();
+  if (bar.abort) return;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar.kv_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&bar.q_full[s], 1);
+      mbar_init(&bar.q_empty[s], 1);
+    }
+    mbar_init(&bar.s_full, 1);
+    mbar_init(&bar.dp_full, 1);
+    mbar_init(&bar.p_ready, 256);
+    mbar_init(&bar.ds_ready, 256);
+    mbar_init(&bar.dv_done, 1);
+    mbar_init(&bar.dq_full, 1);
+    mbar_init(&bar.dq_free, 256);
+    mbar_init(&bar.fin, 1);
+    mbar_init(&bar.drain, 1);
+    bar.nunits = tile_units[(size_t)h * (N / 128) + tile];
+    bar.nsteps = (bar.nunits + 1) >> 1;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bar.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar.tmem_base;
+  const int nsteps = bar.nsteps, nunits = bar.nunits;
+  const uint32_t tV = tmem, tK = tmem + 128, tS = tmem + 256, tP = tmem + 384;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    const int blk[2] = {unit_block[(size_t)h * NB + 2 * tile], unit_block[(size_t)h * NB + 2 * tile + 1]};
+    UnitWalk<2> w;
+    walk_init<2>(w, blk, 2, col_ptr, h * NB);
+    int q_issued = 0;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bar.kv_full, 2 * L::TILE);
+#pragma unroll
+      for (int c = 0; c < L::CHUNKS; ++c) {
+        tma_load_2d(smem + L::OFF_K + c * (128 * 128), &mapK, &bar.kv_full, c * 64, h * N + tile * 128);
+        tma_load_2d(smem + L::OFF_V + c * (128 * 128), &mapV, &bar.kv_full, c * 64, h * N + tile * 128);
+      }
+    }
+    for (int j = 0; j < nsteps; ++j) {
+      const int s = j % NS;
+      uint32_t ua, ub = 0;
+      int ma, mb = 0, nu = 1;
+      walk_next<2>(w, rowidx, blocks_h, ua, ma);
+      if (2 * j + 2 <= nunits) {
+        walk_next<2>(w, rowidx, blocks_h, ub, mb);
+        nu = 2;
+      }
+      PRISM_CHECK(ua < (uint32_t)NB && ub < (uint32_t)NB, status, 129);
+      ua = min(ua, (uint32_t)(NB - 1));
+      ub = min(ub, (uint32_t)(NB - 1));
+      if (lane == 0) {
+        bool ok = true;
+        if (j >= NS) ok = mbar_wait(&bar.q_empty[s], ((j / NS) - 1) & 1, status, 61);
+        if (!ok) bar.abort = 1;
+        if (ok) {
+          bar.meta[s] = nu | (ma << 4) | (mb << 8);
+          bar.unit[s][0] = (int)ua;
+          bar.unit[s][1] = (int)ub;
+          uint8_t *qs = smem + L::OFF_Q + s * L::TILE;
+          uint8_t *os = smem + L::OFF_DO + s * L::TILE;
+          float *st = stat + s * 256;
+          mbar_arrive_expect_tx(&bar.q_full[s], nu * (2 * 64 * D * 2 + 2 * 64 * 4));
+#pragma unroll
+          for (int c = 0; c < L::CHUNKS; ++c) {
+            tma_load_2d(qs + c * (128 * 128), &mapQ, &bar.q_full[s], c * 64, h * N + (int)ua * 64);
+            tma_load_2d(os + c * (128 * 128), &mapDO, &bar.q_full[s], c * 64, h * N + (int)ua * 64);
+            if (nu == 2) {
+              tma_load_2d(qs + c * (128 * 128) + 64 * 128, &mapQ, &bar.q_full[s], c * 64, h * N + (int)ub * 64);
+              tma_load_2d(os + c * (128 * 128) + 64 * 128, &mapDO, &bar.q_full[s], c * 64, h * N + (int)ub * 64);
+            }
+          }
+          bulk_load(st, lse2p + (size_t)h * N + (size_t)ua * 64, 256, &bar.q_full[s]);
+          bulk_load(st + 128, deltap + (size_t)h * N + (size_t)ua * 64, 256, &bar.q_full[s]);
+          if (nu == 2) {
+            bulk_load(st + 64, lse2p + (size_t)h * N + (size_t)ub * 64, 256, &bar.q_full[s]);
+            bulk_load(st + 192, deltap + (size_t)h * N + (size_t)ub * 64, 256, &bar.q_full[s]);
+          }
+          ++q_issued;
+        }
+      }
+      __syncwarp();
+      if (*reinterpret_cast<volatile int *>(&bar.abort)) break;
+    }
+    if (lane == 0) {  // no copy may still be writing when the CTA leaves
+      drain_loads(&bar.kv_full, 1, 1, status, 62);
+      drain_loads(bar.q_full, NS, q_issued, status, 63);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t id_full = idesc_f16(128, 128, 0), id_half = idesc_f16(128, 64, 0);
+      const uint32_t id_acc = idesc_f16(128, D, 1);
+      const uint64_t dKd = sdesc_sw128(smem_u32(smem + L::OFF_K), 16, 1024);
+      const uint64_t dVd = sdesc_sw128(smem_u32(smem + L::OFF_V), 16, 1024);
+      const uint64_t dKmn = sdesc_sw128(smem_u32(smem + L::OFF_K), 128 * 128, 1024);  // K^T as an MN-major A
+      bool ok = mbar_wait(&bar.kv_full, 0, status, 64);
+      tc_fence_after();
+      for (int i = 0; ok && i <= nsteps; ++i) {
+        const int s = i % NS, sp = (i + NS - 1) % NS;
+        const int nup = i >= 1 ? (bar.meta[sp] & 15) : 0;  // stage sp is not refilled before dK(i-1)
+        if (i >= 1) {  // dV += P^T(i-1) dO(i-1)
+          ok = mbar_wait(&bar.p_ready, (i - 1) & 1, status, 65);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t dDOmn = sdesc_sw128(smem_u32(smem + L::OFF_DO + sp * L::TILE), 128 * 128, 1024);
+          for (int ks = 0; ks < 4 * nup; ++ks)
+            mma_ts(tV, tS + pk_col(ks), dDOmn + (uint64_t)ks * 128, id_acc, (i > 1 || ks > 0) ? 1u : 0u);
+          mma_commit(&bar.dv_done);
+        }
+        uint32_t id = id_full;
+        uint64_t dDOs = 0;
+        if (i < nsteps) {  // S^T(i) = K Q(i)^T, into the columns dV(i-1) read P^T(i-1) from
+          ok = mbar_wait(&bar.q_full[s], (i / NS) & 1, status, 66);
+          if (ok && i >= 1) ok = mbar_wait(&bar.dv_done, (i - 1) & 1, status, 67);
+          if (!ok) break;
+          tc_fence_after();
+          const int nu = bar.meta[s] & 15;  // written before the stage's Q arrived
+          id = nu == 2 ? id_full : id_half;
+          const uint64_t dQs = sdesc_sw128(smem_u32(smem + L::OFF_Q + s * L::TILE), 16, 1024);
+          dDOs = sdesc_sw128(smem_u32(smem + L::OFF_DO + s * L::TILE), 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tS, dKd + kslice16(kk, 128 * 128), dQs + kslice16(kk, 128 * 128), id, kk > 0 ? 1u : 0u);
+          mma_commit(&bar.s_full);
+        }
+        if (i >= 1) {  // dQ^T(i-1) = K^T dS^T(i-1) into the dP^T columns; dK += dS^T(i-1) Q(i-1)
+          ok = mbar_wait(&bar.ds_ready, (i - 1) & 1, status, 68);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t dSmn = sdesc_sw128(smem_u32(smem + L::OFF_DO + sp * L::TILE), 128 * 128, 1024);
+          const uint64_t dSk = sdesc_sw128(smem_u32(smem + L::OFF_DO + sp * L::TILE), 16, 1024);
+          const uint32_t id_q = idesc_f16_amn(128, 64 * nup, 1);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) mma_ss(tP, dKmn + (uint64_t)ks * 128, dSmn + (uint64_t)ks * 128, id_q, ks > 0 ? 1u : 0u);
+          mma_commit(&bar.dq_full);
+          const uint64_t dQmn = sdesc_sw128(smem_u32(smem + L::OFF_Q + sp * L::TILE), 128 * 128, 1024);
+          for (int ks = 0; ks < 4 * nup; ++ks)
+            mma_ss(tK, dSk + kslice16(ks, 128 * 128), dQmn + (uint64_t)ks * 128, id_acc, (i > 1 || ks > 0) ? 1u : 0u);
+          mma_commit(&bar.q_empty[sp]);
+        }
+        if (i < nsteps) {  // dP^T(i) = V dO(i)^T, once dQ^T(i-1) has been drained
+          if (i >= 1) ok = mbar_wait(&bar.dq_free, (i - 1) & 1, status, 69);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tP, dVd + kslice16(kk, 128 * 128), dDOs + kslice16(kk, 128 * 128), id, kk > 0 ? 1u : 0u);
+          mma_commit(&bar.dp_full);
+        }
+      }
+      if (ok && nsteps > 0) mma_commit(&bar.fin);
+      if (!ok) {
+        bar.abort = 1;
+        mma_drain(&bar.drain, status, 70);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ compute
+    const int g = (warp - 4) >> 2;   // warpgroup: query unit g of every step
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;  // key row of the tile; the feature index d of dQ^T
+    const int half = row >> 6;       // warp-uniform
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    bool ok = true;
+    for (int i = 0; i < nsteps; ++i) {
+      const int s = i % NS;
+      ok = mbar_wait_warp(&bar.s_full, i & 1, status, 71);
+      if (ok) ok = mbar_wait_warp(&bar.q_full[s], (i / NS) & 1, status, 72);
+      if (!ok) break;
+      tc_fence_after();
+      const int meta = bar.meta[s];
+      const bool active = g < (meta & 15);
+      const bool valid = active && (((meta >> (4 + 4 * g)) >> half) & 1);  // warp-uniform
+      const float *st = stat + s * 256 + 64 * g;
+      float pf[64];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[16];
+        if (valid) {
+          uint32_t sv[32];
+          float nl[32];
+          tmem_ld32(tS + lane_off + 64 * g + 32 * c, sv);
+#pragma unroll
+          for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 lq = reinterpret_cast<const float4 *>(st + 32 * c)[k4];
+            nl[4 * k4] = -lq.x;
+            nl[4 * k4 + 1] = -lq.y;
+            nl[4 * k4 + 2] = -lq.z;
+            nl[4 * k4 + 3] = -lq.w;
+          }
+          tmem_wait_ld();
+          softmax_p32(sv, scale_log2, [&nl](int k) { return make_float2(nl[k], nl[k + 1]); }, pf + 32 * c);
+#pragma unroll
+          for (int k = 0; k < 32; k += 2) pk[k / 2] = pack_f16(pf[32 * c + k], pf[32 * c + k + 1]);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) pk[k] = 0u;
+        }
+        if (active) tmem_st16(tS + lane_off + 64 * g + 16 * c, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar.p_ready);
+      ok = mbar_wait_warp(&bar.dp_full, i & 1, status, 73);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t ds[32];  // dS^T of this row and unit, fp16 pairs
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        if (valid) {
+          uint32_t dv[32];
+          tmem_ld32(tP + lane_off + 64 * g + 32 * c, dv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 dq = reinterpret_cast<const float4 *>(st + 128 + 32 * c)[k4];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int k = 4 * k4 + 2 * u;
+              const float2 dd = u ? make_float2(dq.z, dq.w) : make_float2(dq.x, dq.y);
+              const float2 d = fmul2(make_float2(pf[32 * c + k], pf[32 * c + k + 1]),
+                                     fsub2(make_float2(__uint_as_float(dv[k]), __uint_as_float(dv[k + 1])), dd));
+              ds[16 * c + k / 2] = pack_f16(d.x, d.y);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) ds[16 * c + k] = 0u;
+        }
+      }
+      // dS^T goes over dO(i) in the stage: wait for dV(i) to have read it
+      ok = mbar_wait_warp(&bar.dv_done, i & 1, status, 74);
+      if (!ok) break;
+      if (active) {
+        uint8_t *rowp = smem + L::OFF_DO + s * L::TILE + g * (128 * 128) + row * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4 *>(rowp + ((j ^ (row & 7)) << 4)) =
+              make_uint4(ds[4 * j], ds[4 * j + 1], ds[4 * j + 2], ds[4 * j + 3]);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bar.ds_ready);
+      // drain dQ^T(i): TMEM lane = feature d, column = query of unit g
+      ok = mbar_wait_warp(&bar.dq_full, i & 1, status, 75);
+      if (!ok) break;
+      tc_fence_after();
+      if (active) {
+        int u = bar.unit[s][g];
+        if (!PRISM_CHECK((unsigned)u < (unsigned)NB, status, 130)) u = 0;
+        float *dst = dq_acc + ((size_t)h * N + (size_t)u * 64) * D + row;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t qv[32];
+          tmem_ld32(tP + lane_off + 64 * g + 32 * c, qv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) red_add_f32(dst + (size_t)(32 * c + k) * D, __uint_as_float(qv[k]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bar.dq_free);
+    }
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok && nsteps > 0) ok = mbar_wait_warp(&bar.fin, 0, status, 76);
+    if (ok) {
+      tc_fence_after();
+      const size_t prow = (size_t)h * N + (size_t)tile * 128 + row;
+      int n = perm[prow];
+      if (!PRISM_CHECK((unsigned)n < (unsigned)N, status, 131)) n = 0;
+      const size_t off = ((size_t)n * heads + h) * D;
+      // warpgroup 0 writes dV, warpgroup 1 writes dK
+      const uint32_t src = g == 0 ? tV : tK;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t o[32];
+        if (nsteps > 0) {
+          tmem_ld32(src + lane_off + c, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = 0u;
+        }
+        store_row<D>(g == 0 ? dV : dK, grad_fp32 != 0, off + c, o, g == 0 ? dv_scale : sm_scale);
+      }
+    } else {
+      bar.abort = 1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// dQ[n][h][:] = 2^(edO + eV + eK) * scale * dq_acc[h][p][:] for n = perm[h][p]:
+// the fused kernel's fp32 accumulator in natural order, bf16 or fp32.
+template <int D>
+__global__ void __launch_bounds__(256) dq_convert_kernel(const int32_t *__restrict__ perm, int N, int heads,
+                                                         const float *__restrict__ acc, void *__restrict__ dQ,
+                                                         int grad_fp32, float sm_scale_in,
+                                                         const unsigned *__restrict__ range_max, int *status) {
+  constexpr int G = D / 8;  // 8-feature vectors per row
+  const size_t total = (size_t)heads * N * G;
+  for (size_t q = (size_t)blockIdx.x * blockDim.x + threadIdx.x; q < total; q += (size_t)gridDim.x * blockDim.x) {
+    const size_t r = q / G;
+    const int v = (int)(q % G);
+    const int h = (int)(r / N);
+    const float mul = ldexpf(sm_scale_in, range_exp(range_max[3 * heads + h], 3) +
+                                              range_exp(range_max[2 * heads + h], 2) +
+                                              range_exp(range_max[heads + h], 1));
+    int n = perm[r];
+    if (!PRISM_CHECK((unsigned)n < (unsigned)N, status, 132)) n = 0;
+    const float4 a = __ldg(reinterpret_cast<const float4 *>(acc + r * D + v * 8));
+    const float4 b = __ldg(reinterpret_cast<const float4 *>(acc + r * D + v * 8 + 4));
+    const size_t off = ((size_t)n * heads + h) * D + v * 8;
+    if (grad_fp32) {
+      float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(dQ) + off);
+      dst[0] = make_float4(a.x * mul, a.y * mul, a.z * mul, a.w * mul);
+      dst[1] = make_float4(b.x * mul, b.y * mul, b.z * mul, b.w * mul);
+    } else {
+      *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(dQ) + off) =
+          make_uint4(pack_bf16(a.x * mul, a.y * mul), pack_bf16(a.z * mul, a.w * mul), pack_bf16(b.x * mul, b.y * mul),
+                     pack_bf16(b.z * mul, b.w * mul));
+    }
+  }
+}
+
 }  // namespace bwd
 
 // ---------------------------------------------------------------------------
@@ -797,6 +1203,7 @@ struct BwdWs {
   int32_t *unit_block, *tu_q, *tu_k;
   int32_t *range_flag;   // [4][heads]
   unsigned *range_max;   // [4][heads]
+  float *dq_acc;         // [heads][N][128] fp32, permuted rows (fused path; head_dim 128 only)
 };
 static BwdWs carve_bwd(const prism_params &p, void *ws) {
   const size_t N = (size_t)p.T * p.H * p.W, h = p.heads, D = p.head_dim;
@@ -825,6 +1232,8 @@ static BwdWs carve_bwd(const prism_params &p, void *ws) {
   w += align_up(sizeof(int32_t) * h * (N / 128), 256);
   b.range_flag = reinterpret_cast<int32_t *>(w);
   b.range_max = reinterpret_cast<unsigned *>(w + sizeof(int32_t) * 4 * h);
+  w += align_up(sizeof(int32_t) * 8 * h, 256);
+  b.dq_acc = D == 128 ? reinterpret_cast<float *>(w) : nullptr;
   return b;
 }
 
@@ -832,7 +1241,7 @@ size_t attn_bwd_ws_bytes(const prism_params &p) {
   const size_t N = (size_t)p.T * p.H * p.W, h = p.heads, D = p.head_dim;
   return kWsHeader + 4 * align_up(sizeof(uint16_t) * h * N * D, 256) + 2 * align_up(sizeof(float) * h * N, 256) +
          align_up(sizeof(int32_t) * h * (N / 64), 256) + 2 * align_up(sizeof(int32_t) * h * (N / 128), 256) +
-         align_up(sizeof(int32_t) * 8 * h, 256);
+         align_up(sizeof(int32_t) * 8 * h, 256) + (D == 128 ? align_up(sizeof(float) * h * N * D, 256) : 0);
 }
 
 template <int D>
@@ -873,12 +1282,45 @@ static cudaError_t run_bwd(const prism_params &p, const prism_plan_t &plan, cons
   return cudaGetLastError();
 }
 
+static cudaError_t run_bwd_fused(const prism_params &p, const prism_plan_t &plan, const prism_select_t &sel,
+                                 const BwdWs &w, void *dQ, void *dK, void *dV, int grad_fp32, cudaStream_t st) {
+  constexpr int D = 128;
+  const int N = p.T * p.H * p.W;
+  const long long rows = (long long)p.heads * N;
+  CUtensorMap mQ64, mDO64, mK128, mV128;
+  cudaError_t e;
+  if ((e = make_rows_map(&mQ64, w.Qp, rows, D, 64)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&mDO64, w.dOp, rows, D, 64)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&mK128, w.Kp, rows, D, 128)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&mV128, w.Vp, rows, D, 128)) != cudaSuccess) return e;
+  const float scale = effective_scale(p);
+  const float scale_log2 = scale * bwd::kLog2e;
+  dim3 grid(N / 128, p.heads);
+  const int s1 = bwd::KvSmem<D>::BYTES + 1024;
+  cudaFuncSetAttribute(bwd::dkdvq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, s1);
+  {
+    KernelTimer kt_(KT_ATTN_BWD_FUSED, st);
+    bwd::dkdvq_kernel<<<grid, bwd::kThreads, s1, st>>>(mQ64, mDO64, mK128, mV128, sel.col_ptr, sel.row, plan.blocks,
+                                                        w.unit_block, w.tu_k, plan.perm, w.lse2p, w.deltap, w.dq_acc,
+                                                        dK, dV, grad_fp32, N, p.heads, scale_log2, scale,
+                                                        w.range_max, &w.hdr->status);
+  }
+  {
+    KernelTimer kt_(KT_DQ_CONVERT, st);
+    bwd::dq_convert_kernel<D><<<148 * 8, 256, 0, st>>>(plan.perm, N, p.heads, w.dq_acc, dQ, grad_fp32, scale,
+                                                       w.range_max, &w.hdr->status);
+  }
+  count_launches(2);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_attn_bwd(const prism_params &p, const prism_plan_t &plan, const prism_select_t &sel,
                             const uint16_t *Q, const uint16_t *K, const uint16_t *V, const uint16_t *O,
                             const uint16_t *O_res, const uint16_t *dO, const float *lse, void *dQ, void *dK,
-                            void *dV, int grad_fp32, void *ws, cudaStream_t st) {
+                            void *dV, int grad_fp32, int deterministic, void *ws, cudaStream_t st) {
   const int N = p.T * p.H * p.W, NB = N / 64, D = p.head_dim;
   BwdWs w = carve_bwd(p, ws);
+  const bool fused = D == 128 && !deterministic;
   cudaError_t e;
   if ((e = cudaMemsetAsync(w.range_flag, 0, sizeof(int32_t) * 8 * p.heads, st)) != cudaSuccess) return e;
   if ((e = launch_permute3(plan.perm, N, p.heads, D, Q, K, V, w.Qp, w.Kp, w.Vp, w.range_flag, &w.hdr->status,
@@ -890,11 +1332,12 @@ cudaError_t launch_attn_bwd(const prism_params &p, const prism_plan_t &plan, con
   if (D == 128)
     bwd::bwd_prep_kernel<128><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(plan.perm, N, p.heads, dO, O, O_res, lse,
                                                                               w.dOp, w.lse2p, w.deltap,
-                                                                              w.range_flag + 3 * p.heads);
+                                                                              w.range_flag + 3 * p.heads,
+                                                                              fused ? w.dq_acc : nullptr);
   else
     bwd::bwd_prep_kernel<64><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(plan.perm, N, p.heads, dO, O, O_res, lse,
                                                                              w.dOp, w.lse2p, w.deltap,
-                                                                             w.range_flag + 3 * p.heads);
+                                                                             w.range_flag + 3 * p.heads, nullptr);
   }
   count_launches(1);
   if ((e = launch_range_fix(plan.perm, N, p.heads, D, RangeSrc{{Q, K, V, dO}}, RangeDst{{w.Qp, w.Kp, w.Vp, w.dOp}},
@@ -907,6 +1350,7 @@ cudaError_t launch_attn_bwd(const prism_params &p, const prism_plan_t &plan, con
   if ((e = launch_tile_units(sel.col_ptr, sel.row, plan.blocks, w.unit_block, N, p.heads, 2, w.tu_k, st)) !=
       cudaSuccess)
     return e;
+  if (fused) return run_bwd_fused(p, plan, sel, w, dQ, dK, dV, grad_fp32, st);
   return D == 128 ? run_bwd<128>(p, plan, sel, w, dQ, dK, dV, grad_fp32, st)
                   : run_bwd<64>(p, plan, sel, w, dQ, dK, dV, grad_fp32, st);
 }

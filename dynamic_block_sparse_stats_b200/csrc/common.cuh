@@ -239,6 +239,13 @@ __device__ __forceinline__ void mma_drain(uint64_t *bar, int *status, int where)
   mma_commit(bar);
   mbar_wait(bar, 0, status, where);
 }
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (tcgen05.mma operand reads) before the barrier that publishes them.
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// Fire-and-forget fp32 add to global memory (performed at L2).
+__device__ __forceinline__ void red_add_f32(float *p, float v) {
+  asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 // tcgen05.wait::ld that also names the registers of the load it completes,
@@ -319,6 +326,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16(uint32_t M, uint32_t N, uint32
 }
 __host__ __device__ constexpr uint32_t idesc_f16(uint32_t M, uint32_t N, uint32_t b_mn_major) {
   return (1u << 4) | (b_mn_major << 16) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+// fp16 operands with A MN-major (bit 15) as well: A read as the transpose of a
+// K-major tile already in shared memory.
+__host__ __device__ constexpr uint32_t idesc_f16_amn(uint32_t M, uint32_t N, uint32_t b_mn_major) {
+  return idesc_f16(M, N, b_mn_major) | (1u << 15);
 }
 
 // ---------------------------------------------------------------------------

@@ -51,7 +51,7 @@ size_t attn_bwd_ws_bytes(const prism_params &p);
 cudaError_t launch_attn_bwd(const prism_params &p, const prism_plan_t &plan, const prism_select_t &sel,
                             const uint16_t *Q, const uint16_t *K, const uint16_t *V, const uint16_t *O,
                             const uint16_t *O_res, const uint16_t *dO, const float *lse, void *dQ, void *dK,
-                            void *dV, int grad_fp32, void *ws, cudaStream_t st);
+                            void *dV, int grad_fp32, int deterministic, void *ws, cudaStream_t st);
 
 // shared launch helper: token gather into permuted head-major order with the
 // bf16 -> fp16 conversion of the attention operands:
@@ -123,6 +123,8 @@ enum KernelTimingId {
   KT_BWD_PREP,
   KT_PROJECT_V,
   KT_RANGE_FIX,
+  KT_ATTN_BWD_FUSED,
+  KT_DQ_CONVERT,
   KT_COUNT
 };
 static_assert(KT_COUNT == PRISM_KERNEL_TIMING_IDS, "timing ids");

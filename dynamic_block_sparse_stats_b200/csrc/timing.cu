@@ -12,7 +12,8 @@ const char *const kNames[KT_COUNT] = {
     "zone_video_stats", "block_mean",  "block_score", "select_row", "attn_fwd",  "attn_bwd_dkdv", "attn_bwd_dq",
     "a2v_norm",         "zone_a2v_stats", "plan_finalize", "perm",   "select_scan", "csr_fill",    "csc_count",
     "csc_scan",         "csc_fill",    "csc_sort",    "permute3",   "unit_block", "tile_units",    "bwd_prep",
-    "project_v",        "range_fix"};
+    "project_v",        "range_fix",
+    "attn_bwd_fused",   "dq_convert"};
 
 struct Rec {
   cudaEvent_t a, b;

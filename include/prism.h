@@ -296,7 +296,9 @@ int prism_select(const prism_params *p, const prism_plan_t *plan,
                  void *workspace, size_t ws_bytes, prism_stream_t stream);
 
 /* Bytes of workspace prism_attn_fwd (backward = 0) or prism_attn_bwd
- * (backward = 1) needs (0 on invalid params). */
+ * (backward = 1, either value of its `deterministic`; for head_dim 128 this
+ * includes the fused path's fp32 dQ accumulator, 4 N heads 128 bytes) needs
+ * (0 on invalid params). */
 size_t prism_attn_workspace_size(const prism_params *p, int backward);
 
 /*
@@ -341,6 +343,16 @@ int prism_attn_fwd(const prism_params *p, const prism_plan_t *plan,
  *   O_res     the forward's O_res, or NULL (Delta from the bf16 O alone).
  *   dO        bf16 [N][heads][head_dim] upstream gradient.
  *   dQ,dK,dV  [N][heads][head_dim]; bf16 when grad_fp32 == 0, fp32 else.
+ *   deterministic  0: for head_dim 128, one kernel per 128-key tile forms
+ *             dK, dV and that tile's share of dQ (dQ = scale dS K added into
+ *             an fp32 accumulator in the workspace by fp32 atomic adds, then
+ *             converted to dQ); 10 P D flops for P computed query-key pairs.
+ *             The order of those adds varies from run to run, so dQ may
+ *             differ in its last bits between runs (dK, dV do not).
+ *             1 (and head_dim 64 always): two kernels, one per 128-key tile
+ *             for dK, dV and one per 128-query tile for dQ, which computes
+ *             S and dP a second time (14 P D flops); every output is
+ *             bitwise reproducible.  Any other value is PRISM_ERR_INVALID_ARG.
  * sel must carry the transpose (col_ptr/row non-NULL).
  * Returns PRISM_OK, PRISM_ERR_INVALID_ARG, PRISM_ERR_UNSUPPORTED,
  * PRISM_ERR_CAPACITY or PRISM_ERR_CUDA.
@@ -350,8 +362,8 @@ int prism_attn_bwd(const prism_params *p, const prism_plan_t *plan,
                    const uint16_t *K, const uint16_t *V, const uint16_t *O,
                    const uint16_t *O_res, const uint16_t *dO,
                    const float *lse, void *dQ, void *dK, void *dV,
-                   int grad_fp32, void *workspace, size_t ws_bytes,
-                   prism_stream_t stream);
+                   int grad_fp32, int deterministic, void *workspace,
+                   size_t ws_bytes, prism_stream_t stream);
 
 /* Waits on `stream` and returns the status a kernel recorded in
  * `workspace`: PRISM_OK, PRISM_ERR_TIMEOUT, or PRISM_ERR_RANGE (an attention
@@ -381,8 +393,9 @@ int prism_kernel_timing(int enable);
  * 16 csc_sort, 17 permute3, 18 unit_block, 19 tile_units, 20 bwd_prep,
  * 21 project_v, 22 range_fix (both launches of the pre-scale fix-up of
  * operands above the fp16 range; their blocks return at once when no value
- * is). */
-#define PRISM_KERNEL_TIMING_IDS 23
+ * is), 23 attn_bwd_fused (dK, dV and dQ in one kernel), 24 dq_convert
+ * (the fused kernel's fp32 dQ accumulator to the natural-order output). */
+#define PRISM_KERNEL_TIMING_IDS 25
 
 /* Reads the records of kernel `id` (0 .. PRISM_KERNEL_TIMING_IDS - 1): waits
  * for its events, and returns the number of timed launches, their total

@@ -68,7 +68,7 @@ int main(void) {
   prism_select_t sel = {p256, p256, 10, 0, NULL, NULL};
   size_t ws_b = prism_attn_workspace_size(&small, 1);
   CHECK(prism_attn_bwd(&small, &plan, &sel, V, V, V, V, NULL, V, (const float *)p256, V, V, V, 0,
-                       (void *)(uintptr_t)256, ws_b, NULL) == PRISM_ERR_INVALID_ARG);
+                       0, (void *)(uintptr_t)256, ws_b, NULL) == PRISM_ERR_INVALID_ARG);
 
   /* a2v_norm: n = 0 is a no-op, a width that is not a multiple of 8 is refused */
   CHECK(prism_a2v_norm(V, 0, 64, 64, (float *)p256, NULL) == PRISM_OK);

@@ -91,7 +91,7 @@ def test_null_pointers_and_short_workspace_are_rejected():
     assert lib.prism_select(C.byref(p), C.byref(plan), C.c_void_p(256), C.c_void_p(256), C.byref(sel),
                             C.c_void_p(256), 1 << 30, None) == _lib.PRISM_ERR_INVALID_ARG
     assert lib.prism_attn_bwd(C.byref(p), C.byref(plan), C.byref(_lib.PrismSelect(256, 256, 10, 0, None, None)),
-                              *([C.c_void_p(256)] * 10), 0, C.c_void_p(256), 1 << 30, None) == _lib.PRISM_ERR_INVALID_ARG
+                              *([C.c_void_p(256)] * 10), 0, 0, C.c_void_p(256), 1 << 30, None) == _lib.PRISM_ERR_INVALID_ARG
 
 
 def test_workspace_sizes_grow_with_the_grid():
@@ -137,7 +137,7 @@ def test_misaligned_tensor_pointers_are_rejected_before_any_cuda_call():
                             C.c_void_p(256), ws, 1 << 40, None)
     assert rc == _lib.PRISM_ERR_INVALID_ARG and "V" in lib.prism_last_error().decode()
     rc = lib.prism_attn_bwd(C.byref(p), C.byref(plan), C.byref(sel), *[C.c_void_p(256)] * 5, C.c_void_p(256),
-                            C.c_void_p(256), C.c_void_p(256), C.c_void_p(260), C.c_void_p(256), 1, ws, 1 << 40, None)
+                            C.c_void_p(256), C.c_void_p(256), C.c_void_p(260), C.c_void_p(256), 1, 0, ws, 1 << 40, None)
     assert rc == _lib.PRISM_ERR_INVALID_ARG and "dK" in lib.prism_last_error().decode()
 
 

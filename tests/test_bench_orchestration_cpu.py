@@ -24,7 +24,7 @@ _KERNEL_MS = {"zone_video_stats": 0.1, "block_mean": 0.2, "block_score": 0.05, "
               "plan_finalize": 0.02, "perm": 0.01, "select_scan": 0.01, "csr_fill": 0.01, "csc_count": 0.01,
               "csc_scan": 0.01, "csc_fill": 0.01, "csc_sort": 0.01, "permute3": 0.05, "unit_block": 0.01,
               "tile_units": 0.01, "bwd_prep": 0.03, "project_v": 0.5,
-              "range_fix": 0.01}
+              "range_fix": 0.01, "attn_bwd_fused": 0.0, "dq_convert": 0.0}
 
 
 class _Lib:
@@ -118,7 +118,8 @@ def _oracle_api(monkeypatch, w):
                              ws if ws is not None else torch.zeros(256, dtype=torch.uint8),
                              O_res if O_res is not None else torch.zeros_like(Q))
 
-    def attn_bwd(p, pl, sel, Q, K, V, O, dO, lse, grad_fp32=False, out=None, ws=None, O_res=None, stream=None):
+    def attn_bwd(p, pl, sel, Q, K, V, O, dO, lse, grad_fp32=False, out=None, ws=None, O_res=None, stream=None,
+                 deterministic=False):
         calls.append("attn_bwd")
         return out if out is not None else tuple(torch.zeros_like(Q) for _ in range(3))
 
@@ -144,7 +145,8 @@ def test_run_prism_orchestration_on_cpu(monkeypatch):
     monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
     monkeypatch.setattr(bench, "read_stream_gbs", lambda device: 7000.0)
     args = argparse.Namespace(steps=2, warmup=3, no_e2e=True, no_cpu_baseline=False, no_dense=True,
-                              shard="layers", workload="tiny", backward=True, no_projection=False)
+                              shard="layers", workload="tiny", backward=True, no_projection=False,
+                              deterministic=True)
     line = bench.run_prism(args, w, rank=0, world=1, device=torch.device("cpu"))
     json.dumps(line)                                        # serialisable as one JSON line
 

@@ -205,7 +205,7 @@ def test_marshalling_through_a_fake_library(monkeypatch):
     assert name == "prism_attn_bwd"
     want = (x["Q"], x["K"], x["V"], fw.O, fw.O_res, x["dO"], fw.lse, dQ, dK, dV)
     assert [t.value for t in args[3:13]] == [t.data_ptr() for t in want]
-    assert args[13] == 1 and args[15] == 4096 and dQ.dtype == torch.float32 and dQ.shape == (N, HEADS, D)
+    assert args[13] == 1 and args[14] == 0 and args[16] == 4096 and dQ.dtype == torch.float32 and dQ.shape == (N, HEADS, D)
 
     with pytest.raises(ValueError, match="dQ must be torch.bfloat16"):
         api.attn_bwd(P, pl, sel, x["Q"], x["K"], x["V"], fw.O, x["dO"], fw.lse, out=(dQ, dK, dV))
@@ -246,7 +246,7 @@ def test_buffer_reuse_as_the_benchmark_step_does(monkeypatch):
     names = [c[0] for c in fake.calls]
     assert names == ["prism_a2v_norm", "prism_plan", "prism_select", "prism_attn_fwd", "prism_attn_bwd"] * 2
     bwd = [c[1] for c in fake.calls if c[0] == "prism_attn_bwd"]
-    assert bwd[0][14].value == bws.data_ptr() and bwd[0][15] == 4096
+    assert bwd[0][15].value == bws.data_ptr() and bwd[0][16] == 4096
     assert [t.value for t in bwd[0][10:13]] == [t.data_ptr() for t in grads]
 
 

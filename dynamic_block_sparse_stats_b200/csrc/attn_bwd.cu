@@ -796,32 +796,73 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // Fused dK/dV/dQ kernel (head_dim 128): the dK/dV kernel's walk over a
 // 128-key tile's query units, plus dQ^T(i) = K^T dS^T(i) per step, added
-// into an fp32 [heads][N][128] accumulator in permuted order by fp32
-// reductions at L2 (red.global.add).  No S or dP is recomputed for dQ, so
-// the backward issues 10 P D flops instead of the two-kernel path's 14 P D.
-// The reduction order is not fixed: dQ is not bitwise reproducible from run
-// to run (dK and dV are; each CTA owns its key rows).
+// into an fp32 [heads][N][128] accumulator in permuted order by bulk
+// reductions (cp.reduce.async.bulk .add.f32, performed at L2).  No S or dP
+// is recomputed for dQ, so the backward issues 10 P D flops instead of the
+// two-kernel path's 14 P D.  The order of the reductions is not fixed: dQ is
+// not bitwise reproducible from run to run (dK and dV are; each CTA owns its
+// key rows).
 //   TMEM: dV [0, 128), dK [128, 256), S^T [256, 384) (P^T packed into it,
 //   read by dV as a TS product), dP^T [384, 512), and dQ^T of the same step
 //   in those columns once the compute warps have read dP^T.
-//   Shared memory: dS^T (fp16, 128 keys x 128 queries, 128-byte swizzle)
-//   is written over the step's dO in its ring stage once dV has read dO.  It
-//   is the K-major A operand of dK += dS^T Q and the MN-major B operand of
-//   dQ^T = K^T dS^T, whose A is the resident K tile read MN-major.
-//   MMA issue order of iteration i: dV(i-1), S^T(i), dQ^T(i-1), dK(i-1),
-//   dP^T(i) (the last once the compute warps have drained dQ^T(i-1)).
+//   Shared memory (FusedSmem; 1024-byte-aligned window, no slack): the K and
+//   V tiles; a ring of two stages, each a Q tile (with its rows' lse) and a
+//   dO tile (with their Delta), filled and released separately; dS^T (fp16,
+//   128 keys x 128 queries, 128-byte swizzle), the K-major A operand of
+//   dK += dS^T Q and the MN-major B operand of dQ^T = K^T dS^T, whose A is
+//   the resident K tile read MN-major.
+//   Per step the compute warps load dQ^T(i) from TMEM (freeing the columns
+//   for dP^T(i+1)) and stage it as [64 queries][128] fp32 per unit:
+//   warpgroup 0 into the stage's dO slot (free once dV(i) and dP^T(i) are
+//   done), warpgroup 1 into the dS^T buffer (free once dQ^T(i) and dK(i)
+//   are).  Warp 2 issues one 32 KB bulk reduction per unit (the unit's 64
+//   accumulator rows are contiguous) and releases the two buffers when the
+//   copies have read them, so the reductions run behind the next step.
+//   MMA issue order of iteration i: dV(i-1), S^T(i) (which runs while the
+//   compute warps form dS(i-1)), dQ^T(i-1), dK(i-1), dP^T(i).
 // ---------------------------------------------------------------------------
+struct FusedSmem {
+  static constexpr int TILE = 128 * 128 * 2;  // 128 rows of 128 fp16
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + TILE;
+  static constexpr int OFF_Q = OFF_V + TILE;        // ring of query-unit pairs
+  static constexpr int OFF_DO = OFF_Q + NS * TILE;  // ring of dO-unit pairs; warpgroup 0's dQ staging
+  static constexpr int OFF_DS = OFF_DO + NS * TILE;  // dS^T; warpgroup 1's dQ staging
+  static constexpr int OFF_STAT = OFF_DS + TILE;     // [NS][lse2 128, delta 128] floats
+  static constexpr int OFF_BAR = OFF_STAT + NS * 256 * 4;
+  static constexpr int BYTES = OFF_BAR + 256;
+};
+
 struct FusedBars {
   uint64_t kv_full;
-  uint64_t q_full[NS], q_empty[NS];
-  uint64_t s_full, dp_full, p_ready, ds_ready, dv_done, dq_full, dq_free;
-  uint64_t fin;    // single use: every MMA of the tile has completed
-  uint64_t drain;  // single use: the MMA thread's in-flight products after an abort
-  int meta[NS];    // units | mask_a << 4 | mask_b << 8 (bit = 64-row half of the key tile)
-  int unit[NS][2];  // the stage's query units
+  uint64_t q_full[NS], o_full[NS];      // Q + lse2, dO + Delta of a stage have arrived
+  uint64_t q_empty[NS], o_empty[NS];    // the Q slot (after dK), the dO slot (after its staging was read)
+  uint64_t s_full, dp_full, p_ready, ds_ready, dv_done, dq_full, dk_done, dq_free;
+  uint64_t staged[2];  // warpgroup g has staged its unit's dQ^T
+  uint64_t ds_free;    // the dS^T buffer's staging has been read
+  uint64_t fin;        // single use: every MMA of the tile has completed
+  uint64_t drain;      // single use: the MMA thread's in-flight products after an abort
+  int meta[NS];        // units | mask_a << 4 | mask_b << 8 (bit = 64-row half of the key tile)
+  int unit[NS][2];     // the stage's query units
+  // step i's unit count and units for the reducer, copied by warpgroup 0
+  // (the producer may refill the stage's meta and unit before the reducer
+  // is done with step i)
+  int red_job[2][3];
   uint32_t tmem_base;
   int nsteps, nunits, abort;
 };
+
+__device__ __forceinline__ void bulk_reduce_add_f32(float *gdst, const void *ssrc, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(gdst),
+               "r"(smem_u32(ssrc)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __global__ void __launch_bounds__(kThreads, 1)
     dkdvq_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapDO,
@@ -833,10 +874,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                  void *__restrict__ dK, void *__restrict__ dV, int grad_fp32, int N, int heads,
                  float scale_log2_in, float sm_scale_in, const unsigned *__restrict__ range_max, int *status) {
   constexpr int D = 128;
-  using L = KvSmem<D>;
+  using L = FusedSmem;
   static_assert(sizeof(FusedBars) <= L::BYTES - L::OFF_BAR, "barrier block");
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  // the layout fills the window: it needs the window 1024-byte aligned (as
+  // the B200 places it) and has no slack to align it here
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) record_status(status, PRISM_ERR_UNSUPPORTED, 77);
+    return;
+  }
   FusedBars &bar = *reinterpret_cast<FusedBars *>(smem + L::OFF_BAR);
   float *stat = reinterpret_cast<float *>(smem + L::OFF_STAT);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -858,7 +904,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar.kv_full, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bar.q_full[s], 1);
+      mbar_init(&bar.o_full[s], 1);
       mbar_init(&bar.q_empty[s], 1);
+      mbar_init(&bar.o_empty[s], 1);
     }
     mbar_init(&bar.s_full, 1);
     mbar_init(&bar.dp_full, 1);
@@ -866,7 +914,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar.ds_ready, 256);
     mbar_init(&bar.dv_done, 1);
     mbar_init(&bar.dq_full, 1);
+    mbar_init(&bar.dk_done, 1);
     mbar_init(&bar.dq_free, 256);
+    mbar_init(&bar.staged[0], 128);
+    mbar_init(&bar.staged[1], 128);
+    mbar_init(&bar.ds_free, 1);
     mbar_init(&bar.fin, 1);
     mbar_init(&bar.drain, 1);
     bar.nunits = tile_units[(size_t)h * (N / 128) + tile];
@@ -889,11 +941,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int blk[2] = {unit_block[(size_t)h * NB + 2 * tile], unit_block[(size_t)h * NB + 2 * tile + 1]};
     UnitWalk<2> w;
     walk_init<2>(w, blk, 2, col_ptr, h * NB);
-    int q_issued = 0;
+    int q_issued = 0, o_issued = 0;
     if (lane == 0) {
       mbar_arrive_expect_tx(&bar.kv_full, 2 * L::TILE);
 #pragma unroll
-      for (int c = 0; c < L::CHUNKS; ++c) {
+      for (int c = 0; c < 2; ++c) {
         tma_load_2d(smem + L::OFF_K + c * (128 * 128), &mapK, &bar.kv_full, c * 64, h * N + tile * 128);
         tma_load_2d(smem + L::OFF_V + c * (128 * 128), &mapV, &bar.kv_full, c * 64, h * N + tile * 128);
       }
@@ -913,39 +965,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         bool ok = true;
         if (j >= NS) ok = mbar_wait(&bar.q_empty[s], ((j / NS) - 1) & 1, status, 61);
-        if (!ok) bar.abort = 1;
         if (ok) {
           bar.meta[s] = nu | (ma << 4) | (mb << 8);
           bar.unit[s][0] = (int)ua;
           bar.unit[s][1] = (int)ub;
           uint8_t *qs = smem + L::OFF_Q + s * L::TILE;
-          uint8_t *os = smem + L::OFF_DO + s * L::TILE;
           float *st = stat + s * 256;
-          mbar_arrive_expect_tx(&bar.q_full[s], nu * (2 * 64 * D * 2 + 2 * 64 * 4));
+          mbar_arrive_expect_tx(&bar.q_full[s], nu * (64 * D * 2 + 64 * 4));
 #pragma unroll
-          for (int c = 0; c < L::CHUNKS; ++c) {
+          for (int c = 0; c < 2; ++c) {
             tma_load_2d(qs + c * (128 * 128), &mapQ, &bar.q_full[s], c * 64, h * N + (int)ua * 64);
-            tma_load_2d(os + c * (128 * 128), &mapDO, &bar.q_full[s], c * 64, h * N + (int)ua * 64);
-            if (nu == 2) {
+            if (nu == 2)
               tma_load_2d(qs + c * (128 * 128) + 64 * 128, &mapQ, &bar.q_full[s], c * 64, h * N + (int)ub * 64);
-              tma_load_2d(os + c * (128 * 128) + 64 * 128, &mapDO, &bar.q_full[s], c * 64, h * N + (int)ub * 64);
-            }
           }
           bulk_load(st, lse2p + (size_t)h * N + (size_t)ua * 64, 256, &bar.q_full[s]);
-          bulk_load(st + 128, deltap + (size_t)h * N + (size_t)ua * 64, 256, &bar.q_full[s]);
-          if (nu == 2) {
-            bulk_load(st + 64, lse2p + (size_t)h * N + (size_t)ub * 64, 256, &bar.q_full[s]);
-            bulk_load(st + 192, deltap + (size_t)h * N + (size_t)ub * 64, 256, &bar.q_full[s]);
-          }
+          if (nu == 2) bulk_load(st + 64, lse2p + (size_t)h * N + (size_t)ub * 64, 256, &bar.q_full[s]);
           ++q_issued;
         }
+        if (ok && j >= NS) ok = mbar_wait(&bar.o_empty[s], ((j / NS) - 1) & 1, status, 62);
+        if (ok) {
+          uint8_t *os = smem + L::OFF_DO + s * L::TILE;
+          float *st = stat + s * 256;
+          mbar_arrive_expect_tx(&bar.o_full[s], nu * (64 * D * 2 + 64 * 4));
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            tma_load_2d(os + c * (128 * 128), &mapDO, &bar.o_full[s], c * 64, h * N + (int)ua * 64);
+            if (nu == 2)
+              tma_load_2d(os + c * (128 * 128) + 64 * 128, &mapDO, &bar.o_full[s], c * 64, h * N + (int)ub * 64);
+          }
+          bulk_load(st + 128, deltap + (size_t)h * N + (size_t)ua * 64, 256, &bar.o_full[s]);
+          if (nu == 2) bulk_load(st + 192, deltap + (size_t)h * N + (size_t)ub * 64, 256, &bar.o_full[s]);
+          ++o_issued;
+        }
+        if (!ok) bar.abort = 1;
       }
       __syncwarp();
       if (*reinterpret_cast<volatile int *>(&bar.abort)) break;
     }
     if (lane == 0) {  // no copy may still be writing when the CTA leaves
-      drain_loads(&bar.kv_full, 1, 1, status, 62);
+      drain_loads(&bar.kv_full, 1, 1, status, 63);
       drain_loads(bar.q_full, NS, q_issued, status, 63);
+      drain_loads(bar.o_full, NS, o_issued, status, 63);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -955,6 +1015,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dKd = sdesc_sw128(smem_u32(smem + L::OFF_K), 16, 1024);
       const uint64_t dVd = sdesc_sw128(smem_u32(smem + L::OFF_V), 16, 1024);
       const uint64_t dKmn = sdesc_sw128(smem_u32(smem + L::OFF_K), 128 * 128, 1024);  // K^T as an MN-major A
+      const uint64_t dSmn = sdesc_sw128(smem_u32(smem + L::OFF_DS), 128 * 128, 1024);  // dS^T as an MN-major B
+      const uint64_t dSk = sdesc_sw128(smem_u32(smem + L::OFF_DS), 16, 1024);          // dS^T as a K-major A
       bool ok = mbar_wait(&bar.kv_full, 0, status, 64);
       tc_fence_after();
       for (int i = 0; ok && i <= nsteps; ++i) {
@@ -970,8 +1032,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&bar.dv_done);
         }
         uint32_t id = id_full;
-        uint64_t dDOs = 0;
-        if (i < nsteps) {  // S^T(i) = K Q(i)^T, into the columns dV(i-1) read P^T(i-1) from
+        if (i < nsteps) {  // S^T(i) = K Q(i)^T, into the columns dV(i-1) read P^T(i-1) from; it runs
+                           // while the compute warps form dS(i-1)
           ok = mbar_wait(&bar.q_full[s], (i / NS) & 1, status, 66);
           if (ok && i >= 1) ok = mbar_wait(&bar.dv_done, (i - 1) & 1, status, 67);
           if (!ok) break;
@@ -979,7 +1041,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int nu = bar.meta[s] & 15;  // written before the stage's Q arrived
           id = nu == 2 ? id_full : id_half;
           const uint64_t dQs = sdesc_sw128(smem_u32(smem + L::OFF_Q + s * L::TILE), 16, 1024);
-          dDOs = sdesc_sw128(smem_u32(smem + L::OFF_DO + s * L::TILE), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             mma_ss(tS, dKd + kslice16(kk, 128 * 128), dQs + kslice16(kk, 128 * 128), id, kk > 0 ? 1u : 0u);
@@ -989,21 +1050,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait(&bar.ds_ready, (i - 1) & 1, status, 68);
           if (!ok) break;
           tc_fence_after();
-          const uint64_t dSmn = sdesc_sw128(smem_u32(smem + L::OFF_DO + sp * L::TILE), 128 * 128, 1024);
-          const uint64_t dSk = sdesc_sw128(smem_u32(smem + L::OFF_DO + sp * L::TILE), 16, 1024);
           const uint32_t id_q = idesc_f16_amn(128, 64 * nup, 1);
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) mma_ss(tP, dKmn + (uint64_t)ks * 128, dSmn + (uint64_t)ks * 128, id_q, ks > 0 ? 1u : 0u);
+          for (int ks = 0; ks < 8; ++ks)
+            mma_ss(tP, dKmn + (uint64_t)ks * 128, dSmn + (uint64_t)ks * 128, id_q, ks > 0 ? 1u : 0u);
           mma_commit(&bar.dq_full);
           const uint64_t dQmn = sdesc_sw128(smem_u32(smem + L::OFF_Q + sp * L::TILE), 128 * 128, 1024);
           for (int ks = 0; ks < 4 * nup; ++ks)
             mma_ss(tK, dSk + kslice16(ks, 128 * 128), dQmn + (uint64_t)ks * 128, id_acc, (i > 1 || ks > 0) ? 1u : 0u);
+          mma_commit(&bar.dk_done);
           mma_commit(&bar.q_empty[sp]);
         }
-        if (i < nsteps) {  // dP^T(i) = V dO(i)^T, once dQ^T(i-1) has been drained
-          if (i >= 1) ok = mbar_wait(&bar.dq_free, (i - 1) & 1, status, 69);
+        if (i < nsteps) {  // dP^T(i) = V dO(i)^T, once the compute warps have read dQ^T(i-1)
+          ok = mbar_wait(&bar.o_full[s], (i / NS) & 1, status, 69);
+          if (ok && i >= 1) ok = mbar_wait(&bar.dq_free, (i - 1) & 1, status, 70);
           if (!ok) break;
           tc_fence_after();
+          const uint64_t dDOs = sdesc_sw128(smem_u32(smem + L::OFF_DO + s * L::TILE), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             mma_ss(tP, dVd + kslice16(kk, 128 * 128), dDOs + kslice16(kk, 128 * 128), id, kk > 0 ? 1u : 0u);
@@ -1013,8 +1076,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok && nsteps > 0) mma_commit(&bar.fin);
       if (!ok) {
         bar.abort = 1;
-        mma_drain(&bar.drain, status, 70);
+        mma_drain(&bar.drain, status, 71);
       }
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ dQ reducer
+    if (lane == 0) {
+      bool ok = true;
+      for (int i = 0; ok && i < nsteps; ++i) {
+        const int s = i % NS;
+        // the dS^T buffer first: the compute warps write the next dS^T into
+        // it, while the dO slot is refilled only for step i + 2
+        ok = mbar_wait(&bar.staged[1], i & 1, status, 82);
+        if (ok) ok = mbar_wait(&bar.staged[0], i & 1, status, 81);
+        if (!ok) break;
+        const int *job = bar.red_job[i & 1];  // written before staged[0] (step i+2 rewrites it only
+                                              // after this step's reductions have been read)
+        const int nu = job[0];
+        int ua = job[1], ub = job[2];
+        if (!PRISM_CHECK((unsigned)ua < (unsigned)NB && (unsigned)ub < (unsigned)NB, status, 130)) ua = ub = 0;
+        if (nu == 2)
+          bulk_reduce_add_f32(dq_acc + ((size_t)h * N + (size_t)ub * 64) * D, smem + L::OFF_DS, 64 * D * 4);
+        bulk_commit();
+        bulk_reduce_add_f32(dq_acc + ((size_t)h * N + (size_t)ua * 64) * D, smem + L::OFF_DO + s * L::TILE,
+                            64 * D * 4);
+        bulk_commit();
+        bulk_wait_read<1>();  // the dS^T buffer's staging has been read
+        mbar_arrive(&bar.ds_free);
+        bulk_wait_read<0>();  // and the dO slot's
+        mbar_arrive(&bar.o_empty[s]);
+      }
+      if (!ok) bar.abort = 1;
+      bulk_wait_all();  // every reduction has been performed before the CTA leaves
     }
     __syncwarp();
   } else if (warp >= 4) {
@@ -1027,11 +1121,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int i = 0; i < nsteps; ++i) {
       const int s = i % NS;
-      ok = mbar_wait_warp(&bar.s_full, i & 1, status, 71);
+      ok = mbar_wait_warp(&bar.s_full, i & 1, status, 72);
+      // the stage's statistics were written by the async proxy: observe the
+      // stage's own barriers (already complete) so those writes are visible
       if (ok) ok = mbar_wait_warp(&bar.q_full[s], (i / NS) & 1, status, 72);
       if (!ok) break;
       tc_fence_after();
-      const int meta = bar.meta[s];
+      // the stage's meta and units, read before this step releases the stage
+      const int meta = bar.meta[s], unit0 = bar.unit[s][0], unit1 = bar.unit[s][1];
       const bool active = g < (meta & 15);
       const bool valid = active && (((meta >> (4 + 4 * g)) >> half) & 1);  // warp-uniform
       const float *st = stat + s * 256 + 64 * g;
@@ -1065,6 +1162,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&bar.p_ready);
       ok = mbar_wait_warp(&bar.dp_full, i & 1, status, 73);
+      if (ok) ok = mbar_wait_warp(&bar.o_full[s], (i / NS) & 1, status, 73);
       if (!ok) break;
       tc_fence_after();
       uint32_t ds[32];  // dS^T of this row and unit, fp16 pairs
@@ -1091,11 +1189,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < 16; ++k) ds[16 * c + k] = 0u;
         }
       }
-      // dS^T goes over dO(i) in the stage: wait for dV(i) to have read it
-      ok = mbar_wait_warp(&bar.dv_done, i & 1, status, 74);
+      // the dS^T buffer held the previous step's staging until its reduction read it
+      if (i >= 1) ok = mbar_wait_warp(&bar.ds_free, (i - 1) & 1, status, 74);
       if (!ok) break;
       if (active) {
-        uint8_t *rowp = smem + L::OFF_DO + s * L::TILE + g * (128 * 128) + row * 128;
+        uint8_t *rowp = smem + L::OFF_DS + g * (128 * 128) + row * 128;
 #pragma unroll
         for (int j = 0; j < 8; ++j)
           *reinterpret_cast<uint4 *>(rowp + ((j ^ (row & 7)) << 4)) =
@@ -1104,28 +1202,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(&bar.ds_ready);
-      // drain dQ^T(i): TMEM lane = feature d, column = query of unit g
-      ok = mbar_wait_warp(&bar.dq_full, i & 1, status, 75);
+      // dQ^T(i): TMEM lane = feature d, column = query of unit g.  Staged as
+      // [64 queries][128] fp32: warpgroup 0 into the dO slot once dQ^T(i) is
+      // done (dV(i) and dP^T(i), issued before it, are too), warpgroup 1
+      // into the dS^T buffer once dK(i), the buffer's last reader, is done.
+      // Then dP^T(i+1) may take the columns.
+      ok = g == 0 ? mbar_wait_warp(&bar.dq_full, i & 1, status, 75) : mbar_wait_warp(&bar.dk_done, i & 1, status, 76);
       if (!ok) break;
       tc_fence_after();
       if (active) {
-        int u = bar.unit[s][g];
-        if (!PRISM_CHECK((unsigned)u < (unsigned)NB, status, 130)) u = 0;
-        float *dst = dq_acc + ((size_t)h * N + (size_t)u * 64) * D + row;
+        float *stg = reinterpret_cast<float *>(smem + (g == 0 ? L::OFF_DO + s * L::TILE : L::OFF_DS));
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t qv[32];
           tmem_ld32(tP + lane_off + 64 * g + 32 * c, qv);
           tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 32; ++k) red_add_f32(dst + (size_t)(32 * c + k) * D, __uint_as_float(qv[k]));
+          for (int k = 0; k < 32; ++k) stg[(32 * c + k) * D + row] = __uint_as_float(qv[k]);
         }
       }
       tc_fence_before();
       mbar_arrive(&bar.dq_free);
+      if (g == 0 && q4 == 0 && lane == 0) {
+        bar.red_job[i & 1][0] = meta & 15;
+        bar.red_job[i & 1][1] = unit0;
+        bar.red_job[i & 1][2] = unit1;
+      }
+      fence_async_smem();
+      mbar_arrive(&bar.staged[g]);
     }
     ok = __all_sync(0xffffffffu, ok);
-    if (ok && nsteps > 0) ok = mbar_wait_warp(&bar.fin, 0, status, 76);
+    if (ok && nsteps > 0) ok = mbar_wait_warp(&bar.fin, 0, status, 78);
     if (ok) {
       tc_fence_after();
       const size_t prow = (size_t)h * N + (size_t)tile * 128 + row;
@@ -1296,7 +1403,7 @@ static cudaError_t run_bwd_fused(const prism_params &p, const prism_plan_t &plan
   const float scale = effective_scale(p);
   const float scale_log2 = scale * bwd::kLog2e;
   dim3 grid(N / 128, p.heads);
-  const int s1 = bwd::KvSmem<D>::BYTES + 1024;
+  const int s1 = bwd::FusedSmem::BYTES;  // exactly the layout: the window's base is 1024-byte aligned
   cudaFuncSetAttribute(bwd::dkdvq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, s1);
   {
     KernelTimer kt_(KT_ATTN_BWD_FUSED, st);

@@ -66,6 +66,8 @@ WORKLOADS = {
     # 8x16x16 grid, one head, D=64: four zones; one zone carries an
     # amplitude-3 sinusoid along H, one zone an A2V blob.
     "tiny": Workload("tiny", 8, 16, 16, 1, 64, topk_abs=2, top_p=0.9, kind="tiny"),
+    # the same grid and fields at D=128 (the fused backward's head size)
+    "tiny_d128": Workload("tiny_d128", 8, 16, 16, 1, 128, topk_abs=2, top_p=0.9, kind="tiny"),
     # Parity-test grids: small enough for the oracle, several tiles, and
     # a zone count that is not a multiple of any tile size.
     "small": Workload("small", 16, 24, 40, 2, 128, topk_frac=0.10, top_p=0.9,

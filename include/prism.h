@@ -366,8 +366,10 @@ int prism_attn_bwd(const prism_params *p, const prism_plan_t *plan,
                    size_t ws_bytes, prism_stream_t stream);
 
 /* Waits on `stream` and returns the status a kernel recorded in
- * `workspace`: PRISM_OK, PRISM_ERR_TIMEOUT, or PRISM_ERR_RANGE (an attention
- * call met an infinite or NaN Q/K/V/dO value), or PRISM_ERR_CUDA. */
+ * `workspace`: PRISM_OK, PRISM_ERR_TIMEOUT, PRISM_ERR_RANGE (an attention
+ * call met an infinite or NaN Q/K/V/dO value), PRISM_ERR_UNSUPPORTED (the
+ * fused backward found its shared-memory window not 1024-byte aligned; its
+ * layout fills the window and cannot realign it), or PRISM_ERR_CUDA. */
 int prism_workspace_status(const void *workspace, prism_stream_t stream);
 
 /* Message of the calling thread's last failing call ("" if none).  The

@@ -813,13 +813,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   the resident K tile read MN-major.
 //   Per step the compute warps load dQ^T(i) from TMEM (freeing the columns
 //   for dP^T(i+1)) and stage it as [64 queries][128] fp32 per unit:
-//   warpgroup 0 into the stage's dO slot (free once dV(i) and dP^T(i) are
-//   done), warpgroup 1 into the dS^T buffer (free once dQ^T(i) and dK(i)
-//   are).  Warp 2 issues one 32 KB bulk reduction per unit (the unit's 64
+//   warpgroup 0 into the stage's dO slot, warpgroup 1 into the dS^T buffer
+//   (both free once dQ^T(i), the last product issued that reads them, is
+//   done).  Warp 2 issues one 32 KB bulk reduction per unit (the unit's 64
 //   accumulator rows are contiguous) and releases the two buffers when the
 //   copies have read them, so the reductions run behind the next step.
 //   MMA issue order of iteration i: dV(i-1), S^T(i) (which runs while the
-//   compute warps form dS(i-1)), dQ^T(i-1), dK(i-1), dP^T(i).
+//   compute warps form dS(i-1)), dK(i-1), dQ^T(i-1), dP^T(i).
 // ---------------------------------------------------------------------------
 struct FusedSmem {
   static constexpr int TILE = 128 * 128 * 2;  // 128 rows of 128 fp16
@@ -837,7 +837,7 @@ struct FusedBars {
   uint64_t kv_full;
   uint64_t q_full[NS], o_full[NS];      // Q + lse2, dO + Delta of a stage have arrived
   uint64_t q_empty[NS], o_empty[NS];    // the Q slot (after dK), the dO slot (after its staging was read)
-  uint64_t s_full, dp_full, p_ready, ds_ready, dv_done, dq_full, dk_done, dq_free;
+  uint64_t s_full, dp_full, p_ready, ds_ready, dv_done, dq_full, dq_free;
   uint64_t staged[2];  // warpgroup g has staged its unit's dQ^T
   uint64_t ds_free;    // the dS^T buffer's staging has been read
   uint64_t fin;        // single use: every MMA of the tile has completed
@@ -914,7 +914,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar.ds_ready, 256);
     mbar_init(&bar.dv_done, 1);
     mbar_init(&bar.dq_full, 1);
-    mbar_init(&bar.dk_done, 1);
     mbar_init(&bar.dq_free, 256);
     mbar_init(&bar.staged[0], 128);
     mbar_init(&bar.staged[1], 128);
@@ -1046,20 +1045,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_ss(tS, dKd + kslice16(kk, 128 * 128), dQs + kslice16(kk, 128 * 128), id, kk > 0 ? 1u : 0u);
           mma_commit(&bar.s_full);
         }
-        if (i >= 1) {  // dQ^T(i-1) = K^T dS^T(i-1) into the dP^T columns; dK += dS^T(i-1) Q(i-1)
+        if (i >= 1) {  // dK += dS^T(i-1) Q(i-1); dQ^T(i-1) = K^T dS^T(i-1) into the dP^T columns
           ok = mbar_wait(&bar.ds_ready, (i - 1) & 1, status, 68);
           if (!ok) break;
           tc_fence_after();
+          const uint64_t dQmn = sdesc_sw128(smem_u32(smem + L::OFF_Q + sp * L::TILE), 128 * 128, 1024);
+          for (int ks = 0; ks < 4 * nup; ++ks)
+            mma_ss(tK, dSk + kslice16(ks, 128 * 128), dQmn + (uint64_t)ks * 128, id_acc, (i > 1 || ks > 0) ? 1u : 0u);
+          mma_commit(&bar.q_empty[sp]);
           const uint32_t id_q = idesc_f16_amn(128, 64 * nup, 1);
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
             mma_ss(tP, dKmn + (uint64_t)ks * 128, dSmn + (uint64_t)ks * 128, id_q, ks > 0 ? 1u : 0u);
-          mma_commit(&bar.dq_full);
-          const uint64_t dQmn = sdesc_sw128(smem_u32(smem + L::OFF_Q + sp * L::TILE), 128 * 128, 1024);
-          for (int ks = 0; ks < 4 * nup; ++ks)
-            mma_ss(tK, dSk + kslice16(ks, 128 * 128), dQmn + (uint64_t)ks * 128, id_acc, (i > 1 || ks > 0) ? 1u : 0u);
-          mma_commit(&bar.dk_done);
-          mma_commit(&bar.q_empty[sp]);
+          mma_commit(&bar.dq_full);  // also covers dK(i-1), issued before
         }
         if (i < nsteps) {  // dP^T(i) = V dO(i)^T, once the compute warps have read dQ^T(i-1)
           ok = mbar_wait(&bar.o_full[s], (i / NS) & 1, status, 69);
@@ -1202,12 +1200,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(&bar.ds_ready);
-      // dQ^T(i): TMEM lane = feature d, column = query of unit g.  Staged as
-      // [64 queries][128] fp32: warpgroup 0 into the dO slot once dQ^T(i) is
-      // done (dV(i) and dP^T(i), issued before it, are too), warpgroup 1
-      // into the dS^T buffer once dK(i), the buffer's last reader, is done.
-      // Then dP^T(i+1) may take the columns.
-      ok = g == 0 ? mbar_wait_warp(&bar.dq_full, i & 1, status, 75) : mbar_wait_warp(&bar.dk_done, i & 1, status, 76);
+      // dQ^T(i): TMEM lane = feature d, column = query of unit g.  Once it is
+      // done (and with it every product issued before: dV(i), dP^T(i) and
+      // dK(i), the last readers of the dO slot and of the dS^T buffer), it
+      // is staged as [64 queries][128] fp32, warpgroup 0 into the stage's
+      // dO slot, warpgroup 1 into the dS^T buffer.  Then dP^T(i+1) may take
+      // the columns.
+      ok = mbar_wait_warp(&bar.dq_full, i & 1, status, 75);
       if (!ok) break;
       tc_fence_after();
       if (active) {

@@ -329,7 +329,8 @@ KERNEL_SOURCES = {"project_v": "project.cu", "zone_video_stats": "plan.cu", "zon
                   "range_fix": "range.cu"}
 NCU_KERNEL_NAMES = {"a2v_norm": "a2v_norm_kernel", "zone_video_stats": "zone_video_stats_kernel",
                     "block_mean": "block_mean_kernel", "attn_fwd": "attn_fwd_kernel",
-                    "attn_bwd_dkdv": "dkdv_kernel", "attn_bwd_dq": "dq_kernel"}
+                    "attn_bwd_dkdv": "dkdv_kernel", "attn_bwd_dq": "dq_kernel", "attn_bwd_fused": "dkdvq_kernel",
+                    "project_v": "project_v_kernel"}
 
 
 def strip_comments(text: str) -> str:
@@ -408,20 +409,26 @@ def stored_traffic(kernel):
     return d["bytes_per_launch"]
 
 
-def write_traffic(csv_path, out_path=None):
-    """profiles/traffic.json from an ncu capture of dram__bytes_read.sum and
-    dram__bytes_write.sum (`ncu --csv --log-file`): per timed kernel, the mean
-    of read + write bytes over its captured launches, keyed to the digest of
-    the kernel's code as it is now (run it on the code that was captured)."""
-    rows, start = [], False
-    with open(csv_path) as f:
-        for line in f:
-            if line.startswith('"ID"'):
-                start = True
-            if start:
-                rows.append(line)
+def write_traffic(csv_paths, out_path=None):
+    """profiles/traffic.json from ncu captures of dram__bytes_read.sum and
+    dram__bytes_write.sum (`ncu --csv --log-file`, one or more files): per
+    timed kernel, the mean of read + write bytes over its captured launches,
+    keyed to the digest of the kernel's code as it is now (run it on the code
+    that was captured)."""
+    if isinstance(csv_paths, str):
+        csv_paths = [csv_paths]
+    records = []
+    for k, path in enumerate(csv_paths):
+        rows, start = [], False
+        with open(path) as f:
+            for line in f:
+                if line.startswith('"ID"'):
+                    start = True
+                if start:
+                    rows.append(line)
+        records += [dict(r, ID=f"{k}:{r['ID']}") for r in csv.DictReader(io.StringIO("".join(rows)))]
     per = {}
-    for r in csv.DictReader(io.StringIO("".join(rows))):
+    for r in records:
         if r["Metric Name"] not in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
             continue
         name = next((k for k, frag in NCU_KERNEL_NAMES.items() if frag in r["Kernel Name"]), None)
@@ -843,7 +850,7 @@ def main():
     ap.add_argument("--no-projection", action="store_true",
                     help="plan from a given V (prism_plan) instead of the fused value projection "
                          "(prism_project_v_plan) in the step")
-    ap.add_argument("--write-traffic", metavar="NCU_CSV",
+    ap.add_argument("--write-traffic", metavar="NCU_CSV", nargs="+",
                     help="write profiles/traffic.json from an ncu DRAM-bytes capture and exit (no GPU needed)")
     ap.add_argument("--shard", choices=["layers", "heads"], default="layers",
                     help="N>1: every rank its own layer (weak scaling, default) or one layer's heads split "

@@ -3,7 +3,9 @@ heads gives, bit for bit, the same plan, selection, forward and backward
 outputs as the same heads of the full-layer call.  The path has no
 cross-head step (plan, selection and attention are per head; the A2V map is
 per token and shared), which is what `bench.py --shard heads` relies on when
-it splits one layer's heads over ranks."""
+it splits one layer's heads over ranks.  The fused backward sums dQ in no
+fixed order, so for it dK and dV are compared bit for bit and dQ within a
+few fp32 roundings; the deterministic backward is compared bit for bit."""
 import numpy as np
 import pytest
 import torch
@@ -20,7 +22,8 @@ def _run(w, inp):
     pl = api.plan(p, inp["V"], inp["a"])
     sel = api.select(p, pl, inp["Q"], inp["K"])
     fw = api.attn_fwd(p, pl, sel, inp["Q"], inp["K"], inp["V"])
-    g = api.attn_bwd(p, pl, sel, inp["Q"], inp["K"], inp["V"], fw.O, inp["dO"], fw.lse, O_res=fw.O_res)
+    g = [api.attn_bwd(p, pl, sel, inp["Q"], inp["K"], inp["V"], fw.O, inp["dO"], fw.lse, O_res=fw.O_res,
+                      grad_fp32=True, deterministic=det) for det in (True, False)]
     torch.cuda.synchronize()
     assert api.workspace_status(fw.ws) == 0
     return pl, sel, fw, g
@@ -54,5 +57,9 @@ def test_head_slice_equals_full_layer(h0, h1):
     assert torch.equal(fw_f.O[:, h0:h1], fw_p.O)
     assert torch.equal(fw_f.O_res[:, h0:h1], fw_p.O_res)
     assert torch.equal(fw_f.lse[h0:h1], fw_p.lse)
-    for a, b in zip(g_f, g_p):
+    for a, b in zip(g_f[0], g_p[0]):       # deterministic backward
         assert torch.equal(a[:, h0:h1], b)
+    for a, b in zip(g_f[1][1:], g_p[1][1:]):  # fused: dK, dV
+        assert torch.equal(a[:, h0:h1], b)
+    d = (g_f[1][0][:, h0:h1] - g_p[1][0]).abs().max().item()
+    assert d <= 1e-5 * g_p[1][0].abs().max().item(), d

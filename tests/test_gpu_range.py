@@ -39,12 +39,16 @@ def _close(got, want):
     assert d.max().item() <= MAX_ABS and d.mean().item() <= MEAN_ABS, (d.max().item(), d.mean().item())
 
 
-def _layer(w, Q, K, V, dO, a, sm_scale=0.0):
+def _layer(w, Q, K, V, dO, a, sm_scale=0.0, deterministic=True):
+    """The bit-for-bit comparisons below use the deterministic backward (the
+    fused one sums dQ in no fixed order); the fused path is checked against
+    it on the same out-of-range inputs at the end."""
     p = api.params_for(w, sm_scale=sm_scale)
     pl = api.plan(p, V, a)
     sel = api.select(p, pl, Q, K)
     fw = api.attn_fwd(p, pl, sel, Q, K, V)
-    g = api.attn_bwd(p, pl, sel, Q, K, V, fw.O, dO, fw.lse, grad_fp32=True, O_res=fw.O_res)
+    g = api.attn_bwd(p, pl, sel, Q, K, V, fw.O, dO, fw.lse, grad_fp32=True, O_res=fw.O_res,
+                     deterministic=deterministic)
     torch.cuda.synchronize()
     assert api.workspace_status(fw.ws) == 0
     return sel, fw, g
@@ -103,3 +107,25 @@ def test_large_upstream_gradient(base):
     assert torch.equal(g[2][:, 1], g0[2][:, 1] * S17)
     for k in (0, 1):
         _close(g[k][:, 1] / S17, g0[k][:, 1])
+
+
+@pytest.mark.parametrize("which", ["K", "V", "dO"])
+def test_fused_backward_with_out_of_range_heads(base, which):
+    """The fused backward folds the same pre-scales back (dK, dV in its
+    stores, dQ in the conversion pass): on each out-of-range input it gives
+    the deterministic path's dK and dV bit for bit and its dQ within a few
+    fp32 roundings."""
+    w, inp, _ = base
+    x = dict(Q=inp["Q"], K=inp["K"], V=inp["V"], dO=inp["dO"])
+    sm = 0.0
+    if which == "K":
+        x["K"] = _scaled(_scaled(inp["K"], 0, S17), 1, S17)
+        sm = scale_of(w.head_dim) / S17
+    else:
+        x[which] = _scaled(inp[which], 1, S17)
+    assert x[which].float().abs().max().item() > 65504
+    _, _, gd = _layer(w, x["Q"], x["K"], x["V"], x["dO"], inp["a"], sm_scale=sm, deterministic=True)
+    _, _, gf = _layer(w, x["Q"], x["K"], x["V"], x["dO"], inp["a"], sm_scale=sm, deterministic=False)
+    assert torch.equal(gf[1], gd[1]) and torch.equal(gf[2], gd[2])
+    d = (gf[0] - gd[0]).abs().max().item()
+    assert d <= 1e-5 * gd[0].abs().max().item(), d

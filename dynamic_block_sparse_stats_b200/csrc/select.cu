@@ -286,6 +286,27 @@ __device__ __forceinline__ void block_excl_scan2(int v0, int v1, int &e0, int &e
   __syncthreads();
 }
 
+// One histogram update per distinct bucket and warp instead of one per key:
+// rows whose scores are close together put most keys of a digit into a few
+// buckets, and per-key shared-memory atomics on those serialise.  The lanes
+// with the same bucket sum their counts and weights (each weight < 2^62,
+// at most 32 of them, summed exactly in three 21-bit parts) and the lowest
+// of them adds.  Integer sums, so the histogram is the same in any order.
+// b < 0: the lane adds nothing.  Every lane of the warp calls it.
+__device__ __forceinline__ void hist_add(SelShared &sh, int b, unsigned long long w, bool with_sum) {
+  const unsigned peers = __match_any_sync(0xffffffffu, b);
+  if (b < 0) return;
+  const bool leader = (int)(threadIdx.x & 31) == __ffs(peers) - 1;
+  if (with_sum) {
+    const unsigned s0 = __reduce_add_sync(peers, (unsigned)(w & 0x1fffffu));
+    const unsigned s1 = __reduce_add_sync(peers, (unsigned)((w >> 21) & 0x1fffffu));
+    const unsigned s2 = __reduce_add_sync(peers, (unsigned)(w >> 42));
+    if (leader)
+      atomicAdd(&sh.hsum[b], (unsigned long long)s0 + ((unsigned long long)s1 << 21) + ((unsigned long long)s2 << 42));
+  }
+  if (leader) atomicAdd(&sh.hcnt[b], __popc(peers));
+}
+
 __global__ void __launch_bounds__(kSelThreads) select_row_kernel(float *__restrict__ S, int NB,
                                                                  const int32_t *__restrict__ nb_ptr, float topk_frac,
                                                                  int topk_abs, float top_p,
@@ -391,13 +412,18 @@ __global__ void __launch_bounds__(kSelThreads) select_row_kernel(float *__restri
       }
       __syncthreads();
       const uint32_t prefix = sh.prefix;
-      for (int j = tid; j < nb; j += kSelThreads) {
-        const uint32_t u = key[j];
-        if ((u & pmask) == prefix) {
-          const int b = (u >> shift) & dmask;
-          atomicAdd(&sh.hcnt[b], 1);
-          atomicAdd(&sh.hsum[b], quant_weight(ev[j], qscale));
+      for (int j0 = 0; j0 < nb; j0 += kSelThreads) {  // the same trip count for every thread
+        const int j = j0 + tid;
+        int b = -1;
+        unsigned long long wq = 0;
+        if (j < nb) {
+          const uint32_t u = key[j];
+          if ((u & pmask) == prefix) {
+            b = (int)((u >> shift) & dmask);
+            wq = quant_weight(ev[j], qscale);
+          }
         }
+        hist_add(sh, b, wq, true);
       }
       __syncthreads();
       if (warp == 0) bucket_descent(sh, true, target, 0, shift);
@@ -446,9 +472,14 @@ __global__ void __launch_bounds__(kSelThreads) select_row_kernel(float *__restri
       }
       __syncthreads();
       const uint32_t prefix = sh.prefix;
-      for (int j = tid; j < nb; j += kSelThreads) {
-        const uint32_t u = key[j];
-        if ((u & pmask) == prefix) atomicAdd(&sh.hcnt[(u >> shift) & dmask], 1);
+      for (int j0 = 0; j0 < nb; j0 += kSelThreads) {  // the same trip count for every thread
+        const int j = j0 + tid;
+        int b = -1;
+        if (j < nb) {
+          const uint32_t u = key[j];
+          if ((u & pmask) == prefix) b = (int)((u >> shift) & dmask);
+        }
+        hist_add(sh, b, 0ull, false);
       }
       __syncthreads();
       if (warp == 0) bucket_descent(sh, false, 0ull, n, shift);

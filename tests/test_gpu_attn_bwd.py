@@ -44,8 +44,8 @@ def _run(name, grad_fp32=True, residual=True, deterministic=False, **over):
     return w, inp, p, pl, sel, fw, g
 
 
-def _check(name, heads=None, n_sample=None, seed=0, deterministic=False):
-    w, inp, p, pl, sel, fw, (dQ, dK, dV) = _run(name, deterministic=deterministic)
+def _check(name, heads=None, n_sample=None, seed=0, deterministic=False, **over):
+    w, inp, p, pl, sel, fw, (dQ, dK, dV) = _run(name, deterministic=deterministic, **over)
     NB = w.N // 64
     nb = to_np(pl.n_blocks)
     shapes = to_np(pl.zone_shape)
@@ -96,6 +96,14 @@ def test_bwd_small_d128(deterministic):
 
 def test_bwd_small_d64_multihead():
     _check("small_d64")
+
+
+@pytest.mark.parametrize("deterministic", [False, True])
+def test_bwd_one_block_per_row(deterministic):
+    """Top-k only with k = 1: most key tiles have one or no user, so the
+    kernels' empty walks (zero dK, dV, no dQ reductions) and single-unit
+    steps carry most of the layer."""
+    _check("small", deterministic=deterministic, topk_abs=1, top_p=0.0)
 
 
 @pytest.mark.parametrize("deterministic", [False, True])

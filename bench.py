@@ -205,6 +205,7 @@ def kernel_rooflines(ktimes, P, D, N, h, nb, peaks, peak_src, steps, nnz=0, sm_m
     sustained = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     burst = peaks.get("bf16_tflops", sustained)
     hbm = peaks["hbm_gbs"]
+    fused = bool(ktimes.get("attn_bwd_fused", (0, 0.0))[0])  # the backward ran the fused kernel
     sum_nb2 = float((nb.double() ** 2).sum().item())
     sum_nb = float(nb.double().sum().item())
     Z = N // 512
@@ -244,8 +245,9 @@ def kernel_rooflines(ktimes, P, D, N, h, nb, peaks, peak_src, steps, nnz=0, sm_m
         "tile_units": ("hbm", 3 * 12.0 * nnz, None,
                        "per launch the selection's ids and the block sizes they index (about 12*nnz bytes; "
                        "one launch in the forward, two in the backward)"),
-        "bwd_prep": ("hbm", 8.0 * HBD + 16.0 * HN, None,
-                     "dO, O, O_res read, fp16 dO written (8*N*h*D bytes) + LSE, Delta (16*N*h)"),
+        "bwd_prep": ("hbm", (12.0 if fused else 8.0) * HBD + 16.0 * HN, None,
+                     "dO, O, O_res read, fp16 dO written (8*N*h*D bytes) + LSE, Delta (16*N*h)"
+                     + (" + the fused path's fp32 dQ accumulator zeroed (4*N*h*D)" if fused else "")),
         "a2v_norm": ("hbm", 2.0 * HBD + 4.0 * N, None,
                      "one read of the bridge output (2*N*h*D bytes) + the fp32 norms (4*N)"),
         "range_fix": ("hbm", None, None, "pre-scale fix-up of operands above the fp16 range: every block "

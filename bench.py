@@ -844,7 +844,7 @@ def run_prism(args, w, rank, world, device):
                    "topk_frac": w.topk_frac, "top_p": w.top_p, "backward": backward,
                    "bwd_path": (None if not backward else
                                 "two-kernel, deterministic" if args.deterministic or D != 128 else
-                                "fused dK/dV/dQ, dQ by fp32 atomic adds"),
+                                "fused dK/dV/dQ, dQ summed by fp32 bulk reductions"),
                    "plan_from": ("prism_project_v_plan: V = X Wv^T (C = %d) with the zone statistics in the "
                                  "GEMM epilogue" % X.shape[1]) if proj else "prism_plan of a given V",
                    "parallelism": (f"heads split over {world} ranks (this rank {h0}-{h1 - 1}), no collectives on the path"

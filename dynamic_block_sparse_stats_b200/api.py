@@ -368,8 +368,8 @@ def attn_bwd(p: PrismParams, pl: Plan, sel: Selection, Q, K, V, O, dO, lse, grad
              O_res=None, stream=None, deterministic=False):
     """prism_attn_bwd: dQ, dK, dV through the selected blocks (natural order).
     Pass the forward's O_res for an fp32-accurate Delta.  deterministic=False
-    (head_dim 128) takes the fused kernel, whose dQ is summed by fp32 atomic
-    adds in no fixed order; True takes the two-kernel path, bitwise
+    (head_dim 128) takes the fused kernel, whose dQ is summed by fp32
+    reductions in no fixed order; True takes the two-kernel path, bitwise
     reproducible."""
     N = p.T * p.H * p.W
     shape = (N, p.heads, p.head_dim)

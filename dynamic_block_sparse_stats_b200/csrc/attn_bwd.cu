@@ -9,7 +9,11 @@
 //   P = exp(s*scale - lse), dP = dO V^T, Delta_q = sum_c dO_qc O_qc,
 //   dS = P (dP - Delta), dQ = scale dS K, dK = scale dS^T Q, dV = P^T dO.
 //
-// Two kernels, no atomics (deterministic):
+// Two paths.  The default (head_dim 128) is dkdvq_kernel, one CTA per
+// 128-key tile that forms dK, dV and its share of dQ, summed into an fp32
+// accumulator by bulk reductions (described at the kernel), then
+// dq_convert_kernel.  The deterministic path is two kernels without
+// reductions:
 //   dq_kernel    one CTA per 128-query tile; walks the CSR like the forward,
 //                two key units (128 keys) per step: S = Q K^T and dP = dO V^T
 //                with Q and dO held in TMEM (TS MMAs), dS -> TMEM (fp16),
@@ -21,7 +25,8 @@
 //                softmax of step i overlaps dK(i-1) and dP^T(i), and S^T(i)
 //                waits only for dV(i-1) to have read P^T(i-1).
 // Operands are fp16 conversions of the bf16 inputs (exact for 2^-17 <= |x| <=
-// 65504 and for 0, see the forward).
+// 65504 and for 0, see the forward; heads beyond that range are pre-scaled by
+// a power of two that the kernels fold back).
 // Roles: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer, warps 4-11
 // two compute warpgroups (one thread per TMEM lane), each taking one of the
 // step's two 64-token units.

@@ -345,7 +345,7 @@ int prism_attn_fwd(const prism_params *p, const prism_plan_t *plan,
  *   dQ,dK,dV  [N][heads][head_dim]; bf16 when grad_fp32 == 0, fp32 else.
  *   deterministic  0: for head_dim 128, one kernel per 128-key tile forms
  *             dK, dV and that tile's share of dQ (dQ = scale dS K added into
- *             an fp32 accumulator in the workspace by fp32 atomic adds, then
+ *             an fp32 accumulator in the workspace by fp32 reductions, then
  *             converted to dQ); 10 P D flops for P computed query-key pairs.
  *             The order of those adds varies from run to run, so dQ may
  *             differ in its last bits between runs (dK, dV do not).

@@ -823,8 +823,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   done).  Warp 2 issues one 32 KB bulk reduction per unit (the unit's 64
 //   accumulator rows are contiguous) and releases the two buffers when the
 //   copies have read them, so the reductions run behind the next step.
-//   MMA issue order of iteration i: dV(i-1), S^T(i) (which runs while the
-//   compute warps form dS(i-1)), dK(i-1), dQ^T(i-1), dP^T(i).
+//   MMA issue order of iteration i: dV(i-1), dK(i-1), dQ^T(i-1), S^T(i),
+//   dP^T(i): dQ^T(i-1), which the compute warps wait for, goes ahead of
+//   S^T(i), which they need only after staging it.
 // ---------------------------------------------------------------------------
 struct FusedSmem {
   static constexpr int TILE = 128 * 128 * 2;  // 128 rows of 128 fp16
@@ -1035,21 +1036,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_ts(tV, tS + pk_col(ks), dDOmn + (uint64_t)ks * 128, id_acc, (i > 1 || ks > 0) ? 1u : 0u);
           mma_commit(&bar.dv_done);
         }
-        uint32_t id = id_full;
-        if (i < nsteps) {  // S^T(i) = K Q(i)^T, into the columns dV(i-1) read P^T(i-1) from; it runs
-                           // while the compute warps form dS(i-1)
-          ok = mbar_wait(&bar.q_full[s], (i / NS) & 1, status, 66);
-          if (ok && i >= 1) ok = mbar_wait(&bar.dv_done, (i - 1) & 1, status, 67);
-          if (!ok) break;
-          tc_fence_after();
-          const int nu = bar.meta[s] & 15;  // written before the stage's Q arrived
-          id = nu == 2 ? id_full : id_half;
-          const uint64_t dQs = sdesc_sw128(smem_u32(smem + L::OFF_Q + s * L::TILE), 16, 1024);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tS, dKd + kslice16(kk, 128 * 128), dQs + kslice16(kk, 128 * 128), id, kk > 0 ? 1u : 0u);
-          mma_commit(&bar.s_full);
-        }
         if (i >= 1) {  // dK += dS^T(i-1) Q(i-1); dQ^T(i-1) = K^T dS^T(i-1) into the dP^T columns
           ok = mbar_wait(&bar.ds_ready, (i - 1) & 1, status, 68);
           if (!ok) break;
@@ -1063,6 +1049,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int ks = 0; ks < 8; ++ks)
             mma_ss(tP, dKmn + (uint64_t)ks * 128, dSmn + (uint64_t)ks * 128, id_q, ks > 0 ? 1u : 0u);
           mma_commit(&bar.dq_full);  // also covers dK(i-1), issued before
+        }
+        uint32_t id = id_full;
+        if (i < nsteps) {  // S^T(i) = K Q(i)^T, into the columns dV(i-1) read P^T(i-1) from
+          ok = mbar_wait(&bar.q_full[s], (i / NS) & 1, status, 66);
+          if (ok && i >= 1) ok = mbar_wait(&bar.dv_done, (i - 1) & 1, status, 67);
+          if (!ok) break;
+          tc_fence_after();
+          const int nu = bar.meta[s] & 15;  // written before the stage's Q arrived
+          id = nu == 2 ? id_full : id_half;
+          const uint64_t dQs = sdesc_sw128(smem_u32(smem + L::OFF_Q + s * L::TILE), 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tS, dKd + kslice16(kk, 128 * 128), dQs + kslice16(kk, 128 * 128), id, kk > 0 ? 1u : 0u);
+          mma_commit(&bar.s_full);
         }
         if (i < nsteps) {  // dP^T(i) = V dO(i)^T, once the compute warps have read dQ^T(i-1)
           ok = mbar_wait(&bar.o_full[s], (i / NS) & 1, status, 69);

@@ -139,6 +139,26 @@ def test_misaligned_tensor_pointers_are_rejected_before_any_cuda_call():
     rc = lib.prism_attn_bwd(C.byref(p), C.byref(plan), C.byref(sel), *[C.c_void_p(256)] * 5, C.c_void_p(256),
                             C.c_void_p(256), C.c_void_p(256), C.c_void_p(260), C.c_void_p(256), 1, 0, ws, 1 << 40, None)
     assert rc == _lib.PRISM_ERR_INVALID_ARG and "dK" in lib.prism_last_error().decode()
+    # the backward's path selector takes 0 (fused) or 1 (deterministic) only
+    for det in (2, -1):
+        rc = lib.prism_attn_bwd(C.byref(p), C.byref(plan), C.byref(sel), *[C.c_void_p(256)] * 10, 1, det, ws,
+                                1 << 40, None)
+        assert rc == _lib.PRISM_ERR_INVALID_ARG and "deterministic" in lib.prism_last_error().decode()
+
+
+def test_backward_workspace_holds_the_fused_accumulator():
+    """For head_dim 128 the backward's workspace includes the fused path's
+    fp32 dQ accumulator (4 * N * heads * 128 bytes) on top of the two-kernel
+    path's needs; head_dim 64 has no fused path and no accumulator."""
+    lib = _lib.load()
+    for D in (64, 128):
+        p = api.params(56, 96, 160, 24, D)
+        N = 56 * 96 * 160
+        bwd, fwd = lib.prism_attn_workspace_size(C.byref(p), 1), lib.prism_attn_workspace_size(C.byref(p), 0)
+        copies = 4 * N * 24 * D * 2      # Q, K, V, dO gathered as fp16
+        acc = 4 * N * 24 * D if D == 128 else 0
+        assert copies + acc <= bwd < copies + acc + (256 << 20), (D, bwd)  # + LSE, Delta, walk tables
+        assert fwd < bwd
 
 
 @pytest.mark.parametrize("C_", [0, 32, 100, 70000])

@@ -98,6 +98,11 @@ BENCH = [
  ("stale traffic still reported", "        if source_digest(d[\"source\"]) != d[\"code_digest\"]:", "        if False:"),
  ("clock median as mean", "return {\"sm_mhz\": statistics.median(sm) if sm else None", "return {\"sm_mhz\": statistics.mean(sm) if sm else None"),
  ("throttle reasons ignored", "                if v.strip().lower() == \"active\":", "                if False:"),
+ ("fused backward issued as 14PD", "\"issued_TFLOPs\": (10.0 if one else 14.0)", "\"issued_TFLOPs\": (14.0 if one else 14.0)"),
+ ("accumulator zeroing not counted", "(12.0 if fused else 8.0) * HBD", "8.0 * HBD"),
+ ("e2e: a step does not wait for its inputs", "            cs.wait_event(ev_in[b])\n", "            pass\n"),
+ ("e2e: results copied before the step ends", "            xs.wait_event(ev_done[b])\n            with torch.cuda.stream(xs):\n                for src, dst",
+  "            with torch.cuda.stream(xs):\n                for src, dst"),
 ]
 
 BINDING = [
@@ -112,9 +117,11 @@ BINDING = [
  ("binding: no growth on short capacity", "out.col.numel() < cs.nnz <= 0x7fffffff", "False"),
  ("binding: residual always passed", "_ptr(O_res) if residual else None, _ptr(lse)", "_ptr(O_res), _ptr(lse)"),
  ("binding: gradients in the wrong order", "_ptr(dQ), _ptr(dK), _ptr(dV)", "_ptr(dK), _ptr(dQ), _ptr(dV)"),
+ ("binding: backward path selector dropped", "int(bool(deterministic))", "0"),
 ]
 
 CABI = [  # (file under the package's csrc/, name, old, new); the copy's library is rebuilt for each
+ ("api.cu", "C: backward path selector unchecked", "if (deterministic != 0 && deterministic != 1)", "if (false)"),
  ("api.cu", "C: zone edge unchecked", "if (p->T % 8 || p->H % 8 || p->W % 8)", "if (false)"),
  ("api.cu", "C: head_dim 96 accepted", "if (p->head_dim != 64 && p->head_dim != 128)", "if (false)"),
  ("api.cu", "C: grid size unchecked", "if (N * p->heads * p->head_dim >= (1LL << 40) || N >= (1LL << 30))", "if (false)"),

@@ -100,6 +100,31 @@ def test_computed_pairs_with_a_different_block_table_per_head():
     assert got == _dense_mask_pairs(w, opl, osel)
 
 
+def test_kernel_roofline_arithmetic_on_the_fused_backward():
+    """With the fused kernel (and its dQ conversion) the combined backward
+    is 10PD over those two kernels, issued and algorithmic alike, and
+    bwd_prep's bytes include the accumulator's zeroing."""
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops_sustained": 1000.0, "bf16_tflops": 1200.0}
+    P, D, N, h, steps = 1.0e12, 128, 860160, 24, 2
+    nb = torch.tensor([100, 200])
+    kt = {"attn_fwd": (2, 1000.0), "attn_bwd_fused": (2, 2396.0), "dq_convert": (2, 4.0), "bwd_prep": (2, 10.0),
+          "attn_bwd_dkdv": (0, 0.0), "attn_bwd_dq": (0, 0.0)}
+    out = bench.kernel_rooflines(kt, P, D, N, h, nb, peaks, "measured", steps)
+    assert out["attn_bwd_fused"]["achieved"] == pytest.approx(10 * P * D / 1.198 / 1e12)
+    bwd = out["attn_bwd"]
+    assert bwd["path"] == "fused" and bwd["ms_per_launch"] == pytest.approx(1200.0)
+    assert bwd["achieved"] == pytest.approx(10 * P * D / 1.2 / 1e12)
+    assert bwd["issued_TFLOPs"] == pytest.approx(bwd["achieved"])
+    assert out["attn_fwd_bwd"]["achieved"] == pytest.approx(14 * P * D / 1.7 / 1e12)
+    assert out["dq_convert"]["achieved"] == pytest.approx((6 * N * h * D + 4 * N * h) / 2e-3 / 1e9)
+    assert out["bwd_prep"]["achieved"] == pytest.approx((12 * N * h * D + 16 * N * h) / 5e-3 / 1e9)
+    # the two-kernel path's bwd_prep has no accumulator to zero
+    kt2 = {"attn_bwd_dkdv": (2, 1600.0), "attn_bwd_dq": (2, 1200.0), "bwd_prep": (2, 10.0)}
+    out2 = bench.kernel_rooflines(kt2, P, D, N, h, nb, peaks, "measured", steps)
+    assert out2["bwd_prep"]["achieved"] == pytest.approx((8 * N * h * D + 16 * N * h) / 5e-3 / 1e9)
+    assert out2["attn_bwd"]["path"] == "two-kernel deterministic"
+
+
 def test_kernel_roofline_arithmetic():
     peaks = {"hbm_gbs": 6000.0, "bf16_tflops_sustained": 1000.0, "bf16_tflops": 1200.0, "sm_max_mhz": 2000.0}
     P, D, N, h, steps = 1.0e12, 128, 860160, 24, 2

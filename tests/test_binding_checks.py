@@ -207,6 +207,8 @@ def test_marshalling_through_a_fake_library(monkeypatch):
     assert [t.value for t in args[3:13]] == [t.data_ptr() for t in want]
     assert args[13] == 1 and args[14] == 0 and args[16] == 4096 and dQ.dtype == torch.float32 and dQ.shape == (N, HEADS, D)
 
+    api.attn_bwd(P, pl, sel, x["Q"], x["K"], x["V"], fw.O, x["dO"], fw.lse, grad_fp32=True, deterministic=True)
+    assert fake.calls[-1][1][14] == 1                # the path selector reaches the library
     with pytest.raises(ValueError, match="dQ must be torch.bfloat16"):
         api.attn_bwd(P, pl, sel, x["Q"], x["K"], x["V"], fw.O, x["dO"], fw.lse, out=(dQ, dK, dV))
     assert api.workspace_status(fw.ws) == 0

@@ -591,6 +591,17 @@ def read_stream_gbs(device, nbytes=4 << 30, iters=5):
     return gbs
 
 
+def pinned_like(t):
+    """A page-locked host tensor of t's shape and dtype."""
+    return torch.empty(tuple(t.shape), dtype=t.dtype, pin_memory=True)
+
+
+def pinned_copy(t):
+    """t copied into page-locked host memory directly (no pageable copy in
+    between: each rank holds tens of GB of these at the 2K size)."""
+    return pinned_like(t).copy_(t)
+
+
 def run_e2e(args, primary, step, names, backward, total_flops, world, device):
     """The same metric end to end through the public API with host buffers:
     every step copies its inputs from pinned host memory and its results (O,
@@ -599,9 +610,9 @@ def run_e2e(args, primary, step, names, backward, total_flops, world, device):
     stream while step k (k+1) computes; otherwise the copies run in line with
     the steps.  Timed with CUDA events from before the first copy to after the
     last, over ksteps steps."""
-    hin = {k: primary[k].cpu().pin_memory() for k in names}
+    hin = {k: pinned_copy(primary[k]) for k in names}
     outs_of = lambda b: [b["O"]] + (list(b["grads"]) if backward else [])  # noqa: E731
-    hout = [torch.empty_like(t, device="cpu").pin_memory() for t in outs_of(primary)]
+    hout = [pinned_like(t) for t in outs_of(primary)]
     h2d = sum(t.numel() * t.element_size() for t in hin.values())
     d2h = sum(t.numel() * t.element_size() for t in hout)
     free, _ = torch.cuda.mem_get_info(device)

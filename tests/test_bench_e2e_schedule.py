@@ -116,6 +116,8 @@ def test_e2e_schedule_orders_every_copy(monkeypatch, free_gb, backward):
     monkeypatch.setattr(torch.cuda, "synchronize", lambda *a: None)
     monkeypatch.setattr(torch.cuda, "mem_get_info", lambda *a: (free_gb << 30, 180 << 30))
     monkeypatch.setattr(torch, "empty_like", lambda t, **kw: _Buf("empty"))
+    monkeypatch.setattr(bench, "pinned_copy", lambda t: _Buf("host"))
+    monkeypatch.setattr(bench, "pinned_like", lambda t: _Buf("host"))
     _Sim.current = default
 
     names = ["Q", "K", "X", "hhat"] + (["dO"] if backward else [])

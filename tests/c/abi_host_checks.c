@@ -69,12 +69,18 @@ int main(void) {
   size_t ws_b = prism_attn_workspace_size(&small, 1);
   CHECK(prism_attn_bwd(&small, &plan, &sel, V, V, V, V, NULL, V, (const float *)p256, V, V, V, 0,
                        0, (void *)(uintptr_t)256, ws_b, NULL) == PRISM_ERR_INVALID_ARG);
+  /* and its path selector is 0 (fused) or 1 (deterministic) */
+  sel.col_ptr = p256;
+  sel.row = p256;
+  CHECK(prism_attn_bwd(&small, &plan, &sel, V, V, V, V, NULL, V, (const float *)p256, V, V, V, 0,
+                       2, (void *)(uintptr_t)256, ws_b, NULL) == PRISM_ERR_INVALID_ARG);
+  CHECK(strstr(prism_last_error(), "deterministic") != NULL);
 
   /* a2v_norm: n = 0 is a no-op, a width that is not a multiple of 8 is refused */
   CHECK(prism_a2v_norm(V, 0, 64, 64, (float *)p256, NULL) == PRISM_OK);
   CHECK(prism_a2v_norm(V, 4, 12, 16, (float *)p256, NULL) == PRISM_ERR_INVALID_ARG);
 
-  /* timing ids outside 0..7 are refused */
+  /* timing ids outside 0..PRISM_KERNEL_TIMING_IDS-1 are refused */
   int n = 0;
   double ms = 0.0;
   const char *name = NULL;
